@@ -1,0 +1,161 @@
+/*
+ * tempcache.h - C ABI of the TempCache step on one NVIDIA B200 (sm_100a).
+ *
+ * TempCache (FAST-AR technical summary, section 2.A "TempCache", pt and fr pages)
+ * compresses the temporal KV cache of an autoregressive video-diffusion attention
+ * layer: every new key is hashed with locality-sensitive hashing, matched top-1
+ * against the earlier cache entries, and merged into its match when their
+ * similarity clears a threshold (values averaged, group size n counted); keys
+ * that find no match are appended. Attention then runs over the compressed cache
+ * plus the current chunk and shifts each cache logit by ln n, which Lemma 5.1 of
+ * the paper states is exact when the merged keys are identical.
+ *
+ * Conventions for every call below
+ *   - Token-major tensors K, V, Q, out are row-major [T, H, d] arrays in DEVICE
+ *     memory, in the handle's storage type (bf16 or fp32), 16-byte aligned and
+ *     contiguous. The caller owns them; the library reads K and V only inside the
+ *     stream-ordered work it enqueues and copies them into its own memory.
+ *   - tc_stream is a cudaStream_t value (NULL = the legacy default stream). Calls
+ *     on one handle must use one stream at a time; handles are not thread-safe.
+ *   - Host-detectable errors (bad argument, wrong state, out of memory) return at
+ *     once and change nothing. Errors seen by a kernel are sticky: the next call
+ *     that synchronises (tc_sync, tc_cache_size, the export calls) returns them,
+ *     and every later call returns them too.
+ *   - Every call returns TC_EINVAL for a NULL or destroyed handle.
+ */
+#ifndef TEMPCACHE_H
+#define TEMPCACHE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct tc_ctx* tc_handle;
+typedef void* tc_stream;
+
+typedef enum {
+    TC_OK = 0,
+    TC_EINVAL = 1,     /* bad argument or handle                                   */
+    TC_ENOMEM = 2,     /* device or host allocation failed                         */
+    TC_ECAPACITY = 3,  /* a commit would exceed the per-head capacity              */
+    TC_ECUDA = 4,      /* a CUDA runtime or driver call failed                     */
+    TC_ESTATE = 5,     /* call not valid in the current state                      */
+    TC_ETIMEOUT = 6,   /* a kernel gave up waiting on one of its own barriers      */
+    TC_ENOTIMPL = 7,   /* combination not supported by this build                  */
+    TC_EDEVICE = 8     /* no usable sm_100 device                                  */
+} tc_status;
+
+typedef enum { TC_BF16 = 0, TC_F32 = 1 } tc_dtype;
+
+typedef struct {
+    tc_dtype dtype;            /* storage and I/O type of K, V, Q, out                  */
+    uint64_t seed;             /* seed of the default hyperplanes                      */
+    float softmax_scale;       /* 0 selects 1/sqrt(d)                                  */
+    const float* hyperplanes;  /* HOST [nbits*d] hash normals, each value exactly
+                                  representable in bf16; NULL = N(0,1) draws from seed,
+                                  rounded to bf16. Copied during the call.              */
+} tc_options;
+
+/*
+ * tc_create / tc_create_ex - allocate a TempCache for one attention layer.
+ *   H         heads (>= 1); every head has its own cache.
+ *   d         head dimension: 64 or 128.
+ *   nbits     hash bits, 1..24 (section 2.A: locality-sensitive hashing; the hash
+ *             family is sign-of-random-hyperplane, 2^nbits buckets per head).
+ *   tau       cosine threshold for a merge, -1 <= tau <= 2 (section 2.A: merges
+ *             use a similarity threshold). tau > 1 never merges (dense cache).
+ *   capacity  cache entries per head (>= 1). All device memory for `capacity`
+ *             entries is allocated here.
+ * tc_create uses bf16 storage, seed 0 and scale 1/sqrt(d).
+ * On success *out owns every device buffer of the cache; release it with
+ * tc_destroy. On failure *out is set to NULL. Returns TC_EDEVICE when the
+ * current device is not an sm_100 part.
+ */
+tc_status tc_create(int32_t H, int32_t d, int32_t nbits, float tau, int64_t capacity,
+                    tc_handle* out);
+tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t capacity,
+                       const tc_options* opt, tc_handle* out);
+
+/*
+ * tc_append_chunk - feed the next chunk of T new tokens, K and V [T, H, d].
+ * First commits the chunk staged by the previous call (section 2.A: each new key
+ * is matched top-1 in its hash bucket among the entries committed before; a match
+ * at cosine >= tau merges, v <- (n v + sum v_t)/(n + m), n <- n + m; unmatched
+ * keys are appended in token order), then stages this chunk: copies it into the
+ * library's head-major staging buffer and hashes its keys. Attention sees a staged
+ * chunk raw, with logit shift 0.
+ * Asynchronous on `stream`, except when the committed cache might overflow its
+ * capacity: then the call synchronises to learn the outcome and, if the commit
+ * would overflow, returns TC_ECAPACITY with the cache unchanged, the previous
+ * chunk still staged and this chunk not accepted.
+ * T >= 1. Returns TC_EINVAL for NULL or misaligned K or V.
+ */
+tc_status tc_append_chunk(tc_handle h, const void* K, const void* V, int64_t T,
+                          tc_stream stream);
+
+/*
+ * tc_attend - biased attention of Q [Tq, H, d] over the committed cache entries
+ * (logit shift ln n_j) and the staged chunk (shift 0); writes out [Tq, H, d].
+ * out_t = sum_j exp(s_tj) v_j / sum_j exp(s_tj), s_tj = scale <q_t, k_j> + shift_j,
+ * no mask (section 2.A with Lemma 5.1: averaged values plus a logit shift by the
+ * group size reproduce attention over the identical keys they replace).
+ * bf16 handles compute QK^T and PV on tensor cores with fp32 accumulation and an
+ * fp32 online softmax; fp32 handles compute in fp32 throughout.
+ * Asynchronous on `stream`. Tq >= 1. Returns TC_ESTATE before the first
+ * tc_append_chunk. out must not overlap Q.
+ */
+tc_status tc_attend(tc_handle h, const void* Q, int64_t Tq, void* out, tc_stream stream);
+
+/* tc_flush - commit the staged chunk (if any) and stage nothing. Same capacity
+ * behaviour as tc_append_chunk. */
+tc_status tc_flush(tc_handle h, tc_stream stream);
+
+/* tc_reset - empty the cache and drop any staged chunk, keeping every allocation
+ * (start a new rollout). Asynchronous on `stream`. */
+tc_status tc_reset(tc_handle h, tc_stream stream);
+
+/* tc_cache_size - synchronise and write the committed entry count of every head
+ * to the HOST array sizes_H [H]. */
+tc_status tc_cache_size(tc_handle h, int64_t* sizes_H);
+
+/* tc_sync - synchronise the handle's last stream and return its sticky status. */
+tc_status tc_sync(tc_handle h);
+
+/* tc_destroy - free every buffer of the handle. NULL-safe. Synchronises. */
+void tc_destroy(tc_handle h);
+
+/* tc_status_string - static description of a status code. */
+const char* tc_status_string(tc_status s);
+
+/* ---- inspection (host buffers; every call synchronises) -------------------- */
+
+/* Codes, merge targets (-1 = appended) and final entry index of every token of the
+ * last committed chunk, as HOST arrays [H * T] (head-major); *T_out receives T
+ * (0 if nothing was committed). Any array pointer may be NULL. */
+tc_status tc_debug_last_commit(tc_handle h, int64_t* T_out, uint32_t* codes_HT,
+                               int32_t* match_HT, int32_t* dest_HT);
+
+/* Hash codes of the staged chunk, HOST [H * T_staged]; *T_out receives T_staged. */
+tc_status tc_debug_staged_codes(tc_handle h, int64_t* T_out, uint32_t* codes_HT);
+
+/* Committed entries of head `head` (count from tc_cache_size) into HOST arrays:
+ * K [M*d] in the storage type, V32 [M*d] fp32 running means, n [M], code [M].
+ * Any pointer may be NULL. */
+tc_status tc_export_cache(tc_handle h, int32_t head, void* K, float* V32, int32_t* n,
+                          uint32_t* code);
+
+/* The hash normals in use, HOST [nbits * d]. */
+tc_status tc_get_hyperplanes(tc_handle h, float* R);
+
+/* Kernels this handle has launched so far, and how many hash bits / similarity
+ * decisions needed the exact fp64 re-check (see the search kernel). */
+tc_status tc_stats(tc_handle h, uint64_t* kernel_launches, uint64_t* hash_rechecks,
+                   uint64_t* match_rechecks);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TEMPCACHE_H */

@@ -1,0 +1,232 @@
+"""TempCache on B200: Python binding of the C-ABI library libtempcache.so.
+
+FAST-AR's TempCache (technical summary, section 2.A) compresses the temporal KV
+cache of an autoregressive video-diffusion attention layer: new keys are hashed
+with sign-of-random-hyperplane LSH, matched top-1 against the cache inside their
+bucket, merged into their match above a cosine threshold (values averaged, count n
+kept) or appended; attention then runs over the compressed cache plus the current
+chunk with a +ln n logit shift per cache entry.
+
+This module only marshals arguments: torch tensors supply device memory and the
+current CUDA stream, and every step runs in the library's CUDA kernels. There is
+no CPU fallback; without the built library the import fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "_lib", "libtempcache.so")
+
+TC_OK, TC_EINVAL, TC_ENOMEM, TC_ECAPACITY, TC_ECUDA, TC_ESTATE, TC_ETIMEOUT, TC_ENOTIMPL, TC_EDEVICE = range(9)
+TC_BF16, TC_F32 = 0, 1
+
+API = [
+    "tc_create", "tc_create_ex", "tc_append_chunk", "tc_attend", "tc_flush", "tc_reset", "tc_cache_size", "tc_sync",
+    "tc_destroy", "tc_status_string", "tc_debug_last_commit", "tc_debug_staged_codes", "tc_export_cache",
+    "tc_get_hyperplanes", "tc_stats",
+]
+
+
+class TCOptions(ctypes.Structure):
+    _fields_ = [("dtype", ctypes.c_int), ("seed", ctypes.c_uint64), ("softmax_scale", ctypes.c_float),
+                ("hyperplanes", ctypes.POINTER(ctypes.c_float))]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libtempcache.so is not built ({LIB_PATH}); run "
+                          "`python kv_cache_attention_tempcache_b200/build.py`")
+    lib = ctypes.CDLL(LIB_PATH)
+    H = ctypes.c_void_p
+    i32, i64, f32, vp = ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_void_p
+    sig = {
+        "tc_create": (ctypes.c_int, [i32, i32, i32, f32, i64, ctypes.POINTER(H)]),
+        "tc_create_ex": (ctypes.c_int, [i32, i32, i32, f32, i64, ctypes.POINTER(TCOptions), ctypes.POINTER(H)]),
+        "tc_append_chunk": (ctypes.c_int, [H, vp, vp, i64, vp]),
+        "tc_attend": (ctypes.c_int, [H, vp, i64, vp, vp]),
+        "tc_flush": (ctypes.c_int, [H, vp]),
+        "tc_reset": (ctypes.c_int, [H, vp]),
+        "tc_cache_size": (ctypes.c_int, [H, ctypes.POINTER(i64)]),
+        "tc_sync": (ctypes.c_int, [H]),
+        "tc_destroy": (None, [H]),
+        "tc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "tc_debug_last_commit": (ctypes.c_int, [H, ctypes.POINTER(i64), vp, vp, vp]),
+        "tc_debug_staged_codes": (ctypes.c_int, [H, ctypes.POINTER(i64), vp]),
+        "tc_export_cache": (ctypes.c_int, [H, i32, vp, vp, vp, vp]),
+        "tc_get_hyperplanes": (ctypes.c_int, [H, vp]),
+        "tc_stats": (ctypes.c_int, [H, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64),
+                                    ctypes.POINTER(ctypes.c_uint64)]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+class TempCacheError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lib.tc_status_string(status).decode()} (status {status})")
+
+
+class CapacityError(TempCacheError):
+    pass
+
+
+def _check(status: int, where: str):
+    if status == TC_OK:
+        return
+    if status == TC_ECAPACITY:
+        raise CapacityError(status, where)
+    raise TempCacheError(status, where)
+
+
+def _np_ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+class TempCache:
+    """One attention layer's TempCache on the current CUDA device.
+
+    K, V, Q are [T, H, d] torch tensors in the storage dtype (torch.bfloat16 or
+    torch.float32). CUDA tensors are used in place; CPU tensors are copied to the
+    device on the current stream first (the end-to-end path).
+    """
+
+    def __init__(self, H: int, d: int, nbits: int, tau: float, capacity: int, dtype: str = "bf16",
+                 seed: int = 0, softmax_scale: float = 0.0, hyperplanes=None):
+        self.H, self.d, self.nbits = int(H), int(d), int(nbits)
+        self.dtype = dtype
+        self.torch_dtype = torch.bfloat16 if dtype == "bf16" else torch.float32
+        opt = TCOptions()
+        opt.dtype = TC_BF16 if dtype == "bf16" else TC_F32
+        opt.seed = int(seed)
+        opt.softmax_scale = float(softmax_scale)
+        self._R = None
+        if hyperplanes is not None:
+            R = np.ascontiguousarray(np.asarray(hyperplanes, dtype=np.float32).reshape(-1))
+            self._R = R
+            opt.hyperplanes = R.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
+        self._h = ctypes.c_void_p()
+        _check(lib.tc_create_ex(self.H, self.d, self.nbits, float(tau), int(capacity), ctypes.byref(opt),
+                                ctypes.byref(self._h)), "tc_create_ex")
+        self._keep = []
+
+    # -- helpers ---------------------------------------------------------------
+    def _dev(self, x: torch.Tensor, name: str) -> torch.Tensor:
+        if x.dtype != self.torch_dtype:
+            raise TypeError(f"{name} must be {self.torch_dtype}, got {x.dtype}")
+        if x.dim() != 3 or x.shape[1] != self.H or x.shape[2] != self.d:
+            raise ValueError(f"{name} must be [T, {self.H}, {self.d}], got {tuple(x.shape)}")
+        if not x.is_cuda:
+            x = x.to("cuda", non_blocking=True)
+        return x.contiguous()
+
+    @staticmethod
+    def _stream():
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+    @property
+    def handle(self):
+        return self._h
+
+    # -- verbs -----------------------------------------------------------------
+    def append_chunk(self, K: torch.Tensor, V: torch.Tensor):
+        K = self._dev(K, "K")
+        V = self._dev(V, "V")
+        if K.shape != V.shape:
+            raise ValueError("K and V shapes differ")
+        self._keep = [K, V]  # the kernels read them asynchronously on the stream
+        _check(lib.tc_append_chunk(self._h, K.data_ptr(), V.data_ptr(), K.shape[0], self._stream()),
+               "tc_append_chunk")
+
+    def attend(self, Q: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+        Q = self._dev(Q, "Q")
+        if out is None:
+            out = torch.empty_like(Q)
+        _check(lib.tc_attend(self._h, Q.data_ptr(), Q.shape[0], out.data_ptr(), self._stream()), "tc_attend")
+        return out
+
+    def flush(self):
+        _check(lib.tc_flush(self._h, self._stream()), "tc_flush")
+
+    def reset(self):
+        """Empty the cache (new rollout); allocations are kept."""
+        _check(lib.tc_reset(self._h, self._stream()), "tc_reset")
+
+    def sync(self):
+        _check(lib.tc_sync(self._h), "tc_sync")
+
+    def cache_size(self) -> np.ndarray:
+        out = np.zeros(self.H, dtype=np.int64)
+        _check(lib.tc_cache_size(self._h, out.ctypes.data_as(ctypes.POINTER(ctypes.c_int64))), "tc_cache_size")
+        return out
+
+    def last_commit(self):
+        """(codes, match, dest) of the last committed chunk as [H, T] arrays."""
+        T = ctypes.c_int64()
+        _check(lib.tc_debug_last_commit(self._h, ctypes.byref(T), None, None, None), "tc_debug_last_commit")
+        n = T.value
+        codes = np.zeros((self.H, n), np.uint32)
+        match = np.zeros((self.H, n), np.int32)
+        dest = np.zeros((self.H, n), np.int32)
+        if n:
+            _check(lib.tc_debug_last_commit(self._h, ctypes.byref(T), _np_ptr(codes), _np_ptr(match),
+                                            _np_ptr(dest)), "tc_debug_last_commit")
+        return codes, match, dest
+
+    def staged_codes(self) -> np.ndarray:
+        T = ctypes.c_int64()
+        _check(lib.tc_debug_staged_codes(self._h, ctypes.byref(T), None), "tc_debug_staged_codes")
+        codes = np.zeros((self.H, T.value), np.uint32)
+        if T.value:
+            _check(lib.tc_debug_staged_codes(self._h, ctypes.byref(T), _np_ptr(codes)), "tc_debug_staged_codes")
+        return codes
+
+    def export_cache(self, head: int):
+        """(K [M,d] as fp32, V32 [M,d], n [M], code [M]) of one head's committed entries."""
+        M = int(self.cache_size()[head])
+        K = np.zeros((M, self.d), np.uint16 if self.dtype == "bf16" else np.float32)
+        V = np.zeros((M, self.d), np.float32)
+        n = np.zeros(M, np.int32)
+        code = np.zeros(M, np.uint32)
+        _check(lib.tc_export_cache(self._h, head, _np_ptr(K), _np_ptr(V), _np_ptr(n), _np_ptr(code)),
+               "tc_export_cache")
+        if self.dtype == "bf16":
+            K = (K.astype(np.uint32) << 16).view(np.float32)
+        return K, V, n, code
+
+    def hyperplanes(self) -> np.ndarray:
+        R = np.zeros((self.nbits, self.d), np.float32)
+        _check(lib.tc_get_hyperplanes(self._h, _np_ptr(R)), "tc_get_hyperplanes")
+        return R
+
+    def stats(self):
+        a, b, c = ctypes.c_uint64(), ctypes.c_uint64(), ctypes.c_uint64()
+        _check(lib.tc_stats(self._h, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)), "tc_stats")
+        return {"kernel_launches": a.value, "hash_rechecks": b.value, "match_rechecks": c.value}
+
+    def launch_count(self) -> int:
+        a = ctypes.c_uint64()
+        _check(lib.tc_stats(self._h, ctypes.byref(a), None, None), "tc_stats")
+        return a.value
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            lib.tc_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,78 @@
+// Internal declarations shared by the TempCache host runtime and its kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace tc {
+
+// Device state of one TempCache. Per-head arrays have a padded row stride
+// capP = round_up(capacity, 128) so a 128-row attention tile never leaves its head.
+struct CacheView {
+    int H, d, nbits;
+    int64_t capP;          // padded capacity per head
+    int64_t capacity;      // usable entries per head
+    void* Kc;              // [H][capP][d] storage type, representative keys
+    void* Vc;              // [H][capP][d] storage type, value means (attention operand)
+    float* V32;            // [H][capP][d] fp32 value means (master copy)
+    int32_t* cnt;          // [H][capP] group sizes n
+    float* bias2;          // [H][capP] log2(n); -inf for unused rows
+    uint32_t* code;        // [H][capP]
+    int32_t* bnext;        // [H][capP] next older entry in the same bucket, -1 ends
+    int32_t* bhead;        // [H][2^nbits] newest entry of each bucket, -1 = empty
+    int32_t* mcount;       // [H][capP] tokens merging into the entry in this commit (0 between commits)
+    int32_t* mfill;        // [H][capP] fill cursor of the entry's merge segment (0 between commits)
+    int32_t* moff;         // [H][capP] start of the entry's merge segment
+    int32_t* M;            // [H] committed entries
+};
+
+struct StageView {
+    int64_t TmaxP;         // staging rows per head (multiple of 128)
+    int64_t T;             // tokens staged (or being committed)
+    void* Ks;              // [H][TmaxP][d]
+    void* Vs;              // [H][TmaxP][d]
+    uint32_t* scode;       // [H][TmaxP] hash codes of the staged tokens
+    float* sbias;          // [TmaxP] 0 for t < T, -inf beyond
+    int32_t* match;        // [H][TmaxP] merge target or -1 (last commit)
+    int32_t* dest;         // [H][TmaxP] entry each token ended in (last commit)
+    uint32_t* lcode;       // [H][TmaxP] codes of the last committed chunk
+    int32_t* seg;          // [H][TmaxP] token ids grouped by merge target
+    int32_t* touched;      // [H][TmaxP] entries with at least one merge
+};
+
+// Per-commit counters (int32, reset at the start of every commit):
+//   ctr[0, H)   entries touched by merges, per head
+//   ctr[H, 2H)  cache size after the commit, per head
+//   ctr[2H]     abort flag: some head would exceed its capacity
+constexpr int kCtrInts(int H) { return 2 * H + 2; }
+
+// Sticky device-side statistics and error bits.
+enum : unsigned { kErrBucketList = 1u, kErrTimeout = 2u };
+struct Stats {
+    unsigned long long hash_rechecks;
+    unsigned long long match_rechecks;
+    unsigned int error_bits;
+    unsigned int pad;
+};
+
+// Launchers (tc_commit.cu).
+cudaError_t launch_stage_hash(const CacheView& c, const StageView& s, int dtype,
+                              const void* K, const void* V, const float* R, const float* Rnorm,
+                              Stats* stats, cudaStream_t st);
+cudaError_t launch_commit(const CacheView& c, const StageView& s, int dtype, float tau,
+                          int32_t* ctr, Stats* stats, int* launches, cudaStream_t st);
+
+// Launchers (tc_attn_f32.cu, tc_attn_bf16.cu).
+cudaError_t launch_attend_f32(const CacheView& c, const StageView& s, const float* Q,
+                              int64_t Tq, float* out, float scale_log2, cudaStream_t st);
+
+struct AttnMaps {
+    CUtensorMap q, kc, vc, ks, vs;
+};
+cudaError_t launch_attend_bf16(const CacheView& c, const StageView& s, const AttnMaps& maps,
+                               int64_t Tq, __nv_bfloat16* out, float scale_log2, Stats* stats,
+                               cudaStream_t st);
+
+}  // namespace tc

@@ -1,0 +1,112 @@
+"""Drives the CUDA TempCache and the CPU oracle side by side on one seeded workload.
+
+Used by the GPU parity tests and by the smoke check. Inputs come from the shared
+generator (synthetic/); expected values come only from oracle/.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+from oracle import OracleTempCache
+from synthetic import Workload
+
+
+def f64(x: torch.Tensor) -> np.ndarray:
+    return x.detach().to(torch.float64).cpu().numpy()
+
+
+@dataclass
+class ParityReport:
+    commits: int = 0
+    tokens: int = 0
+    code_mismatch: int = 0
+    match_mismatch: int = 0
+    dest_mismatch: int = 0
+    size_mismatch: int = 0
+    key_mismatch: int = 0
+    count_mismatch: int = 0
+    v32_max_err: float = 0.0
+    attn_max_err: float = 0.0
+    attn_mean_err: float = 0.0
+    attn_checks: int = 0
+    merges: int = 0
+    sizes: list = field(default_factory=list)
+
+
+def compare_state(tc, o, rep: ParityReport, heads):
+    sizes_gpu = tc.cache_size()
+    sizes_ref = o.cache_size()
+    rep.size_mismatch += int((sizes_gpu != sizes_ref).sum())
+    for h in heads:
+        K, V32, n, code = tc.export_cache(h)
+        k_ref, v_ref, n_ref, c_ref = o.export_head(h)
+        if K.shape[0] != k_ref.shape[0]:
+            rep.key_mismatch += 1
+            continue
+        rep.key_mismatch += int((K.astype(np.float64) != k_ref).any(axis=1).sum())
+        rep.count_mismatch += int((n != n_ref).sum()) + int((code != c_ref).sum())
+        if V32.size:
+            rep.v32_max_err = max(rep.v32_max_err, float(np.abs(V32.astype(np.float64) - v_ref).max()))
+
+
+def run_parity(cfg, chunks=None, attends=1, rows=None, state_heads=None, flush=True, device="cuda",
+               check_every_state=True):
+    """Run `chunks` chunks through both implementations and collect the differences.
+
+    rows: query rows checked per attend (None = all). state_heads: heads whose
+    cache contents are compared after every commit (None = all).
+    """
+    from kv_cache_attention_tempcache_b200 import TempCache
+
+    chunks = cfg.chunks if chunks is None else chunks
+    w = Workload(cfg, device=device)
+    R = w.hyperplanes()
+    tc = TempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, dtype=cfg.dtype, hyperplanes=R.numpy())
+    o = OracleTempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, R.double().numpy())
+    heads = range(cfg.H) if state_heads is None else state_heads
+    rep = ParityReport()
+    sum_abs, n_abs = 0.0, 0
+    for c in range(chunks):
+        K, V = w.next_chunk()
+        rec = o.append_chunk(f64(K), f64(V))
+        tc.append_chunk(K, V)
+        rep.code_mismatch += int((tc.staged_codes() != o.staged[2]).sum())
+        if rec is not None:
+            codes, match, dest = tc.last_commit()
+            rep.commits += 1
+            rep.tokens += match.size
+            rep.merges += int((rec.match >= 0).sum())
+            rep.code_mismatch += int((codes != rec.codes).sum())
+            rep.match_mismatch += int((match != rec.match).sum())
+            rep.dest_mismatch += int((dest != rec.dest).sum())
+            if check_every_state or c == chunks - 1:
+                compare_state(tc, o, rep, heads)
+            rep.sizes.append(o.cache_size().tolist())
+        for a in range(attends):
+            Q = w.queries(c, a)
+            out = tc.attend(Q)
+            sel = None if rows is None else np.asarray(rows)
+            ref = o.attend(f64(Q), rows=sel)
+            got = f64(out) if sel is None else f64(out[torch.as_tensor(sel, device=out.device)])
+            err = np.abs(got - ref)
+            rep.attn_max_err = max(rep.attn_max_err, float(err.max()))
+            sum_abs += float(err.sum())
+            n_abs += err.size
+            rep.attn_checks += 1
+    if flush:
+        rec = o.flush()
+        tc.flush()
+        if rec is not None:
+            codes, match, dest = tc.last_commit()
+            rep.commits += 1
+            rep.tokens += match.size
+            rep.code_mismatch += int((codes != rec.codes).sum())
+            rep.match_mismatch += int((match != rec.match).sum())
+            rep.dest_mismatch += int((dest != rec.dest).sum())
+            compare_state(tc, o, rep, heads)
+    rep.attn_mean_err = sum_abs / max(n_abs, 1)
+    tc.sync()
+    return rep, tc, o

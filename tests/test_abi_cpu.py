@@ -1,0 +1,95 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every
+function include/tempcache.h declares, and rejects bad arguments before touching
+the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tempcache.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tc_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def tcmod():
+    import kv_cache_attention_tempcache_b200 as m
+    return m
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("tc_create", "tc_append_chunk", "tc_attend", "tc_cache_size", "tc_destroy"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(tcmod):
+    lib = ctypes.CDLL(tcmod.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(tcmod.API) == set(declared_functions())
+
+
+def test_status_strings(tcmod):
+    for s in range(9):
+        assert tcmod.lib.tc_status_string(s)
+    assert tcmod.lib.tc_status_string(99) == b"unknown status"
+
+
+@pytest.mark.parametrize("args", [
+    (0, 128, 16, 0.95, 100),       # H < 1
+    (4, 96, 16, 0.95, 100),        # d not 64/128
+    (4, 128, 0, 0.95, 100),        # nbits < 1
+    (4, 128, 25, 0.95, 100),       # nbits > 24
+    (4, 128, 16, -1.5, 100),       # tau < -1
+    (4, 128, 16, 2.5, 100),        # tau > 2
+    (4, 128, 16, float("nan"), 100),
+    (4, 128, 16, 0.95, 0),         # capacity < 1
+])
+def test_create_rejects_bad_arguments(tcmod, args):
+    h = ctypes.c_void_p()
+    assert tcmod.lib.tc_create(*args, ctypes.byref(h)) == tcmod.TC_EINVAL
+    assert not h.value
+
+
+def test_create_rejects_non_bf16_hyperplanes(tcmod):
+    import numpy as np
+    R = np.full(2 * 64, 0.1, dtype=np.float32)  # 0.1 is not a bf16 value
+    opt = tcmod.TCOptions()
+    opt.dtype = tcmod.TC_BF16
+    opt.hyperplanes = R.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
+    h = ctypes.c_void_p()
+    assert tcmod.lib.tc_create_ex(1, 64, 2, 0.9, 10, ctypes.byref(opt), ctypes.byref(h)) == tcmod.TC_EINVAL
+
+
+def test_null_handle_is_rejected_everywhere(tcmod):
+    L, E = tcmod.lib, tcmod.TC_EINVAL
+    buf = (ctypes.c_int64 * 4)()
+    assert L.tc_append_chunk(None, None, None, 1, None) == E
+    assert L.tc_attend(None, None, 1, None, None) == E
+    assert L.tc_flush(None, None) == E
+    assert L.tc_reset(None, None) == E
+    assert L.tc_cache_size(None, buf) == E
+    assert L.tc_sync(None) == E
+    assert L.tc_debug_last_commit(None, None, None, None, None) == E
+    assert L.tc_debug_staged_codes(None, None, None) == E
+    assert L.tc_export_cache(None, 0, None, None, None, None) == E
+    assert L.tc_get_hyperplanes(None, None) == E
+    assert L.tc_stats(None, None, None, None) == E
+    L.tc_destroy(None)  # NULL-safe
+
+
+def test_create_without_device_reports_it(tcmod):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    h = ctypes.c_void_p()
+    st = tcmod.lib.tc_create(2, 128, 16, 0.95, 1000, ctypes.byref(h))
+    assert st in (tcmod.TC_EDEVICE, tcmod.TC_ECUDA)
+    assert not h.value
