@@ -1,0 +1,450 @@
+#!/usr/bin/env python
+"""TempCache benchmark: frames/s of the Wan-2.1-1.3B-shaped attention layer.
+
+A step is one full rollout of the workload from an empty cache: 40 chunks of 3
+frames (4680 tokens, 12 heads, d = 128, bf16), each chunk one tc_append_chunk
+(commit of the previous chunk: hash, bucket search, merge, append; staging of this
+one) followed by 4 tc_attend calls. value = frames processed by all ranks / the
+slowest rank's device time. Inputs are generated before timing and stay resident
+in HBM (3.5 GB of distinct K, V, Q per rollout, far larger than the 126 MB L2).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+N > 1 runs under torchrun: each rank runs an independent rollout (its own seed);
+there is no collective in the data path, only the max-over-ranks of the timing.
+--impl reference times the CPU oracle (fp64 NumPy) on the host instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from synthetic import CONFIGS  # noqa: E402
+
+WORKLOAD = "wan1.3b"
+METRIC = "TempCache frames/s (merge+4x attend) at Wan-1.3B shape; attn TFLOP/s vs peak"
+UNIT = "frames/s"
+MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attention_traffic.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- plumbing
+
+def dist_info():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def init_dist(world: int, backend: str):
+    if world > 1 and not torch.distributed.is_initialized():
+        import datetime
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Largest value of x over all ranks (the step time of the slowest GPU)."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_rate(units_per_rank: float, world: int, max_seconds: float) -> float:
+    """Whole-job throughput: the units of every rank over the slowest rank's time."""
+    return units_per_rank * world / max_seconds
+
+
+def rank_seed(base: int, rank: int) -> int:
+    return base + 7919 * rank
+
+
+def barrier(world: int):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def load_peaks():
+    if os.path.exists(MEASURED_PEAKS):
+        with open(MEASURED_PEAKS) as f:
+            return json.load(f), "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                rows.append((float(p[1]), float(p[2]), p[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, fl in rows for i, v in enumerate(fl) if v.lower() == "active"})
+        sm = [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- workload
+
+def generate_inputs(cfg, device, seed):
+    from synthetic import Workload
+
+    w = Workload(cfg.replace(seed=seed), device=device)
+    chunks = []
+    for c in range(cfg.chunks):
+        K, V = w.next_chunk()
+        Qs = [w.queries(c, a) for a in range(cfg.attends)]
+        chunks.append((K, V, Qs))
+    return w.hyperplanes().numpy(), chunks
+
+
+def rollout(tc, chunks, outs, attn_events=None, app_events=None):
+    tc.reset()
+    for c, (K, V, Qs) in enumerate(chunks):
+        if app_events is not None:
+            app_events[c][0].record()
+        tc.append_chunk(K, V)
+        if app_events is not None:
+            app_events[c][1].record()
+        for a, Q in enumerate(Qs):
+            if attn_events is not None:
+                attn_events[c][a][0].record()
+            tc.attend(Q, out=outs[a])
+            if attn_events is not None:
+                attn_events[c][a][1].record()
+
+
+def sizes_per_chunk(tc, chunks, outs, cfg):
+    """Committed entries per head seen by the attends of each chunk, and commit counts."""
+    tc.reset()
+    sizes, commit = [], []
+    for K, V, Qs in chunks:
+        tc.append_chunk(K, V)
+        sizes.append(tc.cache_size().copy())
+        _, match, _ = tc.last_commit()
+        if match.size:
+            touched = sum(len(np.unique(match[h][match[h] >= 0])) for h in range(cfg.H))
+            commit.append(((match < 0).sum(), (match >= 0).sum(), touched, match.shape[1]))
+        else:
+            commit.append((0, 0, 0, 0))
+        for a, Q in enumerate(Qs):
+            tc.attend(Q, out=outs[a])
+    return sizes, commit
+
+
+def attn_flops(cfg, sizes):
+    """4 * Tq * (M_h + T) * d summed over heads, for every attend of the rollout."""
+    per_chunk = [4.0 * cfg.T * float((s + cfg.T).sum()) * cfg.d for s in sizes]
+    return per_chunk  # one attend call of chunk c
+
+
+def commit_bytes(cfg, commit_counts, b=2):
+    """Algorithmic bytes of one tc_append_chunk: staging copy + hash, reading every
+    staged key once for the search, appending unmatched rows (K, V, fp32 V) and
+    updating merged entries (read the matched V rows, read+write fp32 V, write V)."""
+    T, H, d = cfg.T, cfg.H, cfg.d
+    total = []
+    for u, m, e, Tc in commit_counts:
+        stage = 4 * T * H * d * b + 4 * T * H
+        search = Tc * H * d * b + 8 * Tc * H if Tc else 0
+        append = u * (2 * d * b + 2 * d * b + 4 * d + 16)
+        merge = m * (d * b + 4) + e * (2 * 4 * d + d * b + 8)
+        total.append(stage + search + append + merge)
+    return total
+
+
+# ----------------------------------------------------------------------------- CPU oracle leg
+
+def oracle_sample(cfg, chunks_cpu, R, n_chunks, rows_per_attend, time_budget_s, warmup_chunks=0):
+    """Time the CPU oracle over consecutive chunks of the rollout.
+
+    Every chunk runs the oracle's full merge path; attention runs on
+    `rows_per_attend` query rows per call and its time is scaled to all rows.
+    Returns (frames/s, chunks timed, description).
+    """
+    from oracle import OracleTempCache
+
+    o = OracleTempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, R.astype(np.float64))
+    rng = np.random.default_rng(0)
+    total, timed = 0.0, 0
+    for c, (K, V, Qs) in enumerate(chunks_cpu):
+        if c >= warmup_chunks + n_chunks:
+            break
+        t0 = time.perf_counter()
+        o.append_chunk(K, V)
+        t_merge = time.perf_counter() - t0
+        t_attn = 0.0
+        for Q in Qs:
+            rows = np.sort(rng.choice(cfg.T, size=min(rows_per_attend, cfg.T), replace=False))
+            t1 = time.perf_counter()
+            o.attend(Q, rows=rows)
+            t_attn += (time.perf_counter() - t1) * (cfg.T / len(rows))
+        if c >= warmup_chunks:
+            total += t_merge + t_attn
+            timed += 1
+        if total > time_budget_s and timed >= 1:
+            break
+    desc = (f"chunks {warmup_chunks}..{warmup_chunks + timed - 1} of the {WORKLOAD} rollout: full oracle "
+            f"merge path; attention on {rows_per_attend} of {cfg.T} query rows per call, time scaled to all rows")
+    return cfg.F * timed / total, timed, desc
+
+
+def cpu_inputs(chunks):
+    f = lambda x: x.to(torch.float64).cpu().numpy()  # noqa: E731
+    return [(f(K), f(V), [f(Q) for Q in Qs]) for K, V, Qs in chunks]
+
+
+def run_reference(args):
+    rank, world, _ = dist_info()
+    if rank != 0:
+        return
+    cfg = CONFIGS[WORKLOAD]
+    R, chunks = generate_inputs(cfg.replace(chunks=args.warmup + args.steps), "cpu", cfg.seed)
+    value, timed, desc = oracle_sample(cfg, cpu_inputs(chunks), R, args.steps, 256, float("inf"),
+                                       warmup_chunks=args.warmup)
+    cores = len(os.sched_getaffinity(0))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * cfg.F / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{WORKLOAD}: H=12 d=128 P=1560 F=3 S=4096 p_stay=0.8 sigma=0.05 nbits=16 "
+                               f"tau=0.95", "step": "one chunk (commit + 4 attends) of the rollout"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU leg
+
+def time_e2e(tc, cfg, chunks, steps=1):
+    """Frames/s through the public API with inputs in pinned host memory: each chunk's
+    K, V and Q are copied in and every attention output is read back inside the
+    timed region."""
+    host = [(K.cpu().pin_memory(), V.cpu().pin_memory(), [Q.cpu().pin_memory() for Q in Qs])
+            for K, V, Qs in chunks]
+    outs_host = [torch.empty(cfg.T, cfg.H, cfg.d, dtype=torch.bfloat16).pin_memory() for _ in range(cfg.attends)]
+
+    def one():
+        tc.reset()
+        for K, V, Qs in host:
+            tc.append_chunk(K, V)
+            for a, Q in enumerate(Qs):
+                out = tc.attend(Q)
+                outs_host[a].copy_(out, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        one()
+    e1.record()
+    torch.cuda.synchronize()
+    sec = e0.elapsed_time(e1) / 1000.0 / steps
+    per = cfg.T * cfg.H * cfg.d * 2
+    h2d = cfg.chunks * (2 + cfg.attends) * per
+    d2h = cfg.chunks * cfg.attends * per
+    del host
+    return sec, h2d, d2h
+
+
+def run_gpu(args):
+    from kv_cache_attention_tempcache_b200 import TempCache
+
+    rank, world, local = dist_info()
+    torch.cuda.set_device(local)
+    init_dist(world, "nccl")
+    dev = torch.device("cuda", local)
+    cfg = CONFIGS[WORKLOAD]
+    if args.chunks:
+        cfg = cfg.replace(chunks=args.chunks, capacity=args.chunks * cfg.T)
+    R, chunks = generate_inputs(cfg, dev, rank_seed(cfg.seed, rank))
+    tc = TempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, hyperplanes=R)
+    outs = [torch.empty(cfg.T, cfg.H, cfg.d, dtype=torch.bfloat16, device=dev) for _ in range(cfg.attends)]
+
+    sizes, commit_counts = sizes_per_chunk(tc, chunks, outs, cfg)
+    for _ in range(args.warmup):
+        rollout(tc, chunks, outs)
+    torch.cuda.synchronize()
+
+    # timed region: K rollouts, per-call events for the attention and commit kernels
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    attn_ev = [[[[ev(), ev()] for _ in range(cfg.attends)] for _ in range(cfg.chunks)] for _ in range(args.steps)]
+    app_ev = [[[ev(), ev()] for _ in range(cfg.chunks)] for _ in range(args.steps)]
+    launches0 = tc.launch_count()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0, t1 = ev(), ev()
+    torch.cuda.nvtx.range_push("timed")
+    t0.record()
+    for k in range(args.steps):
+        rollout(tc, chunks, outs, attn_ev[k], app_ev[k])
+    t1.record()
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    launches = tc.launch_count() - launches0
+    sec = t0.elapsed_time(t1) / 1000.0
+    sec_max = max_over_ranks(sec, world, dev)
+    value = aggregate_rate(cfg.F * cfg.chunks * args.steps, world, sec_max)
+
+    # roofline of the dominant kernel (attention) from the live per-launch events
+    flops_per_call = attn_flops(cfg, sizes)
+    attn_ms = [[sum(a[0].elapsed_time(a[1]) for a in attn_ev[k][c]) for c in range(cfg.chunks)]
+               for k in range(args.steps)]
+    attn_sec = sum(sum(x) for x in attn_ms) / 1000.0
+    attn_flops_total = args.steps * cfg.attends * sum(flops_per_call)
+    attn_tflops = attn_flops_total / attn_sec / 1e12
+    app_sec = sum(app_ev[k][c][0].elapsed_time(app_ev[k][c][1]) for k in range(args.steps)
+                  for c in range(cfg.chunks)) / 1000.0
+    cbytes = args.steps * sum(commit_bytes(cfg, commit_counts))
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    traffic = None
+    if os.path.exists(TRAFFIC_FILE):
+        with open(TRAFFIC_FILE) as f:
+            tr = json.load(f)
+        # DRAM bytes per unit of work measured by ncu, scaled to an average launch here
+        traffic = tr.get("bytes_per_flop", 0) * (attn_flops_total / (args.steps * cfg.chunks * cfg.attends)) \
+            if tr.get("kernel") == "attend_bf16_kernel" else None
+
+    # dense baseline: the same attention kernel over the uncompressed history (no merges)
+    dense_line = None
+    if not args.profile:
+        dense = TempCache(cfg.H, cfg.d, cfg.nbits, 2.0, cfg.capacity, hyperplanes=R)
+        rollout(dense, chunks, outs)
+        torch.cuda.synchronize()
+        d0, d1 = ev(), ev()
+        d0.record()
+        rollout(dense, chunks, outs)
+        d1.record()
+        torch.cuda.synchronize()
+        dense_sec = d0.elapsed_time(d1) / 1000.0
+        dense_flops = cfg.attends * sum(4.0 * cfg.T * cfg.H * (c * cfg.T + cfg.T) * cfg.d
+                                        for c in range(cfg.chunks))
+        dense.close()
+        dense_line = {"value": cfg.F * cfg.chunks / dense_sec, "unit": UNIT,
+                      "attn_tflops": dense_flops / dense_sec / 1e12,
+                      "note": "same kernels, tau > 1 so nothing merges (uncompressed cache)"}
+
+    e2e = None
+    if not args.profile:
+        e2e_sec, h2d, d2h = time_e2e(tc, cfg, chunks)
+        e2e_value = aggregate_rate(cfg.F * cfg.chunks, world, max_over_ranks(e2e_sec, world, dev))
+        e2e = {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    if rank != 0:
+        return
+    cores = len(os.sched_getaffinity(0))
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline and not args.profile:
+        cpu_chunks = cpu_inputs(chunks[:6])
+        v, n, desc = oracle_sample(cfg, cpu_chunks, R, n_chunks=5, rows_per_attend=256, time_budget_s=20.0,
+                                   warmup_chunks=1)
+        cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * sec_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"{WORKLOAD}: H=12 d=128 P=1560 F=3 chunks=40 attends=4 S=4096 p_stay=0.8 "
+                               f"sigma=0.05 nbits=16 tau=0.95 bf16",
+                   "step": f"one {cfg.chunks}-chunk rollout ({cfg.F * cfg.chunks} frames) from an empty cache",
+                   "l2": "inputs larger than L2 (3.5 GB of distinct K, V, Q per rollout)",
+                   "parallelism": f"independent rollout per rank x{world}"},
+        "roofline": {"bound": "tensor", "kernel": "attend_bf16_kernel", "achieved": attn_tflops,
+                     "peak": peak, "unit": "TFLOP/s", "frac": attn_tflops / peak,
+                     "peak_kind": f"{peak_kind} bf16 dense, sustained", "traffic": traffic,
+                     "flops_per_launch": attn_flops_total / (args.steps * cfg.chunks * cfg.attends),
+                     "avg_launch_ms": 1000.0 * attn_sec / (args.steps * cfg.chunks * cfg.attends)},
+        "merge": {"achieved_gbs": cbytes / app_sec / 1e9, "peak_gbs": float(peaks["hbm_gbs"]),
+                  "frac": cbytes / app_sec / 1e9 / float(peaks["hbm_gbs"]),
+                  "bytes_per_chunk": cbytes / (args.steps * cfg.chunks),
+                  "avg_append_ms": 1000.0 * app_sec / (args.steps * cfg.chunks)},
+        "attn_share": attn_sec / sec,
+        "dense_baseline": dense_line,
+        "cache_entries_per_head_end": float(np.mean(sizes[-1])),
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="timed rollouts only (no dense baseline, end-to-end or CPU legs), for profilers")
+    ap.add_argument("--chunks", type=int, default=0,
+                    help="rollout length in chunks (default: the workload's 40); profiling runs use fewer")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+    if torch.distributed.is_initialized():
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

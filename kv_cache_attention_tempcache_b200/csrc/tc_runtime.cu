@@ -100,9 +100,11 @@ bool encode3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-__global__ void fill_f32(float* p, int64_t n, float v) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-        p[i] = v;
+// p[h * stride + i] = v for i < n, h < rows (one launch over all heads).
+__global__ void fill_f32(float* p, int64_t n, int rows, int64_t stride, float v) {
+    for (int h = blockIdx.y; h < rows; h += gridDim.y)
+        for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+            p[(int64_t)h * stride + i] = v;
 }
 
 }  // namespace
@@ -375,7 +377,7 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
         delete x;
         return cuda_status(e);
     }
-    fill_f32<<<1024, 256>>>(c.bias2, (int64_t)rows, -INFINITY);
+    fill_f32<<<1024, 256>>>(c.bias2, (int64_t)rows, 1, 0, -INFINITY);
     if ((e = cudaDeviceSynchronize()) != cudaSuccess) {
         delete x;
         return cuda_status(e);
@@ -462,12 +464,10 @@ tc_status tc_reset(tc_handle x, tc_stream stream) {
     cudaError_t e = cudaMemsetAsync(x->c.bhead, 0xff, ((size_t)x->H << x->nbits) * 4, cs);
     if (e == cudaSuccess) e = cudaMemsetAsync(x->c.M, 0, (size_t)x->H * 4, cs);
     if (e == cudaSuccess && upto > 0) {
-        for (int h = 0; h < x->H && e == cudaSuccess; ++h) {
-            fill_f32<<<(unsigned)std::min<int64_t>((upto + 255) / 256, 1024), 256, 0, cs>>>(
-                x->c.bias2 + (size_t)h * x->capP, upto, -INFINITY);
-            e = cudaGetLastError();
-        }
-        x->launches += x->H;
+        dim3 grid((unsigned)std::min<int64_t>((upto + 255) / 256, 64), (unsigned)std::min(x->H, 1024));
+        fill_f32<<<grid, 256, 0, cs>>>(x->c.bias2, upto, x->H, x->capP, -INFINITY);
+        e = cudaGetLastError();
+        x->launches += 1;
     }
     if (e != cudaSuccess) return cuda_status(e);
     std::fill(x->m_upper.begin(), x->m_upper.end(), 0);
