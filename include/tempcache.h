@@ -154,6 +154,38 @@ tc_status tc_get_hyperplanes(tc_handle h, float* R);
 tc_status tc_stats(tc_handle h, uint64_t* kernel_launches, uint64_t* hash_rechecks,
                    uint64_t* match_rechecks);
 
+/* ---- allocation-free entry point -------------------------------------------- */
+
+/*
+ * tc_merge_means_noalloc - average matched rows into running means, allocating
+ * nothing. The paper has no counterpart to this call: it exists for callers that
+ * may not allocate device memory once they are running, such as inference
+ * runtimes that reserve a single fixed arena at start-up, or plugins inside a
+ * framework whose allocator owns the whole device. It is the library's merge step
+ * (values averaged, counts added) on buffers the caller owns:
+ *   for every destination row j, with S_j = { i : target[i] == j } in ascending i,
+ *     mean[j]  <- (count[j] * mean[j] + sum_{i in S_j} src[i]) / (count[j] + |S_j|)
+ *     count[j] <- count[j] + |S_j|
+ *   summed in fp32 in ascending i, so the result does not depend on scheduling.
+ *   src     DEVICE [n_src, d] in src_dtype (bf16 or fp32), read only.
+ *   target  DEVICE [n_src] int32 destination row or -1 (skip); values outside
+ *           [0, n_dst) are skipped too.
+ *   mean    DEVICE [n_dst, d] fp32, updated in place; count DEVICE [n_dst] int32,
+ *           updated in place. Rows no source targets are left as they are.
+ *   d       64 or 128.
+ * Limits: n_src <= 65536 and n_dst <= 262144; larger sizes return TC_EINVAL and
+ * launch nothing. Scratch lives in a fixed device array of about 3.4 MB that every
+ * GPU loading the library holds until the process exits; the call never calls
+ * cudaMalloc, cudaFree or any allocating routine. The first call on a device looks
+ * up that array's device address (make it before any stream capture). All calls
+ * share the array: calls whose GPU work overlaps (other streams or host threads on
+ * the same device) race and corrupt each other's results, so keep them ordered.
+ * Asynchronous on `stream`; returns TC_ECUDA if a launch fails.
+ */
+tc_status tc_merge_means_noalloc(const void* src, tc_dtype src_dtype, const int32_t* target,
+                                 int32_t n_src, int32_t d, float* mean, int32_t* count,
+                                 int32_t n_dst, tc_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -28,7 +28,7 @@ TC_BF16, TC_F32 = 0, 1
 API = [
     "tc_create", "tc_create_ex", "tc_append_chunk", "tc_attend", "tc_flush", "tc_reset", "tc_cache_size", "tc_sync",
     "tc_destroy", "tc_status_string", "tc_debug_last_commit", "tc_debug_staged_codes", "tc_export_cache",
-    "tc_get_hyperplanes", "tc_stats",
+    "tc_get_hyperplanes", "tc_stats", "tc_merge_means_noalloc",
 ]
 
 
@@ -61,6 +61,7 @@ def _load():
         "tc_get_hyperplanes": (ctypes.c_int, [H, vp]),
         "tc_stats": (ctypes.c_int, [H, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64),
                                     ctypes.POINTER(ctypes.c_uint64)]),
+        "tc_merge_means_noalloc": (ctypes.c_int, [vp, ctypes.c_int, vp, i32, i32, vp, vp, i32, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
