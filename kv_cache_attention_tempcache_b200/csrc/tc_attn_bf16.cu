@@ -5,19 +5,21 @@
 // summary, section 2.A: Lemma 5.1 makes averaged values with a logit shift by the
 // group size exact for identical keys. Computed in base 2: x = s * log2(e).
 //
-// One CTA = 128 query rows of one head; two CTAs share an SM so one CTA's softmax
-// overlaps the other's MMAs. Warp roles (192 threads):
-//   warps 0-3  softmax: thread r owns query row r (TMEM lane r); online softmax in
-//              fp32 with lazy rescaling of O (only when the running max grows by
-//              more than 2^8); writes P as bf16 into TMEM over S.
-//   warp 4     TMA producer (Q once, then one K and one V tile per step) and TMEM
-//              allocator.
-//   warp 5     MMA issuer: S = Q K^T (SS form, both K-major), O += P V (P from
-//              TMEM, V MN-major), fp32 accumulators in TMEM.
-// TMEM (256 columns): S/P at columns [0,128), O at [128, 128+D).
-// Shared memory: Q, K, V tiles of 128 rows, 128-byte swizzled boxes of 64 columns.
-// Every mbarrier wait is bounded (2 s); a timeout sets an error bit and the CTA
-// drains its own copies and MMAs before releasing TMEM.
+// One CTA = 128 query rows of one head and owns the SM's 512 TMEM columns:
+//   S0 [0,128), S1 [128,256)  scores of consecutive key tiles (P overwrites its S)
+//   O  [256, 256+D)           fp32 output accumulator
+// Warp roles (224 threads):
+//   warps 0-3  softmax: thread r owns query row r (TMEM lane r); one pass per key
+//              tile with an upper-bound reference max, lazy rescaling of O (only when
+//              the reference grows by more than 2^8), P written as bf16 over S.
+//   warp 4     TMA producer for Q and the K ring (2 stages); TMEM allocator.
+//   warp 5     MMA issuer: S_{i+1} = Q K_{i+1}^T is issued before O += P_i V_i, so
+//              the tensor core computes the next scores while softmax works on P_i.
+//   warp 6     TMA producer for the V ring (2 stages).
+// Operands come by 3-D TMA (64-column, 128-byte-swizzled boxes) straight from the
+// token-major Q and the head-major cache/staging buffers. Every mbarrier wait is
+// bounded (2 s); a timeout sets an error bit and the CTA drains its own copies and
+// MMAs before releasing TMEM.
 #include "tc_internal.h"
 
 #include <math.h>
@@ -28,7 +30,7 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBN = 128;
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 
 template <int D>
@@ -37,16 +39,16 @@ struct Cfg {
     static constexpr int BOX = 128 * 128;             // bytes of one 128-row box
     static constexpr int TILE = NB * BOX;             // bytes of a Q, K or V tile
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = TILE;
-    static constexpr int OFF_V = 2 * TILE;
-    static constexpr int OFF_BIAS = 3 * TILE;         // 2 x 128 floats
-    static constexpr int OFF_BAR = OFF_BIAS + 2 * 128 * 4;
-    static constexpr int NBAR = 10;
+    static constexpr int OFF_K = TILE;                // 2 stages
+    static constexpr int OFF_V = 3 * TILE;            // 2 stages
+    static constexpr int OFF_BIAS = 5 * TILE;         // 2 x 128 floats
+    static constexpr int OFF_BMAX = OFF_BIAS + 2 * 128 * 4;  // 2 x 4 floats
+    static constexpr int OFF_BAR = OFF_BMAX + 2 * 4 * 4;
+    static constexpr int NBAR = 16;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM = OFF_MISC + 32 + 1024;  // + slack for 1024-B alignment
-    static constexpr uint32_t TMEM_COLS = 256;
-    static constexpr uint32_t S_COL = 0;
-    static constexpr uint32_t O_COL = 128;
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t O_COL = 256;
     // Instruction descriptors, kind::f16: bits 4-5 D format (1 = f32), 7-9 A format
     // (1 = bf16), 10-12 B format (1 = bf16), 15/16 A/B major (0 = K, 1 = MN),
     // 17-22 N>>3, 24-28 M>>4.
@@ -56,7 +58,9 @@ struct Cfg {
                                          ((uint32_t)(D >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
 };
 
-enum { B_QFULL = 0, B_KFULL, B_KEMPTY, B_VFULL, B_VEMPTY, B_SFULL, B_PFULL, B_ORDY, B_DRAIN };
+// mbarriers: Q full; K full/empty x2; V full/empty x2; S full x2; P full x2; PV done; drain.
+enum { B_QFULL = 0, B_KFULL = 1, B_KEMPTY = 3, B_VFULL = 5, B_VEMPTY = 7, B_SFULL = 9, B_PFULL = 11, B_ODONE = 13,
+       B_DRAIN = 14 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return (uint32_t)__cvta_generic_to_shared(p);
@@ -181,6 +185,40 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void up2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float m;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+    return m;
+}
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
 // Barrier 1 over the 128 softmax threads with an AND of `v` across them.
 __device__ __forceinline__ bool bar_and_128(bool v) {
     uint32_t res;
@@ -194,7 +232,7 @@ __device__ __forceinline__ bool bar_and_128(bool v) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
 attend_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
                    const __grid_constant__ CUtensorMap tmVc, const __grid_constant__ CUtensorMap tmKs,
                    const __grid_constant__ CUtensorMap tmVs, const int32_t* __restrict__ Mdev,
@@ -205,6 +243,7 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     float* sBias = reinterpret_cast<float*>(smem + C::OFF_BIAS);
+    float* sBmax = reinterpret_cast<float*>(smem + C::OFF_BMAX);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -217,13 +256,15 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[B_QFULL], 1);
-        mbar_init(&bars[B_KFULL], 1);
-        mbar_init(&bars[B_KEMPTY], 1);
-        mbar_init(&bars[B_VFULL], 1);
-        mbar_init(&bars[B_VEMPTY], 1);
-        mbar_init(&bars[B_SFULL], 1);
-        mbar_init(&bars[B_PFULL], 128);
-        mbar_init(&bars[B_ORDY], 1);
+        for (int s2 = 0; s2 < 2; ++s2) {
+            mbar_init(&bars[B_KFULL + s2], 1);
+            mbar_init(&bars[B_KEMPTY + s2], 1);
+            mbar_init(&bars[B_VFULL + s2], 1);
+            mbar_init(&bars[B_VEMPTY + s2], 1);
+            mbar_init(&bars[B_SFULL + s2], 1);
+            mbar_init(&bars[B_PFULL + s2], 128);
+        }
+        mbar_init(&bars[B_ODONE], 1);
         mbar_init(&bars[B_DRAIN], 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -238,64 +279,80 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // Let the next attention call on this stream start filling SMs as this grid
+    // drains (it only reads what this kernel reads).
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tS = tmem + C::S_COL;
     const uint32_t tO = tmem + C::O_COL;
     uint8_t* sQ = smem + C::OFF_Q;
     uint8_t* sK = smem + C::OFF_K;
     uint8_t* sV = smem + C::OFF_V;
 
-    if (warp == 4) {
-        // ---------------------------------------------------------------- producer (lane 0)
+    if (warp == 4 || warp == 6) {
+        // ---------------------------------------------------------------- producers (lane 0)
         if (lane == 0) {
-            int lastK = -1, lastV = -1;
-            mbar_expect_tx(&bars[B_QFULL], C::TILE);
-            for (int b = 0; b < C::NB; ++b) tma_load_3d(sQ + b * C::BOX, &tmQ, 64 * b, h, q0, &bars[B_QFULL]);
+            const bool kside = (warp == 4);
+            uint8_t* ring = kside ? sK : sV;
+            uint64_t* full = &bars[kside ? B_KFULL : B_VFULL];
+            uint64_t* empty = &bars[kside ? B_KEMPTY : B_VEMPTY];
+            const CUtensorMap* mc = kside ? &tmKc : &tmVc;
+            const CUtensorMap* ms = kside ? &tmKs : &tmVs;
+            if (kside) {
+                mbar_expect_tx(&bars[B_QFULL], C::TILE);
+                for (int b = 0; b < C::NB; ++b) tma_load_3d(sQ + b * C::BOX, &tmQ, 64 * b, h, q0, &bars[B_QFULL]);
+            }
+            int last = -1;
             for (int i = 0; i < ntiles && !*abort_flag; ++i) {
+                const int st = i & 1;
+                if (i >= 2 && !mbar_wait(&empty[st], ((i >> 1) - 1) & 1)) { *abort_flag = 1; break; }
                 const bool cache = i < nc;
                 const int row0 = (cache ? i : i - nc) * kBN;
-                const CUtensorMap* mk = cache ? &tmKc : &tmKs;
-                const CUtensorMap* mv = cache ? &tmVc : &tmVs;
-                if (i > 0 && !mbar_wait(&bars[B_KEMPTY], (i - 1) & 1)) { *abort_flag = 1; break; }
-                mbar_expect_tx(&bars[B_KFULL], C::TILE);
-                for (int b = 0; b < C::NB; ++b) tma_load_3d(sK + b * C::BOX, mk, 64 * b, row0, h, &bars[B_KFULL]);
-                lastK = i;
-                if (i > 0 && !mbar_wait(&bars[B_VEMPTY], (i - 1) & 1)) { *abort_flag = 1; break; }
-                mbar_expect_tx(&bars[B_VFULL], C::TILE);
-                for (int b = 0; b < C::NB; ++b) tma_load_3d(sV + b * C::BOX, mv, 64 * b, row0, h, &bars[B_VFULL]);
-                lastV = i;
+                mbar_expect_tx(&full[st], C::TILE);
+                for (int b = 0; b < C::NB; ++b)
+                    tma_load_3d(ring + st * C::TILE + b * C::BOX, cache ? mc : ms, 64 * b, row0, h, &full[st]);
+                last = i;
             }
-            // Drain: every issued copy has landed before the CTA can exit (already
-            // true on the normal path, where the MMA thread consumed them all).
-            mbar_wait(&bars[B_QFULL], 0);
-            if (lastK >= 0) mbar_wait(&bars[B_KFULL], lastK & 1);
-            if (lastV >= 0) mbar_wait(&bars[B_VFULL], lastV & 1);
+            // Drain: the copies issued here land before the CTA can exit (already true
+            // on the normal path, where the MMA thread consumed them all).
+            if (kside) mbar_wait(&bars[B_QFULL], 0);
+            for (int i = (last >= 1 ? last - 1 : 0); i <= last; ++i) mbar_wait(&full[i & 1], (i >> 1) & 1);
         }
     } else if (warp == 5) {
         // ---------------------------------------------------------------- MMA issuer (lane 0)
         if (lane == 0) {
             const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
             bool ok = mbar_wait(&bars[B_QFULL], 0);
-            for (int i = 0; i < ntiles && ok && !*abort_flag; ++i) {
-                // S/P of step i-1 must be consumed by its PV before S is overwritten.
-                if (i > 0 && !mbar_wait(&bars[B_ORDY], (i - 1) & 1)) { ok = false; break; }
-                if (!mbar_wait(&bars[B_KFULL], i & 1)) { ok = false; break; }
+            auto issue_qk = [&](int j) -> bool {
+                const int st = j & 1;
+                // S_st held P_{j-2}: wait until O += P_{j-2} V_{j-2} has retired.
+                if (j >= 2 && !mbar_wait(&bars[B_ODONE], (j - 2) & 1)) return false;
+                if (!mbar_wait(&bars[B_KFULL + st], (j >> 1) & 1)) return false;
                 tc_fence_after();
+                const uint32_t aKs = aK + st * C::TILE;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
-                    mma_ss(tS, sdesc(aQ + off, 16, 1024), sdesc(aK + off, 16, 1024), C::IDESC_QK, kk > 0);
+                    mma_ss(tmem + st * 128, sdesc(aQ + off, 16, 1024), sdesc(aKs + off, 16, 1024), C::IDESC_QK,
+                           kk > 0);
                 }
-                tc_commit(&bars[B_SFULL]);
-                tc_commit(&bars[B_KEMPTY]);
-                if (!mbar_wait(&bars[B_PFULL], i & 1)) { ok = false; break; }
-                if (!mbar_wait(&bars[B_VFULL], i & 1)) { ok = false; break; }
+                tc_commit(&bars[B_SFULL + st]);
+                tc_commit(&bars[B_KEMPTY + st]);
+                return true;
+            };
+            if (ok && ntiles > 0) ok = issue_qk(0);
+            for (int i = 0; i < ntiles && ok && !*abort_flag; ++i) {
+                if (i + 1 < ntiles && !(ok = issue_qk(i + 1))) break;
+                const int st = i & 1;
+                if (!mbar_wait(&bars[B_PFULL + st], (i >> 1) & 1)) { ok = false; break; }
+                if (!mbar_wait(&bars[B_VFULL + st], (i >> 1) & 1)) { ok = false; break; }
                 tc_fence_after();
+                const uint32_t aVs = aV + st * C::TILE;
 #pragma unroll
                 for (int kk = 0; kk < kBN / 16; ++kk)
-                    mma_ts(tO, tS + kk * 8, sdesc(aV + kk * 2048, C::BOX, 1024), C::IDESC_PV, (i > 0 || kk > 0));
-                tc_commit(&bars[B_VEMPTY]);
-                tc_commit(&bars[B_ORDY]);
+                    mma_ts(tO, tmem + st * 128 + kk * 8, sdesc(aVs + kk * 2048, C::BOX, 1024), C::IDESC_PV,
+                           (i > 0 || kk > 0));
+                tc_commit(&bars[B_VEMPTY + st]);
+                tc_commit(&bars[B_ODONE]);
             }
             if (!ok) *abort_flag = 1;
             // Drain: every MMA issued here retires before TMEM is released.
@@ -312,39 +369,48 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         auto bias_of = [&](int i) -> float {
             return (i < nc) ? bias_h[(int64_t)i * kBN + r] : sbias[(int64_t)(i - nc) * kBN + r];
         };
+        const uint64_t c2 = pk2(scale_log2, scale_log2);
         float m_run = -INFINITY, l_run = 0.f;
         float bnext = (ntiles > 0) ? bias_of(0) : 0.f;
         bool ok = true;
         for (int i = 0; i < ntiles; ++i) {
-            float* bb = sBias + (i & 1) * kBN;
+            const int st = i & 1;
+            float* bb = sBias + st * kBN;
             bb[r] = bnext;
-            const bool got = !*abort_flag && mbar_wait(&bars[B_SFULL], i & 1);
-            if (!bar_and_128(got)) { ok = false; break; }   // also publishes bb[] to the group
+            float wm = bnext;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, o));
+            if (lane == 0) sBmax[st * 4 + warp] = wm;
+            const bool got = !*abort_flag && mbar_wait(&bars[B_SFULL + st], (i >> 1) & 1);
+            if (!bar_and_128(got)) { ok = false; break; }   // also publishes bb[] and the bias maxima
             if (i + 1 < ntiles) bnext = bias_of(i + 1);
             tc_fence_after();
-            // Pass 1: row max of x = s * scale * log2(e) + log2 n, 32 columns at a time.
-            float mx = -INFINITY;
-#pragma unroll 1
-            for (int cc = 0; cc < kBN / 32; ++cc) {
-                uint32_t xr[32];
-                TC_LD32(tS + lane_base + 32 * cc, xr);
-                tc_wait_ld();
+            const uint32_t tS = tmem + st * 128 + lane_base;
+            uint32_t sr[kBN];
+            TC_LD32(tS + 0, (sr + 0));
+            TC_LD32(tS + 32, (sr + 32));
+            TC_LD32(tS + 64, (sr + 64));
+            TC_LD32(tS + 96, (sr + 96));
+            tc_wait_ld();
+            // Reference max: an upper bound of this tile's row max, (max raw score) *
+            // scale + (max shift of the tile). p = 2^(x - m) stays <= 2^8 below.
+            float smax = -INFINITY;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) mx = fmaxf(mx, fmaf(__uint_as_float(xr[j]), scale_log2, bb[32 * cc + j]));
-            }
-            const float m_new = fmaxf(m_run, mx);
+            for (int j = 0; j < kBN; j += 2) smax = max3(smax, __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
+            const float4 bm4 = *reinterpret_cast<const float4*>(sBmax + st * 4);
+            const float ub = fmaf(smax, scale_log2, fmaxf(fmaxf(bm4.x, bm4.y), fmaxf(bm4.z, bm4.w)));
             if (i == 0) {
-                m_run = m_new;
+                m_run = ub;
             } else {
-                // Lazy rescaling: O and l keep the old reference max until the row max
-                // grows by more than 8 (a factor 256), then both are scaled by alpha.
-                const bool need = m_new > m_run + 8.f;
+                // Lazy rescaling: O and l keep the old reference until it would grow by
+                // more than 8 (a factor 256), then both are scaled by alpha.
+                const bool need = ub > m_run + 8.f;
                 if (__any_sync(0xffffffffu, need)) {
-                    const bool w = mbar_wait(&bars[B_ORDY], (i - 1) & 1);
+                    const bool w = mbar_wait(&bars[B_ODONE], (i - 1) & 1);
                     if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; }
                     if (ok) {
-                        const float alpha = need ? exp2f(m_run - m_new) : 1.f;
-                        if (need) { l_run *= alpha; m_run = m_new; }
+                        const float alpha = need ? ex2(m_run - ub) : 1.f;
+                        if (need) { l_run *= alpha; m_run = ub; }
                         tc_fence_after();
 #pragma unroll 1
                         for (int c = 0; c < D / 32; ++c) {
@@ -359,31 +425,35 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     }
                 }
             }
-            // Pass 2: p = 2^(x - m), row sum, bf16 P written over S. Chunk cc of P
-            // (columns 16cc..16cc+15) only covers S columns already read.
-            float sum = 0.f;
-#pragma unroll 1
-            for (int cc = 0; cc < kBN / 32; ++cc) {
-                uint32_t xr[32];
-                TC_LD32(tS + lane_base + 32 * cc, xr);
-                tc_wait_ld();
-                uint32_t pk[16];
+            // p = 2^(s * scale + log2 n - m): packed fp32x2 FMA/ADD, MUFU ex2, bf16 pack.
+            const uint64_t negm2 = pk2(-m_run, -m_run);
+            uint64_t sum2 = pk2(0.f, 0.f);
+            uint32_t pk[kBN / 2];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float p0 = exp2f(fmaf(__uint_as_float(xr[2 * j]), scale_log2, bb[32 * cc + 2 * j]) - m_run);
-                    const float p1 =
-                        exp2f(fmaf(__uint_as_float(xr[2 * j + 1]), scale_log2, bb[32 * cc + 2 * j + 1]) - m_run);
-                    sum += p0 + p1;
-                    pk[j] = pack_bf16(p0, p1);
-                }
-                TC_ST16(tS + lane_base + 16 * cc, pk);
+            for (int j = 0; j < kBN; j += 4) {
+                const float4 b4 = *reinterpret_cast<const float4*>(bb + j);
+                const uint64_t x01 = fma2(pk2(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), c2,
+                                          add2(pk2(b4.x, b4.y), negm2));
+                const uint64_t x23 = fma2(pk2(__uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3])), c2,
+                                          add2(pk2(b4.z, b4.w), negm2));
+                float a0, a1, a2, a3;
+                up2(x01, a0, a1);
+                up2(x23, a2, a3);
+                const float p0 = ex2(a0), p1 = ex2(a1), p2 = ex2(a2), p3 = ex2(a3);
+                sum2 = add2(sum2, add2(pk2(p0, p1), pk2(p2, p3)));
+                pk[j / 2] = cvt_bf16x2(p0, p1);
+                pk[j / 2 + 1] = cvt_bf16x2(p2, p3);
             }
-            l_run += sum;
+            float s0, s1;
+            up2(sum2, s0, s1);
+            l_run += s0 + s1;
+            TC_ST32(tS + 0, (pk + 0));
+            TC_ST32(tS + 32, (pk + 32));
             tc_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars[B_PFULL]);
+            mbar_arrive(&bars[B_PFULL + st]);
         }
-        const bool fin = ok && ntiles > 0 && mbar_wait(&bars[B_ORDY], (ntiles - 1) & 1);
+        const bool fin = ok && ntiles > 0 && mbar_wait(&bars[B_ODONE], (ntiles - 1) & 1);
         if (bar_and_128(fin)) {
             tc_fence_after();
             const float inv = 1.f / l_run;
@@ -398,10 +468,10 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 #pragma unroll
                     for (int v = 0; v < 4; ++v) {
                         uint4 w;
-                        w.x = pack_bf16(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
-                        w.y = pack_bf16(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
-                        w.z = pack_bf16(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
-                        w.w = pack_bf16(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
+                        w.x = cvt_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
+                        w.y = cvt_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
+                        w.z = cvt_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
+                        w.w = cvt_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
                         dst[v] = w;
                     }
                 }
@@ -418,11 +488,14 @@ attend_bf16_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS)
                      : "memory");
     }
+    // When this grid was allowed to start before the previous one finished, it
+    // completes only after that one: whatever follows on the stream sees both done.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 template <int D>
-cudaError_t launch_t(const CacheView& c, const StageView& s, const AttnMaps& m, int64_t Tq,
-                     __nv_bfloat16* out, float scale_log2, Stats* stats, cudaStream_t st) {
+cudaError_t launch_t(const CacheView& c, const StageView& s, const AttnMaps& m, int64_t Tq, __nv_bfloat16* out,
+                     float scale_log2, Stats* stats, bool overlap_prev, cudaStream_t st) {
     using C = Cfg<D>;
     static bool attr_set = false;
     if (!attr_set) {
@@ -431,18 +504,28 @@ cudaError_t launch_t(const CacheView& c, const StageView& s, const AttnMaps& m, 
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    dim3 grid((unsigned)((Tq + kBM - 1) / kBM), (unsigned)c.H);
-    attend_bf16_kernel<D><<<grid, kThreads, C::SMEM, st>>>(m.q, m.kc, m.vc, m.ks, m.vs, c.M, c.bias2, c.capP,
-                                                           s.sbias, s.T, Tq, c.H, out, scale_log2, stats);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((Tq + kBM - 1) / kBM), (unsigned)c.H);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = overlap_prev ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, attend_bf16_kernel<D>, m.q, m.kc, m.vc, m.ks, m.vs, (const int32_t*)c.M,
+                              (const float*)c.bias2, c.capP, (const float*)s.sbias, s.T, Tq, c.H, out, scale_log2,
+                              stats);
 }
 
 }  // namespace
 
 cudaError_t launch_attend_bf16(const CacheView& c, const StageView& s, const AttnMaps& maps, int64_t Tq,
-                               __nv_bfloat16* out, float scale_log2, Stats* stats, cudaStream_t st) {
-    return c.d == 128 ? launch_t<128>(c, s, maps, Tq, out, scale_log2, stats, st)
-                      : launch_t<64>(c, s, maps, Tq, out, scale_log2, stats, st);
+                               __nv_bfloat16* out, float scale_log2, Stats* stats, bool overlap_prev,
+                               cudaStream_t st) {
+    return c.d == 128 ? launch_t<128>(c, s, maps, Tq, out, scale_log2, stats, overlap_prev, st)
+                      : launch_t<64>(c, s, maps, Tq, out, scale_log2, stats, overlap_prev, st);
 }
 
 }  // namespace tc

@@ -73,6 +73,6 @@ struct AttnMaps {
 };
 cudaError_t launch_attend_bf16(const CacheView& c, const StageView& s, const AttnMaps& maps,
                                int64_t Tq, __nv_bfloat16* out, float scale_log2, Stats* stats,
-                               cudaStream_t st);
+                               bool overlap_prev, cudaStream_t st);
 
 }  // namespace tc

@@ -131,6 +131,13 @@ struct tc_ctx {
     tc_status sticky = TC_OK;
     AttnMaps maps{};
     int64_t maps_T = -1;
+    // The previous launch of this handle, when it was an attention call: its
+    // stream and buffers decide whether the next attention call may overlap it.
+    bool prev_attend = false;
+    cudaStream_t prev_stream = nullptr;
+    const char* prev_q = nullptr;
+    const char* prev_out = nullptr;
+    size_t prev_bytes = 0;
     std::vector<void*> owned;
 
     tc_status alloc(void** p, size_t bytes) {
@@ -402,6 +409,7 @@ tc_status tc_append_chunk(tc_handle x, const void* K, const void* V, int64_t T, 
     if (!K || !V || !aligned16(K) || !aligned16(V) || T < 1 || T > ((int64_t)1 << 28)) return TC_EINVAL;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     x->last_stream = cs;
+    x->prev_attend = false;
     if ((st = commit_staged(x, cs))) return st;
     if ((st = ensure_staging(x, T))) return st;
     x->s.T = T;
@@ -419,6 +427,7 @@ tc_status tc_flush(tc_handle x, tc_stream stream) {
     if (st) return st;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     x->last_stream = cs;
+    x->prev_attend = false;
     if ((st = commit_staged(x, cs))) return st;
     x->s.T = 0;
     return TC_OK;
@@ -443,7 +452,19 @@ tc_status tc_attend(tc_handle x, const void* Q, int64_t Tq, void* out, tc_stream
         AttnMaps m = x->maps;
         if (!encode3d(&m.q, Q, x->d, x->H, Tq, (uint64_t)x->d * 2, (uint64_t)x->H * x->d * 2, 64, 1, 128))
             return TC_EINVAL;
-        e = launch_attend_bf16(x->c, s, m, Tq, static_cast<__nv_bfloat16*>(out), scale_log2, x->stats, cs);
+        // Consecutive attention calls only read the cache and staging buffers, so the
+        // next may start while the previous drains, unless their buffers interact.
+        auto overlaps = [](const char* a, size_t na, const char* b, size_t nb) { return a < b + nb && b < a + na; };
+        const bool overlap = x->prev_attend && x->prev_stream == cs && !overlaps(o, bytes, x->prev_out, x->prev_bytes) &&
+                             !overlaps(o, bytes, x->prev_q, x->prev_bytes) &&
+                             !overlaps(q, bytes, x->prev_out, x->prev_bytes);
+        e = launch_attend_bf16(x->c, s, m, Tq, static_cast<__nv_bfloat16*>(out), scale_log2, x->stats, overlap,
+                               cs);
+        x->prev_attend = (e == cudaSuccess);
+        x->prev_stream = cs;
+        x->prev_q = q;
+        x->prev_out = o;
+        x->prev_bytes = bytes;
     } else {
         e = launch_attend_f32(x->c, s, static_cast<const float*>(Q), Tq, static_cast<float*>(out), scale_log2, cs);
     }
@@ -456,6 +477,7 @@ tc_status tc_reset(tc_handle x, tc_stream stream) {
     if (st) return st;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     x->last_stream = cs;
+    x->prev_attend = false;
     // Rows at or past the committed size only need log2 n = -inf (masked) and finite
     // keys/values, which the previous rollout left there; the bucket lists restart.
     int64_t upto = 0;
