@@ -148,20 +148,21 @@ def generate_inputs(cfg, device, seed):
     return w.hyperplanes().numpy(), chunks
 
 
-def rollout(tc, chunks, outs, attn_events=None, app_events=None):
+def rollout(tc, chunks, outs, events=None):
+    """One rollout from an empty cache. events[c] = (e0, e1, e2) brackets the append
+    (e0..e1) and the block of attention calls (e1..e2) of chunk c; no event sits
+    between two attention calls, so consecutive calls may overlap on the device."""
     tc.reset()
     for c, (K, V, Qs) in enumerate(chunks):
-        if app_events is not None:
-            app_events[c][0].record()
+        if events is not None:
+            events[c][0].record()
         tc.append_chunk(K, V)
-        if app_events is not None:
-            app_events[c][1].record()
+        if events is not None:
+            events[c][1].record()
         for a, Q in enumerate(Qs):
-            if attn_events is not None:
-                attn_events[c][a][0].record()
             tc.attend(Q, out=outs[a])
-            if attn_events is not None:
-                attn_events[c][a][1].record()
+        if events is not None:
+            events[c][2].record()
 
 
 def sizes_per_chunk(tc, chunks, outs, cfg):
@@ -320,8 +321,7 @@ def run_gpu(args):
 
     # timed region: K rollouts, per-call events for the attention and commit kernels
     ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
-    attn_ev = [[[[ev(), ev()] for _ in range(cfg.attends)] for _ in range(cfg.chunks)] for _ in range(args.steps)]
-    app_ev = [[[ev(), ev()] for _ in range(cfg.chunks)] for _ in range(args.steps)]
+    chunk_ev = [[(ev(), ev(), ev()) for _ in range(cfg.chunks)] for _ in range(args.steps)]
     launches0 = tc.launch_count()
     clocks = ClockSampler(local)
     clocks.start()
@@ -332,7 +332,7 @@ def run_gpu(args):
     torch.cuda.nvtx.range_push("timed")
     t0.record()
     for k in range(args.steps):
-        rollout(tc, chunks, outs, attn_ev[k], app_ev[k])
+        rollout(tc, chunks, outs, chunk_ev[k])
     t1.record()
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
@@ -345,12 +345,11 @@ def run_gpu(args):
 
     # roofline of the dominant kernel (attention) from the live per-launch events
     flops_per_call = attn_flops(cfg, sizes)
-    attn_ms = [[sum(a[0].elapsed_time(a[1]) for a in attn_ev[k][c]) for c in range(cfg.chunks)]
-               for k in range(args.steps)]
-    attn_sec = sum(sum(x) for x in attn_ms) / 1000.0
+    attn_sec = sum(chunk_ev[k][c][1].elapsed_time(chunk_ev[k][c][2]) for k in range(args.steps)
+                   for c in range(cfg.chunks)) / 1000.0
     attn_flops_total = args.steps * cfg.attends * sum(flops_per_call)
     attn_tflops = attn_flops_total / attn_sec / 1e12
-    app_sec = sum(app_ev[k][c][0].elapsed_time(app_ev[k][c][1]) for k in range(args.steps)
+    app_sec = sum(chunk_ev[k][c][0].elapsed_time(chunk_ev[k][c][1]) for k in range(args.steps)
                   for c in range(cfg.chunks)) / 1000.0
     cbytes = args.steps * sum(commit_bytes(cfg, commit_counts))
     peaks, peak_kind = load_peaks()
