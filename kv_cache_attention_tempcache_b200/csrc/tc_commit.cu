@@ -1,5 +1,5 @@
 // TempCache commit path: stage + hash, bucketed top-1 search with the merge
-// decision, compaction scan, append, and the deterministic segmented merge.
+// decision, append in token order, and the deterministic list merge.
 //
 // FAST-AR technical summary, section 2.A "TempCache": each key of the current
 // chunk is hashed with locality-sensitive hashing, its top-1 neighbour among the
@@ -95,12 +95,6 @@ __device__ __forceinline__ float warp_sum(float v) {
     return v;
 }
 
-__device__ __forceinline__ int warp_min(int v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
-
 constexpr int kWarps = 8;  // warps per block of the warp-per-row kernels
 
 inline int grid_for_rows(int64_t rows, int per_block, int max_blocks) {
@@ -112,411 +106,768 @@ inline int grid_for_rows(int64_t rows, int per_block, int max_blocks) {
 
 // ------------------------------------------------------------------ stage + hash
 //
-// One warp per input row r = t*H + h of the token-major chunk. The row is copied
-// to the head-major staging buffer; lane b < nbits then forms <R_b, k> in fp32,
-// keeps its sign when |<R_b,k>| exceeds the certified bound
-//   2 (d+2) u |R_b| |k|   (u = 2^-24; any summation order has error <= (d+2) u
-//                         sum|R_bi k_i| <= (d+2) u |R_b||k|, doubled for margin)
-// and otherwise redoes the sum in fp64 in index order. Bit b = [<R_b,k> >= 0].
-template <typename E, int D>
-__global__ void __launch_bounds__(kWarps * 32)
+// One warp per input row r = t*H + h of the token-major chunk, four rows in flight.
+// The row is copied to the head-major staging buffer. Lane l keeps columns
+// [l*EPL, l*EPL + EPL) of every hyperplane in registers (as bf16 pairs: the normals
+// are bf16 values) and forms the partial dot products of its columns; a
+// reduce-scatter butterfly then leaves the full <R_b, k> (fp32) on lane b. Bit b
+// keeps the fp32 sign when
+//   |<R_b,k>| > 2 (d+2) u |R_b| |k|   (u = 2^-24; any summation order errs by at
+//                                      most (d+2) u sum|R_bi k_i| <= (d+2) u |R_b||k|,
+//                                      doubled for margin)
+// and otherwise lane b redoes the sum in fp64 in index order. Bit b = [<R_b,k> >= 0].
+
+// v[0..NBP) summed over the warp's 32 lanes; lane l ends with the total of slot
+// l mod NBP in v[0]. The first NBP-1 shuffles halve the vector (slot bit s-1 decided
+// by lane bit s-1, and so on down), the remaining lane bits are plain sums.
+template <int NBP>
+__device__ __forceinline__ float reduce_scatter(float (&v)[NBP], int lane) {
+#pragma unroll
+    for (int o = NBP / 2, L = NBP; o >= 1; o >>= 1, L >>= 1) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int k = 0; k < L / 2; ++k) {
+            const float send = up ? v[k] : v[k + L / 2];
+            const float keep = up ? v[k + L / 2] : v[k];
+            v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+#pragma unroll
+    for (int o = NBP; o < 32; o <<= 1) v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+    return v[0];
+}
+
+__device__ __forceinline__ uint32_t pack_bf16_exact(float lo, float hi) {
+    return (__float_as_uint(lo) >> 16) | (__float_as_uint(hi) & 0xffff0000u);
+}
+
+template <typename E, int D, int NBP>
+__global__ void __launch_bounds__(kWarps * 32, NBP <= 8 ? 3 : (NBP <= 16 ? 2 : 1))
 stage_hash_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView c, StageView s,
                   const float* __restrict__ R, const float* __restrict__ Rnorm, Stats* stats) {
     constexpr int EPL = D / 32;
+    constexpr int ROWS = 2;
     using IO = RowIO<E, EPL>;
-    extern __shared__ float sm[];
+    __shared__ float sKey[kWarps][D];
     const int nbits = c.nbits, H = c.H;
     const int64_t T = s.T;
-    float* sR = sm;                        // [nbits][D+1], padded: conflict-free column reads
-    float* sKey = sm + nbits * (D + 1);    // [kWarps][D]
-    for (int i = threadIdx.x; i < nbits * D; i += blockDim.x) sR[(i / D) * (D + 1) + (i % D)] = R[i];
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < s.TmaxP;
          i += (int64_t)gridDim.x * blockDim.x)
         s.sbias[i] = (i < T) ? 0.f : -INFINITY;
-    __syncthreads();
-
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-    float* krow = sKey + wib * D;
+    uint32_t Rp[NBP][EPL / 2];   // hyperplane slices, bf16 pairs
+#pragma unroll
+    for (int b = 0; b < NBP; ++b)
+#pragma unroll
+        for (int e = 0; e < EPL / 2; ++e)
+            Rp[b][e] = (b < nbits) ? pack_bf16_exact(R[b * D + lane * EPL + 2 * e], R[b * D + lane * EPL + 2 * e + 1])
+                                   : 0u;
+    const bool mine = lane < nbits;   // lane b reports bit b
     const float gam2 = 2.f * (float)(D + 2) * kU32;
-    const float rn = (lane < nbits) ? Rnorm[lane] : 0.f;
+    const float rn = mine ? Rnorm[lane] : 0.f;
     const unsigned mask = (nbits >= 32) ? 0xffffffffu : ((1u << nbits) - 1u);
     const int64_t rows = T * H;
-    for (int64_t r = (int64_t)blockIdx.x * kWarps + wib; r < rows; r += (int64_t)gridDim.x * kWarps) {
-        const int64_t t = r / H;
-        const int h = (int)(r - t * H);
-        const int64_t srow = ((int64_t)h * s.TmaxP + t) * D;
-        auto kv = IO::load(K + r * D, lane);
-        auto vv = IO::load(V + r * D, lane);
-        IO::store(reinterpret_cast<E*>(s.Ks) + srow, lane, kv);
-        IO::store(reinterpret_cast<E*>(s.Vs) + srow, lane, vv);
-        float x[EPL];
-        IO::to_float(kv, x);
-        float nk = 0.f;
+    const int64_t stride = (int64_t)gridDim.x * kWarps;
+    for (int64_t r0 = (int64_t)blockIdx.x * kWarps + wib; r0 < rows; r0 += ROWS * stride) {
+        typename IO::V kv[ROWS], vv[ROWS];
 #pragma unroll
-        for (int e = 0; e < EPL; ++e) {
-            nk = fmaf(x[e], x[e], nk);
-            krow[lane * EPL + e] = x[e];
-        }
-        nk = warp_sum(nk);
-        __syncwarp();
-        bool bit = false, rechk = false;
-        if (lane < nbits) {
-            const float* rb = sR + lane * (D + 1);
-            float p = 0.f;
-#pragma unroll 16
-            for (int i = 0; i < D; ++i) p = fmaf(rb[i], krow[i], p);
-            const float err = gam2 * rn * sqrtf(nk) + 1e-30f;
-            if (!(fabsf(p) > err)) {  // inside the band (or not finite): exact fp64, index order
-                rechk = true;
-                double q = 0.0;
-                for (int i = 0; i < D; ++i) q = fma((double)rb[i], (double)krow[i], q);
-                bit = (q >= 0.0);
-            } else {
-                bit = (p >= 0.f);
+        for (int q = 0; q < ROWS; ++q) {
+            const int64_t r = r0 + q * stride;
+            if (r < rows) {
+                kv[q] = IO::load(K + r * D, lane);
+                vv[q] = IO::load(V + r * D, lane);
             }
         }
-        const unsigned code = __ballot_sync(0xffffffffu, bit) & mask;
-        const unsigned nre = __popc(__ballot_sync(0xffffffffu, rechk));
-        if (lane == 0) {
-            s.scode[(int64_t)h * s.TmaxP + t] = code;
-            if (nre) atomicAdd(&stats->hash_rechecks, (unsigned long long)nre);
+#pragma unroll
+        for (int q = 0; q < ROWS; ++q) {
+            const int64_t r = r0 + q * stride;
+            if (r >= rows) break;   // warp-uniform
+            const int64_t t = r / H;
+            const int h = (int)(r - t * H);
+            const int64_t sidx = (int64_t)h * s.TmaxP + t;
+            IO::store(reinterpret_cast<E*>(s.Ks) + sidx * D, lane, kv[q]);
+            IO::store(reinterpret_cast<E*>(s.Vs) + sidx * D, lane, vv[q]);
+            float x[EPL];
+            IO::to_float(kv[q], x);
+            float nk = 0.f;
+            float v[NBP];
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) nk = fmaf(x[e], x[e], nk);
+#pragma unroll
+            for (int b = 0; b < NBP; ++b) {
+                float a = 0.f;
+#pragma unroll
+                for (int e = 0; e < EPL / 2; ++e) {
+                    a = fmaf(__uint_as_float(Rp[b][e] << 16), x[2 * e], a);
+                    a = fmaf(__uint_as_float(Rp[b][e] & 0xffff0000u), x[2 * e + 1], a);
+                }
+                v[b] = a;
+            }
+            nk = warp_sum(nk);
+            const float p = reduce_scatter<NBP>(v, lane);
+            const float err = gam2 * rn * sqrtf(nk) + 1e-30f;
+            const bool need = mine && !(fabsf(p) > err);   // inside the band (or not finite)
+            bool bit = p >= 0.f;
+            if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+                for (int e = 0; e < EPL; ++e) sKey[wib][lane * EPL + e] = x[e];
+                __syncwarp();
+                if (need) {   // exact: fp64, index order
+                    double acc = 0.0;
+                    const float* rb = R + lane * D;
+                    for (int i = 0; i < D; ++i) acc = fma((double)rb[i], (double)sKey[wib][i], acc);
+                    bit = (acc >= 0.0);
+                }
+                __syncwarp();
+            }
+            const unsigned code = __ballot_sync(0xffffffffu, mine && bit) & mask;
+            const unsigned nre = __popc(__ballot_sync(0xffffffffu, need));
+            if (lane == 0) {
+                s.scode[sidx] = code;
+                if (nre) atomicAdd(&stats->hash_rechecks, (unsigned long long)nre);
+            }
         }
-        __syncwarp();
     }
+}
+
+// ------------------------------------------------------------------ lane groups
+//
+// The search, append and merge kernels give each row to a group of 8 lanes: lane g
+// of group q (lanes 8q .. 8q+7) holds elements [g*EPG, g*EPG + EPG) of the row, so
+// one warp works on four rows at once and every lane moves 16-byte words.
+template <typename E, int D>
+struct GSlice {
+    static constexpr int EPG = D / 8;
+    static constexpr int NW = EPG * (int)sizeof(E) / 16;
+    uint4 w[NW];
+    __device__ __forceinline__ void load(const E* row, int gl) {
+        const uint4* p = reinterpret_cast<const uint4*>(row) + gl * NW;
+#pragma unroll
+        for (int k = 0; k < NW; ++k) w[k] = p[k];
+    }
+    __device__ __forceinline__ void store(E* row, int gl) const {
+        uint4* p = reinterpret_cast<uint4*>(row) + gl * NW;
+#pragma unroll
+        for (int k = 0; k < NW; ++k) p[k] = w[k];
+    }
+    __device__ __forceinline__ void zero() {
+#pragma unroll
+        for (int k = 0; k < NW; ++k) w[k] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    __device__ __forceinline__ uint32_t word(int i) const {
+        const uint4& q = w[i >> 2];
+        return (i & 3) == 0 ? q.x : (i & 3) == 1 ? q.y : (i & 3) == 2 ? q.z : q.w;
+    }
+    __device__ __forceinline__ void set_word(int i, uint32_t u) {
+        uint4& q = w[i >> 2];
+        if ((i & 3) == 0) q.x = u; else if ((i & 3) == 1) q.y = u; else if ((i & 3) == 2) q.z = u; else q.w = u;
+    }
+    __device__ __forceinline__ float at(int i) const {
+        if constexpr (sizeof(E) == 2) {
+            const uint32_t u = word(i >> 1);
+            return (i & 1) ? __uint_as_float(u & 0xffff0000u) : __uint_as_float(u << 16);
+        } else {
+            return __uint_as_float(word(i));
+        }
+    }
+    // Round EPG floats to the storage type (bf16: nearest even) and keep them.
+    __device__ __forceinline__ void from_floats(const float (&v)[EPG]) {
+        if constexpr (sizeof(E) == 2) {
+#pragma unroll
+            for (int i = 0; i < EPG / 2; ++i) {
+                const __nv_bfloat162 b = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+                set_word(i, *reinterpret_cast<const uint32_t*>(&b));
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < EPG; ++i) set_word(i, __float_as_uint(v[i]));
+        }
+    }
+};
+
+__device__ __forceinline__ float gsum(float v, unsigned gmask) {
+    v += __shfl_xor_sync(gmask, v, 4);
+    v += __shfl_xor_sync(gmask, v, 2);
+    v += __shfl_xor_sync(gmask, v, 1);
+    return v;
+}
+__device__ __forceinline__ double gsum64(double v, unsigned gmask) {
+    v += __shfl_xor_sync(gmask, v, 4);
+    v += __shfl_xor_sync(gmask, v, 2);
+    v += __shfl_xor_sync(gmask, v, 1);
+    return v;
+}
+
+// sum_i a_i b_i in fp64 in index order 0..d-1, handed from lane to lane of the
+// group (each lane continues the previous lane's sum); every lane gets the result.
+template <typename E, int D>
+__device__ __forceinline__ double gchain_dot(const GSlice<E, D>& a, const GSlice<E, D>& b, int gl, int grp,
+                                             unsigned gmask) {
+    double acc = 0.0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        if (gl == k) {
+#pragma unroll
+            for (int i = 0; i < GSlice<E, D>::EPG; ++i) acc = fma((double)a.at(i), (double)b.at(i), acc);
+        }
+        acc = __shfl_sync(gmask, acc, 8 * grp + k);
+    }
+    return acc;
+}
+
+// This lane's part of sum_i a_i b_i in fp64 (its elements in index order).
+template <typename E, int D>
+__device__ __forceinline__ double lane_dot64(const GSlice<E, D>& a, const GSlice<E, D>& b) {
+    double acc = 0.0;
+#pragma unroll
+    for (int i = 0; i < GSlice<E, D>::EPG; ++i) acc = fma((double)a.at(i), (double)b.at(i), acc);
+    return acc;
+}
+
+// Exact fp64 sums of bf16 products. A nonzero bf16 value with exponent field f
+// (f = 0, a subnormal, taken as 1) lies below 2^(f-126) and is a multiple of
+// 2^(f-134). Let span(x) = max f - min f + 7 over the nonzero elements of a row
+// (0 for a zero row). Every product x_i y_i, and so every partial sum in any
+// order, is then a multiple of 2^(minf_x + minf_y - 268), while each partial sum
+// is below d 2^(maxf_x + maxf_y - 252) in magnitude. When
+//   span(x) + span(y) <= 51 - log2(d)
+// every partial sum is an integer below 2^53 times that unit, so fp64 represents
+// all of them exactly: the sum has no rounding at all and any summation order
+// (lane sums, then the group butterfly) yields the bits of the index-order sum.
+// Otherwise the kernels fall back to the index-order chain.
+template <int D>
+constexpr int kSpanLimit = 51 - (D == 128 ? 7 : 6);
+
+template <int D>
+__device__ __forceinline__ int gspan_bf16(const GSlice<__nv_bfloat16, D>& x, unsigned gmask) {
+    int emax = 0, emin = 255;
+#pragma unroll
+    for (int i = 0; i < GSlice<__nv_bfloat16, D>::EPG / 2; ++i) {
+        const uint32_t u = x.word(i);
+        const uint32_t lo = u & 0xffffu, hi = u >> 16;
+        if (lo & 0x7fffu) {
+            const int f = max((int)((lo >> 7) & 0xffu), 1);
+            emax = max(emax, f);
+            emin = min(emin, f);
+        }
+        if (hi & 0x7fffu) {
+            const int f = max((int)((hi >> 7) & 0xffu), 1);
+            emax = max(emax, f);
+            emin = min(emin, f);
+        }
+    }
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) {
+        emax = max(emax, __shfl_xor_sync(gmask, emax, o));
+        emin = min(emin, __shfl_xor_sync(gmask, emin, o));
+    }
+    return emax >= emin ? emax - emin + 7 : 0;
 }
 
 // ------------------------------------------------------------------ search + decide
 //
-// One warp per staged token (h, t). Candidates are the committed entries of the
-// token's bucket (the linked list bhead/bnext holds exactly the entries committed
-// before this commit). fp32 cosine per candidate; with delta a rigorous bound on
-// |sim32 - sim|, the fp32 result decides when
-//   best < tau - delta                         (no merge), or
-//   best > tau + delta and best - second > 2 delta   (merge into the unique best).
-// Any other case recomputes every candidate's cosine exactly as the definition
-// does (fp64, index order) and takes the maximum, lowest entry index on ties.
+// One 8-lane group per staged token (h, t). Candidates are the committed entries of
+// the token's bucket (the list bhead/bnext holds exactly the entries committed
+// before this commit); the four groups of a warp walk their lists in lockstep, so
+// each step has four independent row loads in flight.
+//
+// bf16 storage: every cosine is formed in fp64 exactly as the definition does
+// (dot / sqrt(|k|^2 |e|^2), each sum in index order): the sums are exact by the
+// span rule above (else the index-order chain), |e|^2 was stored the same way when
+// the entry was appended, and the division and square root are IEEE-rounded on
+// both sides. The best candidate (ties to the lowest entry index) merges when its
+// cosine is >= tau.
+//
+// fp32 storage: fp32 cosines first; with delta a rigorous bound on |sim32 - sim|
+// the fp32 result decides when best < tau - delta (no merge) or best > tau + delta
+// and best - second > 2 delta (merge into the unique best). Any other case
+// recomputes every candidate with the index-order chain.
+//
+// A matched token joins its target's merge list; unmatched tokens are counted per
+// 32-token window. The last block to finish turns the window counts into the new
+// cache sizes and raises the abort flag if some head would exceed its capacity.
 template <typename E, int D>
-__global__ void __launch_bounds__(kWarps * 32)
-search_kernel(CacheView c, StageView s, float tau, double tau64, float delta, int32_t* ntouched,
-              Stats* stats) {
-    constexpr int EPL = D / 32;
-    using IO = RowIO<E, EPL>;
-    __shared__ float sTok[kWarps][D];
-    __shared__ float sCand[kWarps][D];
-    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+__global__ void __launch_bounds__(kWarps * 32, 2)
+search_kernel(CacheView c, StageView s, float tau, double tau64, float delta, int32_t* ctr, Stats* stats) {
+    using G = GSlice<E, D>;
+    constexpr int EPG = G::EPG;
+    const int lane = threadIdx.x & 31, gl = lane & 7, grp = lane >> 3;
+    const unsigned gmask = 0xFFu << (8 * grp);
+    const int H = c.H;
     const int64_t T = s.T;
-    const int64_t rows = T * c.H;
+    const int64_t rows = T * H;
     const E* Kc = reinterpret_cast<const E*>(c.Kc);
     const E* Ks = reinterpret_cast<const E*>(s.Ks);
-    for (int64_t r = (int64_t)blockIdx.x * kWarps + wib; r < rows; r += (int64_t)gridDim.x * kWarps) {
-        const int h = (int)(r / T);
-        const int64_t t = r - (int64_t)h * T;
+    int32_t* ntouched = ctr;
+    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;   // global warp
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t r4 = gw * 4; r4 < rows; r4 += nw * 4) {   // warp-uniform loop
+        const int64_t r = r4 + grp;
+        const bool valid = r < rows;
+        const int h = valid ? (int)(r / T) : 0;
+        const int64_t t = valid ? r - (int64_t)h * T : 0;
         const int64_t sidx = (int64_t)h * s.TmaxP + t;
-        float x[EPL];
-        IO::to_float(IO::load(Ks + sidx * D, lane), x);
-        float nk = 0.f;
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) nk = fmaf(x[e], x[e], nk);
-        nk = warp_sum(nk);
-        const uint32_t code = s.scode[sidx];
         const int64_t hrow = (int64_t)h * c.capP;
-        const int first = c.bhead[((int64_t)h << c.nbits) + code];
-        float best = -INFINITY, second = -INFINITY;
-        int bestj = -1, ncand = 0;
-        bool weird = false;
-        for (int j = first; j >= 0; j = c.bnext[hrow + j]) {
-            if (ncand > c.M[h]) {  // a bucket list can never be longer than the cache
-                if (lane == 0) atomicOr(&stats->error_bits, kErrBucketList);
-                break;
+        G x;
+        if (valid) x.load(Ks + sidx * D, gl);
+        else x.zero();
+        const int first = valid ? c.bhead[((int64_t)h << c.nbits) + s.scode[sidx]] : -1;
+        const int Mh = valid ? c.M[h] : 0;
+        int m = -1, nslow = 0;
+        if constexpr (sizeof(E) == 2) {
+            const int spx = gspan_bf16<D>(x, gmask);
+            double n1 = gsum64(lane_dot64(x, x), gmask);
+            if (2 * spx > kSpanLimit<D>) {
+                n1 = gchain_dot(x, x, gl, grp, gmask);
+                ++nslow;
             }
-            float y[EPL];
-            IO::to_float(IO::load(Kc + (hrow + j) * D, lane), y);
-            float dt = 0.f, ne = 0.f;
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) {
-                dt = fmaf(x[e], y[e], dt);
-                ne = fmaf(y[e], y[e], ne);
-            }
-            dt = warp_sum(dt);
-            ne = warp_sum(ne);
-            const float den = nk * ne;
-            float sim = 0.f;
-            if (nk > 1e-30f && ne > 1e-30f && den < 1e38f && fabsf(dt) < 1e38f)
-                sim = dt / sqrtf(den);
-            else
-                weird = true;
-            if (sim > best) {
-                second = best;
-                best = sim;
-                bestj = j;
-            } else if (sim > second) {
-                second = sim;
-            }
-            ++ncand;
-        }
-        int m = -1;
-        bool exact = false;
-        if (ncand > 0) {
-            if (!weird && best < tau - delta) m = -1;
-            else if (!weird && best > tau + delta && (ncand == 1 || best - second > 2.f * delta)) m = bestj;
-            else exact = true;
-        }
-        if (exact) {
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) sTok[wib][lane * EPL + e] = x[e];
-            double bsim = -INFINITY;
-            int bj = -1, guard = 0;
-            for (int j = first; j >= 0; j = c.bnext[hrow + j]) {
-                if (++guard > ncand) break;
-                float y[EPL];
-                IO::to_float(IO::load(Kc + (hrow + j) * D, lane), y);
-                __syncwarp();
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) sCand[wib][lane * EPL + e] = y[e];
-                __syncwarp();
-                double acc = 0.0;
-                if (lane < 3) {
-                    const float* a = (lane == 2) ? sCand[wib] : sTok[wib];
-                    const float* b = (lane == 1) ? sTok[wib] : sCand[wib];
-                    for (int i = 0; i < D; ++i) acc = fma((double)a[i], (double)b[i], acc);
+            double best = -INFINITY;
+            int bestj = -1, ncand = 0;
+            int j = first;
+            while (__any_sync(0xffffffffu, j >= 0)) {
+                const bool act = j >= 0;
+                G y;
+                int nxt = -1;
+                double n2 = 0.0;
+                if (act) {
+                    y.load(Kc + (hrow + j) * D, gl);
+                    nxt = c.bnext[hrow + j];
+                    n2 = c.knorm64[hrow + j];
+                } else {
+                    y.zero();
                 }
-                const double dot = __shfl_sync(0xffffffffu, acc, 0);
-                const double n1 = __shfl_sync(0xffffffffu, acc, 1);
-                const double n2 = __shfl_sync(0xffffffffu, acc, 2);
-                const double sim = (n1 > 0.0 && n2 > 0.0) ? dot / sqrt(n1 * n2) : 0.0;
-                if (sim > bsim || (sim == bsim && j < bj)) {
-                    bsim = sim;
-                    bj = j;
+                const int spy = gspan_bf16<D>(y, gmask);
+                double dot = gsum64(lane_dot64(x, y), gmask);
+                if (act) {
+                    if (spx + spy > kSpanLimit<D>) {
+                        dot = gchain_dot(x, y, gl, grp, gmask);
+                        ++nslow;
+                    }
+                    const double sim = (n1 > 0.0 && n2 > 0.0) ? dot / sqrt(n1 * n2) : 0.0;
+                    if (sim > best || (sim == best && j < bestj)) {
+                        best = sim;
+                        bestj = j;
+                    }
+                    if (++ncand > Mh) {   // a bucket list can never be longer than the cache
+                        if (gl == 0) atomicOr(&stats->error_bits, kErrBucketList);
+                        nxt = -1;
+                    }
                 }
+                j = nxt;
             }
-            m = (bj >= 0 && bsim >= tau64) ? bj : -1;
+            m = (bestj >= 0 && best >= tau64) ? bestj : -1;
+        } else {
+            float nk = 0.f;
+#pragma unroll
+            for (int i = 0; i < EPG; ++i) nk = fmaf(x.at(i), x.at(i), nk);
+            nk = gsum(nk, gmask);
+            float best = -INFINITY, second = -INFINITY;
+            int bestj = -1, ncand = 0;
+            bool weird = false;
+            int j = first;
+            while (__any_sync(0xffffffffu, j >= 0)) {
+                const bool act = j >= 0;
+                G y;
+                int nxt = -1;
+                if (act) {
+                    y.load(Kc + (hrow + j) * D, gl);
+                    nxt = c.bnext[hrow + j];
+                } else {
+                    y.zero();
+                }
+                float dt = 0.f, ne = 0.f;
+#pragma unroll
+                for (int i = 0; i < EPG; ++i) {
+                    dt = fmaf(x.at(i), y.at(i), dt);
+                    ne = fmaf(y.at(i), y.at(i), ne);
+                }
+                dt = gsum(dt, gmask);
+                ne = gsum(ne, gmask);
+                if (act) {
+                    const float den = nk * ne;
+                    float sim = 0.f;
+                    if (nk > 1e-30f && ne > 1e-30f && den < 1e38f && fabsf(dt) < 1e38f)
+                        sim = dt / sqrtf(den);
+                    else
+                        weird = true;
+                    if (sim > best) {
+                        second = best;
+                        best = sim;
+                        bestj = j;
+                    } else if (sim > second) {
+                        second = sim;
+                    }
+                    if (++ncand > Mh) {
+                        if (gl == 0) atomicOr(&stats->error_bits, kErrBucketList);
+                        nxt = -1;
+                    }
+                }
+                j = nxt;
+            }
+            bool exact = false;
+            if (ncand > 0) {
+                if (!weird && best < tau - delta) m = -1;
+                else if (!weird && best > tau + delta && (ncand == 1 || best - second > 2.f * delta)) m = bestj;
+                else exact = true;
+            }
+            if (exact) {   // uniform inside the group
+                nslow = 1;
+                const double n1 = gchain_dot(x, x, gl, grp, gmask);
+                double bsim = -INFINITY;
+                int bj = -1, guard = 0;
+                for (int jj = first; jj >= 0; jj = c.bnext[hrow + jj]) {
+                    if (++guard > ncand) break;
+                    G y;
+                    y.load(Kc + (hrow + jj) * D, gl);
+                    const double dot = gchain_dot(x, y, gl, grp, gmask);
+                    const double n2 = c.knorm64[hrow + jj];
+                    const double sim = (n1 > 0.0 && n2 > 0.0) ? dot / sqrt(n1 * n2) : 0.0;
+                    if (sim > bsim || (sim == bsim && jj < bj)) {
+                        bsim = sim;
+                        bj = jj;
+                    }
+                }
+                m = (bj >= 0 && bsim >= tau64) ? bj : -1;
+            }
         }
-        if (lane == 0) {
+        if (valid && gl == 0) {
             s.match[sidx] = m;
-            if (exact) atomicAdd(&stats->match_rechecks, 1ull);
+            if (nslow) atomicAdd(&stats->match_rechecks, (unsigned long long)nslow);
             if (m >= 0) {
-                const int old = atomicAdd(&c.mcount[hrow + m], 1);
-                if (old == 0) {
-                    const int slot = atomicAdd(&ntouched[h], 1);
-                    s.touched[(int64_t)h * s.TmaxP + slot] = m;
-                }
+                const int old = atomicExch(&c.lhead[hrow + m], (int)t);
+                s.lnext[sidx] = old;
+                if (old < 0) s.touched[(int64_t)h * s.TmaxP + atomicAdd(&ntouched[h], 1)] = m;
+            } else {
+                atomicAdd(&s.wcnt[(int64_t)h * (s.TmaxP >> 5) + (t >> 5)], 1);
             }
         }
         __syncwarp();
     }
-}
-
-// ------------------------------------------------------------------ scan
-//
-// One block per head. (a) dest[t] = M_h + (number of unmatched tokens before t)
-// for unmatched tokens, match[t] otherwise; the new size is M_h + (unmatched
-// count), and any head past capacity raises the abort flag for the whole commit.
-// (b) Merge segments: the entries touched by merges get consecutive ranges of
-// seg[] sized by their merge counts.
-__device__ int block_exclusive_scan(int v, int* total) {
-    __shared__ int wsum[32];
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
-    int inc = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int n = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += n;
-    }
-    if (lane == 31) wsum[w] = inc;
+    // The last block to finish sums the window counts into the new sizes.
+    __shared__ bool last;
+    __threadfence();   // this thread's list and count updates before the ticket
     __syncthreads();
-    if (w == 0) {
-        int x = (lane < nw) ? wsum[lane] : 0;
+    if (threadIdx.x == 0) last = atomicAdd(&ctr[2 * H + 1], 1) == (int)gridDim.x - 1;
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    const int nwin = (int)((T + 31) >> 5);
+    const int warp = threadIdx.x >> 5;
+    for (int h = warp; h < H; h += blockDim.x >> 5) {
+        int u = 0;
+        for (int w = lane; w < nwin; w += 32) u += __ldcg(&s.wcnt[(int64_t)h * (s.TmaxP >> 5) + w]);
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int n = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += n;
+        for (int o = 16; o > 0; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
+        if (lane == 0) {
+            const int nm = c.M[h] + u;
+            ctr[H + h] = nm;
+            if ((int64_t)nm > c.capacity) atomicExch(&ctr[2 * H], 1);
         }
-        wsum[lane] = x;  // inclusive prefix over warps
     }
-    __syncthreads();
-    const int before = (w > 0) ? wsum[w - 1] : 0;
-    *total = wsum[nw - 1];
-    __syncthreads();
-    return before + inc - v;
 }
 
-__global__ void __launch_bounds__(1024) scan_kernel(CacheView c, StageView s, int32_t* ctr) {
-    const int h = blockIdx.x, H = c.H;
-    int32_t* ntouched = ctr;
-    int32_t* newM = ctr + H;
-    int32_t* abort_flag = ctr + 2 * H;
-    const int64_t T = s.T;
-    const int64_t base = (int64_t)h * s.TmaxP;
-    const int nt = blockDim.x;
-    const int64_t per = (T + nt - 1) / nt;
-    const int64_t t0 = min(T, (int64_t)threadIdx.x * per), t1 = min(T, t0 + per);
-    int u = 0;
-    for (int64_t t = t0; t < t1; ++t) u += (s.match[base + t] < 0);
-    int total = 0;
-    const int ex = block_exclusive_scan(u, &total);
-    const int Mh = c.M[h];
-    int pos = Mh + ex;
-    for (int64_t t = t0; t < t1; ++t) {
-        const int m = s.match[base + t];
-        s.dest[base + t] = (m < 0) ? pos++ : m;
-        s.lcode[base + t] = s.scode[base + t];
+// |k|^2 of a row held by a lane group, in fp64 with the value of the index-order
+// sum (exact by the span rule for bf16 rows that satisfy it, else the chain).
+template <typename E, int D>
+__device__ __forceinline__ double gnorm64(const GSlice<E, D>& x, int gl, int grp, unsigned gmask) {
+    if constexpr (sizeof(E) == 2) {
+        if (2 * gspan_bf16<D>(x, gmask) <= kSpanLimit<D>) return gsum64(lane_dot64(x, x), gmask);
     }
-    if (threadIdx.x == 0) {
-        newM[h] = Mh + total;
-        if ((int64_t)Mh + total > c.capacity) atomicExch(abort_flag, 1);
-    }
-    const int ns = ntouched[h];
-    const int per2 = (ns + nt - 1) / nt;
-    const int s0 = min(ns, (int)threadIdx.x * per2), s1 = min(ns, s0 + per2);
-    const int64_t hrow = (int64_t)h * c.capP;
-    int cs = 0;
-    for (int q = s0; q < s1; ++q) cs += c.mcount[hrow + s.touched[base + q]];
-    int tot2 = 0;
-    int off = block_exclusive_scan(cs, &tot2);
-    for (int q = s0; q < s1; ++q) {
-        const int j = s.touched[base + q];
-        c.moff[hrow + j] = off;
-        off += c.mcount[hrow + j];
-    }
+    return gchain_dot(x, x, gl, grp, gmask);
 }
 
 // ------------------------------------------------------------------ append
 //
-// One warp per staged token. Unmatched tokens become entries at dest (key, value
-// mean, n = 1, log2 n = 0, code) and are pushed on their bucket's list; matched
-// tokens claim a slot in their target's merge segment.
+// One warp per 32-token window of one head. Unmatched tokens of the window take
+// consecutive entries in token order: dest = M_h + (unmatched tokens of earlier
+// windows) + (unmatched lanes below). Each becomes an entry (key, value mean, n = 1,
+// log2 n = 0, code, |k|^2 with the value of the fp64 index-order sum) and is pushed
+// on its bucket's list; lane groups copy two rows each per pass.
 template <typename E, int D>
-__global__ void __launch_bounds__(kWarps * 32) append_kernel(CacheView c, StageView s, const int32_t* ctr) {
-    constexpr int EPL = D / 32;
-    using IO = RowIO<E, EPL>;
+__global__ void __launch_bounds__(kWarps * 32, 3) append_kernel(CacheView c, StageView s, const int32_t* ctr) {
+    using G = GSlice<E, D>;
+    constexpr int EPG = G::EPG;
+    __shared__ int sSrc[kWarps][32];
     const int H = c.H;
     if (ctr[2 * H]) return;  // commit aborted: nothing changes
-    if (blockIdx.x == 0)
-        for (int hh = threadIdx.x; hh < H; hh += blockDim.x) c.M[hh] = ctr[H + hh];
-    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31, gl = lane & 7, grp = lane >> 3, wib = threadIdx.x >> 5;
+    const unsigned gmask = 0xFFu << (8 * grp);
     const int64_t T = s.T;
-    const int64_t rows = T * H;
-    for (int64_t r = (int64_t)blockIdx.x * kWarps + wib; r < rows; r += (int64_t)gridDim.x * kWarps) {
-        const int h = (int)(r / T);
-        const int64_t t = r - (int64_t)h * T;
-        const int64_t sidx = (int64_t)h * s.TmaxP + t;
-        const int64_t hrow = (int64_t)h * c.capP;
-        const int m = s.match[sidx];
-        if (m < 0) {
-            const int j = s.dest[sidx];
-            const int64_t e = hrow + j;
-            const auto kv = IO::load(reinterpret_cast<const E*>(s.Ks) + sidx * D, lane);
-            const auto vv = IO::load(reinterpret_cast<const E*>(s.Vs) + sidx * D, lane);
-            IO::store(reinterpret_cast<E*>(c.Kc) + e * D, lane, kv);
-            IO::store(reinterpret_cast<E*>(c.Vc) + e * D, lane, vv);
-            float v[EPL];
-            IO::to_float(vv, v);
+    const int nwin = (int)((T + 31) >> 5);
+    const E* Ks = reinterpret_cast<const E*>(s.Ks);
+    const E* Vs = reinterpret_cast<const E*>(s.Vs);
+    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t wg = gw; wg < (int64_t)H * nwin; wg += nw) {
+        const int h = (int)(wg / nwin);
+        const int w = (int)(wg - (int64_t)h * nwin);
+        const int32_t* wc = s.wcnt + (int64_t)h * (s.TmaxP >> 5);
+        int prefix = 0;
+        for (int q = lane; q < w; q += 32) prefix += wc[q];
 #pragma unroll
-            for (int q = 0; q < EPL; ++q) c.V32[e * D + lane * EPL + q] = v[q];
-            if (lane == 0) {
-                const uint32_t code = s.scode[sidx];
-                c.cnt[e] = 1;
-                c.bias2[e] = 0.f;
-                c.code[e] = code;
-                c.bnext[e] = atomicExch(&c.bhead[((int64_t)h << c.nbits) + code], j);
-            }
-        } else if (lane == 0) {
-            const int pos = c.moff[hrow + m] + atomicAdd(&c.mfill[hrow + m], 1);
-            s.seg[(int64_t)h * s.TmaxP + pos] = (int)t;
+        for (int o = 16; o > 0; o >>= 1) prefix += __shfl_xor_sync(0xffffffffu, prefix, o);
+        const int64_t t = (int64_t)w * 32 + lane;
+        const bool valid = t < T;
+        const int64_t sidx = (int64_t)h * s.TmaxP + t;
+        const int m = valid ? s.match[sidx] : 0;
+        const bool un = valid && m < 0;
+        const unsigned bal = __ballot_sync(0xffffffffu, un);
+        const int rank = __popc(bal & ((1u << lane) - 1u));
+        const int base = c.M[h] + prefix;
+        if (valid) {
+            s.dest[sidx] = un ? base + rank : m;
+            s.lcode[sidx] = s.scode[sidx];
         }
+        if (un) sSrc[wib][rank] = lane;
+        __syncwarp();
+        const int nun = __popc(bal);
+        const int64_t hrow = (int64_t)h * c.capP;
+        const int64_t wrow = (int64_t)h * s.TmaxP + (int64_t)w * 32;
+        for (int k0 = 0; k0 < nun; k0 += 8) {   // warp-uniform
+            G kr[2], vr[2];
+            int64_t st[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int k = k0 + 4 * u + grp;
+                st[u] = k < nun ? wrow + sSrc[wib][k] : -1;
+                if (st[u] >= 0) {
+                    kr[u].load(Ks + st[u] * D, gl);
+                    vr[u].load(Vs + st[u] * D, gl);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                if (st[u] < 0) continue;   // group-uniform
+                const int k = k0 + 4 * u + grp;
+                const int64_t e = hrow + base + k;
+                kr[u].store(reinterpret_cast<E*>(c.Kc) + e * D, gl);
+                vr[u].store(reinterpret_cast<E*>(c.Vc) + e * D, gl);
+                float4* v32 = reinterpret_cast<float4*>(c.V32 + e * D + gl * EPG);
+#pragma unroll
+                for (int q = 0; q < EPG / 4; ++q)
+                    v32[q] = make_float4(vr[u].at(4 * q), vr[u].at(4 * q + 1), vr[u].at(4 * q + 2), vr[u].at(4 * q + 3));
+                const double nk = gnorm64(kr[u], gl, grp, gmask);
+                if (gl == 0) {
+                    const uint32_t code = s.scode[st[u]];
+                    c.knorm64[e] = nk;
+                    c.cnt[e] = 1;
+                    c.bias2[e] = 0.f;
+                    c.code[e] = code;
+                    c.bnext[e] = atomicExch(&c.bhead[((int64_t)h << c.nbits) + code], base + k);
+                }
+            }
+        }
+        __syncwarp();
     }
 }
 
 // ------------------------------------------------------------------ merge
 //
-// One warp per entry touched by merges. The matched tokens' values are summed in
-// fp32 in ascending token order (deterministic whatever order the atomics filled
-// the segment in), then v <- (n v + sum) / (n + m), n <- n + m (Lemma 5.1: the
-// merged entry carries the mean of its group and the group size).
+// One lane group per entry touched by merges. The matched tokens' values are
+// summed in fp32 in ascending token order (whatever order the atomics built the
+// list in), then v <- (n v + sum) / (n + m), n <- n + m (Lemma 5.1: the merged
+// entry carries the mean of its group and the group size). Lists of up to 8 tokens
+// are ordered inside the group; longer ones go to the whole warp, which orders up
+// to kListSmem tokens in shared memory and otherwise gathers them by scanning the
+// head's match targets in token order. The kernel also leaves the per-commit state
+// ready for the next commit (lists emptied, window counts zeroed, sizes published).
+constexpr int kListSmem = 256;
+
 template <typename E, int D>
-__global__ void __launch_bounds__(kWarps * 32) merge_kernel(CacheView c, StageView s, int32_t* ctr) {
+__device__ void merge_long_list(const CacheView& c, const StageView& s, int h, int j, int32_t* sIds,
+                                int32_t* sSorted, int lane) {
     constexpr int EPL = D / 32;
     using IO = RowIO<E, EPL>;
-    const int H = c.H;
-    const bool aborted = ctr[2 * H] != 0;
-    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     const int64_t T = s.T;
-    const int64_t rows = T * H;
+    const int64_t sbase = (int64_t)h * s.TmaxP;
+    const int64_t e = (int64_t)h * c.capP + j;
     const E* Vs = reinterpret_cast<const E*>(s.Vs);
-    for (int64_t r = (int64_t)blockIdx.x * kWarps + wib; r < rows; r += (int64_t)gridDim.x * kWarps) {
-        const int h = (int)(r / T);
-        const int slot = (int)(r - (int64_t)h * T);
-        if (slot >= ctr[h]) continue;
-        const int64_t sbase = (int64_t)h * s.TmaxP;
-        const int64_t hrow = (int64_t)h * c.capP;
-        const int j = s.touched[sbase + slot];
-        const int64_t e = hrow + j;
-        const int cntj = c.mcount[e];
-        if (!aborted) {
-            const int off = c.moff[e];
-            float acc[EPL];
+    int L = 0, id = 0x7fffffff;
+    for (int tt = c.lhead[e]; tt >= 0; tt = s.lnext[sbase + tt]) {
+        if (L < 32 && lane == L) id = tt;
+        if (L < kListSmem && lane == 0) sIds[L] = tt;
+        ++L;
+        if (L > (int)T) break;   // a list is never longer than the chunk
+    }
+    __syncwarp();
+    float acc[EPL];
 #pragma unroll
-            for (int q = 0; q < EPL; ++q) acc[q] = 0.f;
-            if (cntj <= 32) {
-                const int id = (lane < cntj) ? s.seg[sbase + off + lane] : 0x7fffffff;
-                int rank = 0;
-                for (int k = 0; k < 32; ++k) rank += (__shfl_sync(0xffffffffu, id, k) < id);
-                for (int q = 0; q < cntj; ++q) {
-                    const int src = __ffs(__ballot_sync(0xffffffffu, rank == q)) - 1;
-                    const int tt = __shfl_sync(0xffffffffu, id, src);
-                    float v[EPL];
-                    IO::to_float(IO::load(Vs + (sbase + tt) * D, lane), v);
+    for (int q = 0; q < EPL; ++q) acc[q] = 0.f;
+    auto add_row = [&](int tt) {
+        float v[EPL];
+        IO::to_float(IO::load(Vs + (sbase + tt) * D, lane), v);
 #pragma unroll
-                    for (int qq = 0; qq < EPL; ++qq) acc[qq] = __fadd_rn(acc[qq], v[qq]);
-                }
-            } else {
-                int last = -1;
-                for (int q = 0; q < cntj; ++q) {
-                    int mn = 0x7fffffff;
-                    for (int p = lane; p < cntj; p += 32) {
-                        const int id = s.seg[sbase + off + p];
-                        if (id > last && id < mn) mn = id;
-                    }
-                    mn = warp_min(mn);
-                    float v[EPL];
-                    IO::to_float(IO::load(Vs + (sbase + mn) * D, lane), v);
-#pragma unroll
-                    for (int qq = 0; qq < EPL; ++qq) acc[qq] = __fadd_rn(acc[qq], v[qq]);
-                    last = mn;
-                }
-            }
-            const int nold = c.cnt[e];
-            const int ntot = nold + cntj;
-            const float fn = (float)nold, ft = (float)ntot;
-            float nv[EPL];
-#pragma unroll
-            for (int q = 0; q < EPL; ++q) {
-                const float old = c.V32[e * D + lane * EPL + q];
-                nv[q] = __fdiv_rn(__fadd_rn(__fmul_rn(fn, old), acc[q]), ft);
-                c.V32[e * D + lane * EPL + q] = nv[q];
-            }
-            IO::store(reinterpret_cast<E*>(c.Vc) + e * D, lane, IO::from_float(nv));
-            if (lane == 0) {
-                c.cnt[e] = ntot;
-                c.bias2[e] = log2f(ft);
-            }
+        for (int q = 0; q < EPL; ++q) acc[q] = __fadd_rn(acc[q], v[q]);
+    };
+    if (L <= 32) {
+        int rank = 0;
+        for (int k = 0; k < L; ++k) rank += (__shfl_sync(0xffffffffu, id, k) < id);
+        for (int q2 = 0; q2 < L; ++q2) {
+            const int src = __ffs(__ballot_sync(0xffffffffu, rank == q2 && lane < L)) - 1;
+            add_row(__shfl_sync(0xffffffffu, id, src));
         }
-        if (lane == 0) {
-            c.mcount[e] = 0;
-            c.mfill[e] = 0;
+    } else if (L <= kListSmem) {
+        for (int a = lane; a < L; a += 32) {
+            const int mine = sIds[a];
+            int rank = 0;
+            for (int b = 0; b < L; ++b) rank += (sIds[b] < mine);
+            sSorted[rank] = mine;
+        }
+        __syncwarp();
+        for (int q2 = 0; q2 < L; ++q2) add_row(sSorted[q2]);
+    } else {
+        for (int64_t t0 = 0; t0 < T; t0 += 32) {
+            const bool hit = t0 + lane < T && s.match[sbase + t0 + lane] == j;
+            unsigned b = __ballot_sync(0xffffffffu, hit);
+            while (b) {
+                const int src = __ffs(b) - 1;
+                b &= b - 1;
+                add_row((int)t0 + src);
+            }
         }
     }
+    const int nold = c.cnt[e];
+    const int ntot = nold + L;
+    const float fn = (float)nold, ft = (float)ntot;
+    float nv[EPL];
+#pragma unroll
+    for (int q = 0; q < EPL; ++q) {
+        const float old = c.V32[e * D + lane * EPL + q];
+        nv[q] = __fdiv_rn(__fadd_rn(__fmul_rn(fn, old), acc[q]), ft);
+        c.V32[e * D + lane * EPL + q] = nv[q];
+    }
+    IO::store(reinterpret_cast<E*>(c.Vc) + e * D, lane, IO::from_float(nv));
+    __syncwarp();
+    if (lane == 0) {
+        c.cnt[e] = ntot;
+        c.bias2[e] = log2f(ft);
+        c.lhead[e] = -1;
+    }
+    __syncwarp();
+}
+
+template <typename E, int D>
+__global__ void __launch_bounds__(kWarps * 32, 3) merge_kernel(CacheView c, StageView s, int32_t* ctr) {
+    using G = GSlice<E, D>;
+    constexpr int EPG = G::EPG;
+    __shared__ int32_t sIds[kWarps][kListSmem];
+    __shared__ int32_t sSorted[kWarps][kListSmem];
+    const int H = c.H;
+    const bool aborted = ctr[2 * H] != 0;
+    const int lane = threadIdx.x & 31, gl = lane & 7, grp = lane >> 3, wib = threadIdx.x >> 5;
+    const unsigned gmask = 0xFFu << (8 * grp);
+    const int64_t T = s.T;
+    const E* Vs = reinterpret_cast<const E*>(s.Vs);
+    if (!aborted && blockIdx.x == 0)
+        for (int hh = threadIdx.x; hh < H; hh += blockDim.x) c.M[hh] = ctr[H + hh];
+    const int nwin = (int)((T + 31) >> 5);
+    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < (int64_t)H * nwin;
+         q += (int64_t)gridDim.x * blockDim.x)
+        s.wcnt[(q / nwin) * (s.TmaxP >> 5) + (q % nwin)] = 0;
+    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t q4 = gw * 4; q4 < (int64_t)H * T; q4 += nw * 4) {   // warp-uniform
+        const int64_t q = q4 + grp;
+        int h = 0, j = -1;
+        bool act = false, big = false;
+        if (q < (int64_t)H * T) {
+            h = (int)(q / T);
+            const int slot = (int)(q - (int64_t)h * T);
+            act = slot < ctr[h];
+            if (act) j = s.touched[(int64_t)h * s.TmaxP + slot];
+        }
+        if (act) {   // group-uniform
+            const int64_t sbase = (int64_t)h * s.TmaxP;
+            const int64_t e = (int64_t)h * c.capP + j;
+            if (!aborted) {
+                const float4* v32p = reinterpret_cast<const float4*>(c.V32 + e * D + gl * EPG);
+                float4 old[EPG / 4];
+#pragma unroll
+                for (int k = 0; k < EPG / 4; ++k) old[k] = v32p[k];
+                const int nold = c.cnt[e];
+                int L = 0, id = 0x7fffffff;
+                for (int tt = c.lhead[e]; tt >= 0; tt = s.lnext[sbase + tt]) {
+                    if (gl == L) id = tt;
+                    if (++L > 8) break;
+                }
+                if (L > 8) {
+                    big = true;
+                } else {
+                    int rank = 0;
+                    for (int k = 0; k < L; ++k) rank += (__shfl_sync(gmask, id, 8 * grp + k) < id);
+                    int srt = 0;   // lane gl gets the gl-th smallest token
+                    for (int k = 0; k < L; ++k) {
+                        const int idk = __shfl_sync(gmask, id, 8 * grp + k);
+                        const int rk = __shfl_sync(gmask, rank, 8 * grp + k);
+                        if (rk == gl) srt = idk;
+                    }
+                    float acc[EPG];
+#pragma unroll
+                    for (int i = 0; i < EPG; ++i) acc[i] = 0.f;
+                    G cur;
+                    cur.load(Vs + (sbase + __shfl_sync(gmask, srt, 8 * grp)) * D, gl);
+                    for (int k = 0; k < L; ++k) {
+                        G nxt;
+                        const int tn = __shfl_sync(gmask, srt, 8 * grp + ((k + 1) & 7));
+                        if (k + 1 < L) nxt.load(Vs + (sbase + tn) * D, gl);
+#pragma unroll
+                        for (int i = 0; i < EPG; ++i) acc[i] = __fadd_rn(acc[i], cur.at(i));
+                        cur = nxt;
+                    }
+                    const int ntot = nold + L;
+                    const float fn = (float)nold, ft = (float)ntot;
+                    float nv[EPG];
+#pragma unroll
+                    for (int k = 0; k < EPG / 4; ++k) {
+                        nv[4 * k] = __fdiv_rn(__fadd_rn(__fmul_rn(fn, old[k].x), acc[4 * k]), ft);
+                        nv[4 * k + 1] = __fdiv_rn(__fadd_rn(__fmul_rn(fn, old[k].y), acc[4 * k + 1]), ft);
+                        nv[4 * k + 2] = __fdiv_rn(__fadd_rn(__fmul_rn(fn, old[k].z), acc[4 * k + 2]), ft);
+                        nv[4 * k + 3] = __fdiv_rn(__fadd_rn(__fmul_rn(fn, old[k].w), acc[4 * k + 3]), ft);
+                    }
+                    float4* v32w = reinterpret_cast<float4*>(c.V32 + e * D + gl * EPG);
+#pragma unroll
+                    for (int k = 0; k < EPG / 4; ++k)
+                        v32w[k] = make_float4(nv[4 * k], nv[4 * k + 1], nv[4 * k + 2], nv[4 * k + 3]);
+                    G out;
+                    out.from_floats(nv);
+                    out.store(reinterpret_cast<E*>(c.Vc) + e * D, gl);
+                    if (gl == 0) {
+                        c.cnt[e] = ntot;
+                        c.bias2[e] = log2f(ft);
+                    }
+                }
+            }
+            __syncwarp(gmask);
+            if (!big && gl == 0) c.lhead[e] = -1;
+        }
+        // lists longer than 8 tokens: the whole warp, one list at a time
+        unsigned bigm = __ballot_sync(0xffffffffu, big && gl == 0);
+        while (bigm) {
+            const int src = __ffs(bigm) - 1;
+            bigm &= bigm - 1;
+            const int bh = __shfl_sync(0xffffffffu, h, src);
+            const int bj = __shfl_sync(0xffffffffu, j, src);
+            merge_long_list<E, D>(c, s, bh, bj, sIds[wib], sSorted[wib], lane);
+        }
+    }
+}
+
+template <typename E, int D, int NBP>
+cudaError_t stage_hash_n(const CacheView& c, const StageView& s, const void* K, const void* V, const float* R,
+                         const float* Rnorm, Stats* stats, cudaStream_t st) {
+    const int64_t rows = s.T * c.H;
+    const int grid = grid_for_rows(rows > s.TmaxP ? rows : s.TmaxP, 4 * kWarps, 148 * 8);
+    stage_hash_kernel<E, D, NBP><<<grid, kWarps * 32, 0, st>>>(
+        reinterpret_cast<const E*>(K), reinterpret_cast<const E*>(V), c, s, R, Rnorm, stats);
+    return cudaGetLastError();
 }
 
 template <typename E, int D>
 cudaError_t stage_hash_t(const CacheView& c, const StageView& s, const void* K, const void* V,
                          const float* R, const float* Rnorm, Stats* stats, cudaStream_t st) {
-    const int64_t rows = s.T * c.H;
-    const int grid = grid_for_rows(rows > s.TmaxP ? rows : s.TmaxP, kWarps, 148 * 16);
-    const size_t smem = sizeof(float) * ((size_t)c.nbits * (D + 1) + kWarps * D);
-    stage_hash_kernel<E, D><<<grid, kWarps * 32, smem, st>>>(
-        reinterpret_cast<const E*>(K), reinterpret_cast<const E*>(V), c, s, R, Rnorm, stats);
-    return cudaGetLastError();
+    if (c.nbits <= 8) return stage_hash_n<E, D, 8>(c, s, K, V, R, Rnorm, stats, st);
+    if (c.nbits <= 16) return stage_hash_n<E, D, 16>(c, s, K, V, R, Rnorm, stats, st);
+    return stage_hash_n<E, D, 32>(c, s, K, V, R, Rnorm, stats, st);
 }
 
 template <typename E, int D>
@@ -526,14 +877,14 @@ cudaError_t commit_t(const CacheView& c, const StageView& s, float tau, int32_t*
     cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int32_t) * kCtrInts(H), st);
     if (e != cudaSuccess) return e;
     const int64_t rows = s.T * H;
-    const int grid = grid_for_rows(rows, kWarps, 148 * 16);
-    // delta bounds |sim32 - sim| (see the kernel comment): 2 x (2 (d+2) u + 3 u).
+    // delta bounds |sim32 - sim| (see the search kernel): 2 x (2 (d+2) u + 3 u).
     const float delta = 2.f * (2.f * (float)(D + 2) * kU32 + 3.f * kU32);
-    search_kernel<E, D><<<grid, kWarps * 32, 0, st>>>(c, s, tau, (double)tau, delta, ctr, stats);
-    scan_kernel<<<H, 1024, 0, st>>>(c, s, ctr);
-    append_kernel<E, D><<<grid, kWarps * 32, 0, st>>>(c, s, ctr);
-    merge_kernel<E, D><<<grid, kWarps * 32, 0, st>>>(c, s, ctr);
-    *launches += 4;
+    const int sgrid = grid_for_rows(rows, 4 * kWarps, 148 * 16);
+    search_kernel<E, D><<<sgrid, kWarps * 32, 0, st>>>(c, s, tau, (double)tau, delta, ctr, stats);
+    const int64_t wins = (int64_t)H * ((s.T + 31) / 32);
+    append_kernel<E, D><<<grid_for_rows(wins, kWarps, 148 * 16), kWarps * 32, 0, st>>>(c, s, ctr);
+    merge_kernel<E, D><<<grid_for_rows(rows, kWarps, 148 * 8), kWarps * 32, 0, st>>>(c, s, ctr);
+    *launches += 3;
     return cudaGetLastError();
 }
 

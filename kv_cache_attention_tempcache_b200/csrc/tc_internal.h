@@ -22,9 +22,8 @@ struct CacheView {
     uint32_t* code;        // [H][capP]
     int32_t* bnext;        // [H][capP] next older entry in the same bucket, -1 ends
     int32_t* bhead;        // [H][2^nbits] newest entry of each bucket, -1 = empty
-    int32_t* mcount;       // [H][capP] tokens merging into the entry in this commit (0 between commits)
-    int32_t* mfill;        // [H][capP] fill cursor of the entry's merge segment (0 between commits)
-    int32_t* moff;         // [H][capP] start of the entry's merge segment
+    double* knorm64;       // [H][capP] |k|^2 of each entry, fp64 summed in index order
+    int32_t* lhead;        // [H][capP] newest token merging into the entry in this commit (-1 between commits)
     int32_t* M;            // [H] committed entries
 };
 
@@ -38,7 +37,8 @@ struct StageView {
     int32_t* match;        // [H][TmaxP] merge target or -1 (last commit)
     int32_t* dest;         // [H][TmaxP] entry each token ended in (last commit)
     uint32_t* lcode;       // [H][TmaxP] codes of the last committed chunk
-    int32_t* seg;          // [H][TmaxP] token ids grouped by merge target
+    int32_t* lnext;        // [H][TmaxP] next (older) token of the same merge list
+    int32_t* wcnt;         // [H][TmaxP/32] unmatched tokens per 32-token window (0 between commits)
     int32_t* touched;      // [H][TmaxP] entries with at least one merge
 };
 
@@ -46,6 +46,7 @@ struct StageView {
 //   ctr[0, H)   entries touched by merges, per head
 //   ctr[H, 2H)  cache size after the commit, per head
 //   ctr[2H]     abort flag: some head would exceed its capacity
+//   ctr[2H+1]   blocks of the search kernel that have finished
 constexpr int kCtrInts(int H) { return 2 * H + 2; }
 
 // Sticky device-side statistics and error bits.

@@ -149,7 +149,7 @@ struct tc_ctx {
         return TC_OK;
     }
     void free_staging() {
-        void* ptrs[] = {s.Ks, s.Vs, s.scode, s.sbias, s.match, s.dest, s.lcode, s.seg, s.touched};
+        void* ptrs[] = {s.Ks, s.Vs, s.scode, s.sbias, s.match, s.dest, s.lcode, s.lnext, s.wcnt, s.touched};
         for (void* p : ptrs) {
             if (!p) continue;
             owned.erase(std::remove(owned.begin(), owned.end(), p), owned.end());
@@ -202,15 +202,17 @@ tc_status ensure_staging(tc_ctx* x, int64_t T) {
     if ((st = c.alloc(&c.s.Ks, rowsH * x->d * x->esize)) || (st = c.alloc(&c.s.Vs, rowsH * x->d * x->esize)) ||
         (st = c.alloc((void**)&c.s.scode, rowsH * 4)) || (st = c.alloc((void**)&c.s.sbias, P * 4)) ||
         (st = c.alloc((void**)&c.s.match, rowsH * 4)) || (st = c.alloc((void**)&c.s.dest, rowsH * 4)) ||
-        (st = c.alloc((void**)&c.s.lcode, rowsH * 4)) || (st = c.alloc((void**)&c.s.seg, rowsH * 4)) ||
-        (st = c.alloc((void**)&c.s.touched, rowsH * 4))) {
+        (st = c.alloc((void**)&c.s.lcode, rowsH * 4)) || (st = c.alloc((void**)&c.s.lnext, rowsH * 4)) ||
+        (st = c.alloc((void**)&c.s.wcnt, rowsH / 32 * 4)) || (st = c.alloc((void**)&c.s.touched, rowsH * 4))) {
         x->free_staging();
         return st;
     }
     // Zero the staging keys and values once: rows past the staged chunk are only
     // ever read as masked attention operands and must hold finite values.
+    // The window counts start at zero; every commit leaves them at zero.
     if (cudaMemset(c.s.Ks, 0, rowsH * x->d * x->esize) != cudaSuccess ||
-        cudaMemset(c.s.Vs, 0, rowsH * x->d * x->esize) != cudaSuccess)
+        cudaMemset(c.s.Vs, 0, rowsH * x->d * x->esize) != cudaSuccess ||
+        cudaMemset(c.s.wcnt, 0, rowsH / 32 * 4) != cudaSuccess)
         return cuda_status(cudaGetLastError());
     x->s.TmaxP = P;
     x->maps_T = -1;
@@ -355,8 +357,8 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
         (st = x->alloc((void**)&c.V32, rows * d * 4)) || (st = x->alloc((void**)&c.cnt, rows * 4)) ||
         (st = x->alloc((void**)&c.bias2, rows * 4)) || (st = x->alloc((void**)&c.code, rows * 4)) ||
         (st = x->alloc((void**)&c.bnext, rows * 4)) || (st = x->alloc((void**)&c.bhead, ((size_t)H << nbits) * 4)) ||
-        (st = x->alloc((void**)&c.mcount, rows * 4)) || (st = x->alloc((void**)&c.mfill, rows * 4)) ||
-        (st = x->alloc((void**)&c.moff, rows * 4)) || (st = x->alloc((void**)&c.M, (size_t)H * 4)) ||
+        (st = x->alloc((void**)&c.knorm64, rows * 8)) || (st = x->alloc((void**)&c.lhead, rows * 4)) ||
+        (st = x->alloc((void**)&c.M, (size_t)H * 4)) ||
         (st = x->alloc((void**)&x->ctr, (size_t)kCtrInts(H) * 4)) ||
         (st = x->alloc((void**)&x->stats, sizeof(Stats))) ||
         (st = x->alloc((void**)&x->R, (size_t)nbits * d * 4)) || (st = x->alloc((void**)&x->Rnorm, nbits * 4))) {
@@ -375,8 +377,8 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
     if ((e = cudaMemset(c.Kc, 0, rows * d * x->esize)) || (e = cudaMemset(c.Vc, 0, rows * d * x->esize)) ||
         (e = cudaMemset(c.V32, 0, rows * d * 4)) || (e = cudaMemset(c.cnt, 0, rows * 4)) ||
         (e = cudaMemset(c.code, 0, rows * 4)) || (e = cudaMemset(c.bnext, 0xff, rows * 4)) ||
-        (e = cudaMemset(c.bhead, 0xff, ((size_t)H << nbits) * 4)) || (e = cudaMemset(c.mcount, 0, rows * 4)) ||
-        (e = cudaMemset(c.mfill, 0, rows * 4)) || (e = cudaMemset(c.moff, 0, rows * 4)) ||
+        (e = cudaMemset(c.bhead, 0xff, ((size_t)H << nbits) * 4)) || (e = cudaMemset(c.knorm64, 0, rows * 8)) ||
+        (e = cudaMemset(c.lhead, 0xff, rows * 4)) ||
         (e = cudaMemset(c.M, 0, (size_t)H * 4)) || (e = cudaMemset(x->ctr, 0, (size_t)kCtrInts(H) * 4)) ||
         (e = cudaMemset(x->stats, 0, sizeof(Stats))) ||
         (e = cudaMemcpy(x->R, x->Rhost.data(), (size_t)nbits * d * 4, cudaMemcpyHostToDevice)) ||
