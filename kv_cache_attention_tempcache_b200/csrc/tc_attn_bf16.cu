@@ -54,6 +54,18 @@
 #ifndef TC_ATTN_VST
 #define TC_ATTN_VST 2
 #endif
+#ifndef TC_ATTN_SPLIT
+#define TC_ATTN_SPLIT 0
+#endif
+#ifndef TC_ATTN_RING
+#define TC_ATTN_RING 0
+#endif
+#ifndef TC_ATTN_DUO
+#define TC_ATTN_DUO 1
+#endif
+#ifndef TC_ATTN_ONEPASS
+#define TC_ATTN_ONEPASS 0
+#endif
 
 namespace tc {
 
@@ -78,6 +90,12 @@ constexpr int kTeams = TC_ATTN_TEAMS;          // 2: teams on alternate key tile
 constexpr int kSched = TC_ATTN_SCHED;          // MMA issue: 0 blocking, 1 polling, 2 polling with backoff
 constexpr int kKSt = TC_ATTN_KST;               // K ring stages
 constexpr int kVSt = TC_ATTN_VST;               // V ring stages
+constexpr bool kSplit = TC_ATTN_SPLIT != 0;      // teams with two threads per query row
+constexpr int kThreadsSplit = 32 * (16 + 3);
+constexpr bool kRing = TC_ATTN_RING != 0;        // one query tile, 16 softmax warps, three S buffers
+constexpr int kThreadsRing = 32 * (16 + 4);
+constexpr bool kDuo = TC_ATTN_DUO != 0;          // two teams over the ring, one shared O
+constexpr bool kOnePass = TC_ATTN_ONEPASS != 0;  // teams: S read from TMEM once per tile, into registers
 static_assert(kSBuf == 2 || kSBuf == 3, "two or three score buffers");
 static_assert(kKSt >= 2 && kKSt <= 4 && kVSt >= 2 && kVSt <= 4, "ring depths");
 static_assert(!kQinTmem || kSBuf == 2, "Q in TMEM leaves room for two score buffers");
@@ -230,6 +248,13 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t 
           "=r"(r[29]), "=r"(r[30]), "=r"(r[31])                                                              \
         : "r"(taddr))
 
+#define TC_LD16(taddr, r)                                                                                    \
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];" \
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),    \
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),           \
+                   "=r"(r[15])                                                                                       \
+                 : "r"(taddr))
+
 #define TC_LD64(taddr, r)                                                                                    \
     asm volatile(                                                                                            \
         "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17," \
@@ -368,6 +393,18 @@ __device__ __forceinline__ bool bar_and_256(bool v) {
         "bar.red.and.pred q, 1, 256, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(res)
         : "r"((uint32_t)v)
+        : "memory");
+    return res != 0;
+}
+
+// Named barrier `id` over `count` threads with an AND of `v` across them.
+__device__ __forceinline__ bool bar_and(int id, int count, bool v) {
+    uint32_t res;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(res)
+        : "r"((uint32_t)v), "r"(id), "r"(count)
         : "memory");
     return res != 0;
 }
@@ -899,20 +936,37 @@ attend_bf16_teams_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
             if (!bar_and_team(got, t)) { ok = false; break; }
             if (i + 2 < ntiles) bnext = bias_of(i + 2);
             tc_fence_after();
-            // Pass 1: row max of the raw scores, 64 columns at a time.
+            // Row max of the raw scores: with kOnePass the whole 128-column row of S
+            // comes into registers with one wait, otherwise 64 columns at a time.
             float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-            for (int h2 = 0; h2 < 2; ++h2) {
-                uint32_t sr[64];
-                TC_LD32(tS + 64 * h2, (sr + 0));
-                TC_LD32(tS + 64 * h2 + 32, (sr + 32));
+            uint32_t srow[kOnePass ? 128 : 1];
+            if constexpr (kOnePass) {
+                TC_LD32(tS, (srow + 0));
+                TC_LD32(tS + 32, (srow + 32));
+                TC_LD32(tS + 64, (srow + 64));
+                TC_LD32(tS + 96, (srow + 96));
                 tc_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 64; j += 8) {
-                    m4[0] = max3(m4[0], __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
-                    m4[1] = max3(m4[1], __uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3]));
-                    m4[2] = max3(m4[2], __uint_as_float(sr[j + 4]), __uint_as_float(sr[j + 5]));
-                    m4[3] = max3(m4[3], __uint_as_float(sr[j + 6]), __uint_as_float(sr[j + 7]));
+                for (int j = 0; j < 128; j += 8) {
+                    m4[0] = max3(m4[0], __uint_as_float(srow[j]), __uint_as_float(srow[j + 1]));
+                    m4[1] = max3(m4[1], __uint_as_float(srow[j + 2]), __uint_as_float(srow[j + 3]));
+                    m4[2] = max3(m4[2], __uint_as_float(srow[j + 4]), __uint_as_float(srow[j + 5]));
+                    m4[3] = max3(m4[3], __uint_as_float(srow[j + 6]), __uint_as_float(srow[j + 7]));
+                }
+            } else {
+#pragma unroll 1
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint32_t sr[64];
+                    TC_LD32(tS + 64 * h2, (sr + 0));
+                    TC_LD32(tS + 64 * h2 + 32, (sr + 32));
+                    tc_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 64; j += 8) {
+                        m4[0] = max3(m4[0], __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
+                        m4[1] = max3(m4[1], __uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3]));
+                        m4[2] = max3(m4[2], __uint_as_float(sr[j + 4]), __uint_as_float(sr[j + 5]));
+                        m4[3] = max3(m4[3], __uint_as_float(sr[j + 6]), __uint_as_float(sr[j + 7]));
+                    }
                 }
             }
             const float smax = fmaxf(max3(m4[0], m4[1], m4[2]), m4[3]);
@@ -933,14 +987,26 @@ attend_bf16_teams_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
                         const float alpha = need ? ex2(m_run - ub) : 1.f;
                         if (need) { l_run *= alpha; m_run = ub; }
                         tc_fence_after();
+if constexpr (kOnePass) {
 #pragma unroll 1
-                        for (int c = 0; c < D / 32; ++c) {
-                            uint32_t o[32];
-                            TC_LD32(tOt + 32 * c, o);
-                            tc_wait_ld();
+                            for (int c = 0; c < D / 16; ++c) {
+                                uint32_t o[16];
+                                TC_LD16(tOt + 16 * c, o);
+                                tc_wait_ld();
 #pragma unroll
-                            for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
-                            TC_ST32(tOt + 32 * c, o);
+                                for (int q = 0; q < 16; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+                                TC_ST16(tOt + 16 * c, o);
+                            }
+                        } else {
+#pragma unroll 1
+                            for (int c = 0; c < D / 32; ++c) {
+                                uint32_t o[32];
+                                TC_LD32(tOt + 32 * c, o);
+                                tc_wait_ld();
+#pragma unroll
+                                for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+                                TC_ST32(tOt + 32 * c, o);
+                            }
                         }
                         tc_wait_st();
                     }
@@ -951,38 +1017,60 @@ attend_bf16_teams_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
             // pairs of P are written over S columns already read.
             const uint64_t negm2 = pk2(-m_run, -m_run);
             uint64_t sumA = pk2(0.f, 0.f), sumB = pk2(0.f, 0.f);
-#pragma unroll 1
-            for (int h2 = 0; h2 < 2; ++h2) {
-                uint32_t sr[64];
-                TC_LD32(tS + 64 * h2, (sr + 0));
-                TC_LD32(tS + 64 * h2 + 32, (sr + 32));
-                tc_wait_ld();
-                uint32_t pk[32];
-                const float* bh = bb + 64 * h2;
+            if constexpr (kOnePass) {
+                uint32_t pk[64];
 #pragma unroll
-                for (int j = 0; j < 64; j += 4) {
-                    const float4 b4 = *reinterpret_cast<const float4*>(bh + j);
-                    const uint64_t x01 = fma2(pk2(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), c2,
+                for (int j = 0; j < 128; j += 4) {
+                    const float4 b4 = *reinterpret_cast<const float4*>(bb + j);
+                    const uint64_t x01 = fma2(pk2(__uint_as_float(srow[j]), __uint_as_float(srow[j + 1])), c2,
                                               add2(pk2(b4.x, b4.y), negm2));
-                    const uint64_t x23 = fma2(pk2(__uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3])), c2,
+                    const uint64_t x23 = fma2(pk2(__uint_as_float(srow[j + 2]), __uint_as_float(srow[j + 3])), c2,
                                               add2(pk2(b4.z, b4.w), negm2));
                     float a0, a1, a2, a3;
                     up2(x01, a0, a1);
                     up2(x23, a2, a3);
-                    const float p0 = ex2(a0), p1 = ex2(a1);
-                    float p2, p3;
-                    if (kPoly && (j / 4) % 3 != 2) {
-                        exp2_poly2(a2, a3, p2, p3);
-                    } else {
-                        p2 = ex2(a2);
-                        p3 = ex2(a3);
-                    }
+                    const float p0 = ex2(a0), p1 = ex2(a1), p2 = ex2(a2), p3 = ex2(a3);
                     sumA = add2(sumA, pk2(p0, p1));
                     sumB = add2(sumB, pk2(p2, p3));
                     pk[j / 2] = cvt_bf16x2(p0, p1);
                     pk[j / 2 + 1] = cvt_bf16x2(p2, p3);
                 }
-                TC_ST32(tS + 32 * h2, pk);
+                TC_ST32(tS, pk);
+                TC_ST32(tS + 32, (pk + 32));
+            } else {
+    #pragma unroll 1
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint32_t sr[64];
+                    TC_LD32(tS + 64 * h2, (sr + 0));
+                    TC_LD32(tS + 64 * h2 + 32, (sr + 32));
+                    tc_wait_ld();
+                    uint32_t pk[32];
+                    const float* bh = bb + 64 * h2;
+    #pragma unroll
+                    for (int j = 0; j < 64; j += 4) {
+                        const float4 b4 = *reinterpret_cast<const float4*>(bh + j);
+                        const uint64_t x01 = fma2(pk2(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), c2,
+                                                  add2(pk2(b4.x, b4.y), negm2));
+                        const uint64_t x23 = fma2(pk2(__uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3])), c2,
+                                                  add2(pk2(b4.z, b4.w), negm2));
+                        float a0, a1, a2, a3;
+                        up2(x01, a0, a1);
+                        up2(x23, a2, a3);
+                        const float p0 = ex2(a0), p1 = ex2(a1);
+                        float p2, p3;
+                        if (kPoly && (j / 4) % 3 != 2) {
+                            exp2_poly2(a2, a3, p2, p3);
+                        } else {
+                            p2 = ex2(a2);
+                            p3 = ex2(a3);
+                        }
+                        sumA = add2(sumA, pk2(p0, p1));
+                        sumB = add2(sumB, pk2(p2, p3));
+                        pk[j / 2] = cvt_bf16x2(p0, p1);
+                        pk[j / 2 + 1] = cvt_bf16x2(p2, p3);
+                    }
+                    TC_ST32(tS + 32 * h2, pk);
+                }
             }
             float s0, s1, s2, s3;
             up2(sumA, s0, s1);
@@ -1050,30 +1138,1110 @@ attend_bf16_teams_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_c
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+
+// Shared-memory layout of the split kernel: Q tile, K and V rings, then per team t
+// and bias buffer b: log2 n of the tile's keys [t][b][128] and quarter maxima
+// [t][b][4]; the halves' reference maxima [t][g][128]; the epilogue exchange
+// [t][g][m, l][128]; mbarriers.
+template <int D>
+struct CfgS {
+    using C = Cfg<D>;
+    static constexpr int TILE = C::TILE;
+    static constexpr int BOX = C::BOX;
+    static constexpr int NB = C::NB;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = TILE;
+    static constexpr int OFF_V = (1 + kKSt) * TILE;
+    static constexpr int OFF_BIAS = (1 + kKSt + kVSt) * TILE;   // 2 x 2 x 128 floats
+    static constexpr int OFF_BMAX = OFF_BIAS + 2 * 2 * 128 * 4;  // 2 x 2 x 4 floats
+    static constexpr int OFF_UB = OFF_BMAX + 2 * 2 * 4 * 4;      // 2 x 2 x 128 floats
+    static constexpr int OFF_XCH = OFF_UB + 2 * 2 * 128 * 4;     // 2 x 2 x 2 x 128 floats
+    static constexpr int OFF_BAR = OFF_XCH + 2 * 2 * 2 * 128 * 4;
+    static constexpr int OFF_MISC = OFF_BAR + C::NBAR * 8;
+    static constexpr int SMEM = OFF_MISC + 32 + 1024;
+    static_assert(SMEM <= 232448, "shared memory per block");
+};
+
+// Split-row teams. Two softmax teams take alternate key tiles (team t: tiles t, t+2,
+// ...) with their own score buffer S_t = TMEM [128 t, 128 t + 128) and output
+// accumulator O_t = [256 + 128 t, ...). Each team has eight warps: thread (t, g, r)
+// owns columns [64 g, 64 g + 64) of query row r, so every SM sub-partition runs four
+// softmax warps. The halves agree on a reference max per tile through shared memory
+// at one team barrier, keep partial row sums, and each writes its 64 probabilities
+// (bf16) over its own first 32 S columns; the PV product reads the A operand for keys
+// [64 g, 64 g + 64) from columns [128 t + 64 g, ... + 32). The epilogue merges the
+// teams' partial results: O = (O_A 2^(m_A - m) + O_B 2^(m_B - m)) / (l_A 2^.. + l_B 2^..).
+// Warps 16, 17, 18: K producer (and TMEM allocator), MMA issuer, V producer.
+template <int D>
+__global__ void __launch_bounds__(kThreadsSplit, 1)
+attend_bf16_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
+                         const __grid_constant__ CUtensorMap tmVc, const __grid_constant__ CUtensorMap tmKs,
+                         const __grid_constant__ CUtensorMap tmVs, const int32_t* __restrict__ Mdev,
+                         const float* __restrict__ bias2, int64_t capP,
+                         const float* __restrict__ sbias, int64_t Ts, int64_t Tq, int H,
+                         __nv_bfloat16* __restrict__ out, float scale_log2, Stats* stats) {
+    using C = Cfg<D>;
+    using L = CfgS<D>;
+    constexpr int kWK = 16, kWM = 17, kWV = 18;   // control warps
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+    float* sBias = reinterpret_cast<float*>(smem + L::OFF_BIAS);   // [t][b][128]
+    float* sBmax = reinterpret_cast<float*>(smem + L::OFF_BMAX);   // [t][b][4]
+    float* sUb = reinterpret_cast<float*>(smem + L::OFF_UB);       // [t][g][128]
+    float* sXch = reinterpret_cast<float*>(smem + L::OFF_XCH);     // [t][g][m,l][128]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.y;
+    const int q0 = blockIdx.x * kBM;
+    const int Mh = Mdev[h];
+    const int nc = (Mh + kBN - 1) / kBN;
+    const int ntiles = nc + (int)((Ts + kBN - 1) / kBN);
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars[B_QFULL], 1);
+        for (int s2 = 0; s2 < 4; ++s2) {
+            mbar_init(&bars[B_KFULL + s2], 1);
+            mbar_init(&bars[B_KEMPTY + s2], 1);
+            mbar_init(&bars[B_VFULL + s2], 1);
+            mbar_init(&bars[B_VEMPTY + s2], 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&bars[B_SFULL + t], 1);
+            mbar_init(&bars[B_PFULL + t], 256);
+            mbar_init(&bars[B_ODONE + t], 1);
+        }
+        mbar_init(&bars[B_DRAIN], 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == kWK) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(C::TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tO = tmem + 256;
+    uint8_t* sQ = smem + L::OFF_Q;
+    uint8_t* sK = smem + L::OFF_K;
+    uint8_t* sV = smem + L::OFF_V;
+
+    const bool is_kprod = (warp == kWK && lane == 0);
+    const bool is_vprod = (warp == kWV && lane == 0);
+    if (is_kprod || is_vprod) {
+        // ---------------------------------------------------------------- TMA producers
+        const bool kside = is_kprod;
+        const int nst = kside ? kKSt : kVSt;
+        uint8_t* ring = kside ? sK : sV;
+        uint64_t* full = &bars[kside ? B_KFULL : B_VFULL];
+        uint64_t* empty = &bars[kside ? B_KEMPTY : B_VEMPTY];
+        const CUtensorMap* mc = kside ? &tmKc : &tmVc;
+        const CUtensorMap* ms = kside ? &tmKs : &tmVs;
+        if (kside) {
+            mbar_expect_tx(&bars[B_QFULL], C::TILE);
+            for (int b = 0; b < C::NB; ++b) tma_load_3d(sQ + b * C::BOX, &tmQ, 64 * b, h, q0, &bars[B_QFULL]);
+        }
+        int last = -1;
+        for (int i = 0; i < ntiles && !*abort_flag; ++i) {
+            const int st = i % nst;
+            if (i >= nst && !mbar_wait(&empty[st], ((i / nst) - 1) & 1)) { *abort_flag = 1; break; }
+            const bool cache = i < nc;
+            const int row0 = (cache ? i : i - nc) * kBN;
+            mbar_expect_tx(&full[st], C::TILE);
+            for (int b = 0; b < C::NB; ++b)
+                tma_load_3d(ring + st * C::TILE + b * C::BOX, cache ? mc : ms, 64 * b, row0, h, &full[st]);
+            last = i;
+        }
+        if (kside) mbar_wait(&bars[B_QFULL], 0);
+        for (int i = (last >= nst - 1 ? last - nst + 1 : 0); i <= last; ++i) mbar_wait(&full[i % nst], (i / nst) & 1);
+    } else if (warp >= 16) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (warp == kWM && lane == 0) {
+            const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK), aV = smem_u32(sV);
+            bool ok = mbar_wait(&bars[B_QFULL], 0);
+            // S_t = Q K_j^T for tile j of team t = j & 1; S_t held P_{j-2}, so
+            // O_t += P_{j-2} V_{j-2} must have retired first.
+            auto issue_qk = [&](int j) -> bool {
+                const int t = j & 1, st = j % kKSt;
+                if (j >= 2 && !mbar_wait(&bars[B_ODONE + t], ((j - 2) >> 1) & 1)) return false;
+                if (!mbar_wait(&bars[B_KFULL + st], (j / kKSt) & 1)) return false;
+                tc_fence_after();
+                const uint32_t aKs = aK + st * C::TILE;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                    mma_ss(tmem + t * 128, sdesc(aQ + off, 16, 1024), sdesc(aKs + off, 16, 1024), C::IDESC_QK,
+                           kk > 0);
+                }
+                tc_commit(&bars[B_SFULL + t]);
+                tc_commit(&bars[B_KEMPTY + st]);
+                return true;
+            };
+            // O_t += P_t V_i; keys [16 kk, 16 kk + 16) of P sit at TMEM column
+            // 128 t + 64 (kk / 4) + 8 (kk % 4) (each half's P over its own S columns).
+            auto issue_pv = [&](int i) -> bool {
+                const int t = i & 1, st = i % kVSt;
+                if (!mbar_wait(&bars[B_VFULL + st], (i / kVSt) & 1)) return false;
+                tc_fence_after();
+                const uint32_t aVs = aV + st * C::TILE;
+#pragma unroll
+                for (int kk = 0; kk < kBN / 16; ++kk)
+                    mma_ts(tO + t * 128, tmem + t * 128 + 64 * (kk >> 2) + 8 * (kk & 3),
+                           sdesc(aVs + kk * 2048, C::BOX, 1024), C::IDESC_PV, (i >= 2 || kk > 0));
+                tc_commit(&bars[B_VEMPTY + st]);
+                tc_commit(&bars[B_ODONE + t]);
+                return true;
+            };
+            int pv = 0, qk = 0;
+            while (ok && qk < ntiles && qk < 2) ok = issue_qk(qk++);
+            while (ok && pv < ntiles && !*abort_flag) {
+                if (!mbar_wait(&bars[B_PFULL + (pv & 1)], (pv >> 1) & 1) || !issue_pv(pv)) { ok = false; break; }
+                ++pv;
+                if (pv < ntiles && mbar_try(&bars[B_PFULL + (pv & 1)], (pv >> 1) & 1)) {
+                    if (!issue_pv(pv)) { ok = false; break; }
+                    ++pv;
+                }
+                while (ok && qk < ntiles && qk <= pv + 1) ok = issue_qk(qk++);
+            }
+            if (!ok) *abort_flag = 1;
+            tc_commit(&bars[B_DRAIN]);
+            mbar_wait(&bars[B_DRAIN], 0);
+        }
+    } else {
+        // ---------------------------------------------------------------- softmax (warps 0-15)
+        const int t = warp >> 3;             // team: key tiles i = t, t + 2, ...
+        const int g = (warp >> 2) & 1;       // half: key columns [64 g, 64 g + 64) of each tile
+        const int wt = warp & 3;             // TMEM lane quarter (= SM sub-partition)
+        const int r = wt * 32 + lane;        // query row within the tile = TMEM lane
+        const uint32_t lane_base = (uint32_t)(wt * 32) << 16;
+        const uint32_t tS = tmem + t * 128 + 64 * g + lane_base;   // my S columns, then my P
+        const uint32_t tOg = tO + t * 128 + (D / 2) * g + lane_base;  // my O columns
+        const float* bias_h = bias2 + (int64_t)h * capP;
+        auto bias_of = [&](int i) -> float {
+            return (i < nc) ? bias_h[(int64_t)i * kBN + r] : sbias[(int64_t)(i - nc) * kBN + r];
+        };
+        // Half 0 stages each tile's log2 n row (one value per thread) and its quarter maxima.
+        auto stage_bias = [&](int b, float v) {
+            sBias[(t * 2 + b) * 128 + r] = v;
+            float wm = v;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, o));
+            if (lane == 0) sBmax[(t * 2 + b) * 4 + wt] = wm;
+        };
+        const uint64_t c2 = pk2(scale_log2, scale_log2);
+        float m_run = -INFINITY, l_run = 0.f;
+        float bnext = 0.f;
+        if (g == 0) {
+            if (t < ntiles) stage_bias(0, bias_of(t));
+            if (t + 2 < ntiles) bnext = bias_of(t + 2);
+        }
+        bool ok = bar_and(1 + t, 256, true);
+        for (int i = t; i < ntiles; i += 2) {
+            const int k = i >> 1;  // the team's k-th tile
+            const int b = k & 1;
+            // (warp-uniform: the TMEM loads below are warp-collective)
+            const bool got = __all_sync(0xffffffffu, !*abort_flag && mbar_wait(&bars[B_SFULL + t], k & 1));
+            tc_fence_after();
+            // Row max over my 64 raw scores, and the reference for this half.
+            float smax = -INFINITY;
+            if (got) {
+                uint32_t sr[64];
+                TC_LD32(tS, (sr + 0));
+                TC_LD32(tS + 32, (sr + 32));
+                tc_wait_ld();
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int j = 0; j < 64; j += 8) {
+                    m4[0] = max3(m4[0], __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
+                    m4[1] = max3(m4[1], __uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3]));
+                    m4[2] = max3(m4[2], __uint_as_float(sr[j + 4]), __uint_as_float(sr[j + 5]));
+                    m4[3] = max3(m4[3], __uint_as_float(sr[j + 6]), __uint_as_float(sr[j + 7]));
+                }
+                smax = fmaxf(max3(m4[0], m4[1], m4[2]), m4[3]);
+            }
+            const float2 bm = *reinterpret_cast<const float2*>(sBmax + (t * 2 + b) * 4 + 2 * g);
+            sUb[(t * 2 + g) * 128 + r] = fmaf(smax, scale_log2, fmaxf(bm.x, bm.y));
+            // Stage the log2 n row of the team's next tile into the other buffer. Its
+            // previous contents were last read in the team's previous tile, which every
+            // thread finished before S could be refilled.
+            if (g == 0 && i + 2 < ntiles) stage_bias(b ^ 1, bnext);
+            if (!bar_and(1 + t, 256, got)) { ok = false; break; }
+            if (g == 0 && i + 4 < ntiles) bnext = bias_of(i + 4);
+            // Reference max: an upper bound of the row max of this tile, (max raw score)
+            // * scale + (max log2 n), agreed by both halves. p = 2^(x - m) <= 2^8 below.
+            const float ub = fmaxf(sUb[(t * 2 + 0) * 128 + r], sUb[(t * 2 + 1) * 128 + r]);
+            if (k == 0) {
+                m_run = ub;
+            } else {
+                // Lazy rescaling: O_t and l keep the old reference until it would grow by
+                // more than 8 (a factor 256); then both halves scale their parts by alpha.
+                const bool need = ub > m_run + 8.f;
+                if (__any_sync(0xffffffffu, need)) {
+                    const bool w = mbar_wait(&bars[B_ODONE + t], (k - 1) & 1);
+                    if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; }
+                    if (ok) {
+                        const float alpha = need ? ex2(m_run - ub) : 1.f;
+                        if (need) { l_run *= alpha; m_run = ub; }
+                        tc_fence_after();
+#pragma unroll 1
+                        for (int c = 0; c < D / 64; ++c) {
+                            uint32_t o[32];
+                            TC_LD32(tOg + 32 * c, o);
+                            tc_wait_ld();
+#pragma unroll
+                            for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+                            TC_ST32(tOg + 32 * c, o);
+                        }
+                        tc_wait_st();
+                    }
+                }
+            }
+            // p = 2^(s * scale + log2 n - m) over my 64 columns in two chunks of 32,
+            // packed fp32x2 FMA/ADD and MUFU ex2; 16 bf16 pairs per chunk go over S
+            // columns already read.
+            const uint64_t negm2 = pk2(-m_run, -m_run);
+            uint64_t sumA = pk2(0.f, 0.f), sumB = pk2(0.f, 0.f);
+            const float* bh = sBias + (t * 2 + b) * 128 + 64 * g;
+#pragma unroll 1
+            for (int h2 = 0; h2 < 2; ++h2) {
+                uint32_t sr[32];
+                TC_LD32(tS + 32 * h2, sr);
+                tc_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    const float4 b4 = *reinterpret_cast<const float4*>(bh + 32 * h2 + j);
+                    const uint64_t x01 = fma2(pk2(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), c2,
+                                              add2(pk2(b4.x, b4.y), negm2));
+                    const uint64_t x23 = fma2(pk2(__uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3])), c2,
+                                              add2(pk2(b4.z, b4.w), negm2));
+                    float a0, a1, a2, a3;
+                    up2(x01, a0, a1);
+                    up2(x23, a2, a3);
+                    const float p0 = ex2(a0), p1 = ex2(a1), p2 = ex2(a2), p3 = ex2(a3);
+                    sumA = add2(sumA, pk2(p0, p1));
+                    sumB = add2(sumB, pk2(p2, p3));
+                    pk[j / 2] = cvt_bf16x2(p0, p1);
+                    pk[j / 2 + 1] = cvt_bf16x2(p2, p3);
+                }
+                TC_ST16(tS + 16 * h2, pk);
+            }
+            float s0, s1, s2, s3;
+            up2(sumA, s0, s1);
+            up2(sumB, s2, s3);
+            l_run += (s0 + s1) + (s2 + s3);
+            tc_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars[B_PFULL + t]);
+        }
+        // Epilogue: both teams' last products retire; thread (t, g) writes output
+        // columns [D/4 (2t + g), D/4 (2t + g + 1)) of its row.
+        const int lastt = ntiles - 1 - ((ntiles - 1 - t) & 1);   // this team's last tile (or < 0)
+        const bool fin = ok && (lastt < 0 || mbar_wait(&bars[B_ODONE + t], (lastt >> 1) & 1));
+        sXch[((t * 2 + g) * 2 + 0) * 128 + r] = m_run;
+        sXch[((t * 2 + g) * 2 + 1) * 128 + r] = l_run;
+        if (bar_and(3, 512, fin)) {
+            const float mA = sXch[(0 * 2 + 0) * 128 + r];
+            const float lA = sXch[(0 * 2 + 1) * 128 + r] + sXch[(2 * 1 + 1) * 128 + r];
+            const float mB = sXch[(4 + 0) * 128 + r];
+            const float lB = sXch[(4 + 1) * 128 + r] + sXch[(6 + 1) * 128 + r];
+            const float m = fmaxf(mA, mB);
+            const float fA = (lA > 0.f) ? ex2(mA - m) : 0.f;   // a team with no tiles contributes 0
+            const float fB = (lB > 0.f) ? ex2(mB - m) : 0.f;
+            const float inv = 1.f / (lA * fA + lB * fB);
+            const float wA = fA * inv, wB = fB * inv;
+            const bool haveB = ntiles > 1;
+            tc_fence_after();
+            const int64_t row = q0 + r;
+            constexpr int QC = D / 4;   // output columns per thread
+            const int col = QC * (2 * t + g);
+            uint32_t oa[QC], ob[QC];
+            if constexpr (QC == 32) {
+                TC_LD32(tO + lane_base + col, oa);
+                if (haveB) TC_LD32(tO + 128 + lane_base + col, ob);
+            } else {
+                TC_LD16(tO + lane_base + col, oa);
+                if (haveB) TC_LD16(tO + 128 + lane_base + col, ob);
+            }
+            tc_wait_ld();
+            if (row < Tq) {
+                uint4* dst = reinterpret_cast<uint4*>(out + (row * H + h) * D + col);
+#pragma unroll
+                for (int v = 0; v < QC / 8; ++v) {
+                    float e[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        e[q] = __uint_as_float(oa[8 * v + q]) * wA + (haveB ? __uint_as_float(ob[8 * v + q]) * wB : 0.f);
+                    uint4 w4;
+                    w4.x = cvt_bf16x2(e[0], e[1]);
+                    w4.y = cvt_bf16x2(e[2], e[3]);
+                    w4.z = cvt_bf16x2(e[4], e[5]);
+                    w4.w = cvt_bf16x2(e[6], e[7]);
+                    dst[v] = w4;
+                }
+            }
+        } else {
+            *abort_flag = 1;
+        }
+    }
+    if (threadIdx.x == 0 && *abort_flag) atomicOr(&stats->error_bits, 2u);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWK) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS)
+                     : "memory");
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+
+// ---------------------------------------------------------------------------- ring kernel
+// Shared-memory layout: Q tile, K ring (3 stages), V ring (2 stages); log2 n of the
+// keys of three tiles [3][128] and their quarter maxima [3][4]; the quarters' reference
+// maxima [2][4][128]; the epilogue row sums [4][128]; mbarriers.
+constexpr int kRK = 3, kRV = 2;
+enum { R_QFULL = 0, R_KFULL = 1, R_KEMPTY = 4, R_VFULL = 7, R_VEMPTY = 9, R_SFULL = 11, R_PFULL = 14,
+       R_ODONE = 17, R_DRAIN = 20, R_NBAR = 22 };
+template <int D>
+struct CfgR {
+    using C = Cfg<D>;
+    static constexpr int TILE = C::TILE;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = TILE;
+    static constexpr int OFF_V = (1 + kRK) * TILE;
+    static constexpr int OFF_BIAS = (1 + kRK + kRV) * TILE;   // 3 x 128 floats
+    static constexpr int OFF_BMAX = OFF_BIAS + 3 * 128 * 4;    // 3 x 4 floats
+    static constexpr int OFF_UB = OFF_BMAX + 3 * 4 * 4;        // 2 x 4 x 128 floats
+    static constexpr int OFF_L = OFF_UB + 2 * 4 * 128 * 4;     // 4 x 128 floats
+    static constexpr int OFF_BAR = OFF_L + 4 * 128 * 4;
+    static constexpr int OFF_MISC = OFF_BAR + R_NBAR * 8;
+    static constexpr int SMEM = OFF_MISC + 32 + 1024;
+    static_assert(SMEM <= 232448, "shared memory per block");
+    static constexpr uint32_t O_COL = 384;   // S_b = [128 b, 128 b + 128), b < 3; O = [384, 384 + D)
+};
+
+// One CTA = 128 query rows of one head; the key tiles are processed in order.
+//   TMEM: three score buffers S_b (tile i uses b = i mod 3) and one output
+//         accumulator O; P (bf16) overwrites the S columns its quarter has read.
+//   warps 0-15  softmax: thread (q, r) owns columns [32 q, 32 q + 32) of query row r
+//               (TMEM lane r), four softmax warps per SM sub-partition. Per tile: S
+//               into registers once, a reference max agreed by the four quarters at
+//               one barrier (upper bound: max raw score * scale + max log2 n), lazy
+//               rescaling of O and the row sums (only when the reference grows by more
+//               than 2^8), p = 2^(x - m) with packed fp32x2 math and MUFU ex2, P written
+//               as bf16 over its own first 16 S columns.
+//   warp 16     TMEM allocator; lane 0 TMA producer for Q and the K ring.
+//   warp 17     lane 0 issues S_b = Q K_i^T once K_i has landed and PV of tile i - 3
+//               (the last reader of S_b) has retired: up to three tiles ahead.
+//   warp 18     lane 0 TMA producer for the V ring.
+//   warp 19     lane 0 issues O += P_i V_i once P_i is written.
+// Two issuing threads keep the tensor pipe fed while either waits on a barrier;
+// each commit tracks the products its own thread issued.
+template <int D>
+__global__ void __launch_bounds__(kThreadsRing, 1)
+attend_bf16_ring_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
+                        const __grid_constant__ CUtensorMap tmVc, const __grid_constant__ CUtensorMap tmKs,
+                        const __grid_constant__ CUtensorMap tmVs, const int32_t* __restrict__ Mdev,
+                        const float* __restrict__ bias2, int64_t capP,
+                        const float* __restrict__ sbias, int64_t Ts, int64_t Tq, int H,
+                        __nv_bfloat16* __restrict__ out, float scale_log2, Stats* stats) {
+    using C = Cfg<D>;
+    using L = CfgR<D>;
+    constexpr int kWK = 16, kWQK = 17, kWV = 18, kWPV = 19;
+    constexpr int QC = D / 4;   // output (and rescale) columns per softmax thread
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+    float* sBias = reinterpret_cast<float*>(smem + L::OFF_BIAS);   // [3][128]
+    float* sBmax = reinterpret_cast<float*>(smem + L::OFF_BMAX);   // [3][4]
+    float* sUb = reinterpret_cast<float*>(smem + L::OFF_UB);       // [2][4][128]
+    float* sL = reinterpret_cast<float*>(smem + L::OFF_L);         // [4][128]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.y;
+    const int q0 = blockIdx.x * kBM;
+    const int Mh = Mdev[h];
+    const int nc = (Mh + kBN - 1) / kBN;
+    const int ntiles = nc + (int)((Ts + kBN - 1) / kBN);
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars[R_QFULL], 1);
+        for (int s2 = 0; s2 < kRK; ++s2) {
+            mbar_init(&bars[R_KFULL + s2], 1);
+            mbar_init(&bars[R_KEMPTY + s2], 1);
+        }
+        for (int s2 = 0; s2 < kRV; ++s2) {
+            mbar_init(&bars[R_VFULL + s2], 1);
+            mbar_init(&bars[R_VEMPTY + s2], 1);
+        }
+        for (int b = 0; b < 3; ++b) {
+            mbar_init(&bars[R_SFULL + b], 1);
+            mbar_init(&bars[R_PFULL + b], 512);
+            mbar_init(&bars[R_ODONE + b], 1);
+        }
+        mbar_init(&bars[R_DRAIN], 1);
+        mbar_init(&bars[R_DRAIN + 1], 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == kWK) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(C::TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tO = tmem + L::O_COL;
+    uint8_t* sQ = smem + L::OFF_Q;
+    uint8_t* sK = smem + L::OFF_K;
+    uint8_t* sV = smem + L::OFF_V;
+
+    if ((warp == kWK || warp == kWV) && lane == 0) {
+        // ---------------------------------------------------------------- TMA producers
+        const bool kside = warp == kWK;
+        const int nst = kside ? kRK : kRV;
+        uint8_t* ring = kside ? sK : sV;
+        uint64_t* full = &bars[kside ? R_KFULL : R_VFULL];
+        uint64_t* empty = &bars[kside ? R_KEMPTY : R_VEMPTY];
+        const CUtensorMap* mc = kside ? &tmKc : &tmVc;
+        const CUtensorMap* ms = kside ? &tmKs : &tmVs;
+        if (kside) {
+            mbar_expect_tx(&bars[R_QFULL], C::TILE);
+            for (int b = 0; b < C::NB; ++b) tma_load_3d(sQ + b * C::BOX, &tmQ, 64 * b, h, q0, &bars[R_QFULL]);
+        }
+        int last = -1;
+        for (int i = 0; i < ntiles && !*abort_flag; ++i) {
+            const int st = i % nst;
+            if (i >= nst && !mbar_wait(&empty[st], ((i / nst) - 1) & 1)) { *abort_flag = 1; break; }
+            const bool cache = i < nc;
+            const int row0 = (cache ? i : i - nc) * kBN;
+            mbar_expect_tx(&full[st], C::TILE);
+            for (int b = 0; b < C::NB; ++b)
+                tma_load_3d(ring + st * C::TILE + b * C::BOX, cache ? mc : ms, 64 * b, row0, h, &full[st]);
+            last = i;
+        }
+        if (kside) mbar_wait(&bars[R_QFULL], 0);
+        for (int i = (last >= nst - 1 ? last - nst + 1 : 0); i <= last; ++i) mbar_wait(&full[i % nst], (i / nst) & 1);
+    } else if (warp == kWQK && lane == 0) {
+        // ---------------------------------------------------------------- QK issuer
+        const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK);
+        bool ok = mbar_wait(&bars[R_QFULL], 0);
+        for (int j = 0; ok && j < ntiles && !*abort_flag; ++j) {
+            const int b = j % 3, st = j % kRK;
+            if (j >= 3 && !mbar_wait(&bars[R_ODONE + b], ((j - 3) / 3) & 1)) { ok = false; break; }
+            if (!mbar_wait(&bars[R_KFULL + st], (j / kRK) & 1)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t aKs = aK + st * C::TILE;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                mma_ss(tmem + b * 128, sdesc(aQ + off, 16, 1024), sdesc(aKs + off, 16, 1024), C::IDESC_QK, kk > 0);
+            }
+            tc_commit(&bars[R_SFULL + b]);
+            tc_commit(&bars[R_KEMPTY + st]);
+        }
+        if (!ok) *abort_flag = 1;
+        tc_commit(&bars[R_DRAIN]);
+        mbar_wait(&bars[R_DRAIN], 0);
+    } else if (warp == kWPV && lane == 0) {
+        // ---------------------------------------------------------------- PV issuer
+        // O += P_i V_i; keys [16 kk, 16 kk + 16) of P sit at column 128 b + 32 (kk / 2) +
+        // 8 (kk % 2): each quarter's probabilities over its own first S columns.
+        const uint32_t aV = smem_u32(sV);
+        bool ok = true;
+        for (int i = 0; i < ntiles && !*abort_flag; ++i) {
+            const int b = i % 3, st = i % kRV;
+            if (!mbar_wait(&bars[R_PFULL + b], (i / 3) & 1)) { ok = false; break; }
+            if (!mbar_wait(&bars[R_VFULL + st], (i / kRV) & 1)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t aVs = aV + st * C::TILE;
+#pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk)
+                mma_ts(tO, tmem + b * 128 + 32 * (kk >> 1) + 8 * (kk & 1), sdesc(aVs + kk * 2048, C::BOX, 1024),
+                       C::IDESC_PV, (i > 0 || kk > 0));
+            tc_commit(&bars[R_VEMPTY + st]);
+            tc_commit(&bars[R_ODONE + b]);
+        }
+        if (!ok) *abort_flag = 1;
+        tc_commit(&bars[R_DRAIN + 1]);
+        mbar_wait(&bars[R_DRAIN + 1], 0);
+    } else if (warp < 16) {
+        // ---------------------------------------------------------------- softmax (warps 0-15)
+        const int q = warp >> 2;             // column quarter
+        const int wt = warp & 3;             // TMEM lane quarter (= SM sub-partition)
+        const int r = wt * 32 + lane;        // query row within the tile = TMEM lane
+        const uint32_t lane_base = (uint32_t)(wt * 32) << 16;
+        const uint32_t tOq = tO + QC * q + lane_base;
+        const float* bias_h = bias2 + (int64_t)h * capP;
+        auto bias_of = [&](int i) -> float {
+            return (i < nc) ? bias_h[(int64_t)i * kBN + r] : sbias[(int64_t)(i - nc) * kBN + r];
+        };
+        // Quarter 0 stages each tile's log2 n row (one value per thread) and its quarter maxima.
+        auto stage_bias = [&](int b, float v) {
+            sBias[b * 128 + r] = v;
+            float wm = v;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, o));
+            if (lane == 0) sBmax[b * 4 + wt] = wm;
+        };
+        const uint64_t c2 = pk2(scale_log2, scale_log2);
+        float m_run = -INFINITY, l_run = 0.f;
+        float bnext = 0.f;
+        if (q == 0) {
+            stage_bias(0, bias_of(0));
+            if (1 < ntiles) bnext = bias_of(1);
+        }
+        bool ok = bar_and(1, 512, true);
+        for (int i = 0; i < ntiles; ++i) {
+            const int b = i % 3, u = i & 1;
+            // (warp-uniform: the TMEM loads below are warp-collective)
+            const bool got = __all_sync(0xffffffffu, !*abort_flag && mbar_wait(&bars[R_SFULL + b], (i / 3) & 1));
+            tc_fence_after();
+            const uint32_t tS = tmem + b * 128 + 32 * q + lane_base;
+            uint32_t sr[32];
+            float smax = -INFINITY;
+            if (got) {
+                TC_LD32(tS, sr);
+                tc_wait_ld();
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int j = 0; j < 32; j += 8) {
+                    m4[0] = max3(m4[0], __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
+                    m4[1] = max3(m4[1], __uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3]));
+                    m4[2] = max3(m4[2], __uint_as_float(sr[j + 4]), __uint_as_float(sr[j + 5]));
+                    m4[3] = max3(m4[3], __uint_as_float(sr[j + 6]), __uint_as_float(sr[j + 7]));
+                }
+                smax = fmaxf(max3(m4[0], m4[1], m4[2]), m4[3]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) sr[j] = 0u;
+            }
+            sUb[(u * 4 + q) * 128 + r] = fmaf(smax, scale_log2, sBmax[b * 4 + q]);
+            // Stage the next tile's log2 n row. Its buffer was last read two tiles ago,
+            // before the previous barrier.
+            if (q == 0 && i + 1 < ntiles) stage_bias((i + 1) % 3, bnext);
+            if (!bar_and(1, 512, got)) { ok = false; break; }
+            if (q == 0 && i + 2 < ntiles) bnext = bias_of(i + 2);
+            // Reference max: an upper bound of the row max of this tile, agreed by the
+            // four quarters. p = 2^(x - m) <= 2^8 below.
+            const float ub = fmaxf(fmaxf(sUb[(u * 4 + 0) * 128 + r], sUb[(u * 4 + 1) * 128 + r]),
+                                   fmaxf(sUb[(u * 4 + 2) * 128 + r], sUb[(u * 4 + 3) * 128 + r]));
+            if (i == 0) {
+                m_run = ub;
+            } else {
+                // Lazy rescaling: O and l keep the old reference until it would grow by more
+                // than 8 (a factor 256); then, once PV of the previous tile has retired,
+                // each quarter scales its O columns and its partial row sum by alpha.
+                const bool need = ub > m_run + 8.f;
+                if (__any_sync(0xffffffffu, need)) {
+                    const bool w = mbar_wait(&bars[R_ODONE + (i - 1) % 3], ((i - 1) / 3) & 1);
+                    if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; }
+                    if (ok) {
+                        const float alpha = need ? ex2(m_run - ub) : 1.f;
+                        if (need) { l_run *= alpha; m_run = ub; }
+                        tc_fence_after();
+                        uint32_t o[QC];
+                        if constexpr (QC == 32) TC_LD32(tOq, o);
+                        else TC_LD16(tOq, o);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < QC; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                        if constexpr (QC == 32) TC_ST32(tOq, o);
+                        else TC_ST16(tOq, o);
+                        tc_wait_st();
+                    }
+                }
+            }
+            // p = 2^(s * scale + log2 n - m) over my 32 columns: packed fp32x2 FMA/ADD and
+            // MUFU ex2; 16 bf16 pairs go over the first 16 of my S columns.
+            const uint64_t negm2 = pk2(-m_run, -m_run);
+            uint64_t sumA = pk2(0.f, 0.f), sumB = pk2(0.f, 0.f);
+            const float* bh = sBias + b * 128 + 32 * q;
+            uint32_t pk[16];
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                const float4 b4 = *reinterpret_cast<const float4*>(bh + j);
+                const uint64_t x01 = fma2(pk2(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), c2,
+                                          add2(pk2(b4.x, b4.y), negm2));
+                const uint64_t x23 = fma2(pk2(__uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3])), c2,
+                                          add2(pk2(b4.z, b4.w), negm2));
+                float a0, a1, a2, a3;
+                up2(x01, a0, a1);
+                up2(x23, a2, a3);
+                const float p0 = ex2(a0), p1 = ex2(a1), p2 = ex2(a2), p3 = ex2(a3);
+                sumA = add2(sumA, pk2(p0, p1));
+                sumB = add2(sumB, pk2(p2, p3));
+                pk[j / 2] = cvt_bf16x2(p0, p1);
+                pk[j / 2 + 1] = cvt_bf16x2(p2, p3);
+            }
+            TC_ST16(tS, pk);
+            float s0, s1, s2, s3;
+            up2(sumA, s0, s1);
+            up2(sumB, s2, s3);
+            l_run += (s0 + s1) + (s2 + s3);
+            tc_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars[R_PFULL + b]);
+        }
+        // Epilogue: the last product retires (products retire in order: each commit
+        // covers every earlier product of the issuing thread), the quarters add their
+        // row sums, and thread (q, r) writes output columns [QC q, QC q + QC).
+        const int lastt = ntiles - 1;
+        const bool fin = ok && mbar_wait(&bars[R_ODONE + lastt % 3], (lastt / 3) & 1);
+        sL[q * 128 + r] = l_run;
+        if (bar_and(1, 512, fin)) {
+            const float inv = 1.f / ((sL[0 * 128 + r] + sL[1 * 128 + r]) + (sL[2 * 128 + r] + sL[3 * 128 + r]));
+            tc_fence_after();
+            uint32_t o[QC];
+            if constexpr (QC == 32) TC_LD32(tOq, o);
+            else TC_LD16(tOq, o);
+            tc_wait_ld();
+            const int64_t row = q0 + r;
+            if (row < Tq) {
+                uint4* dst = reinterpret_cast<uint4*>(out + (row * H + h) * D + QC * q);
+#pragma unroll
+                for (int v = 0; v < QC / 8; ++v) {
+                    uint4 w4;
+                    w4.x = cvt_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
+                    w4.y = cvt_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
+                    w4.z = cvt_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
+                    w4.w = cvt_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
+                    dst[v] = w4;
+                }
+            }
+        } else {
+            *abort_flag = 1;
+        }
+    }
+    if (threadIdx.x == 0 && *abort_flag) atomicOr(&stats->error_bits, 2u);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWK) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS)
+                     : "memory");
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+
+// ---------------------------------------------------------------------------- duo kernel
+// Two softmax teams over a three-buffer score ring with one shared output accumulator.
+enum { U_QFULL = 0, U_KFULL = 1, U_KEMPTY = 4, U_VFULL = 7, U_VEMPTY = 9, U_SFULL = 11, U_PFULL = 14,
+       U_ODONE = 17, U_DRAIN = 20, U_MREADY = 22, U_NBAR = 24 };
+template <int D>
+struct CfgU {
+    using C = Cfg<D>;
+    static constexpr int TILE = C::TILE;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = TILE;
+    static constexpr int OFF_V = (1 + kRK) * TILE;
+    static constexpr int OFF_BIAS = (1 + kRK + kRV) * TILE;   // [team][3][128] log2 n
+    static constexpr int OFF_BMAX = OFF_BIAS + 2 * 3 * 128 * 4; // [team][3][4]
+    static constexpr int OFF_UB = OFF_BMAX + 2 * 3 * 4 * 4;     // [team][2][half][128]
+    static constexpr int OFF_MREF = OFF_UB + 2 * 2 * 2 * 128 * 4;  // [team][128]
+    static constexpr int OFF_L = OFF_MREF + 2 * 128 * 4;        // [4][128]
+    static constexpr int OFF_BAR = OFF_L + 4 * 128 * 4;
+    static constexpr int OFF_MISC = OFF_BAR + U_NBAR * 8;
+    static constexpr int SMEM = OFF_MISC + 32 + 1024;
+    static_assert(SMEM <= 232448, "shared memory per block");
+    static constexpr uint32_t O_COL = 384;
+};
+
+// One CTA = 128 query rows of one head.
+//   TMEM: score buffers S_b = [128 b, 128 b + 128) (tile i uses b = i mod 3) and one
+//         output accumulator O = [384, 384 + D).
+//   warps 0-15  softmax, two teams of eight warps: team t takes tiles t, t + 2, ...;
+//               thread (t, g, r) owns columns [64 g, 64 g + 64) of query row r (TMEM
+//               lane r), so every SM sub-partition runs two warps of each team and the
+//               teams' phases interleave. Per tile the halves agree on an upper bound of
+//               the row max (max raw score * scale + max log2 n) at a team barrier.
+//               The reference m is shared by both teams and changes lazily: tile i keeps
+//               the reference of tile i - 1 (published by the other team through shared
+//               memory and an mbarrier) unless its bound exceeds it by more than 8, and
+//               then O is rescaled once PV of tile i - 1 has retired. Row sums stay per
+//               thread, rescaled when the reference moves. P (bf16) goes over the first
+//               32 S columns of each half.
+//   warp 16     TMEM allocator; lane 0 TMA producer for Q and the K ring (3 stages).
+//   warp 17     lane 0 issues S_b = Q K_i^T once K_i has landed and PV of tile i - 3 has
+//               retired (up to three tiles ahead).
+//   warp 18     lane 0 TMA producer for the V ring (2 stages).
+//   warp 19     lane 0 issues O += P_i V_i in tile order.
+template <int D>
+__global__ void __launch_bounds__(kThreadsRing, 1)
+attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
+                       const __grid_constant__ CUtensorMap tmVc, const __grid_constant__ CUtensorMap tmKs,
+                       const __grid_constant__ CUtensorMap tmVs, const int32_t* __restrict__ Mdev,
+                       const float* __restrict__ bias2, int64_t capP,
+                       const float* __restrict__ sbias, int64_t Ts, int64_t Tq, int H,
+                       __nv_bfloat16* __restrict__ out, float scale_log2, Stats* stats) {
+    using C = Cfg<D>;
+    using L = CfgU<D>;
+    constexpr int kWK = 16, kWQK = 17, kWV = 18, kWPV = 19;
+    constexpr int QC = D / 4;   // output columns per softmax thread
+    constexpr int HC = D / 2;   // O columns a half rescales
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+    float* sBias = reinterpret_cast<float*>(smem + L::OFF_BIAS);
+    float* sBmax = reinterpret_cast<float*>(smem + L::OFF_BMAX);
+    float* sUb = reinterpret_cast<float*>(smem + L::OFF_UB);
+    float* sMref = reinterpret_cast<float*>(smem + L::OFF_MREF);
+    float* sL = reinterpret_cast<float*>(smem + L::OFF_L);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.y;
+    const int q0 = blockIdx.x * kBM;
+    const int Mh = Mdev[h];
+    const int nc = (Mh + kBN - 1) / kBN;
+    const int ntiles = nc + (int)((Ts + kBN - 1) / kBN);
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars[U_QFULL], 1);
+        for (int s2 = 0; s2 < kRK; ++s2) {
+            mbar_init(&bars[U_KFULL + s2], 1);
+            mbar_init(&bars[U_KEMPTY + s2], 1);
+        }
+        for (int s2 = 0; s2 < kRV; ++s2) {
+            mbar_init(&bars[U_VFULL + s2], 1);
+            mbar_init(&bars[U_VEMPTY + s2], 1);
+        }
+        for (int b = 0; b < 3; ++b) {
+            mbar_init(&bars[U_SFULL + b], 1);
+            mbar_init(&bars[U_PFULL + b], 256);
+            mbar_init(&bars[U_ODONE + b], 1);
+        }
+        mbar_init(&bars[U_DRAIN], 1);
+        mbar_init(&bars[U_DRAIN + 1], 1);
+        mbar_init(&bars[U_MREADY], 128);
+        mbar_init(&bars[U_MREADY + 1], 128);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == kWK) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(C::TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t tO = tmem + L::O_COL;
+    uint8_t* sQ = smem + L::OFF_Q;
+    uint8_t* sK = smem + L::OFF_K;
+    uint8_t* sV = smem + L::OFF_V;
+
+    if ((warp == kWK || warp == kWV) && lane == 0) {
+        // ---------------------------------------------------------------- TMA producers
+        const bool kside = warp == kWK;
+        const int nst = kside ? kRK : kRV;
+        uint8_t* ring = kside ? sK : sV;
+        uint64_t* full = &bars[kside ? U_KFULL : U_VFULL];
+        uint64_t* empty = &bars[kside ? U_KEMPTY : U_VEMPTY];
+        const CUtensorMap* mc = kside ? &tmKc : &tmVc;
+        const CUtensorMap* ms = kside ? &tmKs : &tmVs;
+        if (kside) {
+            mbar_expect_tx(&bars[U_QFULL], C::TILE);
+            for (int b = 0; b < C::NB; ++b) tma_load_3d(sQ + b * C::BOX, &tmQ, 64 * b, h, q0, &bars[U_QFULL]);
+        }
+        int last = -1;
+        for (int i = 0; i < ntiles && !*abort_flag; ++i) {
+            const int st = i % nst;
+            if (i >= nst && !mbar_wait(&empty[st], ((i / nst) - 1) & 1)) { *abort_flag = 1; break; }
+            const bool cache = i < nc;
+            const int row0 = (cache ? i : i - nc) * kBN;
+            mbar_expect_tx(&full[st], C::TILE);
+            for (int b = 0; b < C::NB; ++b)
+                tma_load_3d(ring + st * C::TILE + b * C::BOX, cache ? mc : ms, 64 * b, row0, h, &full[st]);
+            last = i;
+        }
+        if (kside) mbar_wait(&bars[U_QFULL], 0);
+        for (int i = (last >= nst - 1 ? last - nst + 1 : 0); i <= last; ++i) mbar_wait(&full[i % nst], (i / nst) & 1);
+    } else if (warp == kWQK && lane == 0) {
+        // ---------------------------------------------------------------- QK issuer
+        const uint32_t aQ = smem_u32(sQ), aK = smem_u32(sK);
+        bool ok = mbar_wait(&bars[U_QFULL], 0);
+        for (int j = 0; ok && j < ntiles && !*abort_flag; ++j) {
+            const int b = j % 3, st = j % kRK;
+            if (j >= 3 && !mbar_wait(&bars[U_ODONE + b], ((j - 3) / 3) & 1)) { ok = false; break; }
+            if (!mbar_wait(&bars[U_KFULL + st], (j / kRK) & 1)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t aKs = aK + st * C::TILE;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t off = (kk >> 2) * C::BOX + (kk & 3) * 32;
+                mma_ss(tmem + b * 128, sdesc(aQ + off, 16, 1024), sdesc(aKs + off, 16, 1024), C::IDESC_QK, kk > 0);
+            }
+            tc_commit(&bars[U_SFULL + b]);
+            tc_commit(&bars[U_KEMPTY + st]);
+        }
+        if (!ok) *abort_flag = 1;
+        tc_commit(&bars[U_DRAIN]);
+        mbar_wait(&bars[U_DRAIN], 0);
+    } else if (warp == kWPV && lane == 0) {
+        // ---------------------------------------------------------------- PV issuer
+        // O += P_i V_i; keys [16 kk, 16 kk + 16) of P sit at column 128 b + 64 (kk / 4) +
+        // 8 (kk % 4): each half's probabilities over its own first S columns.
+        const uint32_t aV = smem_u32(sV);
+        bool ok = true;
+        for (int i = 0; i < ntiles && !*abort_flag; ++i) {
+            const int b = i % 3, st = i % kRV;
+            if (!mbar_wait(&bars[U_PFULL + b], (i / 3) & 1)) { ok = false; break; }
+            if (!mbar_wait(&bars[U_VFULL + st], (i / kRV) & 1)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t aVs = aV + st * C::TILE;
+#pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk)
+                mma_ts(tO, tmem + b * 128 + 64 * (kk >> 2) + 8 * (kk & 3), sdesc(aVs + kk * 2048, C::BOX, 1024),
+                       C::IDESC_PV, (i > 0 || kk > 0));
+            tc_commit(&bars[U_VEMPTY + st]);
+            tc_commit(&bars[U_ODONE + b]);
+        }
+        if (!ok) *abort_flag = 1;
+        tc_commit(&bars[U_DRAIN + 1]);
+        mbar_wait(&bars[U_DRAIN + 1], 0);
+    } else if (warp < 16) {
+        // ---------------------------------------------------------------- softmax teams
+        const int t = warp >> 3;             // team
+        const int g = (warp >> 2) & 1;       // half: columns [64 g, 64 g + 64)
+        const int wt = warp & 3;             // TMEM lane quarter (= SM sub-partition)
+        const int r = wt * 32 + lane;        // query row within the tile = TMEM lane
+        const uint32_t lane_base = (uint32_t)(wt * 32) << 16;
+        const uint32_t tOh = tO + HC * g + lane_base;
+        const float* bias_h = bias2 + (int64_t)h * capP;
+        auto bias_of = [&](int i) -> float {
+            return (i < nc) ? bias_h[(int64_t)i * kBN + r] : sbias[(int64_t)(i - nc) * kBN + r];
+        };
+        // Half 0 stages the log2 n row of each of its team's tiles and its quarter maxima
+        // (three buffers: a fast thread may stage two tiles ahead of a slow one's reads).
+        auto stage_bias = [&](int buf, float v) {
+            sBias[(t * 3 + buf) * 128 + r] = v;
+            float wm = v;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, o));
+            if (lane == 0) sBmax[(t * 3 + buf) * 4 + wt] = wm;
+        };
+        const uint64_t c2 = pk2(scale_log2, scale_log2);
+        float m_run = -INFINITY, l_run = 0.f;   // l_run is relative to m_run
+        float bnext = 0.f;
+        if (g == 0) {
+            if (t < ntiles) stage_bias(0, bias_of(t));
+            if (t + 2 < ntiles) bnext = bias_of(t + 2);
+        }
+        bool ok = bar_and(1 + t, 256, true);
+        int k = 0;
+        for (int i = t; i < ntiles; i += 2, ++k) {
+            const int b = i % 3, bb = k % 3, u = k & 1;
+            // (warp-uniform: the TMEM loads below are warp-collective)
+            const bool got = __all_sync(0xffffffffu, !*abort_flag && mbar_wait(&bars[U_SFULL + b], (i / 3) & 1));
+            tc_fence_after();
+            const uint32_t tS = tmem + b * 128 + 64 * g + lane_base;
+            float smax = -INFINITY;
+            if (got) {
+                uint32_t sr[64];
+                TC_LD32(tS, (sr + 0));
+                TC_LD32(tS + 32, (sr + 32));
+                tc_wait_ld();
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int j = 0; j < 64; j += 8) {
+                    m4[0] = max3(m4[0], __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
+                    m4[1] = max3(m4[1], __uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3]));
+                    m4[2] = max3(m4[2], __uint_as_float(sr[j + 4]), __uint_as_float(sr[j + 5]));
+                    m4[3] = max3(m4[3], __uint_as_float(sr[j + 6]), __uint_as_float(sr[j + 7]));
+                }
+                smax = fmaxf(max3(m4[0], m4[1], m4[2]), m4[3]);
+            }
+            const float2 bm = *reinterpret_cast<const float2*>(sBmax + (t * 3 + bb) * 4 + 2 * g);
+            sUb[((t * 2 + u) * 2 + g) * 128 + r] = fmaf(smax, scale_log2, fmaxf(bm.x, bm.y));
+            if (g == 0 && i + 2 < ntiles) stage_bias((k + 1) % 3, bnext);
+            if (!bar_and(1 + t, 256, got)) { ok = false; break; }
+            if (g == 0 && i + 4 < ntiles) bnext = bias_of(i + 4);
+            const float ub = fmaxf(sUb[((t * 2 + u) * 2 + 0) * 128 + r], sUb[((t * 2 + u) * 2 + 1) * 128 + r]);
+            // The reference of tile i - 1, decided by the other team.
+            float mprev = -INFINITY;
+            if (i > 0) {
+                const bool w = mbar_wait(&bars[U_MREADY + (t ^ 1)], ((i - 1) >> 1) & 1);
+                if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; }
+                mprev = sMref[(t ^ 1) * 128 + r];
+            }
+            const bool raise = i == 0 || ub > mprev + 8.f;
+            const float mnew = raise ? ub : mprev;
+            if (g == 0) {
+                sMref[t * 128 + r] = mnew;
+                mbar_arrive(&bars[U_MREADY + t]);
+            }
+            // O holds tiles < i relative to mprev: rescale it once PV of tile i - 1 retired.
+            if (i > 0 && __any_sync(0xffffffffu, raise)) {
+                const bool w = mbar_wait(&bars[U_ODONE + (i - 1) % 3], ((i - 1) / 3) & 1);
+                if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; }
+                if (ok) {
+                    const float alpha = raise ? ex2(mprev - mnew) : 1.f;
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int c = 0; c < HC / 32; ++c) {
+                        uint32_t o[32];
+                        TC_LD32(tOh + 32 * c, o);
+                        tc_wait_ld();
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * alpha);
+                        TC_ST32(tOh + 32 * c, o);
+                    }
+                    tc_wait_st();
+                }
+            }
+            if (mnew != m_run) {   // my row sum follows the reference
+                l_run = (l_run > 0.f) ? l_run * ex2(m_run - mnew) : 0.f;
+                m_run = mnew;
+            }
+            // p = 2^(s * scale + log2 n - m) over my 64 columns in two chunks of 32.
+            const uint64_t negm2 = pk2(-m_run, -m_run);
+            uint64_t sumA = pk2(0.f, 0.f), sumB = pk2(0.f, 0.f);
+            const float* bh = sBias + (t * 3 + bb) * 128 + 64 * g;
+#pragma unroll 1
+            for (int h2 = 0; h2 < 2; ++h2) {
+                uint32_t sr[32];
+                TC_LD32(tS + 32 * h2, sr);
+                tc_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    const float4 b4 = *reinterpret_cast<const float4*>(bh + 32 * h2 + j);
+                    const uint64_t x01 = fma2(pk2(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), c2,
+                                              add2(pk2(b4.x, b4.y), negm2));
+                    const uint64_t x23 = fma2(pk2(__uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3])), c2,
+                                              add2(pk2(b4.z, b4.w), negm2));
+                    float a0, a1, a2, a3;
+                    up2(x01, a0, a1);
+                    up2(x23, a2, a3);
+                    const float p0 = ex2(a0), p1 = ex2(a1), p2 = ex2(a2), p3 = ex2(a3);
+                    sumA = add2(sumA, pk2(p0, p1));
+                    sumB = add2(sumB, pk2(p2, p3));
+                    pk[j / 2] = cvt_bf16x2(p0, p1);
+                    pk[j / 2 + 1] = cvt_bf16x2(p2, p3);
+                }
+                TC_ST16(tS + 16 * h2, pk);
+            }
+            float s0, s1, s2, s3;
+            up2(sumA, s0, s1);
+            up2(sumB, s2, s3);
+            l_run += (s0 + s1) + (s2 + s3);
+            tc_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bars[U_PFULL + b]);
+        }
+        // Epilogue: the last product retires (each commit covers every earlier product of
+        // the PV issuer), every row sum moves to the final reference, and thread (t, g, r)
+        // writes output columns [QC (2 t + g), QC (2 t + g + 1)) of its row.
+        const int lastt = ntiles - 1;
+        bool fin = ok && mbar_wait(&bars[U_ODONE + lastt % 3], (lastt / 3) & 1);
+        fin = fin && mbar_wait(&bars[U_MREADY + (lastt & 1)], (lastt >> 1) & 1);
+        const float mfin = sMref[(lastt & 1) * 128 + r];
+        const float lfin = (l_run > 0.f) ? l_run * ex2(m_run - mfin) : 0.f;
+        sL[(t * 2 + g) * 128 + r] = lfin;
+        if (bar_and(3, 512, fin)) {
+            const float inv = 1.f / ((sL[0 * 128 + r] + sL[1 * 128 + r]) + (sL[2 * 128 + r] + sL[3 * 128 + r]));
+            tc_fence_after();
+            const int col = QC * (2 * t + g);
+            uint32_t o[QC];
+            if constexpr (QC == 32) TC_LD32(tO + lane_base + col, o);
+            else TC_LD16(tO + lane_base + col, o);
+            tc_wait_ld();
+            const int64_t row = q0 + r;
+            if (row < Tq) {
+                uint4* dst = reinterpret_cast<uint4*>(out + (row * H + h) * D + col);
+#pragma unroll
+                for (int v = 0; v < QC / 8; ++v) {
+                    uint4 w4;
+                    w4.x = cvt_bf16x2(__uint_as_float(o[8 * v + 0]) * inv, __uint_as_float(o[8 * v + 1]) * inv);
+                    w4.y = cvt_bf16x2(__uint_as_float(o[8 * v + 2]) * inv, __uint_as_float(o[8 * v + 3]) * inv);
+                    w4.z = cvt_bf16x2(__uint_as_float(o[8 * v + 4]) * inv, __uint_as_float(o[8 * v + 5]) * inv);
+                    w4.w = cvt_bf16x2(__uint_as_float(o[8 * v + 6]) * inv, __uint_as_float(o[8 * v + 7]) * inv);
+                    dst[v] = w4;
+                }
+            }
+        } else {
+            *abort_flag = 1;
+        }
+    }
+    if (threadIdx.x == 0 && *abort_flag) atomicOr(&stats->error_bits, 2u);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kWK) {
+        __syncwarp();
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS)
+                     : "memory");
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 template <int D>
 cudaError_t launch_t(const CacheView& c, const StageView& s, const AttnMaps& m, int64_t Tq, __nv_bfloat16* out,
                      float scale_log2, Stats* stats, bool overlap_prev, cudaStream_t st) {
     using C = Cfg<D>;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = kTeams == 2 ? cudaFuncSetAttribute(attend_bf16_teams_kernel<D>,
-                                                           cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM)
-                                    : cudaFuncSetAttribute(attend_bf16_kernel<D>,
-                                                           cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        cudaError_t e = kDuo ? cudaFuncSetAttribute(attend_bf16_duo_kernel<D>,
+                                                    cudaFuncAttributeMaxDynamicSharedMemorySize, CfgU<D>::SMEM)
+                        : kRing ? cudaFuncSetAttribute(attend_bf16_ring_kernel<D>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize, CfgR<D>::SMEM)
+                        : kSplit ? cudaFuncSetAttribute(attend_bf16_split_kernel<D>,
+                                                      cudaFuncAttributeMaxDynamicSharedMemorySize, CfgS<D>::SMEM)
+                        : kTeams == 2 ? cudaFuncSetAttribute(attend_bf16_teams_kernel<D>,
+                                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM)
+                                      : cudaFuncSetAttribute(attend_bf16_kernel<D>,
+                                                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((Tq + kBM - 1) / kBM), (unsigned)c.H);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.blockDim = dim3((kDuo || kRing) ? kThreadsRing : kSplit ? kThreadsSplit : kThreads);
+    cfg.dynamicSmemBytes = kDuo ? CfgU<D>::SMEM : kRing ? CfgR<D>::SMEM : kSplit ? CfgS<D>::SMEM : C::SMEM;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = overlap_prev ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if constexpr (kTeams == 2)
+    if constexpr (kDuo)
+        return cudaLaunchKernelEx(&cfg, attend_bf16_duo_kernel<D>, m.q, m.kc, m.vc, m.ks, m.vs,
+                                  (const int32_t*)c.M, (const float*)c.bias2, c.capP,
+                                  (const float*)s.sbias, s.T, Tq, c.H, out, scale_log2, stats);
+    else if constexpr (kRing)
+        return cudaLaunchKernelEx(&cfg, attend_bf16_ring_kernel<D>, m.q, m.kc, m.vc, m.ks, m.vs,
+                                  (const int32_t*)c.M, (const float*)c.bias2, c.capP,
+                                  (const float*)s.sbias, s.T, Tq, c.H, out, scale_log2, stats);
+    else if constexpr (kSplit)
+        return cudaLaunchKernelEx(&cfg, attend_bf16_split_kernel<D>, m.q, m.kc, m.vc, m.ks, m.vs,
+                                  (const int32_t*)c.M, (const float*)c.bias2, c.capP,
+                                  (const float*)s.sbias, s.T, Tq, c.H, out, scale_log2, stats);
+    else if constexpr (kTeams == 2)
         return cudaLaunchKernelEx(&cfg, attend_bf16_teams_kernel<D>, m.q, m.kc, m.vc, m.ks, m.vs,
                                   (const int32_t*)c.M, (const float*)c.bias2, c.capP,
                                   (const float*)s.sbias, s.T, Tq, c.H, out, scale_log2, stats);

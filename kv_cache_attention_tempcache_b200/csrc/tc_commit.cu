@@ -224,6 +224,7 @@ stage_hash_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView c,
             const unsigned nre = __popc(__ballot_sync(0xffffffffu, need));
             if (lane == 0) {
                 s.scode[sidx] = code;
+                s.sfirst[sidx] = c.bhead[((int64_t)h << c.nbits) + code];
                 if (nre) atomicAdd(&stats->hash_rechecks, (unsigned long long)nre);
             }
         }
@@ -367,9 +368,11 @@ __device__ __forceinline__ int gspan_bf16(const GSlice<__nv_bfloat16, D>& x, uns
 // ------------------------------------------------------------------ search + decide
 //
 // One 8-lane group per staged token (h, t). Candidates are the committed entries of
-// the token's bucket (the list bhead/bnext holds exactly the entries committed
-// before this commit); the four groups of a warp walk their lists in lockstep, so
-// each step has four independent row loads in flight.
+// the token's bucket: the list bhead/bnext holds exactly the entries committed
+// before this commit, and its head was read when the token was staged (nothing
+// changes the cache between staging and commit). The four groups of a warp walk
+// their lists in lockstep, so each step has four independent row loads in flight.
+// The grid is persistent (two blocks per SM).
 //
 // bf16 storage: every cosine is formed in fp64 exactly as the definition does
 // (dot / sqrt(|k|^2 |e|^2), each sum in index order): the sums are exact by the
@@ -411,7 +414,7 @@ search_kernel(CacheView c, StageView s, float tau, double tau64, float delta, in
         G x;
         if (valid) x.load(Ks + sidx * D, gl);
         else x.zero();
-        const int first = valid ? c.bhead[((int64_t)h << c.nbits) + s.scode[sidx]] : -1;
+        const int first = valid ? s.sfirst[sidx] : -1;
         const int Mh = valid ? c.M[h] : 0;
         int m = -1, nslow = 0;
         if constexpr (sizeof(E) == 2) {
@@ -879,7 +882,7 @@ cudaError_t commit_t(const CacheView& c, const StageView& s, float tau, int32_t*
     const int64_t rows = s.T * H;
     // delta bounds |sim32 - sim| (see the search kernel): 2 x (2 (d+2) u + 3 u).
     const float delta = 2.f * (2.f * (float)(D + 2) * kU32 + 3.f * kU32);
-    const int sgrid = grid_for_rows(rows, 4 * kWarps, 148 * 16);
+    const int sgrid = grid_for_rows(rows, 4 * kWarps, 148 * 2);
     search_kernel<E, D><<<sgrid, kWarps * 32, 0, st>>>(c, s, tau, (double)tau, delta, ctr, stats);
     const int64_t wins = (int64_t)H * ((s.T + 31) / 32);
     append_kernel<E, D><<<grid_for_rows(wins, kWarps, 148 * 16), kWarps * 32, 0, st>>>(c, s, ctr);

@@ -33,6 +33,8 @@ struct StageView {
     void* Ks;              // [H][TmaxP][d]
     void* Vs;              // [H][TmaxP][d]
     uint32_t* scode;       // [H][TmaxP] hash codes of the staged tokens
+    int32_t* sfirst;       // [H][TmaxP] newest committed entry of the token's bucket (-1 = empty), read at
+                           // staging; the cache cannot change between staging and commit
     float* sbias;          // [TmaxP] 0 for t < T, -inf beyond
     int32_t* match;        // [H][TmaxP] merge target or -1 (last commit)
     int32_t* dest;         // [H][TmaxP] entry each token ended in (last commit)

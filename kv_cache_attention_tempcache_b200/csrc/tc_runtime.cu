@@ -149,7 +149,7 @@ struct tc_ctx {
         return TC_OK;
     }
     void free_staging() {
-        void* ptrs[] = {s.Ks, s.Vs, s.scode, s.sbias, s.match, s.dest, s.lcode, s.lnext, s.wcnt, s.touched};
+        void* ptrs[] = {s.Ks, s.Vs, s.scode, s.sfirst, s.sbias, s.match, s.dest, s.lcode, s.lnext, s.wcnt, s.touched};
         for (void* p : ptrs) {
             if (!p) continue;
             owned.erase(std::remove(owned.begin(), owned.end(), p), owned.end());
@@ -200,7 +200,7 @@ tc_status ensure_staging(tc_ctx* x, int64_t T) {
     tc_ctx& c = *x;
     tc_status st = TC_OK;
     if ((st = c.alloc(&c.s.Ks, rowsH * x->d * x->esize)) || (st = c.alloc(&c.s.Vs, rowsH * x->d * x->esize)) ||
-        (st = c.alloc((void**)&c.s.scode, rowsH * 4)) || (st = c.alloc((void**)&c.s.sbias, P * 4)) ||
+        (st = c.alloc((void**)&c.s.scode, rowsH * 4)) || (st = c.alloc((void**)&c.s.sfirst, rowsH * 4)) || (st = c.alloc((void**)&c.s.sbias, P * 4)) ||
         (st = c.alloc((void**)&c.s.match, rowsH * 4)) || (st = c.alloc((void**)&c.s.dest, rowsH * 4)) ||
         (st = c.alloc((void**)&c.s.lcode, rowsH * 4)) || (st = c.alloc((void**)&c.s.lnext, rowsH * 4)) ||
         (st = c.alloc((void**)&c.s.wcnt, rowsH / 32 * 4)) || (st = c.alloc((void**)&c.s.touched, rowsH * 4))) {
