@@ -39,7 +39,8 @@ WORKLOAD = "wan1.3b"
 METRIC = "TempCache frames/s (merge+4x attend) at Wan-1.3B shape; attn TFLOP/s vs peak"
 UNIT = "frames/s"
 MEASURED_PEAKS = os.path.join(ROOT, "MEASURED_PEAKS.json")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attention_traffic.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attend_bf16_duo_wan1.3b_traffic.json")
+ATTN_KERNEL = "attend_bf16_duo_kernel"   # the attention kernel the bf16 path launches
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -360,7 +361,7 @@ def run_gpu(args):
             tr = json.load(f)
         # DRAM bytes per unit of work measured by ncu, scaled to an average launch here
         traffic = tr.get("bytes_per_flop", 0) * (attn_flops_total / (args.steps * cfg.chunks * cfg.attends)) \
-            if tr.get("kernel") == "attend_bf16_kernel" else None
+            if tr.get("kernel") == ATTN_KERNEL else None
 
     # dense baseline: the same attention kernel over the uncompressed history (no merges)
     dense_line = None
@@ -405,7 +406,7 @@ def run_gpu(args):
                    "step": f"one {cfg.chunks}-chunk rollout ({cfg.F * cfg.chunks} frames) from an empty cache",
                    "l2": "inputs larger than L2 (3.5 GB of distinct K, V, Q per rollout)",
                    "parallelism": f"independent rollout per rank x{world}"},
-        "roofline": {"bound": "tensor", "kernel": "attend_bf16_kernel", "achieved": attn_tflops,
+        "roofline": {"bound": "tensor", "kernel": ATTN_KERNEL, "achieved": attn_tflops,
                      "peak": peak, "unit": "TFLOP/s", "frac": attn_tflops / peak,
                      "peak_kind": f"{peak_kind} bf16 dense, sustained", "traffic": traffic,
                      "flops_per_launch": attn_flops_total / (args.steps * cfg.chunks * cfg.attends),
@@ -422,6 +423,8 @@ def run_gpu(args):
         "gpu_launches": launches,
         "clocks": clk,
     }
+    if args.profile:   # per-call FLOPs of each chunk's attends, to pair with an ncu capture
+        line["flops_per_chunk"] = flops_per_call
     print(json.dumps(line), flush=True)
 
 
