@@ -149,8 +149,10 @@ tc_status tc_export_cache(tc_handle h, int32_t head, void* K, float* V32, int32_
 /* The hash normals in use, HOST [nbits * d]. */
 tc_status tc_get_hyperplanes(tc_handle h, float* R);
 
-/* Kernels this handle has launched so far, and how many hash bits / similarity
- * decisions needed the exact fp64 re-check (see the search kernel). */
+/* Kernels this handle has launched so far; hash bits that needed the exact fp64
+ * re-check (the fp32 sign was inside its rounding bound); and similarity sums that
+ * took the sequential index-order fp64 path (bf16 rows outside the exact-sum
+ * exponent range, or fp32 decisions inside their rounding bound). */
 tc_status tc_stats(tc_handle h, uint64_t* kernel_launches, uint64_t* hash_rechecks,
                    uint64_t* match_rechecks);
 
