@@ -168,6 +168,8 @@ stage_hash_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView c,
     const unsigned mask = (nbits >= 32) ? 0xffffffffu : ((1u << nbits) - 1u);
     const int64_t rows = T * H;
     const int64_t stride = (int64_t)gridDim.x * kWarps;
+    int nq = 0;                    // rows queued for the bucket-head lookup
+    int64_t q_sidx = 0, q_bucket = 0;
     for (int64_t r0 = (int64_t)blockIdx.x * kWarps + wib; r0 < rows; r0 += ROWS * stride) {
         typename IO::V kv[ROWS], vv[ROWS];
 #pragma unroll
@@ -224,11 +226,21 @@ stage_hash_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView c,
             const unsigned nre = __popc(__ballot_sync(0xffffffffu, need));
             if (lane == 0) {
                 s.scode[sidx] = code;
-                s.sfirst[sidx] = c.bhead[((int64_t)h << c.nbits) + code];
                 if (nre) atomicAdd(&stats->hash_rechecks, (unsigned long long)nre);
+            }
+            // The bucket-head lookups of up to 32 rows are batched, one row per lane, so
+            // their latencies overlap instead of stalling the warp once per row.
+            if (lane == nq) {
+                q_sidx = sidx;
+                q_bucket = ((int64_t)h << c.nbits) + code;
+            }
+            if (++nq == 32) {
+                s.sfirst[q_sidx] = c.bhead[q_bucket];
+                nq = 0;
             }
         }
     }
+    if (lane < nq) s.sfirst[q_sidx] = c.bhead[q_bucket];
 }
 
 // ------------------------------------------------------------------ lane groups
@@ -404,6 +416,23 @@ search_kernel(CacheView c, StageView s, float tau, double tau64, float delta, in
     int32_t* ntouched = ctr;
     const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;   // global warp
     const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    // The next token's key row and list head are loaded while the current token's
+    // decision is published (its atomics wait for their old values).
+    G xn;
+    int first_n = -1;
+    auto fetch = [&](int64_t r4n) {
+        const int64_t rn = r4n + grp;
+        if (rn < rows) {
+            const int hn = (int)(rn / T);
+            const int64_t sn = (int64_t)hn * s.TmaxP + (rn - (int64_t)hn * T);
+            xn.load(Ks + sn * D, gl);
+            first_n = s.sfirst[sn];
+        } else {
+            xn.zero();
+            first_n = -1;
+        }
+    };
+    fetch(gw * 4);
     for (int64_t r4 = gw * 4; r4 < rows; r4 += nw * 4) {   // warp-uniform loop
         const int64_t r = r4 + grp;
         const bool valid = r < rows;
@@ -411,10 +440,8 @@ search_kernel(CacheView c, StageView s, float tau, double tau64, float delta, in
         const int64_t t = valid ? r - (int64_t)h * T : 0;
         const int64_t sidx = (int64_t)h * s.TmaxP + t;
         const int64_t hrow = (int64_t)h * c.capP;
-        G x;
-        if (valid) x.load(Ks + sidx * D, gl);
-        else x.zero();
-        const int first = valid ? s.sfirst[sidx] : -1;
+        const G x = xn;
+        const int first = first_n;
         const int Mh = valid ? c.M[h] : 0;
         int m = -1, nslow = 0;
         if constexpr (sizeof(E) == 2) {
@@ -533,6 +560,7 @@ search_kernel(CacheView c, StageView s, float tau, double tau64, float delta, in
                 m = (bj >= 0 && bsim >= tau64) ? bj : -1;
             }
         }
+        fetch(r4 + nw * 4);
         if (valid && gl == 0) {
             s.match[sidx] = m;
             if (nslow) atomicAdd(&stats->match_rechecks, (unsigned long long)nslow);
