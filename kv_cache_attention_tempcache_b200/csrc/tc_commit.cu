@@ -457,16 +457,16 @@ search_kernel(CacheView c, StageView s, float tau, double tau64, float delta, in
             while (__any_sync(0xffffffffu, j >= 0)) {
                 const bool act = j >= 0;
                 G y;
-                int nxt = -1;
+                int nxt = -1, spy = 0;
                 double n2 = 0.0;
                 if (act) {
                     y.load(Kc + (hrow + j) * D, gl);
                     nxt = c.bnext[hrow + j];
                     n2 = c.knorm64[hrow + j];
+                    spy = c.kspan[hrow + j];   // stored at append
                 } else {
                     y.zero();
                 }
-                const int spy = gspan_bf16<D>(y, gmask);
                 double dot = gsum64(lane_dot64(x, y), gmask);
                 if (act) {
                     if (spx + spy > kSpanLimit<D>) {
@@ -600,9 +600,9 @@ search_kernel(CacheView c, StageView s, float tau, double tau64, float delta, in
 // |k|^2 of a row held by a lane group, in fp64 with the value of the index-order
 // sum (exact by the span rule for bf16 rows that satisfy it, else the chain).
 template <typename E, int D>
-__device__ __forceinline__ double gnorm64(const GSlice<E, D>& x, int gl, int grp, unsigned gmask) {
+__device__ __forceinline__ double gnorm64(const GSlice<E, D>& x, int span, int gl, int grp, unsigned gmask) {
     if constexpr (sizeof(E) == 2) {
-        if (2 * gspan_bf16<D>(x, gmask) <= kSpanLimit<D>) return gsum64(lane_dot64(x, x), gmask);
+        if (2 * span <= kSpanLimit<D>) return gsum64(lane_dot64(x, x), gmask);
     }
     return gchain_dot(x, x, gl, grp, gmask);
 }
@@ -634,7 +634,8 @@ __global__ void __launch_bounds__(kWarps * 32, 3) append_kernel(CacheView c, Sta
         const int w = (int)(wg - (int64_t)h * nwin);
         const int32_t* wc = s.wcnt + (int64_t)h * (s.TmaxP >> 5);
         int prefix = 0;
-        for (int q = lane; q < w; q += 32) prefix += wc[q];
+#pragma unroll 4
+        for (int q = lane; q < w; q += 32) prefix += wc[q];   // independent loads, unrolled
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) prefix += __shfl_xor_sync(0xffffffffu, prefix, o);
         const int64_t t = (int64_t)w * 32 + lane;
@@ -677,10 +678,13 @@ __global__ void __launch_bounds__(kWarps * 32, 3) append_kernel(CacheView c, Sta
 #pragma unroll
                 for (int q = 0; q < EPG / 4; ++q)
                     v32[q] = make_float4(vr[u].at(4 * q), vr[u].at(4 * q + 1), vr[u].at(4 * q + 2), vr[u].at(4 * q + 3));
-                const double nk = gnorm64(kr[u], gl, grp, gmask);
+                int span = 255;
+                if constexpr (sizeof(E) == 2) span = min(gspan_bf16<D>(kr[u], gmask), 255);
+                const double nk = gnorm64(kr[u], span, gl, grp, gmask);
                 if (gl == 0) {
                     const uint32_t code = s.scode[st[u]];
                     c.knorm64[e] = nk;
+                    c.kspan[e] = (uint8_t)span;
                     c.cnt[e] = 1;
                     c.bias2[e] = 0.f;
                     c.code[e] = code;

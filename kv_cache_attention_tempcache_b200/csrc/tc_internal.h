@@ -23,6 +23,7 @@ struct CacheView {
     int32_t* bnext;        // [H][capP] next older entry in the same bucket, -1 ends
     int32_t* bhead;        // [H][2^nbits] newest entry of each bucket, -1 = empty
     double* knorm64;       // [H][capP] |k|^2 of each entry, fp64 summed in index order
+    uint8_t* kspan;        // [H][capP] exponent span of each bf16 key (exact-sum rule of the search), <= 255
     int32_t* lhead;        // [H][capP] newest token merging into the entry in this commit (-1 between commits)
     int32_t* M;            // [H] committed entries
 };

@@ -335,7 +335,7 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
 
     // Memory budget: refuse early instead of failing halfway.
     const size_t rows = (size_t)H * x->capP;
-    const size_t need = rows * d * (2 * x->esize + 4) + rows * 4 * 7 + ((size_t)H << nbits) * 4;
+    const size_t need = rows * d * (2 * x->esize + 4) + rows * (4 * 7 + 1) + ((size_t)H << nbits) * 4;
     size_t fr = 0, tot = 0;
     if (cudaMemGetInfo(&fr, &tot) != cudaSuccess) {
         cudaGetLastError();
@@ -357,7 +357,7 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
         (st = x->alloc((void**)&c.V32, rows * d * 4)) || (st = x->alloc((void**)&c.cnt, rows * 4)) ||
         (st = x->alloc((void**)&c.bias2, rows * 4)) || (st = x->alloc((void**)&c.code, rows * 4)) ||
         (st = x->alloc((void**)&c.bnext, rows * 4)) || (st = x->alloc((void**)&c.bhead, ((size_t)H << nbits) * 4)) ||
-        (st = x->alloc((void**)&c.knorm64, rows * 8)) || (st = x->alloc((void**)&c.lhead, rows * 4)) ||
+        (st = x->alloc((void**)&c.knorm64, rows * 8)) || (st = x->alloc((void**)&c.kspan, rows)) || (st = x->alloc((void**)&c.lhead, rows * 4)) ||
         (st = x->alloc((void**)&c.M, (size_t)H * 4)) ||
         (st = x->alloc((void**)&x->ctr, (size_t)kCtrInts(H) * 4)) ||
         (st = x->alloc((void**)&x->stats, sizeof(Stats))) ||
@@ -377,7 +377,7 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
     if ((e = cudaMemset(c.Kc, 0, rows * d * x->esize)) || (e = cudaMemset(c.Vc, 0, rows * d * x->esize)) ||
         (e = cudaMemset(c.V32, 0, rows * d * 4)) || (e = cudaMemset(c.cnt, 0, rows * 4)) ||
         (e = cudaMemset(c.code, 0, rows * 4)) || (e = cudaMemset(c.bnext, 0xff, rows * 4)) ||
-        (e = cudaMemset(c.bhead, 0xff, ((size_t)H << nbits) * 4)) || (e = cudaMemset(c.knorm64, 0, rows * 8)) ||
+        (e = cudaMemset(c.bhead, 0xff, ((size_t)H << nbits) * 4)) || (e = cudaMemset(c.knorm64, 0, rows * 8)) || (e = cudaMemset(c.kspan, 0, rows)) ||
         (e = cudaMemset(c.lhead, 0xff, rows * 4)) ||
         (e = cudaMemset(c.M, 0, (size_t)H * 4)) || (e = cudaMemset(x->ctr, 0, (size_t)kCtrInts(H) * 4)) ||
         (e = cudaMemset(x->stats, 0, sizeof(Stats))) ||
