@@ -97,6 +97,29 @@ __device__ __forceinline__ float warp_sum(float v) {
 
 constexpr int kWarps = 8;  // warps per block of the warp-per-row kernels
 
+// Programmatic dependent launch: each commit kernel may be scheduled while its
+// predecessor in the stream finishes; it waits here for the predecessor's memory, and
+// lets its own successor be scheduled once every block has passed its main loop.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dependents_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int block, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)block);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 inline int grid_for_rows(int64_t rows, int per_block, int max_blocks) {
     int64_t b = (rows + per_block - 1) / per_block;
     if (b < 1) b = 1;
@@ -144,7 +167,8 @@ __device__ __forceinline__ uint32_t pack_bf16_exact(float lo, float hi) {
 template <typename E, int D, int NBP>
 __global__ void __launch_bounds__(kWarps * 32, NBP <= 8 ? 3 : (NBP <= 16 ? 2 : 1))
 stage_hash_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView c, StageView s,
-                  const float* __restrict__ R, const float* __restrict__ Rnorm, Stats* stats) {
+                  const float* __restrict__ R, const float* __restrict__ Rnorm, int32_t* ctr, Stats* stats) {
+    grid_dependency_wait();
     constexpr int EPL = D / 32;
     constexpr int ROWS = 2;
     using IO = RowIO<E, EPL>;
@@ -154,6 +178,10 @@ stage_hash_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView c,
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < s.TmaxP;
          i += (int64_t)gridDim.x * blockDim.x)
         s.sbias[i] = (i < T) ? 0.f : -INFINITY;
+    // The commit of this chunk starts from zeroed counters (every commit follows the
+    // staging of the chunk it commits; a refused commit is cleared by the host).
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < kCtrInts(H); i += blockDim.x) ctr[i] = 0;
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     uint32_t Rp[NBP][EPL / 2];   // hyperplane slices, bf16 pairs
 #pragma unroll
@@ -241,6 +269,7 @@ stage_hash_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView c,
         }
     }
     if (lane < nq) s.sfirst[q_sidx] = c.bhead[q_bucket];
+    grid_dependents_launch();
 }
 
 // ------------------------------------------------------------------ lane groups
@@ -404,6 +433,7 @@ __device__ __forceinline__ int gspan_bf16(const GSlice<__nv_bfloat16, D>& x, uns
 template <typename E, int D>
 __global__ void __launch_bounds__(kWarps * 32, 2)
 search_kernel(CacheView c, StageView s, float tau, double tau64, float delta, int32_t* ctr, Stats* stats) {
+    grid_dependency_wait();
     using G = GSlice<E, D>;
     constexpr int EPG = G::EPG;
     const int lane = threadIdx.x & 31, gl = lane & 7, grp = lane >> 3;
@@ -574,6 +604,7 @@ search_kernel(CacheView c, StageView s, float tau, double tau64, float delta, in
         }
         __syncwarp();
     }
+    grid_dependents_launch();
     // The last block to finish sums the window counts into the new sizes.
     __shared__ bool last;
     __threadfence();   // this thread's list and count updates before the ticket
@@ -616,6 +647,8 @@ __device__ __forceinline__ double gnorm64(const GSlice<E, D>& x, int span, int g
 // on its bucket's list; lane groups copy two rows each per pass.
 template <typename E, int D>
 __global__ void __launch_bounds__(kWarps * 32, 3) append_kernel(CacheView c, StageView s, const int32_t* ctr) {
+    grid_dependency_wait();
+    grid_dependents_launch();   // the merge only needs this kernel's completion
     using G = GSlice<E, D>;
     constexpr int EPG = G::EPG;
     __shared__ int sSrc[kWarps][32];
@@ -783,6 +816,7 @@ __device__ void merge_long_list(const CacheView& c, const StageView& s, int h, i
 
 template <typename E, int D>
 __global__ void __launch_bounds__(kWarps * 32, 3) merge_kernel(CacheView c, StageView s, int32_t* ctr) {
+    grid_dependency_wait();
     using G = GSlice<E, D>;
     constexpr int EPG = G::EPG;
     __shared__ int32_t sIds[kWarps][kListSmem];
@@ -885,55 +919,57 @@ __global__ void __launch_bounds__(kWarps * 32, 3) merge_kernel(CacheView c, Stag
             merge_long_list<E, D>(c, s, bh, bj, sIds[wib], sSorted[wib], lane);
         }
     }
+    grid_dependents_launch();
 }
 
 template <typename E, int D, int NBP>
 cudaError_t stage_hash_n(const CacheView& c, const StageView& s, const void* K, const void* V, const float* R,
-                         const float* Rnorm, Stats* stats, cudaStream_t st) {
+                         const float* Rnorm, int32_t* ctr, Stats* stats, cudaStream_t st) {
     const int64_t rows = s.T * c.H;
     const int grid = grid_for_rows(rows > s.TmaxP ? rows : s.TmaxP, 4 * kWarps, 148 * 8);
-    stage_hash_kernel<E, D, NBP><<<grid, kWarps * 32, 0, st>>>(
-        reinterpret_cast<const E*>(K), reinterpret_cast<const E*>(V), c, s, R, Rnorm, stats);
-    return cudaGetLastError();
+    return launch_pdl(stage_hash_kernel<E, D, NBP>, grid, kWarps * 32, st, reinterpret_cast<const E*>(K),
+                      reinterpret_cast<const E*>(V), c, s, R, Rnorm, ctr, stats);
 }
 
 template <typename E, int D>
 cudaError_t stage_hash_t(const CacheView& c, const StageView& s, const void* K, const void* V,
-                         const float* R, const float* Rnorm, Stats* stats, cudaStream_t st) {
-    if (c.nbits <= 8) return stage_hash_n<E, D, 8>(c, s, K, V, R, Rnorm, stats, st);
-    if (c.nbits <= 16) return stage_hash_n<E, D, 16>(c, s, K, V, R, Rnorm, stats, st);
-    return stage_hash_n<E, D, 32>(c, s, K, V, R, Rnorm, stats, st);
+                         const float* R, const float* Rnorm, int32_t* ctr, Stats* stats, cudaStream_t st) {
+    if (c.nbits <= 8) return stage_hash_n<E, D, 8>(c, s, K, V, R, Rnorm, ctr, stats, st);
+    if (c.nbits <= 16) return stage_hash_n<E, D, 16>(c, s, K, V, R, Rnorm, ctr, stats, st);
+    return stage_hash_n<E, D, 32>(c, s, K, V, R, Rnorm, ctr, stats, st);
 }
 
+// The counters start at zero: the staging kernel of the chunk cleared them.
 template <typename E, int D>
 cudaError_t commit_t(const CacheView& c, const StageView& s, float tau, int32_t* ctr, Stats* stats,
                      int* launches, cudaStream_t st) {
     const int H = c.H;
-    cudaError_t e = cudaMemsetAsync(ctr, 0, sizeof(int32_t) * kCtrInts(H), st);
-    if (e != cudaSuccess) return e;
     const int64_t rows = s.T * H;
     // delta bounds |sim32 - sim| (see the search kernel): 2 x (2 (d+2) u + 3 u).
     const float delta = 2.f * (2.f * (float)(D + 2) * kU32 + 3.f * kU32);
     const int sgrid = grid_for_rows(rows, 4 * kWarps, 148 * 2);
-    search_kernel<E, D><<<sgrid, kWarps * 32, 0, st>>>(c, s, tau, (double)tau, delta, ctr, stats);
+    cudaError_t e = launch_pdl(search_kernel<E, D>, sgrid, kWarps * 32, st, c, s, tau, (double)tau, delta, ctr, stats);
     const int64_t wins = (int64_t)H * ((s.T + 31) / 32);
-    append_kernel<E, D><<<grid_for_rows(wins, kWarps, 148 * 16), kWarps * 32, 0, st>>>(c, s, ctr);
-    merge_kernel<E, D><<<grid_for_rows(rows, kWarps, 148 * 8), kWarps * 32, 0, st>>>(c, s, ctr);
+    if (e == cudaSuccess)
+        e = launch_pdl(append_kernel<E, D>, grid_for_rows(wins, kWarps, 148 * 16), kWarps * 32, st, c, s,
+                       (const int32_t*)ctr);
+    if (e == cudaSuccess)
+        e = launch_pdl(merge_kernel<E, D>, grid_for_rows(rows, kWarps, 148 * 8), kWarps * 32, st, c, s, ctr);
     *launches += 3;
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace
 
 cudaError_t launch_stage_hash(const CacheView& c, const StageView& s, int dtype, const void* K,
-                              const void* V, const float* R, const float* Rnorm, Stats* stats,
+                              const void* V, const float* R, const float* Rnorm, int32_t* ctr, Stats* stats,
                               cudaStream_t st) {
     if (dtype == 0) {
-        return c.d == 128 ? stage_hash_t<__nv_bfloat16, 128>(c, s, K, V, R, Rnorm, stats, st)
-                          : stage_hash_t<__nv_bfloat16, 64>(c, s, K, V, R, Rnorm, stats, st);
+        return c.d == 128 ? stage_hash_t<__nv_bfloat16, 128>(c, s, K, V, R, Rnorm, ctr, stats, st)
+                          : stage_hash_t<__nv_bfloat16, 64>(c, s, K, V, R, Rnorm, ctr, stats, st);
     }
-    return c.d == 128 ? stage_hash_t<float, 128>(c, s, K, V, R, Rnorm, stats, st)
-                      : stage_hash_t<float, 64>(c, s, K, V, R, Rnorm, stats, st);
+    return c.d == 128 ? stage_hash_t<float, 128>(c, s, K, V, R, Rnorm, ctr, stats, st)
+                      : stage_hash_t<float, 64>(c, s, K, V, R, Rnorm, ctr, stats, st);
 }
 
 cudaError_t launch_commit(const CacheView& c, const StageView& s, int dtype, float tau, int32_t* ctr,

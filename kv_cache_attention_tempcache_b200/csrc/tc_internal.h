@@ -45,12 +45,13 @@ struct StageView {
     int32_t* touched;      // [H][TmaxP] entries with at least one merge
 };
 
-// Per-commit counters (int32, reset at the start of every commit):
+// Per-commit counters (int32; zeroed by the staging kernel of the chunk a commit
+// commits, and by the host after a refused commit):
 //   ctr[0, H)   entries touched by merges, per head
 //   ctr[H, 2H)  cache size after the commit, per head
 //   ctr[2H]     abort flag: some head would exceed its capacity
 //   ctr[2H+1]   blocks of the search kernel that have finished
-constexpr int kCtrInts(int H) { return 2 * H + 2; }
+__host__ __device__ constexpr int kCtrInts(int H) { return 2 * H + 2; }
 
 // Sticky device-side statistics and error bits.
 enum : unsigned { kErrBucketList = 1u, kErrTimeout = 2u };
@@ -64,7 +65,7 @@ struct Stats {
 // Launchers (tc_commit.cu).
 cudaError_t launch_stage_hash(const CacheView& c, const StageView& s, int dtype,
                               const void* K, const void* V, const float* R, const float* Rnorm,
-                              Stats* stats, cudaStream_t st);
+                              int32_t* ctr, Stats* stats, cudaStream_t st);
 cudaError_t launch_commit(const CacheView& c, const StageView& s, int dtype, float tau,
                           int32_t* ctr, Stats* stats, int* launches, cudaStream_t st);
 

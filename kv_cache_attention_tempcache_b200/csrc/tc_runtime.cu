@@ -249,7 +249,11 @@ tc_status commit_staged(tc_ctx* x, cudaStream_t st) {
             cudaMemcpy(M.data(), x->c.M, M.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
             return cuda_status(cudaGetLastError());
         for (int h = 0; h < x->H; ++h) x->m_upper[h] = M[h];
-        if (ctr[2 * x->H]) return TC_ECAPACITY;  // nothing changed; the chunk stays staged
+        if (ctr[2 * x->H]) {
+            // Nothing changed and the chunk stays staged; clear the counters for a retry.
+            if (cudaMemset(x->ctr, 0, ctr.size() * 4) != cudaSuccess) return cuda_status(cudaGetLastError());
+            return TC_ECAPACITY;
+        }
     } else {
         for (auto& m : x->m_upper) m += x->T_staged;
     }
@@ -416,7 +420,7 @@ tc_status tc_append_chunk(tc_handle x, const void* K, const void* V, int64_t T, 
     if ((st = ensure_staging(x, T))) return st;
     x->s.T = T;
     if ((st = encode_stage_maps(x))) return st;
-    cudaError_t e = launch_stage_hash(x->c, x->s, (int)x->dtype, K, V, x->R, x->Rnorm, x->stats, cs);
+    cudaError_t e = launch_stage_hash(x->c, x->s, (int)x->dtype, K, V, x->R, x->Rnorm, x->ctr, x->stats, cs);
     x->launches += 1;
     if (e != cudaSuccess) return cuda_status(e);
     x->T_staged = T;
