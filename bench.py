@@ -246,6 +246,11 @@ def cpu_inputs(chunks):
     return [(f(K), f(V), [f(Q) for Q in Qs]) for K, V, Qs in chunks]
 
 
+def describe(cfg) -> str:
+    return (f"{cfg.name}: H={cfg.H} d={cfg.d} P={cfg.P} F={cfg.F} chunks={cfg.chunks} attends={cfg.attends} "
+            f"S={cfg.S} p_stay={cfg.p_stay} sigma={cfg.sigma} nbits={cfg.nbits} tau={cfg.tau} {cfg.dtype}")
+
+
 def run_reference(args):
     rank, world, _ = dist_info()
     if rank != 0:
@@ -259,8 +264,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * cfg.F / value,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{WORKLOAD}: H=12 d=128 P=1560 F=3 S=4096 p_stay=0.8 sigma=0.05 nbits=16 "
-                               f"tau=0.95", "step": "one chunk (commit + 4 attends) of the rollout"},
+        "config": {"workload": describe(cfg), "step": "one chunk (commit + 4 attends) of the rollout"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -308,10 +312,12 @@ def run_gpu(args):
     torch.cuda.set_device(local)
     init_dist(world, "nccl")
     dev = torch.device("cuda", local)
-    cfg = CONFIGS[WORKLOAD]
+    cfg = CONFIGS[args.workload]
+    headline = args.workload == WORKLOAD and not args.profile
     if args.chunks:
-        cfg = cfg.replace(chunks=args.chunks, capacity=args.chunks * cfg.T)
+        cfg = cfg.replace(chunks=args.chunks, capacity=min(cfg.capacity, args.chunks * cfg.T))
     R, chunks = generate_inputs(cfg, dev, rank_seed(cfg.seed, rank))
+    input_gb = cfg.chunks * cfg.T * cfg.H * cfg.d * 2 * (2 + cfg.attends) / 1e9
     tc = TempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, hyperplanes=R)
     outs = [torch.empty(cfg.T, cfg.H, cfg.d, dtype=torch.bfloat16, device=dev) for _ in range(cfg.attends)]
 
@@ -365,7 +371,7 @@ def run_gpu(args):
 
     # dense baseline: the same attention kernel over the uncompressed history (no merges)
     dense_line = None
-    if not args.profile:
+    if headline:
         dense = TempCache(cfg.H, cfg.d, cfg.nbits, 2.0, cfg.capacity, hyperplanes=R)
         rollout(dense, chunks, outs)
         torch.cuda.synchronize()
@@ -383,7 +389,7 @@ def run_gpu(args):
                       "note": "same kernels, tau > 1 so nothing merges (uncompressed cache)"}
 
     e2e = None
-    if not args.profile:
+    if headline:
         e2e_sec, h2d, d2h = time_e2e(tc, cfg, chunks)
         e2e_value = aggregate_rate(cfg.F * cfg.chunks, world, max_over_ranks(e2e_sec, world, dev))
         e2e = {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
@@ -392,7 +398,7 @@ def run_gpu(args):
         return
     cores = len(os.sched_getaffinity(0))
     cpu = None
-    if world == 1 and not args.no_cpu_baseline and not args.profile:
+    if world == 1 and not args.no_cpu_baseline and headline:
         cpu_chunks = cpu_inputs(chunks[:6])
         v, n, desc = oracle_sample(cfg, cpu_chunks, R, n_chunks=5, rows_per_attend=256, time_budget_s=20.0,
                                    warmup_chunks=1)
@@ -401,10 +407,9 @@ def run_gpu(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1000.0 * sec_max / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"{WORKLOAD}: H=12 d=128 P=1560 F=3 chunks=40 attends=4 S=4096 p_stay=0.8 "
-                               f"sigma=0.05 nbits=16 tau=0.95 bf16",
+        "config": {"workload": describe(cfg),
                    "step": f"one {cfg.chunks}-chunk rollout ({cfg.F * cfg.chunks} frames) from an empty cache",
-                   "l2": "inputs larger than L2 (3.5 GB of distinct K, V, Q per rollout)",
+                   "l2": f"inputs larger than L2 ({input_gb:.1f} GB of distinct K, V, Q per rollout)",
                    "parallelism": f"independent rollout per rank x{world}"},
         "roofline": {"bound": "tensor", "kernel": ATTN_KERNEL, "achieved": attn_tflops,
                      "peak": peak, "unit": "TFLOP/s", "frac": attn_tflops / peak,
@@ -425,6 +430,13 @@ def run_gpu(args):
     }
     if args.profile:   # per-call FLOPs of each chunk's attends, to pair with an ncu capture
         line["flops_per_chunk"] = flops_per_call
+    if args.series:    # per-chunk device time (mean over the timed rollouts)
+        line["series"] = {
+            "append_ms": [float(np.mean([chunk_ev[k][c][0].elapsed_time(chunk_ev[k][c][1]) for k in range(args.steps)]))
+                          for c in range(cfg.chunks)],
+            "attend4_ms": [float(np.mean([chunk_ev[k][c][1].elapsed_time(chunk_ev[k][c][2]) for k in range(args.steps)]))
+                           for c in range(cfg.chunks)],
+            "entries_per_head": [float(np.mean(sz)) for sz in sizes]}
     print(json.dumps(line), flush=True)
 
 
@@ -438,7 +450,10 @@ def main():
     ap.add_argument("--profile", action="store_true",
                     help="timed rollouts only (no dense baseline, end-to-end or CPU legs), for profilers")
     ap.add_argument("--chunks", type=int, default=0,
-                    help="rollout length in chunks (default: the workload's 40); profiling runs use fewer")
+                    help="rollout length in chunks (default: the workload's); profiling runs use fewer")
+    ap.add_argument("--workload", default=WORKLOAD, choices=[k for k, v in CONFIGS.items() if v.dtype == "bf16"],
+                    help="synthetic workload; only the default one adds the dense, end-to-end and CPU legs")
+    ap.add_argument("--series", action="store_true", help="add per-chunk commit and attention times")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
