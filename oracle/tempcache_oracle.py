@@ -33,6 +33,13 @@ silent point is marked READING.
     changes (READING: the pages give no eviction policy).
  9. Deferred commit (READING): the chunk passed to append_chunk(c) is committed at
     the next append_chunk or at flush(); until then attention sees it raw.
+8b. Variant (option intra_chunk; the open point of 8 read the other way): the
+    tokens of a commit are taken in ascending t and the candidates of token t
+    also include the entries created by earlier tokens of the same commit (same
+    code). A token that merges into such an entry joins its group: the entry's
+    value is the mean of its creating token and every later member, n their
+    count. Committed entries precede new ones in index order, so exact ties
+    still go to the lowest entry index.
 10. Attention: out_t = sum_j w_tj v_j / sum_j w_tj with
     w_tj = exp(scale <q_t, k_j> + b_j - max), b_j = ln n_j for committed entries
     and 0 for staged tokens, scale = 1/sqrt(d), no mask (READING: the logit shift
@@ -139,6 +146,12 @@ def top1_in_bucket(keys, codes, cache_keys, cache_codes):
     return best, best_sim
 
 
+def new_entry_members(u, match_row, e) -> np.ndarray:
+    """Tokens of an entry created inside a commit (step 8b): its creating token u
+    and every later token whose match is the new entry e, in ascending t."""
+    return np.concatenate([[u], np.nonzero(np.asarray(match_row) == e)[0]]).astype(np.int64)
+
+
 def merge_decision(best, best_sim, tau) -> np.ndarray:
     """match = best where sim >= tau (tau as fp32 widened to fp64), else -1."""
     tau64 = np.float64(np.float32(tau))
@@ -199,7 +212,8 @@ class OracleTempCache:
     values widened to fp64).
     """
 
-    def __init__(self, H, d, nbits, tau, capacity, hyperplanes, scale=None):
+    def __init__(self, H, d, nbits, tau, capacity, hyperplanes, scale=None, intra_chunk=False):
+        self.intra_chunk = bool(intra_chunk)
         self.H, self.d, self.nbits = int(H), int(d), int(nbits)
         self.tau = float(tau)
         self.capacity = int(capacity)
@@ -220,6 +234,8 @@ class OracleTempCache:
     def _commit(self) -> CommitRecord | None:
         if self.staged is None:
             return None
+        if self.intra_chunk:
+            return self._commit_intra()
         K, V, codes = self.staged
         T = K.shape[1]
         match = np.full((self.H, T), -1, dtype=np.int64)
@@ -247,6 +263,65 @@ class OracleTempCache:
             st.values = np.concatenate([st.values, V[h, new]])
             st.counts = np.concatenate([st.counts, np.ones(new.size, dtype=np.int64)])
             st.codes = np.concatenate([st.codes, codes[h, new]])
+        self.committed_tokens += T
+        self.staged = None
+        return CommitRecord(codes=codes.copy(), match=match, dest=dest, sizes=self.cache_size())
+
+    def _commit_intra(self) -> CommitRecord:
+        """Step 8b: tokens in ascending t, candidates = committed entries of the
+        token's code (snapshot, as in 3) plus the entries created earlier in this
+        commit with the same code; ties to the lowest entry index."""
+        K, V, codes = self.staged
+        T = K.shape[1]
+        tau64 = np.float64(np.float32(self.tau))
+        match = np.full((self.H, T), -1, dtype=np.int64)
+        created = []
+        for h, st in enumerate(self.heads):
+            best, sim = top1_in_bucket(K[h], codes[h], st.keys, st.codes)
+            M0 = st.size
+            new_of_code = {}     # code -> [(entry index, creating token)] in creation order
+            made = []
+            for t in range(T):
+                bj, bs = int(best[t]), float(sim[t])
+                for e, u in new_of_code.get(int(codes[h, t]), []):
+                    s_ = float(cosine_similarity(K[h, t][None, :], K[h, u][None, :])[0])
+                    if s_ > bs:
+                        bj, bs = e, s_
+                if bj >= 0 and bs >= tau64:
+                    match[h, t] = bj
+                else:
+                    e = M0 + len(made)
+                    made.append(t)
+                    new_of_code.setdefault(int(codes[h, t]), []).append((e, t))
+            created.append(made)
+        new_sizes = np.array([st.size + len(c) for st, c in zip(self.heads, created)])
+        if np.any(new_sizes > self.capacity):
+            raise CapacityExceeded(f"commit needs {int(new_sizes.max())} entries, capacity {self.capacity}")
+        dest = match.copy()
+        for h, st in enumerate(self.heads):
+            M0 = st.size
+            made = created[h]
+            dest[h, made] = M0 + np.arange(len(made))
+            # committed targets: step 7
+            for j in np.unique(match[h][(match[h] >= 0) & (match[h] < M0)]):
+                grp = np.nonzero(match[h] == j)[0]
+                n_old = st.counts[j]
+                total = n_old * st.values[j] + V[h, grp].sum(axis=0)
+                st.counts[j] = n_old + grp.size
+                st.values[j] = total / st.counts[j]
+            # new entries: creating token plus later members
+            keys = np.zeros((len(made), self.d))
+            vals = np.zeros((len(made), self.d))
+            cnts = np.zeros(len(made), dtype=np.int64)
+            for k, u in enumerate(made):
+                members = new_entry_members(u, match[h], M0 + k)
+                keys[k] = K[h, u]
+                vals[k] = V[h, members].sum(axis=0) / members.size
+                cnts[k] = members.size
+            st.keys = np.concatenate([st.keys, keys])
+            st.values = np.concatenate([st.values, vals])
+            st.counts = np.concatenate([st.counts, cnts])
+            st.codes = np.concatenate([st.codes, codes[h, made].astype(np.uint32)])
         self.committed_tokens += T
         self.staged = None
         return CommitRecord(codes=codes.copy(), match=match, dest=dest, sizes=self.cache_size())

@@ -80,10 +80,11 @@ def test_golden_hand_example():
 
 # ----------------------------------------------------------------------------- Lemma 5.1
 
-def run_lemma(cfg, calls_per_chunk=2):
+def run_lemma(cfg, calls_per_chunk=2, intra_chunk=False):
     """Max |oracle - uncompressed softmax attention| over a rollout with exact duplicates."""
     w = Workload(cfg)
-    o = OracleTempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, f64(w.hyperplanes()))
+    o = OracleTempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, f64(w.hyperplanes()),
+                        intra_chunk=intra_chunk)
     hist_k, hist_v, worst, merged = [], [], 0.0, 0
     for c in range(cfg.chunks):
         K, V = w.next_chunk()
@@ -389,3 +390,76 @@ def test_planted_mistake_dropping_old_group_breaks_conservation():
             return rec
 
     assert conservation_error(small_cfg(chunks=3), DropsOldGroup) > 1e-3
+
+
+# ----------------------------------------------------------------------------- intra-chunk variant (8b)
+
+def test_intra_exact_duplicates_entry_count_equals_distinct_keys():
+    """With exact duplicates and matching inside a commit, every distinct key seen so
+    far is exactly one entry (a plain set of key bytes counts them)."""
+    cfg = small_cfg(sigma=0.0, tau=1.0 - 1e-6, chunks=5)
+    w = Workload(cfg)
+    o = OracleTempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, f64(w.hyperplanes()),
+                        intra_chunk=True)
+    seen = [set() for _ in range(cfg.H)]
+    for c in range(cfg.chunks):
+        K, V = w.next_chunk()
+        o.append_chunk(f64(K), f64(V))
+        o.flush()
+        Kn = f64(K)
+        for h in range(cfg.H):
+            seen[h].update(Kn[t, h].tobytes() for t in range(cfg.T))
+        np.testing.assert_array_equal(o.cache_size(), [len(x) for x in seen])
+    assert o.cache_size().max() <= cfg.S
+
+
+def test_intra_lemma51_exact_duplicates_equal_uncompressed_attention():
+    cfg = small_cfg(sigma=0.0, tau=1.0 - 1e-6, p_stay=0.7)
+    worst, merged, o = run_lemma(cfg, intra_chunk=True)
+    assert merged > 0
+    assert worst < 1e-9
+
+
+def test_intra_conservation_and_order():
+    cfg = small_cfg(chunks=4, sigma=0.02, tau=0.99)
+    w = Workload(cfg)
+    o = OracleTempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, f64(w.hyperplanes()),
+                        intra_chunk=True)
+    snap = OracleTempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, f64(w.hyperplanes()))
+    all_k = [np.zeros((0, cfg.d)) for _ in range(cfg.H)]
+    all_v = [np.zeros((0, cfg.d)) for _ in range(cfg.H)]
+    for c in range(cfg.chunks):
+        K, V = w.next_chunk()
+        rec = o.append_chunk(f64(K), f64(V))
+        snap.append_chunk(f64(K), f64(V))
+        o.flush()
+        snap.flush()
+        for h in range(cfg.H):
+            all_k[h] = np.concatenate([all_k[h], f64(K)[:, h]])
+            all_v[h] = np.concatenate([all_v[h], f64(V)[:, h]])
+            keys, vals, cnt, _ = o.export_head(h)
+            assert cnt.sum() == all_v[h].shape[0]
+            np.testing.assert_allclose((cnt[:, None] * vals).sum(0), all_v[h].sum(0), rtol=0, atol=1e-9)
+            pos = [int(np.nonzero((all_k[h] == k).all(1))[0][0]) for k in keys]
+            assert pos == sorted(pos)
+    # matching inside a commit can only merge more
+    assert (o.cache_size() <= snap.cache_size()).all() and (o.cache_size() < snap.cache_size()).any()
+
+
+def test_planted_mistake_intra_without_creating_token_breaks_conservation(monkeypatch):
+    """Averaging a new entry's later members without its creating token is caught."""
+    cfg = small_cfg(chunks=3, sigma=0.0, tau=1.0 - 1e-6)
+    real = orc.new_entry_members
+    monkeypatch.setattr(orc, "new_entry_members", lambda u, row, e: real(u, row, e)[1:] if (row == e).any()
+                        else real(u, row, e))
+    w = Workload(cfg)
+    o = OracleTempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, f64(w.hyperplanes()),
+                        intra_chunk=True)
+    total = np.zeros(cfg.d)
+    for c in range(cfg.chunks):
+        K, V = w.next_chunk()
+        o.append_chunk(f64(K), f64(V))
+        o.flush()
+        total += f64(V)[:, 0].sum(0)
+    _, vals, cnt, _ = o.export_head(0)
+    assert np.abs((cnt[:, None] * vals).sum(0) - total).max() > 1e-6
