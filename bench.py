@@ -313,12 +313,12 @@ def run_gpu(args):
     init_dist(world, "nccl")
     dev = torch.device("cuda", local)
     cfg = CONFIGS[args.workload]
-    headline = args.workload == WORKLOAD and not args.profile
+    headline = args.workload == WORKLOAD and not args.profile and not args.intra_chunk
     if args.chunks:
         cfg = cfg.replace(chunks=args.chunks, capacity=min(cfg.capacity, args.chunks * cfg.T))
     R, chunks = generate_inputs(cfg, dev, rank_seed(cfg.seed, rank))
     input_gb = cfg.chunks * cfg.T * cfg.H * cfg.d * 2 * (2 + cfg.attends) / 1e9
-    tc = TempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, hyperplanes=R)
+    tc = TempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, hyperplanes=R, intra_chunk=args.intra_chunk)
     outs = [torch.empty(cfg.T, cfg.H, cfg.d, dtype=torch.bfloat16, device=dev) for _ in range(cfg.attends)]
 
     sizes, commit_counts = sizes_per_chunk(tc, chunks, outs, cfg)
@@ -410,7 +410,8 @@ def run_gpu(args):
         "config": {"workload": describe(cfg),
                    "step": f"one {cfg.chunks}-chunk rollout ({cfg.F * cfg.chunks} frames) from an empty cache",
                    "l2": f"inputs larger than L2 ({input_gb:.1f} GB of distinct K, V, Q per rollout)",
-                   "parallelism": f"independent rollout per rank x{world}"},
+                   "parallelism": f"independent rollout per rank x{world}",
+                   "commit": "matches inside the chunk too" if args.intra_chunk else "snapshot of earlier commits"},
         "roofline": {"bound": "tensor", "kernel": ATTN_KERNEL, "achieved": attn_tflops,
                      "peak": peak, "unit": "TFLOP/s", "frac": attn_tflops / peak,
                      "peak_kind": f"{peak_kind} bf16 dense, sustained", "traffic": traffic,
@@ -454,6 +455,8 @@ def main():
     ap.add_argument("--workload", default=WORKLOAD, choices=[k for k, v in CONFIGS.items() if v.dtype == "bf16"],
                     help="synthetic workload; only the default one adds the dense, end-to-end and CPU legs")
     ap.add_argument("--series", action="store_true", help="add per-chunk commit and attention times")
+    ap.add_argument("--intra-chunk", action="store_true",
+                    help="commits also match tokens against entries created earlier in the same commit")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

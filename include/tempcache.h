@@ -56,6 +56,13 @@ typedef struct {
     const float* hyperplanes;  /* HOST [nbits*d] hash normals, each value exactly
                                   representable in bf16; NULL = N(0,1) draws from seed,
                                   rounded to bf16. Copied during the call.              */
+    int32_t intra_chunk;       /* 0: a commit matches its tokens against the entries
+                                  committed before it only (section 2.A read as a
+                                  snapshot). 1: tokens are taken in ascending t and also
+                                  match entries created earlier in the same commit, so
+                                  duplicates inside one chunk merge too (the other
+                                  reading of the same passage). Costs one more kernel and
+                                  4 * 2^nbits bytes per head.                             */
 } tc_options;
 
 /*

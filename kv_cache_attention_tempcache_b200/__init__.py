@@ -34,7 +34,7 @@ API = [
 
 class TCOptions(ctypes.Structure):
     _fields_ = [("dtype", ctypes.c_int), ("seed", ctypes.c_uint64), ("softmax_scale", ctypes.c_float),
-                ("hyperplanes", ctypes.POINTER(ctypes.c_float))]
+                ("hyperplanes", ctypes.POINTER(ctypes.c_float)), ("intra_chunk", ctypes.c_int32)]
 
 
 def _load():
@@ -104,7 +104,7 @@ class TempCache:
     """
 
     def __init__(self, H: int, d: int, nbits: int, tau: float, capacity: int, dtype: str = "bf16",
-                 seed: int = 0, softmax_scale: float = 0.0, hyperplanes=None):
+                 seed: int = 0, softmax_scale: float = 0.0, hyperplanes=None, intra_chunk: bool = False):
         self.H, self.d, self.nbits = int(H), int(d), int(nbits)
         self.dtype = dtype
         self.torch_dtype = torch.bfloat16 if dtype == "bf16" else torch.float32
@@ -112,6 +112,7 @@ class TempCache:
         opt.dtype = TC_BF16 if dtype == "bf16" else TC_F32
         opt.seed = int(seed)
         opt.softmax_scale = float(softmax_scale)
+        opt.intra_chunk = 1 if intra_chunk else 0
         self._R = None
         if hyperplanes is not None:
             R = np.ascontiguousarray(np.asarray(hyperplanes, dtype=np.float32).reshape(-1))

@@ -406,6 +406,34 @@ __device__ __forceinline__ int gspan_bf16(const GSlice<__nv_bfloat16, D>& x, uns
     return emax >= emin ? emax - emin + 7 : 0;
 }
 
+// The last block of the grid to finish sums the per-window counts of new entries
+// into the new cache sizes and raises the abort flag if a head would exceed its
+// capacity. Every thread of the grid calls it once, after its last update.
+__device__ void publish_sizes(const CacheView& c, const StageView& s, int32_t* ctr) {
+    const int H = c.H;
+    const int lane = threadIdx.x & 31;
+    __shared__ bool last;
+    __threadfence();   // this thread's list and count updates before the ticket
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicAdd(&ctr[2 * H + 1], 1) == (int)gridDim.x - 1;
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    const int nwin = (int)((s.T + 31) >> 5);
+    const int warp = threadIdx.x >> 5;
+    for (int h = warp; h < H; h += blockDim.x >> 5) {
+        int u = 0;
+        for (int w = lane; w < nwin; w += 32) u += __ldcg(&s.wcnt[(int64_t)h * (s.TmaxP >> 5) + w]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
+        if (lane == 0) {
+            const int nm = c.M[h] + u;
+            ctr[H + h] = nm;
+            if ((int64_t)nm > c.capacity) atomicExch(&ctr[2 * H], 1);
+        }
+    }
+}
+
 // ------------------------------------------------------------------ search + decide
 //
 // One 8-lane group per staged token (h, t). Candidates are the committed entries of
@@ -432,7 +460,8 @@ __device__ __forceinline__ int gspan_bf16(const GSlice<__nv_bfloat16, D>& x, uns
 // cache sizes and raises the abort flag if some head would exceed its capacity.
 template <typename E, int D>
 __global__ void __launch_bounds__(kWarps * 32, 2)
-search_kernel(CacheView c, StageView s, float tau, double tau64, float delta, int32_t* ctr, Stats* stats) {
+search_kernel(CacheView c, StageView s, float tau, double tau64, float delta, bool intra, int32_t* ctr,
+              Stats* stats) {
     grid_dependency_wait();
     using G = GSlice<E, D>;
     constexpr int EPG = G::EPG;
@@ -474,6 +503,8 @@ search_kernel(CacheView c, StageView s, float tau, double tau64, float delta, in
         const int first = first_n;
         const int Mh = valid ? c.M[h] : 0;
         int m = -1, nslow = 0;
+        double best64 = -INFINITY;   // exact best committed similarity and its entry
+        int bj64 = -1;
         if constexpr (sizeof(E) == 2) {
             const int spx = gspan_bf16<D>(x, gmask);
             double n1 = gsum64(lane_dot64(x, x), gmask);
@@ -516,6 +547,8 @@ search_kernel(CacheView c, StageView s, float tau, double tau64, float delta, in
                 j = nxt;
             }
             m = (bestj >= 0 && best >= tau64) ? bestj : -1;
+            best64 = best;
+            bj64 = bestj;
         } else {
             float nk = 0.f;
 #pragma unroll
@@ -566,7 +599,8 @@ search_kernel(CacheView c, StageView s, float tau, double tau64, float delta, in
             }
             bool exact = false;
             if (ncand > 0) {
-                if (!weird && best < tau - delta) m = -1;
+                if (intra) exact = true;   // the exact best similarity is needed
+                else if (!weird && best < tau - delta) m = -1;
                 else if (!weird && best > tau + delta && (ncand == 1 || best - second > 2.f * delta)) m = bestj;
                 else exact = true;
             }
@@ -588,9 +622,24 @@ search_kernel(CacheView c, StageView s, float tau, double tau64, float delta, in
                     }
                 }
                 m = (bj >= 0 && bsim >= tau64) ? bj : -1;
+                best64 = bsim;
+                bj64 = bj;
             }
         }
         fetch(r4 + nw * 4);
+        if (intra) {
+            // Matching inside the chunk: keep the committed best for the dedupe kernel
+            // and group the chunk's tokens by bucket.
+            if (valid && gl == 0) {
+                s.match[sidx] = bj64;
+                s.bsim[sidx] = best64;
+                if (nslow) atomicAdd(&stats->match_rechecks, (unsigned long long)nslow);
+                const int old = atomicExch(&c.cbhead[((int64_t)h << c.nbits) + s.scode[sidx]], (int)t);
+                s.cbnext[sidx] = old;
+            }
+            __syncwarp();
+            continue;
+        }
         if (valid && gl == 0) {
             s.match[sidx] = m;
             if (nslow) atomicAdd(&stats->match_rechecks, (unsigned long long)nslow);
@@ -605,27 +654,168 @@ search_kernel(CacheView c, StageView s, float tau, double tau64, float delta, in
         __syncwarp();
     }
     grid_dependents_launch();
-    // The last block to finish sums the window counts into the new sizes.
-    __shared__ bool last;
-    __threadfence();   // this thread's list and count updates before the ticket
-    __syncthreads();
-    if (threadIdx.x == 0) last = atomicAdd(&ctr[2 * H + 1], 1) == (int)gridDim.x - 1;
-    __syncthreads();
-    if (!last) return;
-    __threadfence();
-    const int nwin = (int)((T + 31) >> 5);
-    const int warp = threadIdx.x >> 5;
-    for (int h = warp; h < H; h += blockDim.x >> 5) {
-        int u = 0;
-        for (int w = lane; w < nwin; w += 32) u += __ldcg(&s.wcnt[(int64_t)h * (s.TmaxP >> 5) + w]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) u += __shfl_xor_sync(0xffffffffu, u, o);
-        if (lane == 0) {
-            const int nm = c.M[h] + u;
-            ctr[H + h] = nm;
-            if ((int64_t)nm > c.capacity) atomicExch(&ctr[2 * H], 1);
-        }
+    if (!intra) publish_sizes(c, s, ctr);
+}
+
+// Exact fp64 cosine of two rows held by a lane group (the similarity of the
+// definition; bf16 rows use the exact-sum rule, other rows the index-order chain).
+template <typename E, int D>
+__device__ __forceinline__ double gexact_dot(const GSlice<E, D>& a, int spa, const GSlice<E, D>& b, int spb, int gl,
+                                             int grp, unsigned gmask) {
+    if constexpr (sizeof(E) == 2) {
+        if (spa + spb <= kSpanLimit<D>) return gsum64(lane_dot64(a, b), gmask);
     }
+    return gchain_dot(a, b, gl, grp, gmask);
+}
+
+template <typename E, int D>
+__device__ __forceinline__ int grow_span(const GSlice<E, D>& x, unsigned gmask) {
+    if constexpr (sizeof(E) == 2) return gspan_bf16<D>(x, gmask);
+    return 255;
+}
+
+// ------------------------------------------------------------------ dedupe (matching inside the chunk)
+constexpr int kDedupSmem = 48;   // bucket members ordered in shared memory (more: scan the codes)
+//
+// Used when a commit also matches tokens against entries created earlier in the same
+// commit. The search left, per token, the exact best committed candidate (index and
+// similarity) and grouped the chunk's tokens by (head, code): tokens can only meet
+// tokens of their own bucket, so each bucket is an independent sequence. One lane
+// group per bucket (started by its newest token, the list head) takes the bucket's
+// tokens in ascending t. A token compares the exact cosine against every entry
+// created earlier in the bucket, in creation order; with strict > the committed best
+// (lower entry indices) and earlier creators keep exact ties. It then merges (into a
+// committed entry: the entry's merge list; into a new entry: that entry's member
+// chain, in ascending t) or creates an entry (counted in its 32-token window).
+// Buckets of up to 8 tokens are ordered in the group's lanes, up to kDedupSmem in
+// shared memory; larger ones visit their members by scanning the head's codes in
+// token order. The last block publishes the new sizes.
+template <typename E, int D>
+__global__ void __launch_bounds__(kWarps * 32, 2)
+dedupe_kernel(CacheView c, StageView s, double tau64, int32_t* ctr, Stats* stats) {
+    grid_dependency_wait();
+    __shared__ int sMem[kWarps * 4][kDedupSmem];   // one buffer per lane group
+    __shared__ int sSrt[kWarps * 4][kDedupSmem];
+    using G = GSlice<E, D>;
+    const int lane = threadIdx.x & 31, gl = lane & 7, grp = lane >> 3;
+    const unsigned gmask = 0xFFu << (8 * grp);
+    const int H = c.H;
+    const int64_t T = s.T;
+    const int64_t rows = T * H;
+    const E* Ks = reinterpret_cast<const E*>(s.Ks);
+    int32_t* ntouched = ctr;
+    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t r4 = gw * 4; r4 < rows; r4 += nw * 4) {   // warp-uniform loop
+        const int64_t r = r4 + grp;
+        bool head = false;
+        int h = 0;
+        int64_t t = 0, bucket = 0;
+        uint32_t code = 0;
+        if (r < rows) {
+            h = (int)(r / T);
+            t = r - (int64_t)h * T;
+            code = s.scode[(int64_t)h * s.TmaxP + t];
+            bucket = ((int64_t)h << c.nbits) + code;
+            head = c.cbhead[bucket] == (int)t;
+        }
+        if (!head) continue;   // group-uniform; the loop has no warp-wide operations below
+        const int64_t sbase = (int64_t)h * s.TmaxP;
+        const int64_t hrow = (int64_t)h * c.capP;
+        int cr_head = -1, cr_tail = -1;   // this bucket's new entries, in creation order
+        auto process = [&](int tm) {
+            const int64_t sm = sbase + tm;
+            G x;
+            x.load(Ks + sm * D, gl);
+            const int spx = grow_span<E, D>(x, gmask);
+            const double n1 = gexact_dot(x, spx, x, spx, gl, grp, gmask);
+            int bj = s.match[sm];
+            double bs = s.bsim[sm];
+            int guard = 0;
+            for (int u = cr_head; u >= 0; u = s.crnext[sbase + u]) {
+                if (++guard > (int)T) break;
+                G y;
+                y.load(Ks + (sbase + u) * D, gl);
+                const int spy = grow_span<E, D>(y, gmask);
+                const double n2 = gexact_dot(y, spy, y, spy, gl, grp, gmask);
+                const double dot = gexact_dot(x, spx, y, spy, gl, grp, gmask);
+                const double sim = (n1 > 0.0 && n2 > 0.0) ? dot / sqrt(n1 * n2) : 0.0;
+                if (sim > bs) {
+                    bs = sim;
+                    bj = -2 - u;
+                }
+            }
+            const bool merge = bj != -1 && bs >= tau64;
+            if (gl == 0) {
+                if (merge && bj >= 0) {          // into a committed entry
+                    s.match[sm] = bj;
+                    const int old = atomicExch(&c.lhead[hrow + bj], tm);
+                    s.lnext[sm] = old;
+                    if (old < 0) s.touched[sbase + atomicAdd(&ntouched[h], 1)] = bj;
+                } else if (merge) {              // into an entry created by token u
+                    const int u = -2 - bj;
+                    s.match[sm] = bj;
+                    s.icnext[sm] = -1;
+                    if (s.ichead[sbase + u] < 0) s.ichead[sbase + u] = tm;
+                    else s.icnext[sbase + s.ictail[sbase + u]] = tm;
+                    s.ictail[sbase + u] = tm;
+                } else {                         // creates an entry
+                    s.match[sm] = -1;
+                    s.crnext[sm] = -1;
+                    if (cr_tail >= 0) s.crnext[sbase + cr_tail] = tm;
+                    atomicAdd(&s.wcnt[(int64_t)h * (s.TmaxP >> 5) + (tm >> 5)], 1);
+                }
+            }
+            __syncwarp(gmask);
+            if (!merge) {
+                if (cr_head < 0) cr_head = tm;
+                cr_tail = tm;
+            }
+        };
+        // members: walk the bucket's token list (newest first) into the lanes, and up
+        // to kDedupSmem of them into this group's shared buffer
+        int* buf = sMem[threadIdx.x >> 3];
+        int L = 0, id = 0x7fffffff;
+        for (int u = (int)t; u >= 0; u = s.cbnext[sbase + u]) {
+            if (gl == L) id = u;
+            if (gl == 0 && L < kDedupSmem) buf[L] = u;
+            if (++L > kDedupSmem) break;
+        }
+        __syncwarp(gmask);
+        if (L <= 8) {
+            int rank = 0;
+            for (int k = 0; k < L; ++k) rank += (__shfl_sync(gmask, id, 8 * grp + k) < id);
+            for (int q = 0; q < L; ++q) {
+                const int src = __ffs((__ballot_sync(gmask, rank == q && gl < L) >> (8 * grp)) & 0xFFu) - 1;
+                process(__shfl_sync(gmask, id, 8 * grp + src));
+            }
+        } else if (L <= kDedupSmem) {
+            // order the ids in shared memory: each lane places its ids at their ranks
+            int* srt = sSrt[threadIdx.x >> 3];
+            for (int a = gl; a < L; a += 8) {
+                const int mine = buf[a];
+                int rank = 0;
+                for (int b2 = 0; b2 < L; ++b2) rank += (buf[b2] < mine);
+                srt[rank] = mine;
+            }
+            __syncwarp(gmask);
+            for (int q = 0; q < L; ++q) process(srt[q]);
+        } else {
+            for (int64_t t0 = 0; t0 < T; t0 += 8) {
+                const bool hit = t0 + gl < T && s.scode[sbase + t0 + gl] == code;
+                unsigned b = (__ballot_sync(gmask, hit) >> (8 * grp)) & 0xFFu;
+                while (b) {
+                    const int k = __ffs(b) - 1;
+                    b &= b - 1;
+                    process((int)t0 + k);
+                }
+            }
+        }
+        if (gl == 0) c.cbhead[bucket] = -1;
+        __syncwarp(gmask);
+    }
+    grid_dependents_launch();
+    publish_sizes(c, s, ctr);
 }
 
 // |k|^2 of a row held by a lane group, in fp64 with the value of the index-order
@@ -675,12 +865,12 @@ __global__ void __launch_bounds__(kWarps * 32, 3) append_kernel(CacheView c, Sta
         const bool valid = t < T;
         const int64_t sidx = (int64_t)h * s.TmaxP + t;
         const int m = valid ? s.match[sidx] : 0;
-        const bool un = valid && m < 0;
+        const bool un = valid && m == -1;   // -2 - u: joins the entry token u creates
         const unsigned bal = __ballot_sync(0xffffffffu, un);
         const int rank = __popc(bal & ((1u << lane) - 1u));
         const int base = c.M[h] + prefix;
         if (valid) {
-            s.dest[sidx] = un ? base + rank : m;
+            if (m >= -1) s.dest[sidx] = un ? base + rank : m;
             s.lcode[sidx] = s.scode[sidx];
         }
         if (un) sSrc[wib][rank] = lane;
@@ -706,11 +896,43 @@ __global__ void __launch_bounds__(kWarps * 32, 3) append_kernel(CacheView c, Sta
                 const int k = k0 + 4 * u + grp;
                 const int64_t e = hrow + base + k;
                 kr[u].store(reinterpret_cast<E*>(c.Kc) + e * D, gl);
-                vr[u].store(reinterpret_cast<E*>(c.Vc) + e * D, gl);
                 float4* v32 = reinterpret_cast<float4*>(c.V32 + e * D + gl * EPG);
+                int members = 0;   // later tokens of this chunk that joined this new entry
+                const int64_t sbase = (int64_t)h * s.TmaxP;
+                int tm = s.ichead[st[u]];
+                if (tm < 0) {
+                    vr[u].store(reinterpret_cast<E*>(c.Vc) + e * D, gl);
 #pragma unroll
-                for (int q = 0; q < EPG / 4; ++q)
-                    v32[q] = make_float4(vr[u].at(4 * q), vr[u].at(4 * q + 1), vr[u].at(4 * q + 2), vr[u].at(4 * q + 3));
+                    for (int q = 0; q < EPG / 4; ++q)
+                        v32[q] = make_float4(vr[u].at(4 * q), vr[u].at(4 * q + 1), vr[u].at(4 * q + 2),
+                                             vr[u].at(4 * q + 3));
+                } else {   // group-uniform: mean of the creating token and its members, in t order
+                    float acc[EPG];
+#pragma unroll
+                    for (int i = 0; i < EPG; ++i) acc[i] = 0.f;
+                    for (; tm >= 0; tm = s.icnext[sbase + tm]) {
+                        G vm;
+                        vm.load(Vs + (sbase + tm) * D, gl);
+#pragma unroll
+                        for (int i = 0; i < EPG; ++i) acc[i] = __fadd_rn(acc[i], vm.at(i));
+                        if (gl == 0) {
+                            s.match[sbase + tm] = base + k;
+                            s.dest[sbase + tm] = base + k;
+                        }
+                        if (++members > (int)T) break;
+                    }
+                    const float ft = (float)(1 + members);
+                    float nv[EPG];
+#pragma unroll
+                    for (int i = 0; i < EPG; ++i) nv[i] = __fdiv_rn(__fadd_rn(vr[u].at(i), acc[i]), ft);
+#pragma unroll
+                    for (int q = 0; q < EPG / 4; ++q)
+                        v32[q] = make_float4(nv[4 * q], nv[4 * q + 1], nv[4 * q + 2], nv[4 * q + 3]);
+                    G out;
+                    out.from_floats(nv);
+                    out.store(reinterpret_cast<E*>(c.Vc) + e * D, gl);
+                    if (gl == 0) s.ichead[st[u]] = -1;
+                }
                 int span = 255;
                 if constexpr (sizeof(E) == 2) span = min(gspan_bf16<D>(kr[u], gmask), 255);
                 const double nk = gnorm64(kr[u], span, gl, grp, gmask);
@@ -718,8 +940,8 @@ __global__ void __launch_bounds__(kWarps * 32, 3) append_kernel(CacheView c, Sta
                     const uint32_t code = s.scode[st[u]];
                     c.knorm64[e] = nk;
                     c.kspan[e] = (uint8_t)span;
-                    c.cnt[e] = 1;
-                    c.bias2[e] = 0.f;
+                    c.cnt[e] = 1 + members;
+                    c.bias2[e] = log2f((float)(1 + members));
                     c.code[e] = code;
                     c.bnext[e] = atomicExch(&c.bhead[((int64_t)h << c.nbits) + code], base + k);
                 }
@@ -827,6 +1049,10 @@ __global__ void __launch_bounds__(kWarps * 32, 3) merge_kernel(CacheView c, Stag
     const unsigned gmask = 0xFFu << (8 * grp);
     const int64_t T = s.T;
     const E* Vs = reinterpret_cast<const E*>(s.Vs);
+    if (aborted)   // a refused commit leaves no member chains behind (matching inside the chunk)
+        for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < (int64_t)H * T;
+             q += (int64_t)gridDim.x * blockDim.x)
+            s.ichead[(q / T) * s.TmaxP + (q % T)] = -1;
     if (!aborted && blockIdx.x == 0)
         for (int hh = threadIdx.x; hh < H; hh += blockDim.x) c.M[hh] = ctr[H + hh];
     const int nwin = (int)((T + 31) >> 5);
@@ -941,14 +1167,19 @@ cudaError_t stage_hash_t(const CacheView& c, const StageView& s, const void* K, 
 
 // The counters start at zero: the staging kernel of the chunk cleared them.
 template <typename E, int D>
-cudaError_t commit_t(const CacheView& c, const StageView& s, float tau, int32_t* ctr, Stats* stats,
+cudaError_t commit_t(const CacheView& c, const StageView& s, float tau, bool intra, int32_t* ctr, Stats* stats,
                      int* launches, cudaStream_t st) {
     const int H = c.H;
     const int64_t rows = s.T * H;
     // delta bounds |sim32 - sim| (see the search kernel): 2 x (2 (d+2) u + 3 u).
     const float delta = 2.f * (2.f * (float)(D + 2) * kU32 + 3.f * kU32);
     const int sgrid = grid_for_rows(rows, 4 * kWarps, 148 * 2);
-    cudaError_t e = launch_pdl(search_kernel<E, D>, sgrid, kWarps * 32, st, c, s, tau, (double)tau, delta, ctr, stats);
+    cudaError_t e = launch_pdl(search_kernel<E, D>, sgrid, kWarps * 32, st, c, s, tau, (double)tau, delta, intra,
+                               ctr, stats);
+    if (e == cudaSuccess && intra) {
+        e = launch_pdl(dedupe_kernel<E, D>, sgrid, kWarps * 32, st, c, s, (double)tau, ctr, stats);
+        *launches += 1;
+    }
     const int64_t wins = (int64_t)H * ((s.T + 31) / 32);
     if (e == cudaSuccess)
         e = launch_pdl(append_kernel<E, D>, grid_for_rows(wins, kWarps, 148 * 16), kWarps * 32, st, c, s,
@@ -972,14 +1203,14 @@ cudaError_t launch_stage_hash(const CacheView& c, const StageView& s, int dtype,
                       : stage_hash_t<float, 64>(c, s, K, V, R, Rnorm, ctr, stats, st);
 }
 
-cudaError_t launch_commit(const CacheView& c, const StageView& s, int dtype, float tau, int32_t* ctr,
+cudaError_t launch_commit(const CacheView& c, const StageView& s, int dtype, float tau, bool intra, int32_t* ctr,
                           Stats* stats, int* launches, cudaStream_t st) {
     if (dtype == 0) {
-        return c.d == 128 ? commit_t<__nv_bfloat16, 128>(c, s, tau, ctr, stats, launches, st)
-                          : commit_t<__nv_bfloat16, 64>(c, s, tau, ctr, stats, launches, st);
+        return c.d == 128 ? commit_t<__nv_bfloat16, 128>(c, s, tau, intra, ctr, stats, launches, st)
+                          : commit_t<__nv_bfloat16, 64>(c, s, tau, intra, ctr, stats, launches, st);
     }
-    return c.d == 128 ? commit_t<float, 128>(c, s, tau, ctr, stats, launches, st)
-                      : commit_t<float, 64>(c, s, tau, ctr, stats, launches, st);
+    return c.d == 128 ? commit_t<float, 128>(c, s, tau, intra, ctr, stats, launches, st)
+                      : commit_t<float, 64>(c, s, tau, intra, ctr, stats, launches, st);
 }
 
 }  // namespace tc

@@ -26,6 +26,8 @@ struct CacheView {
     uint8_t* kspan;        // [H][capP] exponent span of each bf16 key (exact-sum rule of the search), <= 255
     int32_t* lhead;        // [H][capP] newest token merging into the entry in this commit (-1 between commits)
     int32_t* M;            // [H] committed entries
+    int32_t* cbhead;       // [H][2^nbits] newest staged token of each bucket during a commit that matches
+                           // inside the chunk (-1 between commits); null when that mode is off
 };
 
 struct StageView {
@@ -43,6 +45,13 @@ struct StageView {
     int32_t* lnext;        // [H][TmaxP] next (older) token of the same merge list
     int32_t* wcnt;         // [H][TmaxP/32] unmatched tokens per 32-token window (0 between commits)
     int32_t* touched;      // [H][TmaxP] entries with at least one merge
+    // matching inside the chunk (see the dedupe kernel):
+    double* bsim;          // [H][TmaxP] best committed similarity of each token (-inf: none)
+    int32_t* cbnext;       // [H][TmaxP] next older staged token with the same code
+    int32_t* crnext;       // [H][TmaxP] next token that created an entry in the same bucket
+    int32_t* ichead;       // [H][TmaxP] first token merging into the entry this token created (-1: none)
+    int32_t* ictail;       // [H][TmaxP] last such token
+    int32_t* icnext;       // [H][TmaxP] next token merging into the same new entry
 };
 
 // Per-commit counters (int32; zeroed by the staging kernel of the chunk a commit
@@ -66,7 +75,7 @@ struct Stats {
 cudaError_t launch_stage_hash(const CacheView& c, const StageView& s, int dtype,
                               const void* K, const void* V, const float* R, const float* Rnorm,
                               int32_t* ctr, Stats* stats, cudaStream_t st);
-cudaError_t launch_commit(const CacheView& c, const StageView& s, int dtype, float tau,
+cudaError_t launch_commit(const CacheView& c, const StageView& s, int dtype, float tau, bool intra_chunk,
                           int32_t* ctr, Stats* stats, int* launches, cudaStream_t st);
 
 // Launchers (tc_attn_f32.cu, tc_attn_bf16.cu).

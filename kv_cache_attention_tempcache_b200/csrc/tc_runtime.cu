@@ -114,6 +114,7 @@ struct tc_ctx {
     int H = 0, d = 0, nbits = 0, esize = 2;
     float tau = 0.f, scale = 0.f;
     tc_dtype dtype = TC_BF16;
+    bool intra = false;            // commits also match inside the chunk
     int64_t capacity = 0, capP = 0;
     int device = 0;
     CacheView c{};
@@ -149,7 +150,8 @@ struct tc_ctx {
         return TC_OK;
     }
     void free_staging() {
-        void* ptrs[] = {s.Ks, s.Vs, s.scode, s.sfirst, s.sbias, s.match, s.dest, s.lcode, s.lnext, s.wcnt, s.touched};
+        void* ptrs[] = {s.Ks,    s.Vs,     s.scode,  s.sfirst, s.sbias,  s.match,  s.dest,   s.lcode,
+                        s.lnext, s.wcnt,   s.touched, s.bsim,  s.cbnext, s.crnext, s.ichead, s.ictail, s.icnext};
         for (void* p : ptrs) {
             if (!p) continue;
             owned.erase(std::remove(owned.begin(), owned.end(), p), owned.end());
@@ -203,16 +205,21 @@ tc_status ensure_staging(tc_ctx* x, int64_t T) {
         (st = c.alloc((void**)&c.s.scode, rowsH * 4)) || (st = c.alloc((void**)&c.s.sfirst, rowsH * 4)) || (st = c.alloc((void**)&c.s.sbias, P * 4)) ||
         (st = c.alloc((void**)&c.s.match, rowsH * 4)) || (st = c.alloc((void**)&c.s.dest, rowsH * 4)) ||
         (st = c.alloc((void**)&c.s.lcode, rowsH * 4)) || (st = c.alloc((void**)&c.s.lnext, rowsH * 4)) ||
-        (st = c.alloc((void**)&c.s.wcnt, rowsH / 32 * 4)) || (st = c.alloc((void**)&c.s.touched, rowsH * 4))) {
+        (st = c.alloc((void**)&c.s.wcnt, rowsH / 32 * 4)) || (st = c.alloc((void**)&c.s.touched, rowsH * 4)) ||
+        (st = c.alloc((void**)&c.s.bsim, rowsH * 8)) || (st = c.alloc((void**)&c.s.cbnext, rowsH * 4)) ||
+        (st = c.alloc((void**)&c.s.crnext, rowsH * 4)) || (st = c.alloc((void**)&c.s.ichead, rowsH * 4)) ||
+        (st = c.alloc((void**)&c.s.ictail, rowsH * 4)) || (st = c.alloc((void**)&c.s.icnext, rowsH * 4))) {
         x->free_staging();
         return st;
     }
     // Zero the staging keys and values once: rows past the staged chunk are only
     // ever read as masked attention operands and must hold finite values.
-    // The window counts start at zero; every commit leaves them at zero.
+    // The window counts start at zero and the in-chunk member chains empty (-1);
+    // every commit leaves them so.
     if (cudaMemset(c.s.Ks, 0, rowsH * x->d * x->esize) != cudaSuccess ||
         cudaMemset(c.s.Vs, 0, rowsH * x->d * x->esize) != cudaSuccess ||
-        cudaMemset(c.s.wcnt, 0, rowsH / 32 * 4) != cudaSuccess)
+        cudaMemset(c.s.wcnt, 0, rowsH / 32 * 4) != cudaSuccess ||
+        cudaMemset(c.s.ichead, 0xff, rowsH * 4) != cudaSuccess)
         return cuda_status(cudaGetLastError());
     x->s.TmaxP = P;
     x->maps_T = -1;
@@ -235,7 +242,7 @@ tc_status commit_staged(tc_ctx* x, cudaStream_t st) {
     StageView s = x->s;
     s.T = x->T_staged;
     int launches = 0;
-    cudaError_t e = launch_commit(x->c, s, (int)x->dtype, x->tau, x->ctr, x->stats, &launches, st);
+    cudaError_t e = launch_commit(x->c, s, (int)x->dtype, x->tau, x->intra, x->ctr, x->stats, &launches, st);
     x->launches += launches;
     if (e != cudaSuccess) return cuda_status(e);
     int64_t worst = 0;
@@ -296,11 +303,11 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
                        tc_handle* out) {
     if (!out) return TC_EINVAL;
     *out = nullptr;
-    tc_options o{TC_BF16, 0, 0.f, nullptr};
+    tc_options o{TC_BF16, 0, 0.f, nullptr, 0};
     if (opt) o = *opt;
     if (H < 1 || H > 4096 || (d != 64 && d != 128) || nbits < 1 || nbits > 24 || !(tau >= -1.f && tau <= 2.f) ||
         capacity < 1 || capacity > (int64_t)1 << 30 || (o.dtype != TC_BF16 && o.dtype != TC_F32) ||
-        !(o.softmax_scale >= 0.f) || !std::isfinite(o.softmax_scale))
+        !(o.softmax_scale >= 0.f) || !std::isfinite(o.softmax_scale) || (o.intra_chunk != 0 && o.intra_chunk != 1))
         return TC_EINVAL;
     if (o.hyperplanes) {
         for (int i = 0; i < nbits * d; ++i)
@@ -326,6 +333,7 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
     x->nbits = nbits;
     x->tau = tau;
     x->dtype = o.dtype;
+    x->intra = o.intra_chunk != 0;
     x->esize = (o.dtype == TC_BF16) ? 2 : 4;
     x->capacity = capacity;
     x->capP = round_up(capacity, 128);
@@ -363,6 +371,7 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
         (st = x->alloc((void**)&c.bnext, rows * 4)) || (st = x->alloc((void**)&c.bhead, ((size_t)H << nbits) * 4)) ||
         (st = x->alloc((void**)&c.knorm64, rows * 8)) || (st = x->alloc((void**)&c.kspan, rows)) || (st = x->alloc((void**)&c.lhead, rows * 4)) ||
         (st = x->alloc((void**)&c.M, (size_t)H * 4)) ||
+        (x->intra && (st = x->alloc((void**)&c.cbhead, ((size_t)H << nbits) * 4))) ||
         (st = x->alloc((void**)&x->ctr, (size_t)kCtrInts(H) * 4)) ||
         (st = x->alloc((void**)&x->stats, sizeof(Stats))) ||
         (st = x->alloc((void**)&x->R, (size_t)nbits * d * 4)) || (st = x->alloc((void**)&x->Rnorm, nbits * 4))) {
@@ -383,7 +392,8 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
         (e = cudaMemset(c.code, 0, rows * 4)) || (e = cudaMemset(c.bnext, 0xff, rows * 4)) ||
         (e = cudaMemset(c.bhead, 0xff, ((size_t)H << nbits) * 4)) || (e = cudaMemset(c.knorm64, 0, rows * 8)) || (e = cudaMemset(c.kspan, 0, rows)) ||
         (e = cudaMemset(c.lhead, 0xff, rows * 4)) ||
-        (e = cudaMemset(c.M, 0, (size_t)H * 4)) || (e = cudaMemset(x->ctr, 0, (size_t)kCtrInts(H) * 4)) ||
+        (e = cudaMemset(c.M, 0, (size_t)H * 4)) ||
+        (x->intra && (e = cudaMemset(c.cbhead, 0xff, ((size_t)H << nbits) * 4))) || (e = cudaMemset(x->ctr, 0, (size_t)kCtrInts(H) * 4)) ||
         (e = cudaMemset(x->stats, 0, sizeof(Stats))) ||
         (e = cudaMemcpy(x->R, x->Rhost.data(), (size_t)nbits * d * 4, cudaMemcpyHostToDevice)) ||
         (e = cudaMemcpy(x->Rnorm, rnorm.data(), nbits * 4, cudaMemcpyHostToDevice))) {

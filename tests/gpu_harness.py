@@ -53,7 +53,7 @@ def compare_state(tc, o, rep: ParityReport, heads):
 
 
 def run_parity(cfg, chunks=None, attends=1, rows=None, state_heads=None, flush=True, device="cuda",
-               check_every_state=True):
+               check_every_state=True, intra_chunk=False):
     """Run `chunks` chunks through both implementations and collect the differences.
 
     rows: query rows checked per attend (None = all). state_heads: heads whose
@@ -64,8 +64,10 @@ def run_parity(cfg, chunks=None, attends=1, rows=None, state_heads=None, flush=T
     chunks = cfg.chunks if chunks is None else chunks
     w = Workload(cfg, device=device)
     R = w.hyperplanes()
-    tc = TempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, dtype=cfg.dtype, hyperplanes=R.numpy())
-    o = OracleTempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, R.double().numpy())
+    tc = TempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, dtype=cfg.dtype, hyperplanes=R.numpy(),
+                   intra_chunk=intra_chunk)
+    o = OracleTempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, R.double().numpy(),
+                        intra_chunk=intra_chunk)
     heads = range(cfg.H) if state_heads is None else state_heads
     rep = ParityReport()
     sum_abs, n_abs = 0.0, 0
