@@ -257,7 +257,7 @@ def run_reference(args):
         return
     cfg = CONFIGS[WORKLOAD]
     R, chunks = generate_inputs(cfg.replace(chunks=args.warmup + args.steps), "cpu", cfg.seed)
-    value, timed, desc = oracle_sample(cfg, cpu_inputs(chunks), R, args.steps, 256, float("inf"),
+    value, timed, desc = oracle_sample(cfg, cpu_inputs(chunks), R, args.steps, 64, float("inf"),
                                        warmup_chunks=args.warmup)
     cores = len(os.sched_getaffinity(0))
     line = {
