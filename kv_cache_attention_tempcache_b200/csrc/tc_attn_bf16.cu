@@ -260,7 +260,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
                        const __grid_constant__ CUtensorMap tmVc, const __grid_constant__ CUtensorMap tmKs,
                        const __grid_constant__ CUtensorMap tmVs, const int32_t* __restrict__ Mdev,
-                       const float* __restrict__ bias2, int64_t capP,
+                       const float* __restrict__ bias2, const float* __restrict__ kmax2c,
+                       const float* __restrict__ kmax2s, const float* __restrict__ bmaxh, int64_t capP,
                        const float* __restrict__ sbias, int64_t Ts, int64_t Tq, int H,
                        __nv_bfloat16* __restrict__ out, float scale_log2, Stats* stats) {
     using C = Cfg<D>;
@@ -417,12 +418,90 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         };
         const uint64_t c2 = pk2(scale_log2, scale_log2);
         float m_run = -INFINITY, l_run = 0.f;   // l_run is relative to m_run
+        // A fixed reference per row: the Cauchy-Schwarz bound of its logits,
+        //   x_j = s_j * scale * log2 e + log2 n_j <= |q| max|k| scale log2 e + max log2 n,
+        // rounded up past the fp32 errors of the norms and of the product. When every row
+        // of the CTA has a bound <= 60, p = 2^(x - m) <= 1 cannot overflow and the largest
+        // p of a row is >= 2^-120 (x_max >= -|q| max|k| scale log2 e), so the tiles need no
+        // max pass, no agreement between threads and no rescaling. Otherwise the CTA runs
+        // the lazy online reference below.
+        bool ok = mbar_wait(&bars[U_QFULL], 0);
+        float q2 = 0.f;
+        {
+            const uint8_t* qrow = sQ + r * 128;
+#pragma unroll 1
+            for (int bx = 0; bx < C::NB; ++bx) {
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const uint4 w4 = *reinterpret_cast<const uint4*>(qrow + bx * C::BOX + ((ch ^ (r & 7)) << 4));
+                    const uint32_t wd[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                    for (int e2 = 0; e2 < 4; ++e2) {
+                        const float lo = __uint_as_float(wd[e2] << 16), hi = __uint_as_float(wd[e2] & 0xffff0000u);
+                        q2 = fmaf(lo, lo, fmaf(hi, hi, q2));
+                    }
+                }
+            }
+        }
+        const float mfix = sqrtf(q2 * fmaxf(kmax2c[h], kmax2s[0])) * scale_log2 * (1.f + 1.f / 256.f) +
+                           bmaxh[h] + 1.f / 256.f;
+        const bool fixed = bar_and(3, 512, ok && mfix <= 60.f);   // uniform over the CTA
+        if (fixed) {
+            m_run = mfix;
+            const uint64_t negm2 = pk2(-mfix, -mfix);
+            auto bias_row = [&](int i) -> const float* {
+                return ((i < nc) ? bias_h + (int64_t)i * kBN : sbias + (int64_t)(i - nc) * kBN) + 64 * g;
+            };
+            if (lane < 2 && t < ntiles) asm volatile("prefetch.global.L1 [%0];" ::"l"(bias_row(t) + 32 * lane));
+            for (int i = t; i < ntiles; i += 2) {
+                const int b = i % 3;
+                const bool got = __all_sync(0xffffffffu, !*abort_flag && mbar_wait(&bars[U_SFULL + b], (i / 3) & 1));
+                if (!got) { ok = false; *abort_flag = 1; break; }
+                tc_fence_after();
+                if (lane < 2 && i + 2 < ntiles)
+                    asm volatile("prefetch.global.L1 [%0];" ::"l"(bias_row(i + 2) + 32 * lane));
+                const uint32_t tS = tmem + b * 128 + 64 * g + lane_base;
+                const float4* brow = reinterpret_cast<const float4*>(bias_row(i));
+                uint64_t sumA = pk2(0.f, 0.f), sumB = pk2(0.f, 0.f);
+#pragma unroll 1
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    uint32_t sr[32];
+                    TC_LD32(tS + 32 * h2, sr);
+                    tc_wait_ld();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4) {
+                        const float4 b4 = __ldg(brow + 8 * h2 + j / 4);
+                        const uint64_t x01 = fma2(pk2(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), c2,
+                                                  add2(pk2(b4.x, b4.y), negm2));
+                        const uint64_t x23 = fma2(pk2(__uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3])), c2,
+                                                  add2(pk2(b4.z, b4.w), negm2));
+                        float a0, a1, a2, a3;
+                        up2(x01, a0, a1);
+                        up2(x23, a2, a3);
+                        const float p0 = ex2(a0), p1 = ex2(a1), p2 = ex2(a2), p3 = ex2(a3);
+                        sumA = add2(sumA, pk2(p0, p1));
+                        sumB = add2(sumB, pk2(p2, p3));
+                        pk[j / 2] = cvt_bf16x2(p0, p1);
+                        pk[j / 2 + 1] = cvt_bf16x2(p2, p3);
+                    }
+                    TC_ST16(tS + 16 * h2, pk);
+                }
+                float s0, s1, s2, s3;
+                up2(sumA, s0, s1);
+                up2(sumB, s2, s3);
+                l_run += (s0 + s1) + (s2 + s3);
+                tc_wait_st();
+                tc_fence_before();
+                mbar_arrive(&bars[U_PFULL + b]);
+            }
+        } else {
         float bnext = 0.f;
         if (g == 0) {
             if (t < ntiles) stage_bias(0, bias_of(t));
             if (t + 2 < ntiles) bnext = bias_of(t + 2);
         }
-        bool ok = bar_and(1 + t, 256, true);
+        ok = bar_and(1 + t, 256, true) && ok;
         int k = 0;
         for (int i = t; i < ntiles; i += 2, ++k) {
             const int b = i % 3, bb = k % 3, u = k & 1;
@@ -524,13 +603,17 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             tc_fence_before();
             mbar_arrive(&bars[U_PFULL + b]);
         }
+        }
         // Epilogue: the last product retires (each commit covers every earlier product of
         // the PV issuer), every row sum moves to the final reference, and thread (t, g, r)
         // writes output columns [QC (2 t + g), QC (2 t + g + 1)) of its row.
         const int lastt = ntiles - 1;
         bool fin = ok && mbar_wait(&bars[U_ODONE + lastt % 3], (lastt / 3) & 1);
-        fin = fin && mbar_wait(&bars[U_MREADY + (lastt & 1)], (lastt >> 1) & 1);
-        const float mfin = sMref[(lastt & 1) * 128 + r];
+        float mfin = mfix;
+        if (!fixed) {
+            fin = fin && mbar_wait(&bars[U_MREADY + (lastt & 1)], (lastt >> 1) & 1);
+            mfin = sMref[(lastt & 1) * 128 + r];
+        }
         const float lfin = (l_run > 0.f) ? l_run * ex2(m_run - mfin) : 0.f;
         sL[(t * 2 + g) * 128 + r] = lfin;
         if (bar_and(3, 512, fin)) {
@@ -591,7 +674,8 @@ cudaError_t launch_t(const CacheView& c, const StageView& s, const AttnMaps& m, 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, attend_bf16_duo_kernel<D>, m.q, m.kc, m.vc, m.ks, m.vs, (const int32_t*)c.M,
-                              (const float*)c.bias2, c.capP, (const float*)s.sbias, s.T, Tq, c.H, out, scale_log2,
+                              (const float*)c.bias2, (const float*)c.kmax2, (const float*)c.kmax2s,
+                              (const float*)c.bmax, c.capP, (const float*)s.sbias, s.T, Tq, c.H, out, scale_log2,
                               stats);
 }
 

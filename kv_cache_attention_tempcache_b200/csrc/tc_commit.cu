@@ -198,6 +198,7 @@ stage_hash_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView c,
     const int64_t stride = (int64_t)gridDim.x * kWarps;
     int nq = 0;                    // rows queued for the bucket-head lookup
     int64_t q_sidx = 0, q_bucket = 0;
+    float kmax = 0.f;              // largest |k|^2 this warp staged
     for (int64_t r0 = (int64_t)blockIdx.x * kWarps + wib; r0 < rows; r0 += ROWS * stride) {
         typename IO::V kv[ROWS], vv[ROWS];
 #pragma unroll
@@ -234,6 +235,7 @@ stage_hash_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView c,
                 v[b] = a;
             }
             nk = warp_sum(nk);
+            kmax = fmaxf(kmax, nk);
             const float p = reduce_scatter<NBP>(v, lane);
             const float err = gam2 * rn * sqrtf(nk) + 1e-30f;
             const bool need = mine && !(fabsf(p) > err);   // inside the band (or not finite)
@@ -269,6 +271,15 @@ stage_hash_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView c,
         }
     }
     if (lane < nq) s.sfirst[q_sidx] = c.bhead[q_bucket];
+    // one bound per block: |k|^2 of the staged keys, rounded up past the fp32 sums' error
+    __shared__ float sKmax[kWarps];
+    if (lane == 0) sKmax[wib] = kmax * (1.f + 1.f / 1024.f);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float m = 0.f;
+        for (int w = 0; w < kWarps; ++w) m = fmaxf(m, sKmax[w]);
+        atomicMax(reinterpret_cast<int*>(c.kmax2s), __float_as_int(m));
+    }
     grid_dependents_launch();
 }
 
@@ -878,6 +889,7 @@ __global__ void __launch_bounds__(kWarps * 32, 3) append_kernel(CacheView c, Sta
         const int nun = __popc(bal);
         const int64_t hrow = (int64_t)h * c.capP;
         const int64_t wrow = (int64_t)h * s.TmaxP + (int64_t)w * 32;
+        float kmax = 0.f;   // largest |k|^2 of the entries this warp creates
         for (int k0 = 0; k0 < nun; k0 += 8) {   // warp-uniform
             G kr[2], vr[2];
             int64_t st[2];
@@ -936,17 +948,22 @@ __global__ void __launch_bounds__(kWarps * 32, 3) append_kernel(CacheView c, Sta
                 int span = 255;
                 if constexpr (sizeof(E) == 2) span = min(gspan_bf16<D>(kr[u], gmask), 255);
                 const double nk = gnorm64(kr[u], span, gl, grp, gmask);
+                kmax = fmaxf(kmax, __double2float_ru(nk));
                 if (gl == 0) {
                     const uint32_t code = s.scode[st[u]];
                     c.knorm64[e] = nk;
                     c.kspan[e] = (uint8_t)span;
                     c.cnt[e] = 1 + members;
                     c.bias2[e] = log2f((float)(1 + members));
+                    if (members) atomicMax(reinterpret_cast<int*>(&c.bmax[h]), __float_as_int(log2f((float)(1 + members))));
                     c.code[e] = code;
                     c.bnext[e] = atomicExch(&c.bhead[((int64_t)h << c.nbits) + code], base + k);
                 }
             }
         }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) kmax = fmaxf(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+        if (lane == 0 && nun > 0) atomicMax(reinterpret_cast<int*>(&c.kmax2[h]), __float_as_int(kmax));
         __syncwarp();
     }
 }
@@ -1032,6 +1049,7 @@ __device__ void merge_long_list(const CacheView& c, const StageView& s, int h, i
         c.cnt[e] = ntot;
         c.bias2[e] = log2f(ft);
         c.lhead[e] = -1;
+        atomicMax(reinterpret_cast<int*>(&c.bmax[h]), __float_as_int(log2f(ft)));   // log2 n >= 0
     }
     __syncwarp();
 }
@@ -1129,6 +1147,7 @@ __global__ void __launch_bounds__(kWarps * 32, 3) merge_kernel(CacheView c, Stag
                     if (gl == 0) {
                         c.cnt[e] = ntot;
                         c.bias2[e] = log2f(ft);
+                        atomicMax(reinterpret_cast<int*>(&c.bmax[h]), __float_as_int(log2f(ft)));   // log2 n >= 0
                     }
                 }
             }

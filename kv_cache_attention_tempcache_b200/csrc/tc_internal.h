@@ -26,6 +26,12 @@ struct CacheView {
     uint8_t* kspan;        // [H][capP] exponent span of each bf16 key (exact-sum rule of the search), <= 255
     int32_t* lhead;        // [H][capP] newest token merging into the entry in this commit (-1 between commits)
     int32_t* M;            // [H] committed entries
+    // Upper bounds for the attention's fixed softmax reference (floats >= 0, raised with
+    // integer atomicMax on their bits): |k|^2 of any committed entry per head, |k|^2 of
+    // any staged token (all heads), log2 n of any committed entry per head.
+    float* kmax2;          // [H]
+    float* kmax2s;         // [1] (cleared before each staging)
+    float* bmax;           // [H]
     int32_t* cbhead;       // [H][2^nbits] newest staged token of each bucket during a commit that matches
                            // inside the chunk (-1 between commits); null when that mode is off
 };

@@ -370,7 +370,8 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
         (st = x->alloc((void**)&c.bias2, rows * 4)) || (st = x->alloc((void**)&c.code, rows * 4)) ||
         (st = x->alloc((void**)&c.bnext, rows * 4)) || (st = x->alloc((void**)&c.bhead, ((size_t)H << nbits) * 4)) ||
         (st = x->alloc((void**)&c.knorm64, rows * 8)) || (st = x->alloc((void**)&c.kspan, rows)) || (st = x->alloc((void**)&c.lhead, rows * 4)) ||
-        (st = x->alloc((void**)&c.M, (size_t)H * 4)) ||
+        (st = x->alloc((void**)&c.M, (size_t)H * 4)) || (st = x->alloc((void**)&c.kmax2, (size_t)H * 4)) ||
+        (st = x->alloc((void**)&c.kmax2s, 4)) || (st = x->alloc((void**)&c.bmax, (size_t)H * 4)) ||
         (x->intra && (st = x->alloc((void**)&c.cbhead, ((size_t)H << nbits) * 4))) ||
         (st = x->alloc((void**)&x->ctr, (size_t)kCtrInts(H) * 4)) ||
         (st = x->alloc((void**)&x->stats, sizeof(Stats))) ||
@@ -392,7 +393,8 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
         (e = cudaMemset(c.code, 0, rows * 4)) || (e = cudaMemset(c.bnext, 0xff, rows * 4)) ||
         (e = cudaMemset(c.bhead, 0xff, ((size_t)H << nbits) * 4)) || (e = cudaMemset(c.knorm64, 0, rows * 8)) || (e = cudaMemset(c.kspan, 0, rows)) ||
         (e = cudaMemset(c.lhead, 0xff, rows * 4)) ||
-        (e = cudaMemset(c.M, 0, (size_t)H * 4)) ||
+        (e = cudaMemset(c.M, 0, (size_t)H * 4)) || (e = cudaMemset(c.kmax2, 0, (size_t)H * 4)) ||
+        (e = cudaMemset(c.kmax2s, 0, 4)) || (e = cudaMemset(c.bmax, 0, (size_t)H * 4)) ||
         (x->intra && (e = cudaMemset(c.cbhead, 0xff, ((size_t)H << nbits) * 4))) || (e = cudaMemset(x->ctr, 0, (size_t)kCtrInts(H) * 4)) ||
         (e = cudaMemset(x->stats, 0, sizeof(Stats))) ||
         (e = cudaMemcpy(x->R, x->Rhost.data(), (size_t)nbits * d * 4, cudaMemcpyHostToDevice)) ||
@@ -430,7 +432,9 @@ tc_status tc_append_chunk(tc_handle x, const void* K, const void* V, int64_t T, 
     if ((st = ensure_staging(x, T))) return st;
     x->s.T = T;
     if ((st = encode_stage_maps(x))) return st;
-    cudaError_t e = launch_stage_hash(x->c, x->s, (int)x->dtype, K, V, x->R, x->Rnorm, x->ctr, x->stats, cs);
+    cudaError_t e = cudaMemsetAsync(x->c.kmax2s, 0, 4, cs);   // the staged keys' bound starts over
+    if (e == cudaSuccess)
+        e = launch_stage_hash(x->c, x->s, (int)x->dtype, K, V, x->R, x->Rnorm, x->ctr, x->stats, cs);
     x->launches += 1;
     if (e != cudaSuccess) return cuda_status(e);
     x->T_staged = T;
@@ -501,6 +505,8 @@ tc_status tc_reset(tc_handle x, tc_stream stream) {
     upto = std::min(round_up(upto, 128), x->capP);
     cudaError_t e = cudaMemsetAsync(x->c.bhead, 0xff, ((size_t)x->H << x->nbits) * 4, cs);
     if (e == cudaSuccess) e = cudaMemsetAsync(x->c.M, 0, (size_t)x->H * 4, cs);
+    if (e == cudaSuccess) e = cudaMemsetAsync(x->c.kmax2, 0, (size_t)x->H * 4, cs);
+    if (e == cudaSuccess) e = cudaMemsetAsync(x->c.bmax, 0, (size_t)x->H * 4, cs);
     if (e == cudaSuccess && upto > 0) {
         dim3 grid((unsigned)std::min<int64_t>((upto + 255) / 256, 64), (unsigned)std::min(x->H, 1024));
         fill_f32<<<grid, 256, 0, cs>>>(x->c.bias2, upto, x->H, x->capP, -INFINITY);
