@@ -216,7 +216,7 @@ __device__ __forceinline__ bool bar_and(int id, int count, bool v) {
 // the halves' reference bounds [2][half][128]; the teams' references [team][128]; the
 // epilogue row sums [4][128].
 enum { U_QFULL = 0, U_KFULL = 1, U_KEMPTY = 4, U_VFULL = 7, U_VEMPTY = 9, U_SFULL = 11, U_PFULL = 14,
-       U_ODONE = 17, U_DRAIN = 20, U_MREADY = 22, U_NBAR = 24 };
+       U_ODONE = 20, U_DRAIN = 23, U_MREADY = 25, U_NBAR = 27 };   // P full: per buffer and half
 template <int D>
 struct CfgU {
     using C = Cfg<D>;
@@ -279,6 +279,7 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     float* sL = reinterpret_cast<float*>(smem + L::OFF_L);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
+    volatile int* sFixed = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 8);   // fixed reference in use
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.y;
@@ -299,7 +300,8 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         }
         for (int b = 0; b < 3; ++b) {
             mbar_init(&bars[U_SFULL + b], 1);
-            mbar_init(&bars[U_PFULL + b], 256);
+            mbar_init(&bars[U_PFULL + 2 * b], 128);
+            mbar_init(&bars[U_PFULL + 2 * b + 1], 128);
             mbar_init(&bars[U_ODONE + b], 1);
         }
         mbar_init(&bars[U_DRAIN], 1);
@@ -377,18 +379,29 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         // ---------------------------------------------------------------- PV issuer
         // O += P_i V_i; keys [16 kk, 16 kk + 16) of P sit at column 128 b + 64 (kk / 4) +
         // 8 (kk % 4): each half's probabilities over its own first S columns.
+        // With the fixed reference the keys of half 0 go in as soon as that half's P is
+        // written; with the online reference a tile may rescale all of O first, so both
+        // halves must be done.
         const uint32_t aV = smem_u32(sV);
-        bool ok = true;
+        bool ok = true, fixed = false;
         for (int i = 0; i < ntiles && !*abort_flag; ++i) {
             const int b = i % 3, st = i % kRV;
-            if (!mbar_wait(&bars[U_PFULL + b], (i / 3) & 1)) { ok = false; break; }
+            if (!mbar_wait(&bars[U_PFULL + 2 * b], (i / 3) & 1)) { ok = false; break; }
+            if (i == 0) fixed = *sFixed != 0;   // written before the first P
+            if (!fixed && !mbar_wait(&bars[U_PFULL + 2 * b + 1], (i / 3) & 1)) { ok = false; break; }
             if (!mbar_wait(&bars[U_VFULL + st], (i / kRV) & 1)) { ok = false; break; }
             tc_fence_after();
             const uint32_t aVs = aV + st * C::TILE;
 #pragma unroll
-            for (int kk = 0; kk < kBN / 16; ++kk)
+            for (int kk = 0; kk < kBN / 16; ++kk) {
+                if (kk == 4 && fixed) {
+                    if (!mbar_wait(&bars[U_PFULL + 2 * b + 1], (i / 3) & 1)) { ok = false; break; }
+                    tc_fence_after();
+                }
                 mma_ts(tO, tmem + b * 128 + 64 * (kk >> 2) + 8 * (kk & 3), sdesc(aVs + kk * 2048, C::BOX, 1024),
                        C::IDESC_PV, (i > 0 || kk > 0));
+            }
+            if (!ok) break;
             tc_commit(&bars[U_VEMPTY + st]);
             tc_commit(&bars[U_ODONE + b]);
         }
@@ -446,6 +459,7 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         const float mfix = sqrtf(q2 * fmaxf(kmax2c[h], kmax2s[0])) * scale_log2 * (1.f + 1.f / 256.f) +
                            bmaxh[h] + 1.f / 256.f;
         const bool fixed = bar_and(3, 512, ok && mfix <= 60.f);   // uniform over the CTA
+        if (threadIdx.x == 0) *sFixed = fixed ? 1 : 0;             // before thread 0's first P
         if (fixed) {
             m_run = mfix;
             const uint64_t negm2 = pk2(-mfix, -mfix);
@@ -493,7 +507,7 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 l_run += (s0 + s1) + (s2 + s3);
                 tc_wait_st();
                 tc_fence_before();
-                mbar_arrive(&bars[U_PFULL + b]);
+                mbar_arrive(&bars[U_PFULL + 2 * b + g]);
             }
         } else {
         float bnext = 0.f;
@@ -601,7 +615,7 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             l_run += (s0 + s1) + (s2 + s3);
             tc_wait_st();
             tc_fence_before();
-            mbar_arrive(&bars[U_PFULL + b]);
+            mbar_arrive(&bars[U_PFULL + 2 * b + g]);
         }
         }
         // Epilogue: the last product retires (each commit covers every earlier product of
