@@ -109,7 +109,10 @@ tc_status tc_append_chunk(tc_handle h, const void* K, const void* V, int64_t T,
  * no mask (section 2.A with Lemma 5.1: averaged values plus a logit shift by the
  * group size reproduce attention over the identical keys they replace).
  * bf16 handles compute QK^T and PV on tensor cores with fp32 accumulation and an
- * fp32 online softmax; fp32 handles compute in fp32 throughout.
+ * fp32 softmax whose reference per query row is a bound of its logits (|q| times
+ * the largest key norm, scaled, plus the largest ln n) when that bound is small
+ * enough to rule out underflow, else a running maximum; fp32 handles compute in
+ * fp32 throughout.
  * Asynchronous on `stream`. Tq >= 1. Returns TC_ESTATE before the first
  * tc_append_chunk. out must not overlap Q.
  */

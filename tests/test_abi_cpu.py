@@ -93,3 +93,22 @@ def test_create_without_device_reports_it(tcmod):
     st = tcmod.lib.tc_create(2, 128, 16, 0.95, 1000, ctypes.byref(h))
     assert st in (tcmod.TC_EDEVICE, tcmod.TC_ECUDA)
     assert not h.value
+
+
+def test_reference_arm_prints_the_contract_line():
+    """bench.py --impl reference runs the CPU oracle and prints one JSON line with the
+    keys the benchmark contract names (no GPU needed)."""
+    import json
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--steps", "1",
+                          "--warmup", "0"], capture_output=True, text=True, timeout=600, cwd=root)
+    assert out.returncode == 0, out.stderr[-2000:]
+    line = json.loads([x for x in out.stdout.splitlines() if x.startswith("{")][-1])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference" and line["value"] > 0
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
