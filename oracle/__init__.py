@@ -16,3 +16,7 @@ from .tempcache_oracle import (  # noqa: F401
     simhash_codes,
     top1_in_bucket,
 )
+from .annca_oracle import (  # noqa: F401
+    annca_cross_attention,
+    kept_prompt_tokens,
+)

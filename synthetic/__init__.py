@@ -11,3 +11,9 @@ from .workload import (  # noqa: F401
     round_to_bf16,
     draw_hyperplanes,
 )
+from .cross import (  # noqa: F401
+    CROSS_CONFIGS,
+    CrossConfig,
+    CrossWorkload,
+    draw_cross_hyperplanes,
+)
