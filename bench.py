@@ -9,6 +9,7 @@ slowest rank's device time. Inputs are generated before timing and stay resident
 in HBM (3.5 GB of distinct K, V, Q per rollout, far larger than the 126 MB L2).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+  python bench.py --workload annca-wan1.3b     (AnnCA cross-attention, its own line)
 
 N > 1 runs under torchrun: each rank runs an independent rollout (its own seed);
 there is no collective in the data path, only the max-over-ranks of the timing.
@@ -33,7 +34,7 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from synthetic import CONFIGS  # noqa: E402
+from synthetic import CONFIGS, CROSS_CONFIGS  # noqa: E402
 
 WORKLOAD = "wan1.3b"
 METRIC = "TempCache frames/s (merge+4x attend) at Wan-1.3B shape; attn TFLOP/s vs peak"
@@ -441,6 +442,141 @@ def run_gpu(args):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- AnnCA leg
+
+ANNCA_METRIC = "AnnCA cross-attention frames/s at Wan-1.3B shape (512 prompt tokens)"
+
+
+def annca_bytes(cfg, kept):
+    """Algorithmic HBM bytes of one tc_annca_attend: the queries read twice (hash, then
+    attention: the kept set of a frame needs all its queries first), the output written
+    once, the query codes written, and every kept key and value row read by the packing
+    kernel, written packed and read by the attention kernel."""
+    q = cfg.T * cfg.H * cfg.d * 2
+    return 2 * q + q + cfg.T * cfg.H * 4 + 3 * kept * cfg.d * 2 * 2
+
+
+def run_annca(args):
+    from kv_cache_attention_tempcache_b200 import AnnCA
+    from synthetic import CrossWorkload
+
+    rank, world, local = dist_info()
+    torch.cuda.set_device(local)
+    init_dist(world, "nccl")
+    dev = torch.device("cuda", local)
+    cfg = CROSS_CONFIGS[args.workload]
+    cfg = cfg.replace(seed=rank_seed(cfg.seed, rank))
+    calls = 40   # one rollout's worth of query blocks (120 frames), 0.6 GB: larger than L2
+    w = CrossWorkload(cfg, device=dev)
+    R = w.hyperplanes().numpy()
+    Kp, Vp = w.prompt()
+    Qs = [w.queries(c) for c in range(calls)]
+    outs = [torch.empty_like(Qs[0]) for _ in range(2)]
+    ann = AnnCA(cfg.H, cfg.d, cfg.nbits, hyperplanes=R)
+    ann.set_prompt(Kp, Vp)
+    kept = []
+    for c in range(calls):
+        ann.attend(Qs[c], cfg.P, out=outs[0])
+        kept.append(int(ann.kept()[0].sum()))
+
+    def step():
+        for c in range(calls):
+            ann.attend(Qs[c], cfg.P, out=outs[c & 1])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0, t1 = ev(), ev()
+    t0.record()
+    for _ in range(args.steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    sec = t0.elapsed_time(t1) / 1000.0
+    sec_max = max_over_ranks(sec, world, dev)
+    value = aggregate_rate(cfg.F * calls * args.steps, world, sec_max)
+    call_sec = sec / (args.steps * calls)
+    nbytes = float(np.mean([annca_bytes(cfg, k) for k in kept]))
+    peaks, peak_kind = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+
+    # every prompt token kept (1-bit hash, both buckets present): the same kernels
+    # over the whole prompt
+    dense = AnnCA(cfg.H, cfg.d, 1, hyperplanes=R[:1])
+    dense.set_prompt(Kp, Vp)
+    for c in range(calls):
+        dense.attend(Qs[c], cfg.P, out=outs[c & 1])
+    dense_kept = dense.kept()[0].mean()
+    torch.cuda.synchronize()
+    d0, d1 = ev(), ev()
+    d0.record()
+    for c in range(calls):
+        dense.attend(Qs[c], cfg.P, out=outs[c & 1])
+    d1.record()
+    torch.cuda.synchronize()
+    dense_sec = d0.elapsed_time(d1) / 1000.0
+    dense.close()
+
+    # end to end: queries from pinned host memory, outputs read back, per call
+    host_q = [q.cpu().pin_memory() for q in Qs]
+    host_o = torch.empty(cfg.T, cfg.H, cfg.d, dtype=torch.bfloat16).pin_memory()
+    e0, e1 = ev(), ev()
+    e0.record()
+    for c in range(calls):
+        host_o.copy_(ann.attend(host_q[c], cfg.P), non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_sec = max_over_ranks(e0.elapsed_time(e1) / 1000.0, world, dev)
+    qb = cfg.T * cfg.H * cfg.d * 2
+
+    if rank != 0:
+        ann.close()
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        from oracle import annca_cross_attention
+        f = lambda x: x.to(torch.float64).cpu().numpy()  # noqa: E731
+        Kn, Vn, Qn = f(Kp), f(Vp), f(Qs[0])
+        t = time.perf_counter()
+        annca_cross_attention(Qn, Kn, Vn, R.astype(np.float64), cfg.P)
+        tcpu = time.perf_counter() - t
+        cpu = {"value": cfg.F / tcpu, "unit": UNIT, "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+               "sample": "one query block (3 frames x 1560 tokens, 12 heads) in full"}
+    line = {
+        "metric": ANNCA_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * sec_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": (f"{cfg.name}: H={cfg.H} d={cfg.d} P={cfg.P} F={cfg.F} L={cfg.L} C={cfg.C} "
+                                f"A={cfg.A} sigma={cfg.sigma} nbits={cfg.nbits} bf16"),
+                   "step": f"{calls} tc_annca_attend calls ({cfg.F * calls} frames), prompt set once before",
+                   "l2": f"inputs larger than L2 ({calls * qb / 1e9:.2f} GB of distinct queries per step)",
+                   "parallelism": f"independent layer per rank x{world}"},
+        "roofline": {"bound": "hbm", "kernel": "annca_mark_kernel + annca_pack_kernel + attend_bf16_duo_kernel "
+                                                "(cross), one call",
+                     "achieved": nbytes / call_sec / 1e9, "peak": hbm, "unit": "GB/s",
+                     "frac": nbytes / call_sec / 1e9 / hbm, "peak_kind": f"{peak_kind} copy bandwidth",
+                     "traffic": None, "bytes_per_call": nbytes, "avg_call_us": 1e6 * call_sec},
+        "kept_fraction": float(np.mean(kept)) / (cfg.H * cfg.F * cfg.L),
+        "dense_baseline": {"value": cfg.F * calls / dense_sec, "unit": UNIT, "kept_fraction": float(dense_kept),
+                           "note": "same kernels with a 1-bit hash: every prompt token kept"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": aggregate_rate(cfg.F * calls, world, e2e_sec), "unit": UNIT,
+                "h2d_bytes_per_step": calls * qb, "d2h_bytes_per_step": calls * qb},
+        "gpu_launches": 3 * calls * args.steps,
+        "clocks": clk,
+    }
+    ann.close()
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -452,14 +588,18 @@ def main():
                     help="timed rollouts only (no dense baseline, end-to-end or CPU legs), for profilers")
     ap.add_argument("--chunks", type=int, default=0,
                     help="rollout length in chunks (default: the workload's); profiling runs use fewer")
-    ap.add_argument("--workload", default=WORKLOAD, choices=[k for k, v in CONFIGS.items() if v.dtype == "bf16"],
-                    help="synthetic workload; only the default one adds the dense, end-to-end and CPU legs")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    choices=[k for k, v in CONFIGS.items() if v.dtype == "bf16"] + ["annca-wan1.3b"],
+                    help="synthetic workload; only the default one adds the dense, end-to-end and CPU legs "
+                         "(annca-wan1.3b: AnnCA cross-attention, with its own legs)")
     ap.add_argument("--series", action="store_true", help="add per-chunk commit and attention times")
     ap.add_argument("--intra-chunk", action="store_true",
                     help="commits also match tokens against entries created earlier in the same commit")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.workload in CROSS_CONFIGS:
+        run_annca(args)
     else:
         run_gpu(args)
     if torch.distributed.is_initialized():

@@ -97,7 +97,7 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
  * capacity: then the call synchronises to learn the outcome and, if the commit
  * would overflow, returns TC_ECAPACITY with the cache unchanged, the previous
  * chunk still staged and this chunk not accepted.
- * T >= 1. Returns TC_EINVAL for NULL or misaligned K or V.
+ * T >= 1 and T * H < 2^31. Returns TC_EINVAL for NULL or misaligned K or V.
  */
 tc_status tc_append_chunk(tc_handle h, const void* K, const void* V, int64_t T,
                           tc_stream stream);
@@ -197,6 +197,76 @@ tc_status tc_stats(tc_handle h, uint64_t* kernel_launches, uint64_t* hash_rechec
 tc_status tc_merge_means_noalloc(const void* src, tc_dtype src_dtype, const int32_t* target,
                                  int32_t n_src, int32_t d, float* mean, int32_t* count,
                                  int32_t n_dst, tc_stream stream);
+
+/* ---- AnnCA: cross-attention over the prompt tokens a frame shares buckets with -- */
+
+/*
+ * AnnCA (FAST-AR technical summary, section 2.B "AnnCA", pt and fr pages): the
+ * latent queries of a frame and the prompt keys are hashed into one space; a prompt
+ * token is kept for the frame when its bucket holds at least one of the frame's
+ * queries, and the frame's cross-attention runs over the kept tokens only. Here
+ * the hash is the sign of nbits random hyperplanes (the TempCache hash, with the
+ * cross-attention layer's own normals, shared by the heads), buckets are exact
+ * codes, and the kept set is decided per frame and per head. A frame whose queries
+ * share no bucket with the prompt gets zero output rows (the empty sum).
+ * Same conventions as above; bf16 only.
+ */
+typedef struct tc_annca_ctx* tc_annca_handle;
+
+/*
+ * tc_annca_create - a cross-attention layer with H heads of dimension d (64 or
+ * 128) and nbits hash bits (1..24). opt may be NULL (seed 0, scale 1/sqrt(d));
+ * opt->dtype must be TC_BF16 (TC_F32 returns TC_ENOTIMPL) and opt->intra_chunk 0.
+ * Allocates nothing until the prompt is set. *out is NULL on failure.
+ */
+tc_status tc_annca_create(int32_t H, int32_t d, int32_t nbits, const tc_options* opt,
+                          tc_annca_handle* out);
+
+/*
+ * tc_annca_set_prompt - the prompt keys and values, Kp and Vp DEVICE [L, H, d]
+ * bf16, 1 <= L <= 4096. The library copies them into its own memory, hashes the
+ * keys and sorts their codes, all on `stream`; the caller may free Kp and Vp once
+ * that work has run. Growing L past the largest earlier value reallocates (and
+ * synchronises first).
+ */
+tc_status tc_annca_set_prompt(tc_annca_handle h, const void* Kp, const void* Vp, int32_t L,
+                              tc_stream stream);
+
+/*
+ * tc_annca_attend - cross-attention of the query block Q DEVICE [Tq, H, d] bf16,
+ * Tq = F P: F frames of P consecutive tokens (frame f is rows f P .. f P + P - 1).
+ * For frame f and head h the kept tokens are the prompt tokens whose code equals
+ * the code of at least one query of that frame and head; then
+ *   out_t = sum_{l kept} exp(scale <q_t, k_l>) v_l / sum_{l kept} exp(scale <q_t, k_l>)
+ * on tensor cores (bf16 products, fp32 accumulation and softmax), and zero rows
+ * where nothing is kept. Writes out DEVICE [Tq, H, d] bf16, which must not overlap
+ * Q. Asynchronous on `stream`: one hash-and-mark kernel, one packing kernel and the
+ * attention kernel. Returns TC_ESTATE before a prompt is set and TC_EINVAL unless
+ * P >= 1, Tq is a positive multiple of P and Tq * H < 2^31. Growing Tq or F past the largest
+ * earlier value reallocates (and synchronises first).
+ */
+tc_status tc_annca_attend(tc_annca_handle h, const void* Q, int64_t Tq, int32_t P, void* out,
+                          tc_stream stream);
+
+/*
+ * tc_annca_kept - inspection of the last tc_annca_attend (HOST buffers; synchronises).
+ * *T_out receives its Tq, *F_out its F and *L_out the prompt length (0 before any). counts [H*F]: kept tokens of slot
+ * h F + f; index [H*F*L]: slot z's kept prompt tokens in ascending order in
+ * index[z*L .. z*L + counts[z]) (the rest unspecified); qcodes [H*Tq] head-major
+ * query codes; pcodes [H*L] prompt codes. Any array pointer may be NULL.
+ */
+tc_status tc_annca_kept(tc_annca_handle h, int64_t* T_out, int64_t* F_out, int32_t* L_out,
+                        int32_t* counts, int32_t* index, uint32_t* qcodes, uint32_t* pcodes);
+
+/* tc_annca_get_hyperplanes - the hash normals in use, HOST [nbits * d]. */
+tc_status tc_annca_get_hyperplanes(tc_annca_handle h, float* R);
+
+/* tc_annca_sync - synchronise the handle's last stream and return its sticky status
+ * (TC_ETIMEOUT if an attention kernel gave up on one of its barriers). */
+tc_status tc_annca_sync(tc_annca_handle h);
+
+/* tc_annca_destroy - free every buffer of the handle. NULL-safe. Synchronises. */
+void tc_annca_destroy(tc_annca_handle h);
 
 #ifdef __cplusplus
 }

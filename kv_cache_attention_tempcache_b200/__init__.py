@@ -29,6 +29,8 @@ API = [
     "tc_create", "tc_create_ex", "tc_append_chunk", "tc_attend", "tc_flush", "tc_reset", "tc_cache_size", "tc_sync",
     "tc_destroy", "tc_status_string", "tc_debug_last_commit", "tc_debug_staged_codes", "tc_export_cache",
     "tc_get_hyperplanes", "tc_stats", "tc_merge_means_noalloc",
+    "tc_annca_create", "tc_annca_set_prompt", "tc_annca_attend", "tc_annca_kept", "tc_annca_get_hyperplanes",
+    "tc_annca_sync", "tc_annca_destroy",
 ]
 
 
@@ -62,6 +64,14 @@ def _load():
         "tc_stats": (ctypes.c_int, [H, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64),
                                     ctypes.POINTER(ctypes.c_uint64)]),
         "tc_merge_means_noalloc": (ctypes.c_int, [vp, ctypes.c_int, vp, i32, i32, vp, vp, i32, vp]),
+        "tc_annca_create": (ctypes.c_int, [i32, i32, i32, ctypes.POINTER(TCOptions), ctypes.POINTER(H)]),
+        "tc_annca_set_prompt": (ctypes.c_int, [H, vp, vp, i32, vp]),
+        "tc_annca_attend": (ctypes.c_int, [H, vp, i64, i32, vp, vp]),
+        "tc_annca_kept": (ctypes.c_int, [H, ctypes.POINTER(i64), ctypes.POINTER(i64), ctypes.POINTER(i32), vp, vp,
+                                          vp, vp]),
+        "tc_annca_get_hyperplanes": (ctypes.c_int, [H, vp]),
+        "tc_annca_sync": (ctypes.c_int, [H]),
+        "tc_annca_destroy": (None, [H]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -225,6 +235,97 @@ class TempCache:
     def close(self):
         if getattr(self, "_h", None) is not None and self._h.value:
             lib.tc_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class AnnCA:
+    """AnnCA cross-attention of one layer on the current CUDA device (bf16).
+
+    FAST-AR summary, section 2.B: for every frame of a query block, only the prompt
+    tokens that share a hash bucket with one of the frame's queries take part in the
+    frame's cross-attention. Kp, Vp are [L, H, d] and Q is [F*P, H, d] torch.bfloat16
+    tensors; CPU tensors are copied to the device on the current stream first.
+    """
+
+    def __init__(self, H: int, d: int, nbits: int, seed: int = 0, softmax_scale: float = 0.0, hyperplanes=None):
+        self.H, self.d, self.nbits = int(H), int(d), int(nbits)
+        opt = TCOptions()
+        opt.dtype = TC_BF16
+        opt.seed = int(seed)
+        opt.softmax_scale = float(softmax_scale)
+        opt.intra_chunk = 0
+        self._R = None
+        if hyperplanes is not None:
+            self._R = np.ascontiguousarray(np.asarray(hyperplanes, dtype=np.float32).reshape(-1))
+            opt.hyperplanes = self._R.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
+        self._h = ctypes.c_void_p()
+        _check(lib.tc_annca_create(self.H, self.d, self.nbits, ctypes.byref(opt), ctypes.byref(self._h)),
+               "tc_annca_create")
+        self._keep = []
+
+    def _dev(self, x: torch.Tensor, name: str) -> torch.Tensor:
+        if x.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be torch.bfloat16, got {x.dtype}")
+        if x.dim() != 3 or x.shape[1] != self.H or x.shape[2] != self.d:
+            raise ValueError(f"{name} must be [n, {self.H}, {self.d}], got {tuple(x.shape)}")
+        if not x.is_cuda:
+            x = x.to("cuda", non_blocking=True)
+        return x.contiguous()
+
+    def set_prompt(self, Kp: torch.Tensor, Vp: torch.Tensor):
+        Kp = self._dev(Kp, "Kp")
+        Vp = self._dev(Vp, "Vp")
+        if Kp.shape != Vp.shape:
+            raise ValueError("Kp and Vp shapes differ")
+        self._keep = [Kp, Vp]
+        _check(lib.tc_annca_set_prompt(self._h, Kp.data_ptr(), Vp.data_ptr(), Kp.shape[0], TempCache._stream()),
+               "tc_annca_set_prompt")
+
+    def attend(self, Q: torch.Tensor, P: int, out: torch.Tensor | None = None) -> torch.Tensor:
+        Q = self._dev(Q, "Q")
+        if out is None:
+            out = torch.empty_like(Q)
+        _check(lib.tc_annca_attend(self._h, Q.data_ptr(), Q.shape[0], int(P), out.data_ptr(), TempCache._stream()),
+               "tc_annca_attend")
+        return out
+
+    def kept(self):
+        """Inspection of the last attend: (keep [H, F, L] bool, query codes [H, T], prompt codes [H, L])."""
+        T, F, L = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int32()
+        _check(lib.tc_annca_kept(self._h, ctypes.byref(T), ctypes.byref(F), ctypes.byref(L), None, None, None, None),
+               "tc_annca_kept")
+        T, F, L = T.value, F.value, L.value
+        counts = np.zeros(self.H * F, np.int32)
+        index = np.zeros(self.H * F * L, np.int32)
+        qcodes = np.zeros((self.H, T), np.uint32)
+        pcodes = np.zeros((self.H, L), np.uint32)
+        _check(lib.tc_annca_kept(self._h, None, None, None, _np_ptr(counts), _np_ptr(index), _np_ptr(qcodes),
+                                 _np_ptr(pcodes)), "tc_annca_kept")
+        keep = np.zeros((self.H, F, L), bool)
+        for z in range(self.H * F):
+            ids = index[z * L: z * L + counts[z]]
+            if counts[z] > 1 and not np.all(np.diff(ids) > 0):
+                raise TempCacheError(TC_ESTATE, "tc_annca_kept: kept list not ascending")
+            keep[z // F, z % F, ids] = True
+        return keep, qcodes, pcodes
+
+    def hyperplanes(self) -> np.ndarray:
+        R = np.zeros((self.nbits, self.d), np.float32)
+        _check(lib.tc_annca_get_hyperplanes(self._h, _np_ptr(R)), "tc_annca_get_hyperplanes")
+        return R
+
+    def sync(self):
+        _check(lib.tc_annca_sync(self._h), "tc_annca_sync")
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            lib.tc_annca_destroy(self._h)
             self._h = ctypes.c_void_p()
 
     def __del__(self):

@@ -1,0 +1,716 @@
+// AnnCA cross-attention: keep, per frame and head, the prompt tokens whose hash
+// bucket holds at least one of the frame's queries, then attend over those only.
+//
+// FAST-AR technical summary, section 2.B "AnnCA": latent queries and prompt keys are
+// projected into one hashed space, prompt tokens without a bucket shared with the
+// current frame's queries are pruned for that frame, and cross-attention skips them.
+//
+// Kernels:
+//   annca_prompt_kernel   once per prompt: copy Kp, Vp head-major, hash every key,
+//                         bound |k|^2 per head.
+//   annca_sort_kernel     once per prompt: sort each head's (code, token) pairs; every
+//                         prompt token learns where its code's run starts.
+//   annca_mark_kernel     per call: hash every query (four rows in flight per warp); each
+//                         lane of a warp then looks one query's code up (a table of the
+//                         head's codes for nbits <= 16, else a binary search of its sorted
+//                         codes) and, if the prompt has that code, stamps the bucket with
+//                         the call's number for the query's frame (written only while the
+//                         stamp differs, so the many queries of one bucket rarely store).
+//   annca_pack_kernel     per call: a few blocks per (head, frame) list the prompt tokens
+//                         whose bucket carries this call's stamp, in ascending order, and
+//                         pack their keys and values into 128-row tiles for the attention
+//                         kernel (zero rows and a -inf logit shift past the last kept
+//                         token). Stamps are never cleared: the next call has a new number.
+//   attention             the tcgen05 flash-attention kernel of tc_attn_bf16.cu in its
+//                         cross mode: the keys of a CTA are the packed tokens of its slot.
+// Hash bits are exact as in the TempCache staging kernel: the fp32 sign is kept only
+// outside its rounding bound, else the bit is recomputed as an fp64 sum in index order.
+#include "../../include/tempcache.h"
+#include "tc_internal.h"
+#include "tc_device.cuh"
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <vector>
+
+namespace tc {
+
+namespace {
+
+constexpr int kMaxPrompt = 4096;   // prompt tokens (the sort runs in one block's shared memory)
+
+// Code of the bf16 row x held by the warp (lane l: elements [l EPL, l EPL + EPL)),
+// with the normals' bf16 pairs in Rp and |R_b| (rounded up) in rn on lane b. Returns
+// the code on every lane; nk receives the fp32 |x|^2 and nre the re-checked bits.
+template <int D, int NBP>
+__device__ __forceinline__ unsigned hash_row(const float (&x)[D / 32], const uint32_t (&Rp)[NBP][D / 64],
+                                             const float* __restrict__ R, float rn, int nbits, float* sRow,
+                                             int lane, float& nk, unsigned& nre) {
+    constexpr int EPL = D / 32;
+    float n2 = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) n2 = fmaf(x[e], x[e], n2);
+    float v[NBP];
+#pragma unroll
+    for (int b = 0; b < NBP; ++b) {
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL / 2; ++e) {
+            a = fmaf(__uint_as_float(Rp[b][e] << 16), x[2 * e], a);
+            a = fmaf(__uint_as_float(Rp[b][e] & 0xffff0000u), x[2 * e + 1], a);
+        }
+        v[b] = a;
+    }
+    n2 = warp_sum(n2);
+    const float p = reduce_scatter<NBP>(v, lane);
+    const bool mine = lane < nbits;
+    // |<R_b,x>| > 2 (d+2) u |R_b||x| certifies the fp32 sign (any summation order errs
+    // by at most (d+2) u |R_b||x|; doubled for margin)
+    const float err = 2.f * (float)(D + 2) * kU32 * rn * sqrtf(n2) + 1e-30f;
+    const bool need = mine && !(fabsf(p) > err);
+    bool bit = p >= 0.f;
+    if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) sRow[lane * EPL + e] = x[e];
+        __syncwarp();
+        if (need) {
+            double acc = 0.0;
+            const float* rb = R + lane * D;
+            for (int i = 0; i < D; ++i) acc = fma((double)rb[i], (double)sRow[i], acc);
+            bit = acc >= 0.0;
+        }
+        __syncwarp();
+    }
+    nk = n2;
+    nre = __popc(__ballot_sync(0xffffffffu, need));
+    const unsigned mask = (nbits >= 32) ? 0xffffffffu : ((1u << nbits) - 1u);
+    return __ballot_sync(0xffffffffu, mine && bit) & mask;
+}
+
+template <int D, int NBP>
+__device__ __forceinline__ void load_planes(const float* __restrict__ R, int nbits, int lane,
+                                            uint32_t (&Rp)[NBP][D / 64]) {
+    constexpr int EPL = D / 32;
+#pragma unroll
+    for (int b = 0; b < NBP; ++b)
+#pragma unroll
+        for (int e = 0; e < EPL / 2; ++e)
+            Rp[b][e] = (b < nbits) ? pack_bf16_exact(R[b * D + lane * EPL + 2 * e], R[b * D + lane * EPL + 2 * e + 1])
+                                   : 0u;
+}
+
+// One warp per prompt row r = l H + h.
+template <int D, int NBP>
+__global__ void __launch_bounds__(kWarps * 32) annca_prompt_kernel(const __nv_bfloat16* __restrict__ Kp,
+                                                                   const __nv_bfloat16* __restrict__ Vp, AnnView a,
+                                                                   const float* __restrict__ R,
+                                                                   const float* __restrict__ Rnorm, Stats* stats) {
+    constexpr int EPL = D / 32;
+    using IO = RowIO<__nv_bfloat16, EPL>;
+    __shared__ float sRow[kWarps][D];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    uint32_t Rp[NBP][D / 64];
+    load_planes<D, NBP>(R, a.nbits, lane, Rp);
+    const float rn = lane < a.nbits ? Rnorm[lane] : 0.f;
+    const int64_t rows = (int64_t)a.L * a.H;
+    for (int64_t r = (int64_t)blockIdx.x * kWarps + wib; r < rows; r += (int64_t)gridDim.x * kWarps) {
+        const int l = (int)((uint32_t)r / (uint32_t)a.H), h = (int)(r - (int64_t)l * a.H);
+        const typename IO::V kv = IO::load(Kp + r * D, lane);
+        const typename IO::V vv = IO::load(Vp + r * D, lane);
+        const int64_t dst = (int64_t)h * a.Lp + l;
+        IO::store(a.Kh + dst * D, lane, kv);
+        IO::store(a.Vh + dst * D, lane, vv);
+        float x[EPL];
+        IO::to_float(kv, x);
+        float nk;
+        unsigned nre;
+        const unsigned code = hash_row<D, NBP>(x, Rp, R, rn, a.nbits, sRow[wib], lane, nk, nre);
+        if (lane == 0) {
+            a.pcode[dst] = code;
+            // |k|^2 rounded up past the fp32 sum's error; floats >= 0 order like their bits
+            atomicMax(reinterpret_cast<int*>(a.kmax2 + h), __float_as_int(nk * (1.f + 1.f / 1024.f)));
+            if (nre) atomicAdd(&stats->hash_rechecks, (unsigned long long)nre);
+        }
+    }
+}
+
+// One block per head: bitonic sort of the (code, token) pairs in shared memory.
+__global__ void __launch_bounds__(1024) annca_sort_kernel(AnnView a) {
+    __shared__ unsigned long long key[kMaxPrompt];
+    const int h = blockIdx.x;
+    int n = 1;
+    while (n < a.L) n <<= 1;
+    for (int i = threadIdx.x; i < n; i += blockDim.x)
+        key[i] = (i < a.L) ? ((unsigned long long)a.pcode[(int64_t)h * a.Lp + i] << 32) | (unsigned)i : ~0ull;
+    __syncthreads();
+    for (int k = 2; k <= n; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = threadIdx.x; i < n; i += blockDim.x) {
+                const int p = i ^ j;
+                if (p > i) {
+                    const unsigned long long u = key[i], w = key[p];
+                    if ((u > w) == ((i & k) == 0)) {
+                        key[i] = w;
+                        key[p] = u;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int i = threadIdx.x; i < a.L; i += blockDim.x) {
+        const uint32_t c = (uint32_t)(key[i] >> 32);
+        const int32_t l = (int32_t)(key[i] & 0xffffffffu);
+        int lo = 0, hi = i;   // first sorted position of code c
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if ((uint32_t)(key[mid] >> 32) < c) lo = mid + 1;
+            else hi = mid;
+        }
+        a.pcs[(int64_t)h * a.Lp + i] = c;
+        a.pix[(int64_t)h * a.Lp + i] = l;
+        a.prun[(int64_t)h * a.Lp + l] = lo;
+        if (a.ptab && lo == i) a.ptab[((int64_t)h << a.nbits) + c] = i;   // (cleared to -1 by the host)
+    }
+}
+
+// Stamps the prompt bucket `code` of head h for slot z, if the prompt has that code.
+// Many queries of a frame share a code: the stamp is only written while it reads
+// different (a stale read just repeats the store).
+__device__ __forceinline__ void flag_bucket(const AnnView& a, int h, int64_t z, uint32_t code) {
+    int lo;
+    if (a.ptab) {
+        lo = a.ptab[((int64_t)h << a.nbits) + code];
+    } else {
+        const uint32_t* cs = a.pcs + (int64_t)h * a.Lp;
+        int hi = a.L;   // first sorted position with code >= `code`
+        lo = 0;
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if (cs[mid] < code) lo = mid + 1;
+            else hi = mid;
+        }
+        if (lo >= a.L || cs[lo] != code) lo = -1;
+    }
+    if (lo >= 0) {
+        uint32_t* f = a.keep + z * a.Lp + lo;
+        if (*f != a.gen) *f = a.gen;
+    }
+}
+
+constexpr int kMarkRows = 4;   // rows a warp of the mark kernel loads before hashing them
+
+// One warp per query row r = t H + h; the lookups of up to 32 rows are batched, one
+// row per lane, so their dependent loads overlap.
+template <int D, int NBP>
+__global__ void __launch_bounds__(kWarps * 32, NBP <= 16 ? 2 : 1)
+annca_mark_kernel(const __nv_bfloat16* __restrict__ Q, int64_t Tq, int P, int F, AnnView a,
+                  const float* __restrict__ R, const float* __restrict__ Rnorm, Stats* stats) {
+    grid_dependency_wait();
+    constexpr int EPL = D / 32;
+    using IO = RowIO<__nv_bfloat16, EPL>;
+    __shared__ float sRow[kWarps][D];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    uint32_t Rp[NBP][D / 64];
+    load_planes<D, NBP>(R, a.nbits, lane, Rp);
+    const float rn = lane < a.nbits ? Rnorm[lane] : 0.f;
+    const int64_t rows = Tq * a.H;
+    const int64_t stride = (int64_t)gridDim.x * kWarps;
+    int nq = 0, q_h = 0;
+    int64_t q_z = 0;
+    uint32_t q_code = 0;
+    unsigned rechecks = 0;
+    for (int64_t r0 = (int64_t)blockIdx.x * kWarps + wib; r0 < rows; r0 += kMarkRows * stride) {
+        typename IO::V raw[kMarkRows];
+#pragma unroll
+        for (int k = 0; k < kMarkRows; ++k)
+            if (r0 + k * stride < rows) raw[k] = IO::load(Q + (r0 + k * stride) * D, lane);
+#pragma unroll
+        for (int k = 0; k < kMarkRows; ++k) {
+            const int64_t r = r0 + k * stride;
+            if (r >= rows) break;   // warp-uniform
+            const int t = (int)((uint32_t)r / (uint32_t)a.H);   // rows < 2^31 (host check)
+            const int h = (int)(r - (int64_t)t * a.H);
+            float x[EPL];
+            IO::to_float(raw[k], x);
+            float nk;
+            unsigned nre;
+            const unsigned code = hash_row<D, NBP>(x, Rp, R, rn, a.nbits, sRow[wib], lane, nk, nre);
+            rechecks += nre;
+            if (lane == 0) a.qcode[(int64_t)h * a.Tmax + t] = code;
+            if (lane == nq) {
+                q_h = h;
+                q_z = (int64_t)h * F + (int)((uint32_t)t / (uint32_t)P);
+                q_code = code;
+            }
+            if (++nq == 32) {
+                flag_bucket(a, q_h, q_z, q_code);
+                nq = 0;
+            }
+        }
+    }
+    if (lane < nq) flag_bucket(a, q_h, q_z, q_code);
+    if (lane == 0 && rechecks) atomicAdd(&stats->hash_rechecks, (unsigned long long)rechecks);
+    grid_dependents_launch();
+}
+
+// Exclusive scan of one value per thread over the block (blockDim.x <= 1024).
+__device__ int block_exclusive_scan(int v, int* total) {
+    __shared__ int wsum[32];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+    int inc = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+    }
+    if (lane == 31) wsum[w] = inc;
+    __syncthreads();
+    if (w == 0) {
+        int y = (lane < nw) ? wsum[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int s = __shfl_up_sync(0xffffffffu, y, o);
+            if (lane >= o) y += s;
+        }
+        wsum[lane] = y;
+    }
+    __syncthreads();
+    const int before = (w > 0) ? wsum[w - 1] : 0;
+    *total = wsum[nw - 1];
+    __syncthreads();
+    return before + inc - v;
+}
+
+// Blocks (z, part) for slot z = h F + f: every part lists the kept tokens (the list is
+// short), part 0 publishes it with the count and the logit shifts, and each part packs
+// its share of the rows.
+constexpr int kPackParts = 4;
+
+template <int D>
+__global__ void __launch_bounds__(256) annca_pack_kernel(int F, AnnView a) {
+    grid_dependency_wait();
+    constexpr int W = D / 8;   // 16-byte words per row
+    __shared__ int32_t sList[kMaxPrompt];
+    const int64_t z = blockIdx.x;
+    const int part = blockIdx.y;
+    const int h = (int)(z / F);
+    const uint32_t* stamp = a.keep + z * a.Lp;
+    const int32_t* run = a.prun + (int64_t)h * a.Lp;
+    const int per = (a.L + blockDim.x - 1) / blockDim.x;
+    const int l0 = min(a.L, (int)threadIdx.x * per), l1 = min(a.L, l0 + per);
+    int c = 0;
+    for (int l = l0; l < l1; ++l) c += stamp[run[l]] == a.gen;
+    int n = 0;
+    int pos = block_exclusive_scan(c, &n);
+    for (int l = l0; l < l1; ++l)
+        if (stamp[run[l]] == a.gen) sList[pos++] = l;
+    __syncthreads();
+    const int nt = (n + 127) & ~127;
+    if (part == 0) {
+        for (int j = threadIdx.x; j < n; j += blockDim.x) a.sidx[z * a.Lp + j] = sList[j];
+        for (int j = threadIdx.x; j < nt; j += blockDim.x) a.sbias[z * a.Lp + j] = (j < n) ? 0.f : -INFINITY;
+        if (threadIdx.x == 0) a.nsel[z] = n;
+    }
+    const int share = (nt / 32 + gridDim.y - 1) / gridDim.y * 32;   // rows per part, whole warps of rows
+    const int j0 = min(nt, part * share), j1 = min(nt, j0 + share);
+    const uint4* Kh = reinterpret_cast<const uint4*>(a.Kh + (int64_t)h * a.Lp * D);
+    const uint4* Vh = reinterpret_cast<const uint4*>(a.Vh + (int64_t)h * a.Lp * D);
+    uint4* Ks = reinterpret_cast<uint4*>(a.Ks + z * a.Lp * D);
+    uint4* Vs = reinterpret_cast<uint4*>(a.Vs + z * a.Lp * D);
+    for (int i = j0 * W + threadIdx.x; i < j1 * W; i += blockDim.x) {
+        const int j = i / W, w = i - j * W;
+        uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = kv;
+        if (j < n) {
+            const int64_t l = sList[j];
+            kv = Kh[l * W + w];
+            vv = Vh[l * W + w];
+        }
+        Ks[(int64_t)j * W + w] = kv;
+        Vs[(int64_t)j * W + w] = vv;
+    }
+    grid_dependents_launch();
+}
+
+template <int D>
+cudaError_t prompt_t(const AnnView& a, const void* Kp, const void* Vp, const float* R, const float* Rnorm,
+                     Stats* stats, cudaStream_t st) {
+    const int grid = grid_for_rows((int64_t)a.L * a.H, kWarps, 148 * 8);
+    const auto* K = reinterpret_cast<const __nv_bfloat16*>(Kp);
+    const auto* V = reinterpret_cast<const __nv_bfloat16*>(Vp);
+    if (a.nbits <= 8) annca_prompt_kernel<D, 8><<<grid, kWarps * 32, 0, st>>>(K, V, a, R, Rnorm, stats);
+    else if (a.nbits <= 16) annca_prompt_kernel<D, 16><<<grid, kWarps * 32, 0, st>>>(K, V, a, R, Rnorm, stats);
+    else annca_prompt_kernel<D, 32><<<grid, kWarps * 32, 0, st>>>(K, V, a, R, Rnorm, stats);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    annca_sort_kernel<<<a.H, 1024, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t select_t(const AnnView& a, const void* Qv, int64_t Tq, int P, int F, const float* R,
+                     const float* Rnorm, Stats* stats, cudaStream_t st) {
+    const auto* Q = reinterpret_cast<const __nv_bfloat16*>(Qv);
+    const int grid = grid_for_rows(Tq * a.H, kWarps * kMarkRows, 148 * (a.nbits <= 16 ? 2 : 1));
+    cudaError_t e;
+    if (a.nbits <= 8) e = launch_pdl(annca_mark_kernel<D, 8>, grid, kWarps * 32, st, Q, Tq, P, F, a, R, Rnorm, stats);
+    else if (a.nbits <= 16)
+        e = launch_pdl(annca_mark_kernel<D, 16>, grid, kWarps * 32, st, Q, Tq, P, F, a, R, Rnorm, stats);
+    else e = launch_pdl(annca_mark_kernel<D, 32>, grid, kWarps * 32, st, Q, Tq, P, F, a, R, Rnorm, stats);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a.H * F), (unsigned)kPackParts);
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, annca_pack_kernel<D>, F, a);
+}
+
+}  // namespace
+
+cudaError_t launch_annca_prompt(const AnnView& a, const void* Kp, const void* Vp, const float* R,
+                                const float* Rnorm, Stats* stats, cudaStream_t st) {
+    return a.d == 128 ? prompt_t<128>(a, Kp, Vp, R, Rnorm, stats, st) : prompt_t<64>(a, Kp, Vp, R, Rnorm, stats, st);
+}
+
+cudaError_t launch_annca_select(const AnnView& a, const void* Q, int64_t Tq, int P, int F, const float* R,
+                                const float* Rnorm, Stats* stats, cudaStream_t st) {
+    return a.d == 128 ? select_t<128>(a, Q, Tq, P, F, R, Rnorm, stats, st)
+                      : select_t<64>(a, Q, Tq, P, F, R, Rnorm, stats, st);
+}
+
+}  // namespace tc
+
+// ------------------------------------------------------------------ C ABI
+
+using namespace tc;
+
+namespace {
+
+constexpr uint32_t kAnnMagic = 0x7c7ca2c3u;
+
+int64_t up128(int64_t x) { return (x + 127) / 128 * 128; }
+
+}  // namespace
+
+struct tc_annca_ctx {
+    uint32_t magic = kAnnMagic;
+    int H = 0, d = 0, nbits = 0;
+    float scale = 0.f;
+    int device = 0;
+    AnnView a{};
+    int64_t Lcap = 0;       // padded prompt rows allocated (a.Lp is this prompt's)
+    bool prompt_set = false;
+    int64_t last_T = 0, last_F = 0;
+    float* R = nullptr;
+    float* Rnorm = nullptr;
+    Stats* stats = nullptr;
+    std::vector<float> Rhost;
+    AttnMaps maps{};
+    int64_t maps_Lp = -1;   // row stride the key/value maps were encoded with
+    cudaStream_t last_stream = nullptr;
+    tc_status sticky = TC_OK;
+
+    void release(void*& p) {
+        if (p) cudaFree(p);
+        p = nullptr;
+    }
+    template <typename T>
+    tc_status grab(T*& p, size_t bytes) {
+        void* q = nullptr;
+        if (dev_alloc(&q, bytes) != cudaSuccess) {
+            cudaGetLastError();
+            return TC_ENOMEM;
+        }
+        p = static_cast<T*>(q);
+        return TC_OK;
+    }
+    void free_prompt() {
+        void* ps[] = {a.Kh, a.Vh, a.pcode, a.pcs, a.pix, a.prun};
+        for (void* p : ps) if (p) cudaFree(p);
+        a.Kh = a.Vh = nullptr;
+        a.pcode = a.pcs = nullptr;
+        a.pix = a.prun = nullptr;
+        // (ptab depends only on H and nbits: kept until the handle goes)
+        Lcap = 0;
+    }
+    void free_queries() {
+        if (a.qcode) cudaFree(a.qcode);
+        a.qcode = nullptr;
+        a.Tmax = 0;
+    }
+    void free_slots() {
+        void* ps[] = {a.keep, a.nsel, a.sidx, a.Ks, a.Vs, a.sbias};
+        for (void* p : ps) if (p) cudaFree(p);
+        a.keep = nullptr;
+        a.nsel = a.sidx = nullptr;
+        a.Ks = a.Vs = nullptr;
+        a.sbias = nullptr;
+        a.Zmax = 0;
+    }
+    ~tc_annca_ctx() {
+        free_prompt();
+        free_queries();
+        free_slots();
+        void* ps[] = {R, Rnorm, stats, a.kmax2, a.zeros, a.ptab};
+        for (void* p : ps) if (p) cudaFree(p);
+        magic = 0;
+    }
+};
+
+namespace {
+
+bool valid(tc_annca_handle h) { return h != nullptr && h->magic == kAnnMagic; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+tc_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return TC_OK;
+    cudaGetLastError();
+    return e == cudaErrorMemoryAllocation ? TC_ENOMEM : TC_ECUDA;
+}
+
+tc_status check_call(tc_annca_ctx* x) {
+    if (!valid(x)) return TC_EINVAL;
+    if (x->sticky != TC_OK) return x->sticky;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != x->device) {
+        cudaGetLastError();
+        return TC_EDEVICE;
+    }
+    return TC_OK;
+}
+
+// Per-slot arrays for Z = H F slots of the current prompt length; re-encodes the
+// key and value tensor maps.
+tc_status ensure_slots(tc_annca_ctx* x, int64_t Z) {
+    AnnView& a = x->a;
+    if (a.keep && Z <= a.Zmax && x->maps_Lp == a.Lp) return TC_OK;
+    if (cudaDeviceSynchronize() != cudaSuccess) return cuda_status(cudaGetLastError());
+    const int64_t Zn = std::max<int64_t>(Z, a.Zmax);
+    x->free_slots();
+    const size_t rows = (size_t)Zn * x->Lcap;
+    tc_status st;
+    if ((st = x->grab(a.keep, rows * 4)) || (st = x->grab(a.nsel, (size_t)Zn * 4)) || (st = x->grab(a.sidx, rows * 4)) ||
+        (st = x->grab(a.Ks, rows * x->d * 2)) || (st = x->grab(a.Vs, rows * x->d * 2)) ||
+        (st = x->grab(a.sbias, rows * 4))) {
+        x->free_slots();
+        return st;
+    }
+    if (cudaMemset(a.keep, 0, rows * 4) != cudaSuccess || cudaMemset(a.nsel, 0, (size_t)Zn * 4) != cudaSuccess) {
+        x->free_slots();
+        return cuda_status(cudaGetLastError());
+    }
+    a.Zmax = Zn;
+    const uint64_t d = x->d;
+    if (!encode3d(&x->maps.kc, a.Ks, d, a.Lp, Zn, d * 2, a.Lp * d * 2, 64, 128, 1) ||
+        !encode3d(&x->maps.vc, a.Vs, d, a.Lp, Zn, d * 2, a.Lp * d * 2, 64, 128, 1)) {
+        x->free_slots();
+        return TC_ECUDA;
+    }
+    x->maps_Lp = a.Lp;
+    return TC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+tc_status tc_annca_create(int32_t H, int32_t d, int32_t nbits, const tc_options* opt, tc_annca_handle* out) {
+    if (!out) return TC_EINVAL;
+    *out = nullptr;
+    tc_options o{TC_BF16, 0, 0.f, nullptr, 0};
+    if (opt) o = *opt;
+    if (H < 1 || H > 4096 || (d != 64 && d != 128) || nbits < 1 || nbits > 24 || !(o.softmax_scale >= 0.f) ||
+        !std::isfinite(o.softmax_scale) || o.intra_chunk != 0 || (o.dtype != TC_BF16 && o.dtype != TC_F32))
+        return TC_EINVAL;
+    if (o.dtype != TC_BF16) return TC_ENOTIMPL;
+    if (o.hyperplanes) {
+        for (int i = 0; i < nbits * d; ++i)
+            if (!std::isfinite(o.hyperplanes[i]) || !is_bf16_value(o.hyperplanes[i])) return TC_EINVAL;
+    }
+    int dev = 0;
+    cudaDeviceProp prop;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return TC_EDEVICE;
+    }
+    if (prop.major != 10) return TC_EDEVICE;
+    if (!get_encoder()) return TC_ECUDA;
+    tc_annca_ctx* x = new (std::nothrow) tc_annca_ctx;
+    if (!x) return TC_ENOMEM;
+    x->H = H;
+    x->d = d;
+    x->nbits = nbits;
+    x->device = dev;
+    x->scale = (o.softmax_scale > 0.f) ? o.softmax_scale : (float)(1.0 / std::sqrt((double)d));
+    if (o.hyperplanes)
+        x->Rhost.assign(o.hyperplanes, o.hyperplanes + (size_t)nbits * d);
+    else
+        default_hyperplanes(o.seed, nbits * d, x->Rhost);
+    std::vector<float> rnorm(nbits);
+    for (int b = 0; b < nbits; ++b) {
+        double s2 = 0.0;
+        for (int i = 0; i < d; ++i) s2 += (double)x->Rhost[(size_t)b * d + i] * x->Rhost[(size_t)b * d + i];
+        rnorm[b] = std::nextafter((float)std::sqrt(s2), INFINITY);
+    }
+    AnnView& a = x->a;
+    a.H = H;
+    a.d = d;
+    a.nbits = nbits;
+    tc_status st;
+    cudaError_t e;
+    if ((st = x->grab(x->R, (size_t)nbits * d * 4)) || (st = x->grab(x->Rnorm, (size_t)nbits * 4)) ||
+        (st = x->grab(x->stats, sizeof(Stats))) || (st = x->grab(a.kmax2, (size_t)H * 4)) ||
+        (st = x->grab(a.zeros, (size_t)H * 4)) ||
+        (nbits <= 16 && (st = x->grab(a.ptab, ((size_t)H << nbits) * 4)))) {
+        delete x;
+        return st;
+    }
+    if ((e = cudaMemcpy(x->R, x->Rhost.data(), (size_t)nbits * d * 4, cudaMemcpyHostToDevice)) ||
+        (e = cudaMemcpy(x->Rnorm, rnorm.data(), (size_t)nbits * 4, cudaMemcpyHostToDevice)) ||
+        (e = cudaMemset(x->stats, 0, sizeof(Stats))) || (e = cudaMemset(a.kmax2, 0, (size_t)H * 4)) ||
+        (e = cudaMemset(a.zeros, 0, (size_t)H * 4))) {
+        delete x;
+        return cuda_status(e);
+    }
+    *out = x;
+    return TC_OK;
+}
+
+tc_status tc_annca_set_prompt(tc_annca_handle x, const void* Kp, const void* Vp, int32_t L, tc_stream stream) {
+    tc_status st = check_call(x);
+    if (st) return st;
+    if (!Kp || !Vp || !aligned16(Kp) || !aligned16(Vp) || L < 1 || L > kMaxPrompt) return TC_EINVAL;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    AnnView& a = x->a;
+    const int64_t Lp = up128(L);
+    if (Lp > x->Lcap) {
+        if (cudaDeviceSynchronize() != cudaSuccess) return cuda_status(cudaGetLastError());
+        x->free_prompt();
+        x->free_slots();   // their row stride follows the prompt's
+        const size_t rows = (size_t)x->H * Lp;
+        if ((st = x->grab(a.Kh, rows * x->d * 2)) || (st = x->grab(a.Vh, rows * x->d * 2)) ||
+            (st = x->grab(a.pcode, rows * 4)) || (st = x->grab(a.pcs, rows * 4)) || (st = x->grab(a.pix, rows * 4)) ||
+            (st = x->grab(a.prun, rows * 4))) {
+            x->free_prompt();
+            x->prompt_set = false;
+            return st;
+        }
+        x->Lcap = Lp;
+    }
+    a.L = L;
+    a.Lp = x->Lcap;   // one row stride for every prompt this allocation holds
+    x->last_stream = cs;
+    cudaError_t e = cudaMemsetAsync(a.kmax2, 0, (size_t)x->H * 4, cs);
+    if (e == cudaSuccess && a.ptab) e = cudaMemsetAsync(a.ptab, 0xff, ((size_t)x->H << x->nbits) * 4, cs);
+    if (e == cudaSuccess) e = launch_annca_prompt(a, Kp, Vp, x->R, x->Rnorm, x->stats, cs);
+    if (e != cudaSuccess) {
+        x->prompt_set = false;
+        return cuda_status(e);
+    }
+    x->prompt_set = true;
+    return TC_OK;
+}
+
+tc_status tc_annca_attend(tc_annca_handle x, const void* Q, int64_t Tq, int32_t P, void* out, tc_stream stream) {
+    tc_status st = check_call(x);
+    if (st) return st;
+    if (!Q || !out || !aligned16(Q) || !aligned16(out) || P < 1 || Tq < 1 || Tq > ((int64_t)1 << 26) || Tq % P ||
+        Tq * x->H >= ((int64_t)1 << 31))   // the kernels index rows t H + h in 32 bits
+        return TC_EINVAL;
+    const size_t bytes = (size_t)Tq * x->H * x->d * 2;
+    const char* q = static_cast<const char*>(Q);
+    const char* o = static_cast<const char*>(out);
+    if (q < o + bytes && o < q + bytes) return TC_EINVAL;
+    if (!x->prompt_set) return TC_ESTATE;
+    const int64_t F = Tq / P;
+    if ((int64_t)x->H * F > (1 << 30) || F * ((P + 127) / 128) > (1 << 30)) return TC_EINVAL;
+    AnnView& a = x->a;
+    if (!a.qcode || Tq > a.Tmax) {
+        if (cudaDeviceSynchronize() != cudaSuccess) return cuda_status(cudaGetLastError());
+        x->free_queries();
+        if ((st = x->grab(a.qcode, (size_t)x->H * Tq * 4))) return st;
+        a.Tmax = Tq;
+    }
+    if ((st = ensure_slots(x, (int64_t)x->H * F))) return st;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    x->last_stream = cs;
+    AttnMaps m = x->maps;
+    if (!encode3d(&m.q, Q, x->d, x->H, Tq, (uint64_t)x->d * 2, (uint64_t)x->H * x->d * 2, 64, 1, 128))
+        return TC_EINVAL;
+    cudaError_t e = cudaSuccess;
+    if (++a.gen == 0) {   // the stamps wrapped: start them over
+        e = cudaMemsetAsync(a.keep, 0, (size_t)a.Zmax * a.Lp * 4, cs);
+        a.gen = 1;
+    }
+    if (e == cudaSuccess) e = launch_annca_select(a, Q, Tq, P, (int)F, x->R, x->Rnorm, x->stats, cs);
+    if (e == cudaSuccess)
+        e = launch_attend_cross_bf16(a, m, Tq, P, (int)F, static_cast<__nv_bfloat16*>(out),
+                                     (float)((double)x->scale * 1.4426950408889634), x->stats, cs);
+    if (e != cudaSuccess) return cuda_status(e);
+    x->last_T = Tq;
+    x->last_F = F;
+    return TC_OK;
+}
+
+tc_status tc_annca_sync(tc_annca_handle x) {
+    if (!valid(x)) return TC_EINVAL;
+    if (x->sticky != TC_OK) return x->sticky;
+    if (cudaStreamSynchronize(x->last_stream) != cudaSuccess) {
+        cudaGetLastError();
+        x->sticky = TC_ECUDA;
+        return x->sticky;
+    }
+    Stats s{};
+    if (cudaMemcpy(&s, x->stats, sizeof(Stats), cudaMemcpyDeviceToHost) != cudaSuccess) {
+        cudaGetLastError();
+        x->sticky = TC_ECUDA;
+    } else if (s.error_bits & kErrTimeout) {
+        x->sticky = TC_ETIMEOUT;
+    }
+    return x->sticky;
+}
+
+tc_status tc_annca_kept(tc_annca_handle x, int64_t* T_out, int64_t* F_out, int32_t* L_out, int32_t* counts,
+                        int32_t* index, uint32_t* qcodes, uint32_t* pcodes) {
+    tc_status st = tc_annca_sync(x);
+    if (st) return st;
+    const AnnView& a = x->a;
+    const int64_t F = x->last_F, Z = (int64_t)x->H * F;
+    if (T_out) *T_out = x->last_T;
+    if (F_out) *F_out = F;
+    if (L_out) *L_out = x->prompt_set ? a.L : 0;
+    cudaError_t e = cudaSuccess;
+    if (counts && Z) e = cudaMemcpy(counts, a.nsel, (size_t)Z * 4, cudaMemcpyDeviceToHost);
+    for (int64_t z = 0; index && e == cudaSuccess && z < Z; ++z)
+        e = cudaMemcpy(index + z * a.L, a.sidx + z * a.Lp, (size_t)a.L * 4, cudaMemcpyDeviceToHost);
+    for (int h = 0; qcodes && e == cudaSuccess && h < x->H && x->last_T; ++h)
+        e = cudaMemcpy(qcodes + (int64_t)h * x->last_T, a.qcode + (int64_t)h * a.Tmax, (size_t)x->last_T * 4,
+                       cudaMemcpyDeviceToHost);
+    for (int h = 0; pcodes && e == cudaSuccess && h < x->H && x->prompt_set; ++h)
+        e = cudaMemcpy(pcodes + (int64_t)h * a.L, a.pcode + (int64_t)h * a.Lp, (size_t)a.L * 4,
+                       cudaMemcpyDeviceToHost);
+    return cuda_status(e);
+}
+
+tc_status tc_annca_get_hyperplanes(tc_annca_handle x, float* R) {
+    if (!valid(x) || !R) return TC_EINVAL;
+    std::memcpy(R, x->Rhost.data(), x->Rhost.size() * sizeof(float));
+    return TC_OK;
+}
+
+void tc_annca_destroy(tc_annca_handle x) {
+    if (!valid(x)) return;
+    cudaDeviceSynchronize();
+    cudaGetLastError();
+    delete x;
+}
+
+}  // extern "C"

@@ -255,14 +255,14 @@ struct CfgU {
 //               retired (up to three tiles ahead).
 //   warp 18     lane 0 TMA producer for the V ring (2 stages).
 //   warp 19     lane 0 issues O += P_i V_i in tile order.
-template <int D>
+template <int D, bool CROSS>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
                        const __grid_constant__ CUtensorMap tmVc, const __grid_constant__ CUtensorMap tmKs,
                        const __grid_constant__ CUtensorMap tmVs, const int32_t* __restrict__ Mdev,
                        const float* __restrict__ bias2, const float* __restrict__ kmax2c,
                        const float* __restrict__ kmax2s, const float* __restrict__ bmaxh, int64_t capP,
-                       const float* __restrict__ sbias, int64_t Ts, int64_t Tq, int H,
+                       const float* __restrict__ sbias, int64_t Ts, int64_t Tq, int H, int Pf, int Ff,
                        __nv_bfloat16* __restrict__ out, float scale_log2, Stats* stats) {
     using C = Cfg<D>;
     using L = CfgU<D>;
@@ -283,10 +283,42 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.y;
-    const int q0 = blockIdx.x * kBM;
-    const int Mh = Mdev[h];
+    // Self-attention: CTA x covers query rows [128 x, 128 x + 128) of all Tq, the keys
+    // are committed entries (slot h of the cache arrays) then staged tokens.
+    // Cross-attention: the query rows are Ff frames of Pf rows; CTA x covers rows of one
+    // frame f, and the keys are the kept prompt tokens of slot h Ff + f, nothing staged.
+    int q0, zc;
+    int64_t qend;
+    if constexpr (CROSS) {
+        // launched as a programmatic dependent of the kernel that packs the keys: wait
+        // for it before reading anything it writes
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        const int tpf = (Pf + kBM - 1) / kBM;
+        const int f = blockIdx.x / tpf;
+        q0 = f * Pf + (blockIdx.x - f * tpf) * kBM;
+        qend = (int64_t)(f + 1) * Pf;
+        zc = h * Ff + f;
+    } else {
+        q0 = blockIdx.x * kBM;
+        qend = Tq;
+        zc = h;
+    }
+    const int Mh = Mdev[zc];
     const int nc = (Mh + kBN - 1) / kBN;
-    const int ntiles = nc + (int)((Ts + kBN - 1) / kBN);
+    const int ntiles = nc + (CROSS ? 0 : (int)((Ts + kBN - 1) / kBN));
+    if constexpr (CROSS) {
+        if (ntiles == 0) {   // no key: the rows are the empty sum, zero
+            constexpr int W = D / 8;   // 16-byte words per row
+            for (int i = threadIdx.x; i < kBM * W; i += kThreads) {
+                const int64_t row = q0 + i / W;
+                if (row < qend)
+                    reinterpret_cast<uint4*>(out + (row * H + h) * D)[i % W] = make_uint4(0u, 0u, 0u, 0u);
+            }
+            asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            return;
+        }
+    }
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[U_QFULL], 1);
@@ -349,7 +381,8 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             const int row0 = (cache ? i : i - nc) * kBN;
             mbar_expect_tx(&full[st], C::TILE);
             for (int b = 0; b < C::NB; ++b)
-                tma_load_3d(ring + st * C::TILE + b * C::BOX, cache ? mc : ms, 64 * b, row0, h, &full[st]);
+                tma_load_3d(ring + st * C::TILE + b * C::BOX, cache ? mc : ms, 64 * b, row0, cache ? zc : h,
+                            &full[st]);
             last = i;
         }
         if (kside) mbar_wait(&bars[U_QFULL], 0);
@@ -416,7 +449,7 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         const int r = wt * 32 + lane;        // query row within the tile = TMEM lane
         const uint32_t lane_base = (uint32_t)(wt * 32) << 16;
         const uint32_t tOh = tO + HC * g + lane_base;
-        const float* bias_h = bias2 + (int64_t)h * capP;
+        const float* bias_h = bias2 + (int64_t)zc * capP;
         auto bias_of = [&](int i) -> float {
             return (i < nc) ? bias_h[(int64_t)i * kBN + r] : sbias[(int64_t)(i - nc) * kBN + r];
         };
@@ -639,7 +672,7 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             else TC_LD16(tO + lane_base + col, o);
             tc_wait_ld();
             const int64_t row = q0 + r;
-            if (row < Tq) {
+            if (row < qend) {
                 uint4* dst = reinterpret_cast<uint4*>(out + (row * H + h) * D + col);
 #pragma unroll
                 for (int v = 0; v < QC / 8; ++v) {
@@ -667,16 +700,23 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-template <int D>
-cudaError_t launch_t(const CacheView& c, const StageView& s, const AttnMaps& m, int64_t Tq, __nv_bfloat16* out,
-                     float scale_log2, Stats* stats, bool overlap_prev, cudaStream_t st) {
+template <int D, bool CROSS>
+cudaError_t set_smem_attr() {
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(attend_bf16_duo_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             CfgU<D>::SMEM);
+        cudaError_t e = cudaFuncSetAttribute(attend_bf16_duo_kernel<D, CROSS>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, CfgU<D>::SMEM);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
+    return cudaSuccess;
+}
+
+template <int D>
+cudaError_t launch_t(const CacheView& c, const StageView& s, const AttnMaps& m, int64_t Tq, __nv_bfloat16* out,
+                     float scale_log2, Stats* stats, bool overlap_prev, cudaStream_t st) {
+    cudaError_t e = set_smem_attr<D, false>();
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((Tq + kBM - 1) / kBM), (unsigned)c.H);
     cfg.blockDim = dim3(kThreads);
@@ -687,10 +727,35 @@ cudaError_t launch_t(const CacheView& c, const StageView& s, const AttnMaps& m, 
     attr[0].val.programmaticStreamSerializationAllowed = overlap_prev ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, attend_bf16_duo_kernel<D>, m.q, m.kc, m.vc, m.ks, m.vs, (const int32_t*)c.M,
-                              (const float*)c.bias2, (const float*)c.kmax2, (const float*)c.kmax2s,
-                              (const float*)c.bmax, c.capP, (const float*)s.sbias, s.T, Tq, c.H, out, scale_log2,
-                              stats);
+    return cudaLaunchKernelEx(&cfg, attend_bf16_duo_kernel<D, false>, m.q, m.kc, m.vc, m.ks, m.vs,
+                              (const int32_t*)c.M, (const float*)c.bias2, (const float*)c.kmax2,
+                              (const float*)c.kmax2s, (const float*)c.bmax, c.capP, (const float*)s.sbias, s.T, Tq,
+                              c.H, (int)Tq, 1, out, scale_log2, stats);
+}
+
+// Cross-attention over the kept prompt tokens: grid (F frames x tiles per frame, H),
+// launched as a programmatic dependent of the packing kernel (the kernel waits for it
+// before its first read).
+template <int D>
+cudaError_t launch_cross_t(const AnnView& a, const AttnMaps& m, int64_t Tq, int P, int F, __nv_bfloat16* out,
+                           float scale_log2, Stats* stats, cudaStream_t st) {
+    cudaError_t e = set_smem_attr<D, true>();
+    if (e != cudaSuccess) return e;
+    const int tpf = (P + kBM - 1) / kBM;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(F * tpf), (unsigned)a.H);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = CfgU<D>::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, attend_bf16_duo_kernel<D, true>, m.q, m.kc, m.vc, m.kc, m.vc,
+                              (const int32_t*)a.nsel, (const float*)a.sbias, (const float*)a.kmax2,
+                              (const float*)a.zeros, (const float*)a.zeros, a.Lp, (const float*)nullptr, (int64_t)0,
+                              Tq, a.H, P, F, out, scale_log2, stats);
 }
 
 }  // namespace
@@ -700,6 +765,12 @@ cudaError_t launch_attend_bf16(const CacheView& c, const StageView& s, const Att
                                cudaStream_t st) {
     return c.d == 128 ? launch_t<128>(c, s, maps, Tq, out, scale_log2, stats, overlap_prev, st)
                       : launch_t<64>(c, s, maps, Tq, out, scale_log2, stats, overlap_prev, st);
+}
+
+cudaError_t launch_attend_cross_bf16(const AnnView& a, const AttnMaps& maps, int64_t Tq, int P, int F,
+                                     __nv_bfloat16* out, float scale_log2, Stats* stats, cudaStream_t st) {
+    return a.d == 128 ? launch_cross_t<128>(a, maps, Tq, P, F, out, scale_log2, stats, st)
+                      : launch_cross_t<64>(a, maps, Tq, P, F, out, scale_log2, stats, st);
 }
 
 }  // namespace tc

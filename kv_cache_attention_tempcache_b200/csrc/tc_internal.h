@@ -6,6 +6,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <vector>
+
 namespace tc {
 
 // Device state of one TempCache. Per-head arrays have a padded row stride
@@ -94,5 +96,56 @@ struct AttnMaps {
 cudaError_t launch_attend_bf16(const CacheView& c, const StageView& s, const AttnMaps& maps,
                                int64_t Tq, __nv_bfloat16* out, float scale_log2, Stats* stats,
                                bool overlap_prev, cudaStream_t st);
+
+
+// Device state of one AnnCA cross-attention layer (tc_annca.cu). The prompt is kept
+// head-major with a padded row stride Lp = round_up(L, 128); the query block being
+// attended holds F frames, and (head h, frame f) is slot z = h F + f of the per-frame
+// arrays, each Lp rows long.
+struct AnnView {
+    int H, d, nbits;
+    int L;                 // prompt tokens
+    int64_t Lp;            // padded prompt rows per head (and per slot)
+    __nv_bfloat16* Kh;     // [H][Lp][d] prompt keys
+    __nv_bfloat16* Vh;     // [H][Lp][d] prompt values
+    uint32_t* pcode;       // [H][Lp] hash codes of the prompt keys
+    uint32_t* pcs;         // [H][Lp] the same codes in ascending order
+    int32_t* pix;          // [H][Lp] prompt token of each sorted code (ties by token)
+    int32_t* prun;         // [H][Lp] first sorted position of each prompt token's code
+    int32_t* ptab;         // [H][2^nbits] first sorted position of each code, -1 if the prompt has
+                           // none (nbits <= 16; null otherwise: binary search in pcs)
+    float* kmax2;          // [H] upper bound of |k|^2 over the prompt keys
+    float* zeros;          // [H] zeros: log2 n bound and staged-key bound of the attention
+    int64_t Tmax;          // query rows the per-query arrays hold
+    uint32_t* qcode;       // [H][Tmax] hash codes of the last query block
+    int64_t Zmax;          // slots the per-frame arrays hold
+    uint32_t* keep;        // [Zmax][Lp] per slot, one stamp per bucket of the prompt, at the
+                           // bucket's first sorted position: equal to gen when a query of the
+                           // slot has that code in the current call
+    uint32_t gen;          // stamp of the current call (>= 1; the stamps start at 0)
+    int32_t* nsel;         // [Zmax] kept prompt tokens per slot
+    int32_t* sidx;         // [Zmax][Lp] kept prompt tokens in ascending order
+    __nv_bfloat16* Ks;     // [Zmax][Lp][d] kept keys, packed; rows up to the next multiple of 128 zeroed
+    __nv_bfloat16* Vs;     // [Zmax][Lp][d] kept values, packed the same way
+    float* sbias;          // [Zmax][Lp] 0 for kept rows, -inf for the rest of the last tile
+};
+
+// Launchers (tc_annca.cu, tc_attn_bf16.cu).
+cudaError_t launch_annca_prompt(const AnnView& a, const void* Kp, const void* Vp, const float* R,
+                                const float* Rnorm, Stats* stats, cudaStream_t st);
+cudaError_t launch_annca_select(const AnnView& a, const void* Q, int64_t Tq, int P, int F, const float* R,
+                                const float* Rnorm, Stats* stats, cudaStream_t st);
+cudaError_t launch_attend_cross_bf16(const AnnView& a, const AttnMaps& maps, int64_t Tq, int P, int F,
+                                     __nv_bfloat16* out, float scale_log2, Stats* stats, cudaStream_t st);
+
+// Host helpers (tc_runtime.cu).
+cudaError_t dev_alloc(void** p, size_t bytes);   // cudaMalloc with the TC_FAULT_ALLOC_AT injection
+float round_bf16(float x);
+bool is_bf16_value(float x);
+void default_hyperplanes(uint64_t seed, int n, std::vector<float>& out);
+bool get_encoder();
+// 3-D bf16 tensor map with a 128-byte swizzle; dims and box innermost first, strides in bytes.
+bool encode3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1, uint64_t s2,
+              uint32_t b0, uint32_t b1, uint32_t b2);
 
 }  // namespace tc

@@ -11,13 +11,7 @@
 #include <new>
 #include <vector>
 
-using namespace tc;
-
-namespace {
-
-constexpr uint32_t kMagic = 0x7c7ca5e1u;
-
-inline int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+namespace tc {
 
 // ---- allocation with host-side fault injection (TC_FAULT_ALLOC_AT=n fails the
 // n-th allocation of the process, counting from 1), used by the failure tests.
@@ -99,6 +93,16 @@ bool encode3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+}  // namespace tc
+
+using namespace tc;
+
+namespace {
+
+constexpr uint32_t kMagic = 0x7c7ca5e1u;
+
+inline int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
 
 // p[h * stride + i] = v for i < n, h < rows (one launch over all heads).
 __global__ void fill_f32(float* p, int64_t n, int rows, int64_t stride, float v) {
@@ -424,7 +428,9 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
 tc_status tc_append_chunk(tc_handle x, const void* K, const void* V, int64_t T, tc_stream stream) {
     tc_status st = check_call(x);
     if (st) return st;
-    if (!K || !V || !aligned16(K) || !aligned16(V) || T < 1 || T > ((int64_t)1 << 28)) return TC_EINVAL;
+    if (!K || !V || !aligned16(K) || !aligned16(V) || T < 1 || T > ((int64_t)1 << 28) ||
+        T * x->H >= ((int64_t)1 << 31))   // the kernels index rows t H + h in 32 bits
+        return TC_EINVAL;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     x->last_stream = cs;
     x->prev_attend = false;

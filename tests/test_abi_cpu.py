@@ -112,3 +112,34 @@ def test_reference_arm_prints_the_contract_line():
         assert key in line, key
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["cpu_baseline"]["kind"] == "oracle"
+
+
+@pytest.mark.parametrize("args", [
+    (0, 128, 10),      # H < 1
+    (4, 96, 10),       # d not 64/128
+    (4, 128, 0),       # nbits < 1
+    (4, 128, 25),      # nbits > 24
+])
+def test_annca_create_rejects_bad_arguments(tcmod, args):
+    h = ctypes.c_void_p()
+    assert tcmod.lib.tc_annca_create(*args, None, ctypes.byref(h)) == tcmod.TC_EINVAL
+    assert not h.value
+
+
+def test_annca_is_bf16_only(tcmod):
+    opt = tcmod.TCOptions()
+    opt.dtype = tcmod.TC_F32
+    h = ctypes.c_void_p()
+    assert tcmod.lib.tc_annca_create(4, 128, 10, ctypes.byref(opt), ctypes.byref(h)) == tcmod.TC_ENOTIMPL
+    opt.dtype = tcmod.TC_BF16
+    opt.intra_chunk = 1   # a TempCache option, meaningless here
+    assert tcmod.lib.tc_annca_create(4, 128, 10, ctypes.byref(opt), ctypes.byref(h)) == tcmod.TC_EINVAL
+
+
+def test_annca_calls_reject_a_null_handle(tcmod):
+    lib = tcmod.lib
+    assert lib.tc_annca_set_prompt(None, None, None, 1, None) == tcmod.TC_EINVAL
+    assert lib.tc_annca_attend(None, None, 1, 1, None, None) == tcmod.TC_EINVAL
+    assert lib.tc_annca_kept(None, None, None, None, None, None, None, None) == tcmod.TC_EINVAL
+    assert lib.tc_annca_sync(None) == tcmod.TC_EINVAL
+    lib.tc_annca_destroy(None)
