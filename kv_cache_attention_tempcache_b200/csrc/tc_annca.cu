@@ -10,12 +10,12 @@
 //                         bound |k|^2 per head.
 //   annca_sort_kernel     once per prompt: sort each head's (code, token) pairs; every
 //                         prompt token learns where its code's run starts.
-//   annca_mark_kernel     per call: hash every query (four rows in flight per warp); each
-//                         lane of a warp then looks one query's code up (a table of the
-//                         head's codes for nbits <= 16, else a binary search of its sorted
-//                         codes) and, if the prompt has that code, stamps the bucket with
-//                         the call's number for the query's frame (written only while the
-//                         stamp differs, so the many queries of one bucket rarely store).
+//   annca_mark_kernel     per call: one lane per query row hashes it, then looks its code
+//                         up (a table of the head's codes for nbits <= 16, else a binary
+//                         search of its sorted codes) and, if the prompt has that code,
+//                         stamps the bucket with the call's number for the query's frame
+//                         (written only while the stamp differs, so the many queries of
+//                         one bucket rarely store).
 //   annca_pack_kernel     per call: a few blocks per (head, frame) list the prompt tokens
 //                         whose bucket carries this call's stamp, in ascending order, and
 //                         pack their keys and values into 128-row tiles for the attention
@@ -200,59 +200,106 @@ __device__ __forceinline__ void flag_bucket(const AnnView& a, int h, int64_t z, 
     }
 }
 
-constexpr int kMarkRows = 4;   // rows a warp of the mark kernel loads before hashing them
+// Shared memory of the mark kernel: per warp 32 staged rows (row stride padded by 16
+// bytes so that lanes reading their own rows hit distinct banks).
+template <int D>
+struct MarkSmem {
+    static constexpr int RB = D * 2 + 16;
+    static constexpr int BYTES = kWarps * 32 * RB;
+};
 
-// One warp per query row r = t H + h; the lookups of up to 32 rows are batched, one
-// row per lane, so their dependent loads overlap.
+// The normals as fp32 [NBP][D] (zero rows past nbits) and their rounded-up norms, passed
+// by value: a kernel parameter sits in the constant bank, so with every index known at
+// compile time each FMA reads its normal as a constant operand, with no load.
 template <int D, int NBP>
-__global__ void __launch_bounds__(kWarps * 32, NBP <= 16 ? 2 : 1)
-annca_mark_kernel(const __nv_bfloat16* __restrict__ Q, int64_t Tq, int P, int F, AnnView a,
-                  const float* __restrict__ R, const float* __restrict__ Rnorm, Stats* stats) {
-    grid_dependency_wait();
-    constexpr int EPL = D / 32;
-    using IO = RowIO<__nv_bfloat16, EPL>;
-    __shared__ float sRow[kWarps][D];
+struct Planes {
+    float v[NBP * D];
+    float rn[NBP];
+};
+
+// One lane per query row, 32 consecutive rows r = t H + h per warp: the warp copies
+// its rows (one contiguous block of the token-major input) into shared memory with
+// coalesced loads, then every lane forms the NBP projections of its own row in fp32
+// (normals broadcast from shared memory), keeps the sign of each bit outside its
+// rounding bound and recomputes the rest in fp64 in index order. The code is stored
+// token-major, and the lane stamps its code's prompt bucket for its frame.
+template <int D, int NBP>
+__global__ void __launch_bounds__(kWarps * 32)
+annca_mark_kernel(const __nv_bfloat16* __restrict__ Q, int rows, int P, int F, AnnView a,
+                  const float* __restrict__ R, const __grid_constant__ Planes<D, NBP> pl, Stats* stats) {
+    using S = MarkSmem<D>;
+    constexpr int W = D / 8;   // 16-byte words per row
+    extern __shared__ __align__(16) uint8_t mk_smem[];
+    uint8_t* sRows = mk_smem;
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-    uint32_t Rp[NBP][D / 64];
-    load_planes<D, NBP>(R, a.nbits, lane, Rp);
-    const float rn = lane < a.nbits ? Rnorm[lane] : 0.f;
-    const int64_t rows = Tq * a.H;
-    const int64_t stride = (int64_t)gridDim.x * kWarps;
-    int nq = 0, q_h = 0;
-    int64_t q_z = 0;
-    uint32_t q_code = 0;
+    const int nbits = a.nbits;
+    grid_dependency_wait();
+    uint8_t* mine = sRows + wib * 32 * S::RB;
+    const float gam2 = 2.f * (float)(D + 2) * kU32;
     unsigned rechecks = 0;
-    for (int64_t r0 = (int64_t)blockIdx.x * kWarps + wib; r0 < rows; r0 += kMarkRows * stride) {
-        typename IO::V raw[kMarkRows];
-#pragma unroll
-        for (int k = 0; k < kMarkRows; ++k)
-            if (r0 + k * stride < rows) raw[k] = IO::load(Q + (r0 + k * stride) * D, lane);
-#pragma unroll
-        for (int k = 0; k < kMarkRows; ++k) {
-            const int64_t r = r0 + k * stride;
-            if (r >= rows) break;   // warp-uniform
-            const int t = (int)((uint32_t)r / (uint32_t)a.H);   // rows < 2^31 (host check)
-            const int h = (int)(r - (int64_t)t * a.H);
-            float x[EPL];
-            IO::to_float(raw[k], x);
-            float nk;
-            unsigned nre;
-            const unsigned code = hash_row<D, NBP>(x, Rp, R, rn, a.nbits, sRow[wib], lane, nk, nre);
-            rechecks += nre;
-            if (lane == 0) a.qcode[(int64_t)h * a.Tmax + t] = code;
-            if (lane == nq) {
-                q_h = h;
-                q_z = (int64_t)h * F + (int)((uint32_t)t / (uint32_t)P);
-                q_code = code;
-            }
-            if (++nq == 32) {
-                flag_bucket(a, q_h, q_z, q_code);
-                nq = 0;
-            }
+    for (int base = (blockIdx.x * kWarps + wib) * 32; base < rows; base += gridDim.x * kWarps * 32) {
+        const int n = min(32, rows - base);
+        const uint4* src = reinterpret_cast<const uint4*>(Q + (int64_t)base * D);
+#pragma unroll 4
+        for (int w = lane; w < n * W; w += 32) {
+            const int row = w / W, col = w - row * W;
+            *reinterpret_cast<uint4*>(mine + row * S::RB + col * 16) = src[w];
         }
+        __syncwarp();
+        if (lane < n) {
+            const uint8_t* rowp = mine + lane * S::RB;
+            float acc[NBP];
+#pragma unroll
+            for (int b = 0; b < NBP; ++b) acc[b] = 0.f;
+            float n2 = 0.f;
+#pragma unroll
+            for (int c = 0; c < W; ++c) {
+                const uint4 v = *reinterpret_cast<const uint4*>(rowp + c * 16);
+                const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+                float x[8];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    x[2 * k] = __uint_as_float(wd[k] << 16);
+                    x[2 * k + 1] = __uint_as_float(wd[k] & 0xffff0000u);
+                }
+#pragma unroll
+                for (int k = 0; k < 8; ++k) n2 = fmaf(x[k], x[k], n2);
+#pragma unroll
+                for (int b = 0; b < NBP; ++b) {
+                    float t = acc[b];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) t = fmaf(pl.v[b * D + c * 8 + k], x[k], t);
+                    acc[b] = t;
+                }
+            }
+            // |<R_b,x>| > 2 (d+2) u |R_b||x| certifies the fp32 sign (any summation order
+            // errs by at most (d+2) u |R_b||x|; doubled for margin); else fp64, index order
+            const float nx = sqrtf(n2);
+            uint32_t code = 0;
+#pragma unroll
+            for (int b = 0; b < NBP; ++b) {
+                if (b >= nbits) break;
+                bool bit = acc[b] >= 0.f;
+                if (!(fabsf(acc[b]) > gam2 * pl.rn[b] * nx + 1e-30f)) {
+                    double s64 = 0.0;
+                    for (int i = 0; i < D; ++i) {
+                        const uint16_t u = *reinterpret_cast<const uint16_t*>(rowp + 2 * i);
+                        s64 = fma((double)R[b * D + i], (double)__uint_as_float((uint32_t)u << 16), s64);
+                    }
+                    bit = s64 >= 0.0;
+                    ++rechecks;
+                }
+                code |= (uint32_t)bit << b;
+            }
+            const int r = base + lane;
+            a.qcode[r] = code;
+            const int t = (int)((uint32_t)r / (uint32_t)a.H);
+            const int h = r - t * a.H;
+            flag_bucket(a, h, (int64_t)h * F + (int)((uint32_t)t / (uint32_t)P), code);
+        }
+        __syncwarp();
     }
-    if (lane < nq) flag_bucket(a, q_h, q_z, q_code);
-    if (lane == 0 && rechecks) atomicAdd(&stats->hash_rechecks, (unsigned long long)rechecks);
+    if (rechecks) atomicAdd(&stats->hash_rechecks, (unsigned long long)rechecks);
     grid_dependents_launch();
 }
 
@@ -349,16 +396,44 @@ cudaError_t prompt_t(const AnnView& a, const void* Kp, const void* Vp, const flo
     return cudaGetLastError();
 }
 
+template <int D, int NBP>
+cudaError_t mark_t(const __nv_bfloat16* Q, int rows, int P, int F, const AnnView& a, const float* R,
+                   const float* Rhost, const float* Rnorm_host, Stats* stats, cudaStream_t st) {
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(annca_mark_kernel<D, NBP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             MarkSmem<D>::BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    Planes<D, NBP> pl;
+    for (int b = 0; b < NBP; ++b) {
+        for (int i = 0; i < D; ++i) pl.v[b * D + i] = (b < a.nbits) ? Rhost[b * D + i] : 0.f;
+        pl.rn[b] = (b < a.nbits) ? Rnorm_host[b] : 0.f;
+    }
+    const int grid = (rows + kWarps * 32 - 1) / (kWarps * 32);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kWarps * 32);
+    cfg.dynamicSmemBytes = MarkSmem<D>::BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, annca_mark_kernel<D, NBP>, Q, rows, P, F, a, R, pl, stats);
+}
+
 template <int D>
 cudaError_t select_t(const AnnView& a, const void* Qv, int64_t Tq, int P, int F, const float* R,
-                     const float* Rnorm, Stats* stats, cudaStream_t st) {
+                     const float* Rhost, const float* Rnorm_host, Stats* stats, cudaStream_t st) {
     const auto* Q = reinterpret_cast<const __nv_bfloat16*>(Qv);
-    const int grid = grid_for_rows(Tq * a.H, kWarps * kMarkRows, 148 * (a.nbits <= 16 ? 2 : 1));
+    const int rows = (int)(Tq * a.H);   // < 2^31 (host check)
     cudaError_t e;
-    if (a.nbits <= 8) e = launch_pdl(annca_mark_kernel<D, 8>, grid, kWarps * 32, st, Q, Tq, P, F, a, R, Rnorm, stats);
-    else if (a.nbits <= 16)
-        e = launch_pdl(annca_mark_kernel<D, 16>, grid, kWarps * 32, st, Q, Tq, P, F, a, R, Rnorm, stats);
-    else e = launch_pdl(annca_mark_kernel<D, 32>, grid, kWarps * 32, st, Q, Tq, P, F, a, R, Rnorm, stats);
+    if (a.nbits <= 8) e = mark_t<D, 8>(Q, rows, P, F, a, R, Rhost, Rnorm_host, stats, st);
+    else if (a.nbits <= 16) e = mark_t<D, 16>(Q, rows, P, F, a, R, Rhost, Rnorm_host, stats, st);
+    else e = mark_t<D, 24>(Q, rows, P, F, a, R, Rhost, Rnorm_host, stats, st);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a.H * F), (unsigned)kPackParts);
@@ -380,9 +455,9 @@ cudaError_t launch_annca_prompt(const AnnView& a, const void* Kp, const void* Vp
 }
 
 cudaError_t launch_annca_select(const AnnView& a, const void* Q, int64_t Tq, int P, int F, const float* R,
-                                const float* Rnorm, Stats* stats, cudaStream_t st) {
-    return a.d == 128 ? select_t<128>(a, Q, Tq, P, F, R, Rnorm, stats, st)
-                      : select_t<64>(a, Q, Tq, P, F, R, Rnorm, stats, st);
+                                const float* Rhost, const float* Rnorm_host, Stats* stats, cudaStream_t st) {
+    return a.d == 128 ? select_t<128>(a, Q, Tq, P, F, R, Rhost, Rnorm_host, stats, st)
+                      : select_t<64>(a, Q, Tq, P, F, R, Rhost, Rnorm_host, stats, st);
 }
 
 }  // namespace tc
@@ -412,6 +487,7 @@ struct tc_annca_ctx {
     float* Rnorm = nullptr;
     Stats* stats = nullptr;
     std::vector<float> Rhost;
+    std::vector<float> Rnorm_host;
     AttnMaps maps{};
     int64_t maps_Lp = -1;   // row stride the key/value maps were encoded with
     cudaStream_t last_stream = nullptr;
@@ -560,6 +636,7 @@ tc_status tc_annca_create(int32_t H, int32_t d, int32_t nbits, const tc_options*
         for (int i = 0; i < d; ++i) s2 += (double)x->Rhost[(size_t)b * d + i] * x->Rhost[(size_t)b * d + i];
         rnorm[b] = std::nextafter((float)std::sqrt(s2), INFINITY);
     }
+    x->Rnorm_host = rnorm;
     AnnView& a = x->a;
     a.H = H;
     a.d = d;
@@ -650,7 +727,8 @@ tc_status tc_annca_attend(tc_annca_handle x, const void* Q, int64_t Tq, int32_t 
         e = cudaMemsetAsync(a.keep, 0, (size_t)a.Zmax * a.Lp * 4, cs);
         a.gen = 1;
     }
-    if (e == cudaSuccess) e = launch_annca_select(a, Q, Tq, P, (int)F, x->R, x->Rnorm, x->stats, cs);
+    if (e == cudaSuccess)
+        e = launch_annca_select(a, Q, Tq, P, (int)F, x->R, x->Rhost.data(), x->Rnorm_host.data(), x->stats, cs);
     if (e == cudaSuccess)
         e = launch_attend_cross_bf16(a, m, Tq, P, (int)F, static_cast<__nv_bfloat16*>(out),
                                      (float)((double)x->scale * 1.4426950408889634), x->stats, cs);
@@ -691,9 +769,12 @@ tc_status tc_annca_kept(tc_annca_handle x, int64_t* T_out, int64_t* F_out, int32
     if (counts && Z) e = cudaMemcpy(counts, a.nsel, (size_t)Z * 4, cudaMemcpyDeviceToHost);
     for (int64_t z = 0; index && e == cudaSuccess && z < Z; ++z)
         e = cudaMemcpy(index + z * a.L, a.sidx + z * a.Lp, (size_t)a.L * 4, cudaMemcpyDeviceToHost);
-    for (int h = 0; qcodes && e == cudaSuccess && h < x->H && x->last_T; ++h)
-        e = cudaMemcpy(qcodes + (int64_t)h * x->last_T, a.qcode + (int64_t)h * a.Tmax, (size_t)x->last_T * 4,
-                       cudaMemcpyDeviceToHost);
+    if (qcodes && e == cudaSuccess && x->last_T) {   // stored token-major, returned head-major
+        std::vector<uint32_t> tm((size_t)x->last_T * x->H);
+        e = cudaMemcpy(tm.data(), a.qcode, tm.size() * 4, cudaMemcpyDeviceToHost);
+        for (int64_t t = 0; e == cudaSuccess && t < x->last_T; ++t)
+            for (int h = 0; h < x->H; ++h) qcodes[(int64_t)h * x->last_T + t] = tm[(size_t)t * x->H + h];
+    }
     for (int h = 0; pcodes && e == cudaSuccess && h < x->H && x->prompt_set; ++h)
         e = cudaMemcpy(pcodes + (int64_t)h * a.L, a.pcode + (int64_t)h * a.Lp, (size_t)a.L * 4,
                        cudaMemcpyDeviceToHost);

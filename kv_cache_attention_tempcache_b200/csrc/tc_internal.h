@@ -117,7 +117,7 @@ struct AnnView {
     float* kmax2;          // [H] upper bound of |k|^2 over the prompt keys
     float* zeros;          // [H] zeros: log2 n bound and staged-key bound of the attention
     int64_t Tmax;          // query rows the per-query arrays hold
-    uint32_t* qcode;       // [H][Tmax] hash codes of the last query block
+    uint32_t* qcode;       // [Tmax][H] hash codes of the last query block (token-major)
     int64_t Zmax;          // slots the per-frame arrays hold
     uint32_t* keep;        // [Zmax][Lp] per slot, one stamp per bucket of the prompt, at the
                            // bucket's first sorted position: equal to gen when a query of the
@@ -133,8 +133,10 @@ struct AnnView {
 // Launchers (tc_annca.cu, tc_attn_bf16.cu).
 cudaError_t launch_annca_prompt(const AnnView& a, const void* Kp, const void* Vp, const float* R,
                                 const float* Rnorm, Stats* stats, cudaStream_t st);
+// R: device normals (fp64 re-checks); Rhost, Rnorm_host: host copies, passed to the
+// hash kernel by value.
 cudaError_t launch_annca_select(const AnnView& a, const void* Q, int64_t Tq, int P, int F, const float* R,
-                                const float* Rnorm, Stats* stats, cudaStream_t st);
+                                const float* Rhost, const float* Rnorm_host, Stats* stats, cudaStream_t st);
 cudaError_t launch_attend_cross_bf16(const AnnView& a, const AttnMaps& maps, int64_t Tq, int P, int F,
                                      __nv_bfloat16* out, float scale_log2, Stats* stats, cudaStream_t st);
 
