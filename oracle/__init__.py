@@ -20,3 +20,7 @@ from .annca_oracle import (  # noqa: F401
     annca_cross_attention,
     kept_prompt_tokens,
 )
+from .annsa_oracle import (  # noqa: F401
+    annsa_attention,
+    same_bucket_groups,
+)
