@@ -258,6 +258,26 @@ tc_status tc_annca_attend(tc_annca_handle h, const void* Q, int64_t Tq, int32_t 
 tc_status tc_annca_kept(tc_annca_handle h, int64_t* T_out, int64_t* F_out, int32_t* L_out,
                         int32_t* counts, int32_t* index, uint32_t* qcodes, uint32_t* pcodes);
 
+/*
+ * tc_annsa_attend - AnnSA (FAST-AR technical summary, section 2.C "AnnSA", pt and fr
+ * pages): self-attention of the block whose cross-attention the last tc_annca_attend
+ * of this handle pruned, restricted to the buckets that pruning found. Token t's bucket
+ * in head h is the code of its AnnCA query there; its self-attention query sees only
+ * the keys of the tokens in its own bucket:
+ *   out_t = sum_{j: b(j) = b(t)} exp(scale <q_t, k_j>) v_j / sum_{same j} exp(...)
+ * (never empty: t is in its own bucket). Q, K, V, out DEVICE [T, H, d] bf16 are the
+ * self-attention projections of the same T tokens; out must not overlap Q, K or V.
+ * The tokens are put in bucket order per head and packed; the attention runs every
+ * 128-row query tile against the 128-row key tiles spanning its buckets, on tensor
+ * cores with the same-bucket mask applied per element (block-sparse).
+ * Asynchronous on `stream` (an ordering kernel, a packing kernel and the attention
+ * kernel). Returns TC_ESTATE unless the last tc_annca_attend had Tq == T, and
+ * TC_EINVAL unless 1 <= T <= 16384. Growing T past the largest earlier value
+ * reallocates (and synchronises first).
+ */
+tc_status tc_annsa_attend(tc_annca_handle h, const void* Q, const void* K, const void* V,
+                          int64_t T, void* out, tc_stream stream);
+
 /* tc_annca_get_hyperplanes - the hash normals in use, HOST [nbits * d]. */
 tc_status tc_annca_get_hyperplanes(tc_annca_handle h, float* R);
 

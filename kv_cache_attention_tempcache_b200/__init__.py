@@ -30,7 +30,7 @@ API = [
     "tc_destroy", "tc_status_string", "tc_debug_last_commit", "tc_debug_staged_codes", "tc_export_cache",
     "tc_get_hyperplanes", "tc_stats", "tc_merge_means_noalloc",
     "tc_annca_create", "tc_annca_set_prompt", "tc_annca_attend", "tc_annca_kept", "tc_annca_get_hyperplanes",
-    "tc_annca_sync", "tc_annca_destroy",
+    "tc_annca_sync", "tc_annca_destroy", "tc_annsa_attend",
 ]
 
 
@@ -72,6 +72,7 @@ def _load():
         "tc_annca_get_hyperplanes": (ctypes.c_int, [H, vp]),
         "tc_annca_sync": (ctypes.c_int, [H]),
         "tc_annca_destroy": (None, [H]),
+        "tc_annsa_attend": (ctypes.c_int, [H, vp, vp, vp, i64, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -314,6 +315,22 @@ class AnnCA:
                 raise TempCacheError(TC_ESTATE, "tc_annca_kept: kept list not ascending")
             keep[z // F, z % F, ids] = True
         return keep, qcodes, pcodes
+
+    def self_attend(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor,
+                    out: torch.Tensor | None = None) -> torch.Tensor:
+        """AnnSA (FAST-AR summary, section 2.C): self-attention of the block the last
+        attend() pruned, each token seeing only the tokens of its own AnnCA bucket."""
+        Q = self._dev(Q, "Q")
+        K = self._dev(K, "K")
+        V = self._dev(V, "V")
+        if not (Q.shape == K.shape == V.shape):
+            raise ValueError("Q, K and V shapes differ")
+        if out is None:
+            out = torch.empty_like(Q)
+        self._keep_sa = [Q, K, V]
+        _check(lib.tc_annsa_attend(self._h, Q.data_ptr(), K.data_ptr(), V.data_ptr(), Q.shape[0], out.data_ptr(),
+                                   TempCache._stream()), "tc_annsa_attend")
+        return out
 
     def hyperplanes(self) -> np.ndarray:
         R = np.zeros((self.nbits, self.d), np.float32)

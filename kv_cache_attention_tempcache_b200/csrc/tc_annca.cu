@@ -447,7 +447,148 @@ cudaError_t select_t(const AnnView& a, const void* Qv, int64_t Tq, int P, int F,
     return cudaLaunchKernelEx(&cfg, annca_pack_kernel<D>, F, a);
 }
 
+// ------------------------------------------------------------------ AnnSA
+//
+// FAST-AR technical summary, section 2.C "AnnSA": the buckets found while pruning the
+// cross-attention are reused and every token's self-attention query only sees the keys
+// of its own bucket. Here a token's bucket is its AnnCA query code in the same head; the
+// tokens of the block are put in bucket order per head, packed, and the attention
+// kernel's sparse mode runs every 128-row query tile against the key tiles spanning its
+// buckets, masked per element to the same bucket.
+
+constexpr int kMaxSparseT = 16384;   // tokens per block (the ordering sorts in shared memory)
+
+// One block per head: bitonic sort of (code, token); per packed row its token and code;
+// per query tile the key tiles from the start of its first row's bucket to the end of its
+// last row's bucket.
+__global__ void __launch_bounds__(1024) annsa_order_kernel(SparseBufs b) {
+    extern __shared__ unsigned long long okey[];
+    const int h = blockIdx.x;
+    const int T = (int)b.T;
+    int n = 1;
+    while (n < T) n <<= 1;
+    for (int i = threadIdx.x; i < n; i += blockDim.x)
+        okey[i] = (i < T) ? ((unsigned long long)b.codes[(int64_t)i * b.H + h] << 32) | (unsigned)i : ~0ull;
+    __syncthreads();
+    for (int k = 2; k <= n; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = threadIdx.x; i < n; i += blockDim.x) {
+                const int p = i ^ j;
+                if (p > i) {
+                    const unsigned long long u = okey[i], w = okey[p];
+                    if ((u > w) == ((i & k) == 0)) {
+                        okey[i] = w;
+                        okey[p] = u;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int64_t i = threadIdx.x; i < b.Tp; i += blockDim.x) {
+        const int64_t o = (int64_t)h * b.Tp + i;
+        b.perm[o] = (i < T) ? (int32_t)(okey[i] & 0xffffffffu) : -1;
+        b.grp[o] = (i < T) ? (uint32_t)(okey[i] >> 32) : 0xffffffffu;
+    }
+    const int nqt = (int)(b.Tp / 128);   // row stride of tiles
+    for (int k = threadIdx.x; k < (T + 127) / 128; k += blockDim.x) {
+        const int f = 128 * k, l = min(f + 127, T - 1);
+        const uint32_t cf = (uint32_t)(okey[f] >> 32), cl = (uint32_t)(okey[l] >> 32);
+        int lo = 0, hi = f;   // first row of cf's bucket
+        while (lo < hi) {
+            const int mid = (lo + hi) >> 1;
+            if ((uint32_t)(okey[mid] >> 32) < cf) lo = mid + 1;
+            else hi = mid;
+        }
+        int lo2 = l, hi2 = T;   // one past the last row of cl's bucket
+        while (lo2 < hi2) {
+            const int mid = (lo2 + hi2) >> 1;
+            if ((uint32_t)(okey[mid] >> 32) <= cl) lo2 = mid + 1;
+            else hi2 = mid;
+        }
+        b.tiles[(int64_t)h * nqt + k] = make_int2(lo / 128, (lo2 + 127) / 128);
+    }
+}
+
+// One warp per packed row r = h Tp + i: copy the token's q, k, v rows (zeros past T),
+// its own logit scale log2(e) <q, k> (the first softmax reference when the kernel cannot
+// use a fixed one) and the head's bound of |k|^2.
+template <int D>
+__global__ void __launch_bounds__(kWarps * 32) annsa_pack_kernel(SparseBufs b, const __nv_bfloat16* __restrict__ Q,
+                                                                 const __nv_bfloat16* __restrict__ K,
+                                                                 const __nv_bfloat16* __restrict__ V,
+                                                                 float scale_log2) {
+    grid_dependency_wait();
+    constexpr int W = D / 8;   // 16-byte words per row (<= 16)
+    const int lane = threadIdx.x & 31;
+    const int64_t Tr = (b.T + 127) / 128 * 128;   // packed rows per head the attention reads
+    const int64_t rows = (int64_t)b.H * Tr;
+    const uint4* Q4 = reinterpret_cast<const uint4*>(Q);
+    const uint4* K4 = reinterpret_cast<const uint4*>(K);
+    const uint4* V4 = reinterpret_cast<const uint4*>(V);
+    uint4* Qs4 = reinterpret_cast<uint4*>(b.Qs);
+    uint4* Ks4 = reinterpret_cast<uint4*>(b.Ks);
+    uint4* Vs4 = reinterpret_cast<uint4*>(b.Vs);
+    for (int64_t rr = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; rr < rows;
+         rr += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+        const int h = (int)(rr / Tr);
+        const int64_t r = (int64_t)h * b.Tp + (rr - (int64_t)h * Tr);
+        const int32_t t = b.perm[r];
+        float qk = 0.f, kk = 0.f;
+        if (lane < W) {
+            uint4 q4 = make_uint4(0u, 0u, 0u, 0u), k4 = q4, v4 = q4;
+            if (t >= 0) {
+                const int64_t src = ((int64_t)t * b.H + h) * W + lane;
+                q4 = Q4[src];
+                k4 = K4[src];
+                v4 = V4[src];
+            }
+            Qs4[r * W + lane] = q4;
+            Ks4[r * W + lane] = k4;
+            Vs4[r * W + lane] = v4;
+            const uint32_t qw[4] = {q4.x, q4.y, q4.z, q4.w}, kw[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float ql = __uint_as_float(qw[e] << 16), qh = __uint_as_float(qw[e] & 0xffff0000u);
+                const float kl = __uint_as_float(kw[e] << 16), kh = __uint_as_float(kw[e] & 0xffff0000u);
+                qk = fmaf(ql, kl, fmaf(qh, kh, qk));
+                kk = fmaf(kl, kl, fmaf(kh, kh, kk));
+            }
+        }
+        qk = warp_sum(qk);
+        kk = warp_sum(kk);
+        if (lane == 0) {
+            b.xself[r] = qk * scale_log2;
+            atomicMax(reinterpret_cast<int*>(b.kmax2 + h), __float_as_int(kk * (1.f + 1.f / 1024.f)));
+        }
+    }
+    grid_dependents_launch();
+}
+
 }  // namespace
+
+cudaError_t launch_annsa_pack(const SparseBufs& b, const void* Q, const void* K, const void* V, float scale_log2,
+                              cudaStream_t st) {
+    int n = 1;
+    while (n < b.T) n <<= 1;
+    const int smem = n * 8;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(annsa_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kMaxSparseT * 8);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    annsa_order_kernel<<<b.H, 1024, smem, st>>>(b);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int grid = grid_for_rows((int64_t)b.H * ((b.T + 127) / 128 * 128), kWarps, 148 * 8);
+    const auto* q = reinterpret_cast<const __nv_bfloat16*>(Q);
+    const auto* k = reinterpret_cast<const __nv_bfloat16*>(K);
+    const auto* v = reinterpret_cast<const __nv_bfloat16*>(V);
+    return b.d == 128 ? launch_pdl(annsa_pack_kernel<128>, grid, kWarps * 32, st, b, q, k, v, scale_log2)
+                      : launch_pdl(annsa_pack_kernel<64>, grid, kWarps * 32, st, b, q, k, v, scale_log2);
+}
 
 cudaError_t launch_annca_prompt(const AnnView& a, const void* Kp, const void* Vp, const float* R,
                                 const float* Rnorm, Stats* stats, cudaStream_t st) {
@@ -490,6 +631,11 @@ struct tc_annca_ctx {
     std::vector<float> Rnorm_host;
     AttnMaps maps{};
     int64_t maps_Lp = -1;   // row stride the key/value maps were encoded with
+    // AnnSA buffers, sized for sp_Tp packed rows per head
+    SparseBufs sb{};
+    int64_t sp_Tp = 0;
+    float* sp_kmax2 = nullptr;
+    AttnMaps sp_maps{};
     cudaStream_t last_stream = nullptr;
     tc_status sticky = TC_OK;
 
@@ -530,10 +676,18 @@ struct tc_annca_ctx {
         a.sbias = nullptr;
         a.Zmax = 0;
     }
+    void free_sparse() {
+        void* ps[] = {sb.perm, sb.grp, sb.tiles, sb.xself, sb.Qs, sb.Ks, sb.Vs};
+        for (void* p : ps) if (p) cudaFree(p);
+        sb = SparseBufs{};
+        sp_Tp = 0;
+    }
     ~tc_annca_ctx() {
         free_prompt();
         free_queries();
         free_slots();
+        free_sparse();
+        if (sp_kmax2) cudaFree(sp_kmax2);
         void* ps[] = {R, Rnorm, stats, a.kmax2, a.zeros, a.ptab};
         for (void* p : ps) if (p) cudaFree(p);
         magic = 0;
@@ -778,6 +932,64 @@ tc_status tc_annca_kept(tc_annca_handle x, int64_t* T_out, int64_t* F_out, int32
     for (int h = 0; pcodes && e == cudaSuccess && h < x->H && x->prompt_set; ++h)
         e = cudaMemcpy(pcodes + (int64_t)h * a.L, a.pcode + (int64_t)h * a.Lp, (size_t)a.L * 4,
                        cudaMemcpyDeviceToHost);
+    return cuda_status(e);
+}
+
+tc_status tc_annsa_attend(tc_annca_handle x, const void* Q, const void* K, const void* V, int64_t T, void* out,
+                          tc_stream stream) {
+    tc_status st = check_call(x);
+    if (st) return st;
+    if (!Q || !K || !V || !out || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(out) || T < 1 ||
+        T > kMaxSparseT)
+        return TC_EINVAL;
+    const size_t bytes = (size_t)T * x->H * x->d * 2;
+    const char* o = static_cast<const char*>(out);
+    for (const void* in : {Q, K, V}) {
+        const char* p = static_cast<const char*>(in);
+        if (p < o + bytes && o < p + bytes) return TC_EINVAL;
+    }
+    if (!x->prompt_set || x->last_T != T) return TC_ESTATE;   // the buckets of this block come from AnnCA
+    if (up128(T) > x->sp_Tp) {
+        const int64_t Tp = up128(T);
+        if (cudaDeviceSynchronize() != cudaSuccess) return cuda_status(cudaGetLastError());
+        x->free_sparse();
+        SparseBufs& b = x->sb;
+        const size_t rows = (size_t)x->H * Tp;
+        if ((st = x->grab(b.perm, rows * 4)) || (st = x->grab(b.grp, rows * 4)) ||
+            (st = x->grab(b.tiles, rows / 128 * sizeof(int2))) || (st = x->grab(b.xself, rows * 4)) ||
+            (st = x->grab(b.Qs, rows * x->d * 2)) || (st = x->grab(b.Ks, rows * x->d * 2)) ||
+            (st = x->grab(b.Vs, rows * x->d * 2)) ||
+            (!x->sp_kmax2 && (st = x->grab(x->sp_kmax2, (size_t)x->H * 4)))) {
+            x->free_sparse();
+            return st;
+        }
+        const uint64_t d = x->d;
+        if (!encode3d(&x->sp_maps.q, b.Qs, d, Tp, x->H, d * 2, Tp * d * 2, 64, 128, 1) ||
+            !encode3d(&x->sp_maps.kc, b.Ks, d, Tp, x->H, d * 2, Tp * d * 2, 64, 128, 1) ||
+            !encode3d(&x->sp_maps.vc, b.Vs, d, Tp, x->H, d * 2, Tp * d * 2, 64, 128, 1)) {
+            x->free_sparse();
+            return TC_ECUDA;
+        }
+        x->sp_Tp = Tp;
+    }
+    const int64_t Tp = x->sp_Tp;   // row stride of the packed arrays (their allocation)
+    SparseBufs b = x->sb;
+    b.H = x->H;
+    b.d = x->d;
+    b.T = T;
+    b.Tp = Tp;
+    b.codes = x->a.qcode;
+    b.kmax2 = x->sp_kmax2;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    x->last_stream = cs;
+    const float scale_log2 = (float)((double)x->scale * 1.4426950408889634);
+    cudaError_t e = cudaMemsetAsync(x->sp_kmax2, 0, (size_t)x->H * 4, cs);
+    if (e == cudaSuccess) e = launch_annsa_pack(b, Q, K, V, scale_log2, cs);
+    if (e == cudaSuccess) {
+        SparseArgs sp{b.tiles, b.grp, b.perm, b.xself, Tp, (int)(Tp / 128)};
+        e = launch_attend_sparse_bf16(x->H, x->d, sp, x->sp_maps, T, x->sp_kmax2, x->a.zeros,
+                                      static_cast<__nv_bfloat16*>(out), scale_log2, x->stats, cs);
+    }
     return cuda_status(e);
 }
 

@@ -255,7 +255,16 @@ struct CfgU {
 //               retired (up to three tiles ahead).
 //   warp 18     lane 0 TMA producer for the V ring (2 stages).
 //   warp 19     lane 0 issues O += P_i V_i in tile order.
-template <int D, bool CROSS>
+enum { kSelf = 0, kCross = 1, kSparse = 2 };   // kernel modes (see the prologue)
+
+// A bucket code as a float's bits -> logit shift 0 when it equals the row's code, else
+// -inf (same-bucket mask of the sparse mode).
+__device__ __forceinline__ float4 mask4(float4 c, uint32_t gq) {
+    return make_float4(__float_as_uint(c.x) == gq ? 0.f : -INFINITY, __float_as_uint(c.y) == gq ? 0.f : -INFINITY,
+                       __float_as_uint(c.z) == gq ? 0.f : -INFINITY, __float_as_uint(c.w) == gq ? 0.f : -INFINITY);
+}
+
+template <int D, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
                        const __grid_constant__ CUtensorMap tmVc, const __grid_constant__ CUtensorMap tmKs,
@@ -263,7 +272,9 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                        const float* __restrict__ bias2, const float* __restrict__ kmax2c,
                        const float* __restrict__ kmax2s, const float* __restrict__ bmaxh, int64_t capP,
                        const float* __restrict__ sbias, int64_t Ts, int64_t Tq, int H, int Pf, int Ff,
-                       __nv_bfloat16* __restrict__ out, float scale_log2, Stats* stats) {
+                       const SparseArgs sp, __nv_bfloat16* __restrict__ out, float scale_log2, Stats* stats) {
+    constexpr bool CROSS = MODE == kCross;
+    constexpr bool SPARSE = MODE == kSparse;
     using C = Cfg<D>;
     using L = CfgU<D>;
     constexpr int kWK = 16, kWQK = 17, kWV = 18, kWPV = 19;
@@ -287,9 +298,20 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     // are committed entries (slot h of the cache arrays) then staged tokens.
     // Cross-attention: the query rows are Ff frames of Pf rows; CTA x covers rows of one
     // frame f, and the keys are the kept prompt tokens of slot h Ff + f, nothing staged.
-    int q0, zc;
+    // Sparse (same-bucket) self-attention: rows are in bucket order (packed, head-major);
+    // CTA x covers packed rows [128 x, 128 x + 128) of head h, the keys are the packed
+    // tiles [kt0, kt1) that hold its rows' buckets, masked per element to the same bucket.
+    int q0, zc, kt0 = 0, nsp = 0;
     int64_t qend;
-    if constexpr (CROSS) {
+    if constexpr (SPARSE) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");   // the packing kernel's output
+        q0 = blockIdx.x * kBM;
+        qend = Tq;
+        zc = h;
+        const int2 kr = sp.tiles[(int64_t)h * sp.nqt + blockIdx.x];
+        kt0 = kr.x;
+        nsp = kr.y - kr.x;
+    } else if constexpr (CROSS) {
         // launched as a programmatic dependent of the kernel that packs the keys: wait
         // for it before reading anything it writes
         asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -303,9 +325,8 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         qend = Tq;
         zc = h;
     }
-    const int Mh = Mdev[zc];
-    const int nc = (Mh + kBN - 1) / kBN;
-    const int ntiles = nc + (CROSS ? 0 : (int)((Ts + kBN - 1) / kBN));
+    const int nc = SPARSE ? nsp : (Mdev[zc] + kBN - 1) / kBN;
+    const int ntiles = nc + ((CROSS || SPARSE) ? 0 : (int)((Ts + kBN - 1) / kBN));
     if constexpr (CROSS) {
         if (ntiles == 0) {   // no key: the rows are the empty sum, zero
             constexpr int W = D / 8;   // 16-byte words per row
@@ -371,14 +392,19 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         const CUtensorMap* ms = kside ? &tmKs : &tmVs;
         if (kside) {
             mbar_expect_tx(&bars[U_QFULL], C::TILE);
-            for (int b = 0; b < C::NB; ++b) tma_load_3d(sQ + b * C::BOX, &tmQ, 64 * b, h, q0, &bars[U_QFULL]);
+            for (int b = 0; b < C::NB; ++b) {
+                if constexpr (SPARSE)   // packed queries, head-major
+                    tma_load_3d(sQ + b * C::BOX, &tmQ, 64 * b, q0, h, &bars[U_QFULL]);
+                else
+                    tma_load_3d(sQ + b * C::BOX, &tmQ, 64 * b, h, q0, &bars[U_QFULL]);
+            }
         }
         int last = -1;
         for (int i = 0; i < ntiles && !*abort_flag; ++i) {
             const int st = i % nst;
             if (i >= nst && !mbar_wait(&empty[st], ((i / nst) - 1) & 1)) { *abort_flag = 1; break; }
             const bool cache = i < nc;
-            const int row0 = (cache ? i : i - nc) * kBN;
+            const int row0 = ((cache ? i : i - nc) + kt0) * kBN;
             mbar_expect_tx(&full[st], C::TILE);
             for (int b = 0; b < C::NB; ++b)
                 tma_load_3d(ring + st * C::TILE + b * C::BOX, cache ? mc : ms, 64 * b, row0, cache ? zc : h,
@@ -449,7 +475,11 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         const int r = wt * 32 + lane;        // query row within the tile = TMEM lane
         const uint32_t lane_base = (uint32_t)(wt * 32) << 16;
         const uint32_t tOh = tO + HC * g + lane_base;
-        const float* bias_h = bias2 + (int64_t)zc * capP;
+        // (sparse mode: the "bias" rows are the packed rows' bucket codes, as float bits,
+        // and turn into 0 / -inf by comparison with the row's own code gq)
+        const float* bias_h = SPARSE ? reinterpret_cast<const float*>(sp.grp) + (int64_t)h * sp.Tp + (int64_t)kt0 * kBN
+                                     : bias2 + (int64_t)zc * capP;
+        const uint32_t gq = SPARSE ? sp.grp[(int64_t)h * sp.Tp + q0 + r] : 0u;
         auto bias_of = [&](int i) -> float {
             return (i < nc) ? bias_h[(int64_t)i * kBN + r] : sbias[(int64_t)(i - nc) * kBN + r];
         };
@@ -508,7 +538,7 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 if (lane < 2 && i + 2 < ntiles)
                     asm volatile("prefetch.global.L1 [%0];" ::"l"(bias_row(i + 2) + 32 * lane));
                 const uint32_t tS = tmem + b * 128 + 64 * g + lane_base;
-                const float4* brow = reinterpret_cast<const float4*>(bias_row(i));
+                const float4* brow = reinterpret_cast<const float4*>(bias_row(i));   // (codes when sparse)
                 uint64_t sumA = pk2(0.f, 0.f), sumB = pk2(0.f, 0.f);
 #pragma unroll 1
                 for (int h2 = 0; h2 < 2; ++h2) {
@@ -518,7 +548,8 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     uint32_t pk[16];
 #pragma unroll
                     for (int j = 0; j < 32; j += 4) {
-                        const float4 b4 = __ldg(brow + 8 * h2 + j / 4);
+                        float4 b4 = __ldg(brow + 8 * h2 + j / 4);
+                        if constexpr (SPARSE) b4 = mask4(b4, gq);
                         const uint64_t x01 = fma2(pk2(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), c2,
                                                   add2(pk2(b4.x, b4.y), negm2));
                         const uint64_t x23 = fma2(pk2(__uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3])), c2,
@@ -563,6 +594,12 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 TC_LD32(tS + 32, (sr + 32));
                 tc_wait_ld();
                 float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                if constexpr (SPARSE) {   // only the row's own bucket counts towards its bound
+                    const float* ch = sBias + (t * 3 + bb) * 128 + 64 * g;
+#pragma unroll
+                    for (int j = 0; j < 64; ++j)
+                        if (__float_as_uint(ch[j]) != gq) sr[j] = __float_as_uint(-INFINITY);
+                }
 #pragma unroll
                 for (int j = 0; j < 64; j += 8) {
                     m4[0] = max3(m4[0], __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
@@ -572,20 +609,23 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 }
                 smax = fmaxf(max3(m4[0], m4[1], m4[2]), m4[3]);
             }
-            const float2 bm = *reinterpret_cast<const float2*>(sBmax + (t * 3 + bb) * 4 + 2 * g);
+            const float2 bm = SPARSE ? make_float2(0.f, 0.f)
+                                     : *reinterpret_cast<const float2*>(sBmax + (t * 3 + bb) * 4 + 2 * g);
             sUb[((t * 2 + u) * 2 + g) * 128 + r] = fmaf(smax, scale_log2, fmaxf(bm.x, bm.y));
             if (g == 0 && i + 2 < ntiles) stage_bias((k + 1) % 3, bnext);
             if (!bar_and(1 + t, 256, got)) { ok = false; break; }
             if (g == 0 && i + 4 < ntiles) bnext = bias_of(i + 4);
             const float ub = fmaxf(sUb[((t * 2 + u) * 2 + 0) * 128 + r], sUb[((t * 2 + u) * 2 + 1) * 128 + r]);
-            // The reference of tile i - 1, decided by the other team.
-            float mprev = -INFINITY;
+            // The reference of tile i - 1, decided by the other team. In the sparse mode a
+            // tile may hold no key of a row's bucket (bound -inf), so the first reference
+            // is the row's own logit, which is finite and never above the row's maximum.
+            float mprev = SPARSE ? sp.xself[(int64_t)h * sp.Tp + q0 + r] : -INFINITY;
             if (i > 0) {
                 const bool w = mbar_wait(&bars[U_MREADY + (t ^ 1)], ((i - 1) >> 1) & 1);
                 if (!__all_sync(0xffffffffu, w)) { ok = false; *abort_flag = 1; }
                 mprev = sMref[(t ^ 1) * 128 + r];
             }
-            const bool raise = i == 0 || ub > mprev + 8.f;
+            const bool raise = (!SPARSE && i == 0) || ub > mprev + 8.f;
             const float mnew = raise ? ub : mprev;
             if (g == 0) {
                 sMref[t * 128 + r] = mnew;
@@ -626,7 +666,8 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 uint32_t pk[16];
 #pragma unroll
                 for (int j = 0; j < 32; j += 4) {
-                    const float4 b4 = *reinterpret_cast<const float4*>(bh + 32 * h2 + j);
+                    float4 b4 = *reinterpret_cast<const float4*>(bh + 32 * h2 + j);
+                    if constexpr (SPARSE) b4 = mask4(b4, gq);
                     const uint64_t x01 = fma2(pk2(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), c2,
                                               add2(pk2(b4.x, b4.y), negm2));
                     const uint64_t x23 = fma2(pk2(__uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3])), c2,
@@ -673,7 +714,8 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             tc_wait_ld();
             const int64_t row = q0 + r;
             if (row < qend) {
-                uint4* dst = reinterpret_cast<uint4*>(out + (row * H + h) * D + col);
+                const int64_t tok = SPARSE ? (int64_t)sp.perm[(int64_t)h * sp.Tp + row] : row;
+                uint4* dst = reinterpret_cast<uint4*>(out + (tok * H + h) * D + col);
 #pragma unroll
                 for (int v = 0; v < QC / 8; ++v) {
                     uint4 w4;
@@ -700,11 +742,11 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-template <int D, bool CROSS>
+template <int D, int MODE>
 cudaError_t set_smem_attr() {
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(attend_bf16_duo_kernel<D, CROSS>,
+        cudaError_t e = cudaFuncSetAttribute(attend_bf16_duo_kernel<D, MODE>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, CfgU<D>::SMEM);
         if (e != cudaSuccess) return e;
         attr_set = true;
@@ -715,7 +757,7 @@ cudaError_t set_smem_attr() {
 template <int D>
 cudaError_t launch_t(const CacheView& c, const StageView& s, const AttnMaps& m, int64_t Tq, __nv_bfloat16* out,
                      float scale_log2, Stats* stats, bool overlap_prev, cudaStream_t st) {
-    cudaError_t e = set_smem_attr<D, false>();
+    cudaError_t e = set_smem_attr<D, kSelf>();
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((Tq + kBM - 1) / kBM), (unsigned)c.H);
@@ -727,10 +769,10 @@ cudaError_t launch_t(const CacheView& c, const StageView& s, const AttnMaps& m, 
     attr[0].val.programmaticStreamSerializationAllowed = overlap_prev ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, attend_bf16_duo_kernel<D, false>, m.q, m.kc, m.vc, m.ks, m.vs,
+    return cudaLaunchKernelEx(&cfg, attend_bf16_duo_kernel<D, kSelf>, m.q, m.kc, m.vc, m.ks, m.vs,
                               (const int32_t*)c.M, (const float*)c.bias2, (const float*)c.kmax2,
                               (const float*)c.kmax2s, (const float*)c.bmax, c.capP, (const float*)s.sbias, s.T, Tq,
-                              c.H, (int)Tq, 1, out, scale_log2, stats);
+                              c.H, (int)Tq, 1, SparseArgs{}, out, scale_log2, stats);
 }
 
 // Cross-attention over the kept prompt tokens: grid (F frames x tiles per frame, H),
@@ -739,7 +781,7 @@ cudaError_t launch_t(const CacheView& c, const StageView& s, const AttnMaps& m, 
 template <int D>
 cudaError_t launch_cross_t(const AnnView& a, const AttnMaps& m, int64_t Tq, int P, int F, __nv_bfloat16* out,
                            float scale_log2, Stats* stats, cudaStream_t st) {
-    cudaError_t e = set_smem_attr<D, true>();
+    cudaError_t e = set_smem_attr<D, kCross>();
     if (e != cudaSuccess) return e;
     const int tpf = (P + kBM - 1) / kBM;
     cudaLaunchConfig_t cfg = {};
@@ -752,10 +794,33 @@ cudaError_t launch_cross_t(const AnnView& a, const AttnMaps& m, int64_t Tq, int 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, attend_bf16_duo_kernel<D, true>, m.q, m.kc, m.vc, m.kc, m.vc,
+    return cudaLaunchKernelEx(&cfg, attend_bf16_duo_kernel<D, kCross>, m.q, m.kc, m.vc, m.kc, m.vc,
                               (const int32_t*)a.nsel, (const float*)a.sbias, (const float*)a.kmax2,
                               (const float*)a.zeros, (const float*)a.zeros, a.Lp, (const float*)nullptr, (int64_t)0,
-                              Tq, a.H, P, F, out, scale_log2, stats);
+                              Tq, a.H, P, F, SparseArgs{}, out, scale_log2, stats);
+}
+
+// Same-bucket self-attention over packed rows: grid (query tiles, H), a programmatic
+// dependent of the packing kernel.
+template <int D>
+cudaError_t launch_sparse_t(int H, const SparseArgs& sp, const AttnMaps& m, int64_t T, const float* kmax2,
+                            const float* zeros, __nv_bfloat16* out, float scale_log2, Stats* stats,
+                            cudaStream_t st) {
+    cudaError_t e = set_smem_attr<D, kSparse>();
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((T + kBM - 1) / kBM), (unsigned)H);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = CfgU<D>::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, attend_bf16_duo_kernel<D, kSparse>, m.q, m.kc, m.vc, m.kc, m.vc,
+                              (const int32_t*)nullptr, (const float*)nullptr, kmax2, zeros, zeros, sp.Tp,
+                              (const float*)nullptr, (int64_t)0, T, H, (int)T, 1, sp, out, scale_log2, stats);
 }
 
 }  // namespace
@@ -771,6 +836,13 @@ cudaError_t launch_attend_cross_bf16(const AnnView& a, const AttnMaps& maps, int
                                      __nv_bfloat16* out, float scale_log2, Stats* stats, cudaStream_t st) {
     return a.d == 128 ? launch_cross_t<128>(a, maps, Tq, P, F, out, scale_log2, stats, st)
                       : launch_cross_t<64>(a, maps, Tq, P, F, out, scale_log2, stats, st);
+}
+
+cudaError_t launch_attend_sparse_bf16(int H, int d, const SparseArgs& sp, const AttnMaps& maps, int64_t T,
+                                      const float* kmax2, const float* zeros, __nv_bfloat16* out,
+                                      float scale_log2, Stats* stats, cudaStream_t st) {
+    return d == 128 ? launch_sparse_t<128>(H, sp, maps, T, kmax2, zeros, out, scale_log2, stats, st)
+                    : launch_sparse_t<64>(H, sp, maps, T, kmax2, zeros, out, scale_log2, stats, st);
 }
 
 }  // namespace tc

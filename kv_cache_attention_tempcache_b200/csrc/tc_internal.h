@@ -130,6 +130,17 @@ struct AnnView {
     float* sbias;          // [Zmax][Lp] 0 for kept rows, -inf for the rest of the last tile
 };
 
+// AnnSA (same-bucket self-attention) arrays read by the attention kernel's sparse mode:
+// the tokens of one block in bucket order per head ("packed" rows, Tp = round_up(T, 128)).
+struct SparseArgs {
+    const int2* tiles;     // [H][nqt] key tiles [x, y) holding the buckets of each query tile
+    const uint32_t* grp;   // [H][Tp] bucket code of each packed row (0xffffffff past T)
+    const int32_t* perm;   // [H][Tp] token of each packed row
+    const float* xself;    // [H][Tp] the row's own logit, scale log2(e) <q, k>
+    int64_t Tp;            // row stride per head (>= round_up(T, 128))
+    int nqt;               // Tp / 128, the row stride of tiles
+};
+
 // Launchers (tc_annca.cu, tc_attn_bf16.cu).
 cudaError_t launch_annca_prompt(const AnnView& a, const void* Kp, const void* Vp, const float* R,
                                 const float* Rnorm, Stats* stats, cudaStream_t st);
@@ -139,6 +150,26 @@ cudaError_t launch_annca_select(const AnnView& a, const void* Q, int64_t Tq, int
                                 const float* Rhost, const float* Rnorm_host, Stats* stats, cudaStream_t st);
 cudaError_t launch_attend_cross_bf16(const AnnView& a, const AttnMaps& maps, int64_t Tq, int P, int F,
                                      __nv_bfloat16* out, float scale_log2, Stats* stats, cudaStream_t st);
+// maps.q: packed queries [H][Tp][d]; maps.kc / maps.vc: packed keys and values, same shape.
+cudaError_t launch_attend_sparse_bf16(int H, int d, const SparseArgs& sp, const AttnMaps& maps, int64_t T,
+                                      const float* kmax2, const float* zeros, __nv_bfloat16* out,
+                                      float scale_log2, Stats* stats, cudaStream_t st);
+// Bucket order and packing of one block for the sparse attention (tc_annca.cu).
+struct SparseBufs {
+    int H, d;
+    int64_t T, Tp;          // tokens; row stride per head of the packed arrays (>= round_up(T, 128))
+    const uint32_t* codes;  // [T][H] bucket codes (token-major)
+    int32_t* perm;          // [H][Tp]
+    uint32_t* grp;          // [H][Tp]
+    int2* tiles;            // [H][Tp/128]
+    float* xself;           // [H][Tp]
+    __nv_bfloat16* Qs;      // [H][Tp][d]
+    __nv_bfloat16* Ks;
+    __nv_bfloat16* Vs;
+    float* kmax2;           // [H], zeroed by the caller
+};
+cudaError_t launch_annsa_pack(const SparseBufs& b, const void* Q, const void* K, const void* V, float scale_log2,
+                              cudaStream_t st);
 
 // Host helpers (tc_runtime.cu).
 cudaError_t dev_alloc(void** p, size_t bytes);   // cudaMalloc with the TC_FAULT_ALLOC_AT injection

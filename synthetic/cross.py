@@ -84,6 +84,14 @@ class CrossWorkload:
         V = torch.randn(cfg.L, cfg.H, cfg.d, generator=g, device=self.device)
         return K.transpose(0, 1).contiguous().to(torch.bfloat16), V.to(torch.bfloat16)
 
+    def self_qkv(self, call: int):
+        """Self-attention projections Q, K, V [F*P, H, d] of the block of call `call`:
+        N(0, 1) draws rounded to bf16 (the buckets come from the cross-attention queries)."""
+        cfg = self.cfg
+        g = torch.Generator(device=self.device).manual_seed((cfg.seed * 7_000_003 + call * 104_729 + 11) % (2 ** 62))
+        return tuple(torch.randn(cfg.T, cfg.H, cfg.d, generator=g, device=self.device).to(torch.bfloat16)
+                     for _ in range(3))
+
     def queries(self, call: int) -> torch.Tensor:
         cfg = self.cfg
         g = torch.Generator(device=self.device).manual_seed((cfg.seed * 1_000_003 + call * 7919 + 3) % (2 ** 62))
