@@ -10,6 +10,7 @@ in HBM (3.5 GB of distinct K, V, Q per rollout, far larger than the 126 MB L2).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
   python bench.py --workload annca-wan1.3b     (AnnCA cross-attention, its own line)
+  python bench.py --workload annsa-wan1.3b     (AnnSA same-bucket self-attention, its own line)
 
 N > 1 runs under torchrun: each rank runs an independent rollout (its own seed);
 there is no collective in the data path, only the max-over-ranks of the timing.
@@ -577,6 +578,143 @@ def run_annca(args):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- AnnSA leg
+
+ANNSA_METRIC = "AnnSA same-bucket self-attention frames/s at Wan-1.3B shape (AnnCA buckets)"
+
+
+def run_annsa(args):
+    from kv_cache_attention_tempcache_b200 import AnnCA, TempCache
+    from synthetic import CrossWorkload
+
+    rank, world, local = dist_info()
+    torch.cuda.set_device(local)
+    init_dist(world, "nccl")
+    dev = torch.device("cuda", local)
+    cfg = CROSS_CONFIGS["annca-wan1.3b"]
+    cfg = cfg.replace(seed=rank_seed(cfg.seed, rank))
+    calls = 40   # 120 frames; 1.7 GB of distinct Q, K, V per step: larger than L2
+    w = CrossWorkload(cfg, device=dev)
+    R = w.hyperplanes().numpy()
+    Kp, Vp = w.prompt()
+    Qc = [w.queries(c) for c in range(calls)]
+    QKV = [w.self_qkv(c) for c in range(calls)]
+    out = torch.empty_like(Qc[0])
+    xout = torch.empty_like(Qc[0])
+    ann = AnnCA(cfg.H, cfg.d, cfg.nbits, hyperplanes=R)
+    ann.set_prompt(Kp, Vp)
+    flops = []
+    for c in range(calls):   # the algorithmic work: 4 n^2 d per bucket of n tokens, every head
+        ann.attend(Qc[c], cfg.P, out=xout)
+        _, qcodes, _ = ann.kept()
+        flops.append(sum(4.0 * float((np.unique(qcodes[h], return_counts=True)[1].astype(np.float64) ** 2).sum())
+                         * cfg.d for h in range(cfg.H)))
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    marks = [[(ev(), ev()) for _ in range(calls)] for _ in range(args.steps)]
+
+    def step(k=None):
+        for c in range(calls):
+            ann.attend(Qc[c], cfg.P, out=xout)   # the buckets of block c (not timed below)
+            if k is not None:
+                marks[k][c][0].record()
+            ann.self_attend(*QKV[c], out=out)
+            if k is not None:
+                marks[k][c][1].record()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        step(k)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    sec = sum(a.elapsed_time(b) for row in marks for a, b in row) / 1000.0
+    sec_max = max_over_ranks(sec, world, dev)
+    value = aggregate_rate(cfg.F * calls * args.steps, world, sec_max)
+    call_sec = sec / (args.steps * calls)
+    tflops = args.steps * sum(flops) / sec / 1e12
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks.get("bf16_tflops", 1590.0))
+
+    # dense baseline: the same attention kernel over the whole block (a TempCache whose
+    # only content is the block, staged)
+    dense = TempCache(cfg.H, cfg.d, 16, 2.0, cfg.T, hyperplanes=np.zeros((16, cfg.d), np.float32))
+    d0, d1 = ev(), ev()
+    dense_sec = 0.0
+    for c in range(calls):
+        Q, K, V = QKV[c]
+        dense.reset()
+        dense.append_chunk(K, V)
+        d0.record()
+        dense.attend(Q, out=out)
+        d1.record()
+        torch.cuda.synchronize()
+        dense_sec += d0.elapsed_time(d1) / 1000.0
+    dense.close()
+
+    # end to end: Q, K, V from pinned host memory and the output read back, per call (the
+    # AnnCA call that finds the buckets stays outside the events)
+    hq = [tuple(x.cpu().pin_memory() for x in qkv) for qkv in QKV[:8]]
+    ho = torch.empty(cfg.T, cfg.H, cfg.d, dtype=torch.bfloat16).pin_memory()
+    e2e_sec = 0.0
+    for c in range(8):
+        ann.attend(Qc[c], cfg.P, out=xout)
+        a0, a1 = ev(), ev()
+        a0.record()
+        ho.copy_(ann.self_attend(*hq[c]), non_blocking=True)
+        a1.record()
+        torch.cuda.synchronize()
+        e2e_sec += a0.elapsed_time(a1) / 1000.0
+    e2e_sec = max_over_ranks(e2e_sec, world, dev)
+    blk = cfg.T * cfg.H * cfg.d * 2
+
+    if rank != 0:
+        ann.close()
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        from oracle import annsa_attention
+        f = lambda x: x.to(torch.float64).cpu().numpy()  # noqa: E731
+        ann.attend(Qc[0], cfg.P, out=xout)
+        _, qcodes, _ = ann.kept()
+        t = time.perf_counter()
+        annsa_attention(*(f(x) for x in QKV[0]), qcodes)
+        cpu = {"value": cfg.F / (time.perf_counter() - t), "unit": UNIT, "cores": len(os.sched_getaffinity(0)),
+               "kind": "oracle", "sample": "one block (3 frames x 1560 tokens, 12 heads) in full"}
+    line = {
+        "metric": ANNSA_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * sec_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": (f"annsa-wan1.3b: H={cfg.H} d={cfg.d} T={cfg.T} (F={cfg.F} x P={cfg.P}), buckets "
+                                f"= {cfg.nbits}-bit AnnCA query codes (annca-wan1.3b), Q K V ~ N(0,1) bf16"),
+                   "step": f"{calls} tc_annsa_attend calls ({cfg.F * calls} frames); the AnnCA call that "
+                           "finds each block's buckets runs before it, outside the timed events",
+                   "l2": f"inputs larger than L2 ({calls * 3 * cfg.T * cfg.H * cfg.d * 2 / 1e9:.2f} GB of "
+                         "distinct Q, K, V per step)",
+                   "parallelism": f"independent layer per rank x{world}"},
+        "roofline": {"bound": "tensor", "kernel": "annsa_order_kernel + annsa_pack_kernel + attend_bf16_duo_kernel "
+                                                  "(sparse), one call",
+                     "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
+                     "peak_kind": f"{peak_kind} bf16 dense, burst", "traffic": None,
+                     "flops_per_call": float(np.mean(flops)), "avg_call_us": 1e6 * call_sec},
+        "dense_baseline": {"value": cfg.F * calls / dense_sec, "unit": UNIT,
+                           "note": "same attention kernel over the whole block (every token sees every token)"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": aggregate_rate(cfg.F * 8, world, e2e_sec), "unit": UNIT,
+                "h2d_bytes_per_step": 3 * blk * calls, "d2h_bytes_per_step": blk * calls},
+        "gpu_launches": 3 * calls * args.steps,
+        "clocks": clk,
+    }
+    ann.close()
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -589,7 +727,8 @@ def main():
     ap.add_argument("--chunks", type=int, default=0,
                     help="rollout length in chunks (default: the workload's); profiling runs use fewer")
     ap.add_argument("--workload", default=WORKLOAD,
-                    choices=[k for k, v in CONFIGS.items() if v.dtype == "bf16"] + ["annca-wan1.3b"],
+                    choices=[k for k, v in CONFIGS.items() if v.dtype == "bf16"] + ["annca-wan1.3b",
+                                                                                      "annsa-wan1.3b"],
                     help="synthetic workload; only the default one adds the dense, end-to-end and CPU legs "
                          "(annca-wan1.3b: AnnCA cross-attention, with its own legs)")
     ap.add_argument("--series", action="store_true", help="add per-chunk commit and attention times")
@@ -600,6 +739,8 @@ def main():
         run_reference(args)
     elif args.workload in CROSS_CONFIGS:
         run_annca(args)
+    elif args.workload == "annsa-wan1.3b":
+        run_annsa(args)
     else:
         run_gpu(args)
     if torch.distributed.is_initialized():
