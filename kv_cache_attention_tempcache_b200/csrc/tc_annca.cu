@@ -510,6 +510,91 @@ __global__ void __launch_bounds__(1024) annsa_order_kernel(SparseBufs b) {
     }
 }
 
+// The same order by counting, for codes below 2^kCountBits (one block per head, 1024
+// threads): bucket sizes by shared-memory atomics, bucket starts by a scan, then the
+// tokens are placed chunk by chunk in token order: inside a warp, lanes with the same
+// code rank themselves with a match mask, and the warps of a chunk take their places in
+// order, one warp per step, from a running cursor per code. The result equals the sort
+// of (code, token) above.
+constexpr int kCountBits = 13;
+
+__global__ void __launch_bounds__(1024) annsa_count_kernel(SparseBufs b, int nbits) {
+    extern __shared__ int32_t cs_smem[];
+    const int ncodes = 1 << nbits;
+    int32_t* cnt = cs_smem;              // [ncodes]
+    int32_t* cur = cs_smem + ncodes;     // [ncodes] running cursor, finally the bucket end
+    int32_t* sBase = cur + ncodes;       // [32][32] base position of each (warp, lane) group
+    __shared__ int wsum[32];
+    const int h = blockIdx.x, T = (int)b.T;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int c = threadIdx.x; c < ncodes; c += blockDim.x) cnt[c] = 0;
+    __syncthreads();
+    for (int t = threadIdx.x; t < T; t += blockDim.x) atomicAdd(&cnt[b.codes[(int64_t)t * b.H + h]], 1);
+    __syncthreads();
+    {   // exclusive scan of cnt into cur: each thread a contiguous run of codes
+        const int per = (ncodes + blockDim.x - 1) / blockDim.x;
+        const int c0 = min(ncodes, (int)threadIdx.x * per), c1 = min(ncodes, c0 + per);
+        int run = 0;
+        for (int c = c0; c < c1; ++c) run += cnt[c];
+        int inc = run;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+        }
+        if (lane == 31) wsum[warp] = inc;
+        __syncthreads();
+        if (warp == 0) {
+            int y = wsum[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int z = __shfl_up_sync(0xffffffffu, y, o);
+                if (lane >= o) y += z;
+            }
+            wsum[lane] = y;
+        }
+        __syncthreads();
+        int pos = (warp > 0 ? wsum[warp - 1] : 0) + inc - run;
+        for (int c = c0; c < c1; ++c) {
+            cur[c] = pos;
+            pos += cnt[c];
+        }
+    }
+    __syncthreads();
+    const unsigned lt = (1u << lane) - 1u;
+    for (int base = 0; base < T; base += blockDim.x) {
+        const int t = base + threadIdx.x;
+        const bool valid = t < T;
+        const uint32_t c = valid ? b.codes[(int64_t)t * b.H + h] : 0xffffffffu;
+        const unsigned same = __match_any_sync(0xffffffffu, c);
+        const int rank = __popc(same & lt), lead = __ffs(same) - 1;
+        for (int w = 0; w < 32; ++w) {
+            if (warp == w && valid && lane == lead) {
+                sBase[w * 32 + lane] = cur[c];
+                cur[c] += __popc(same);
+            }
+            __syncthreads();
+        }
+        if (valid) {
+            const int64_t o = (int64_t)h * b.Tp + sBase[warp * 32 + lead] + rank;
+            b.perm[o] = t;
+            b.grp[o] = c;
+        }
+        __syncthreads();
+    }
+    for (int64_t i = T + threadIdx.x; i < b.Tp; i += blockDim.x) {
+        b.perm[(int64_t)h * b.Tp + i] = -1;
+        b.grp[(int64_t)h * b.Tp + i] = 0xffffffffu;
+    }
+    __syncthreads();   // (this block's own global writes, read back below)
+    const int nqt = (int)(b.Tp / 128);
+    for (int k = threadIdx.x; k < (T + 127) / 128; k += blockDim.x) {
+        const int f = 128 * k, l = min(f + 127, T - 1);
+        const uint32_t cf = b.grp[(int64_t)h * b.Tp + f], cl = b.grp[(int64_t)h * b.Tp + l];
+        b.tiles[(int64_t)h * nqt + k] = make_int2((cur[cf] - cnt[cf]) / 128, (cur[cl] + 127) / 128);
+    }
+}
+
 // One warp per packed row r = h Tp + i: copy the token's q, k, v rows (zeros past T),
 // its own logit scale log2(e) <q, k> (the first softmax reference when the kernel cannot
 // use a fixed one) and the head's bound of |k|^2.
@@ -519,8 +604,9 @@ __global__ void __launch_bounds__(kWarps * 32) annsa_pack_kernel(SparseBufs b, c
                                                                  const __nv_bfloat16* __restrict__ V,
                                                                  float scale_log2) {
     grid_dependency_wait();
-    constexpr int W = D / 8;   // 16-byte words per row (<= 16)
-    const int lane = threadIdx.x & 31;
+    constexpr int W = D / 8;        // 16-byte words per row: W lanes per row
+    constexpr int RPW = 32 / W;     // rows per warp and step
+    const int lane = threadIdx.x & 31, sub = lane / W, w = lane % W;
     const int64_t Tr = (b.T + 127) / 128 * 128;   // packed rows per head the attention reads
     const int64_t rows = (int64_t)b.H * Tr;
     const uint4* Q4 = reinterpret_cast<const uint4*>(Q);
@@ -529,35 +615,40 @@ __global__ void __launch_bounds__(kWarps * 32) annsa_pack_kernel(SparseBufs b, c
     uint4* Qs4 = reinterpret_cast<uint4*>(b.Qs);
     uint4* Ks4 = reinterpret_cast<uint4*>(b.Ks);
     uint4* Vs4 = reinterpret_cast<uint4*>(b.Vs);
-    for (int64_t rr = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; rr < rows;
-         rr += ((int64_t)gridDim.x * blockDim.x) >> 5) {
-        const int h = (int)(rr / Tr);
+    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t rr0 = (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5) * RPW; rr0 < rows; rr0 += nw * RPW) {
+        const int64_t rr = rr0 + sub;
+        const bool live = rr < rows;
+        const int h = live ? (int)(rr / Tr) : 0;
         const int64_t r = (int64_t)h * b.Tp + (rr - (int64_t)h * Tr);
-        const int32_t t = b.perm[r];
-        float qk = 0.f, kk = 0.f;
-        if (lane < W) {
-            uint4 q4 = make_uint4(0u, 0u, 0u, 0u), k4 = q4, v4 = q4;
-            if (t >= 0) {
-                const int64_t src = ((int64_t)t * b.H + h) * W + lane;
-                q4 = Q4[src];
-                k4 = K4[src];
-                v4 = V4[src];
-            }
-            Qs4[r * W + lane] = q4;
-            Ks4[r * W + lane] = k4;
-            Vs4[r * W + lane] = v4;
-            const uint32_t qw[4] = {q4.x, q4.y, q4.z, q4.w}, kw[4] = {k4.x, k4.y, k4.z, k4.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float ql = __uint_as_float(qw[e] << 16), qh = __uint_as_float(qw[e] & 0xffff0000u);
-                const float kl = __uint_as_float(kw[e] << 16), kh = __uint_as_float(kw[e] & 0xffff0000u);
-                qk = fmaf(ql, kl, fmaf(qh, kh, qk));
-                kk = fmaf(kl, kl, fmaf(kh, kh, kk));
-            }
+        const int32_t t = live ? b.perm[r] : -1;
+        uint4 q4 = make_uint4(0u, 0u, 0u, 0u), k4 = q4, v4 = q4;
+        if (t >= 0) {
+            const int64_t src = ((int64_t)t * b.H + h) * W + w;
+            q4 = Q4[src];
+            k4 = K4[src];
+            v4 = V4[src];
         }
-        qk = warp_sum(qk);
-        kk = warp_sum(kk);
-        if (lane == 0) {
+        if (live) {
+            Qs4[r * W + w] = q4;
+            Ks4[r * W + w] = k4;
+            Vs4[r * W + w] = v4;
+        }
+        const uint32_t qw[4] = {q4.x, q4.y, q4.z, q4.w}, kw[4] = {k4.x, k4.y, k4.z, k4.w};
+        float qk = 0.f, kk = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float ql = __uint_as_float(qw[e] << 16), qh = __uint_as_float(qw[e] & 0xffff0000u);
+            const float kl = __uint_as_float(kw[e] << 16), kh = __uint_as_float(kw[e] & 0xffff0000u);
+            qk = fmaf(ql, kl, fmaf(qh, kh, qk));
+            kk = fmaf(kl, kl, fmaf(kh, kh, kk));
+        }
+#pragma unroll
+        for (int o = 1; o < W; o <<= 1) {   // sums over the W lanes of this row
+            qk += __shfl_xor_sync(0xffffffffu, qk, o);
+            kk += __shfl_xor_sync(0xffffffffu, kk, o);
+        }
+        if (live && w == 0) {
             b.xself[r] = qk * scale_log2;
             atomicMax(reinterpret_cast<int*>(b.kmax2 + h), __float_as_int(kk * (1.f + 1.f / 1024.f)));
         }
@@ -567,22 +658,28 @@ __global__ void __launch_bounds__(kWarps * 32) annsa_pack_kernel(SparseBufs b, c
 
 }  // namespace
 
-cudaError_t launch_annsa_pack(const SparseBufs& b, const void* Q, const void* K, const void* V, float scale_log2,
-                              cudaStream_t st) {
-    int n = 1;
-    while (n < b.T) n <<= 1;
-    const int smem = n * 8;
-    static bool attr_set = false;
+cudaError_t launch_annsa_pack(const SparseBufs& b, int nbits, const void* Q, const void* K, const void* V,
+                              float scale_log2, cudaStream_t st) {
+static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(annsa_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              kMaxSparseT * 8);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(annsa_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (2 << kCountBits) * 4 + 32 * 32 * 4);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    annsa_order_kernel<<<b.H, 1024, smem, st>>>(b);
+    if (nbits <= kCountBits) {
+        annsa_count_kernel<<<b.H, 1024, (2 << nbits) * 4 + 32 * 32 * 4, st>>>(b, nbits);
+    } else {
+        int n = 1;
+        while (n < b.T) n <<= 1;
+        annsa_order_kernel<<<b.H, 1024, n * 8, st>>>(b);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const int grid = grid_for_rows((int64_t)b.H * ((b.T + 127) / 128 * 128), kWarps, 148 * 8);
+    const int grid = grid_for_rows((int64_t)b.H * ((b.T + 127) / 128 * 128), kWarps * (32 / (b.d / 8)), 148 * 8);
     const auto* q = reinterpret_cast<const __nv_bfloat16*>(Q);
     const auto* k = reinterpret_cast<const __nv_bfloat16*>(K);
     const auto* v = reinterpret_cast<const __nv_bfloat16*>(V);
@@ -984,7 +1081,7 @@ tc_status tc_annsa_attend(tc_annca_handle x, const void* Q, const void* K, const
     x->last_stream = cs;
     const float scale_log2 = (float)((double)x->scale * 1.4426950408889634);
     cudaError_t e = cudaMemsetAsync(x->sp_kmax2, 0, (size_t)x->H * 4, cs);
-    if (e == cudaSuccess) e = launch_annsa_pack(b, Q, K, V, scale_log2, cs);
+    if (e == cudaSuccess) e = launch_annsa_pack(b, x->nbits, Q, K, V, scale_log2, cs);
     if (e == cudaSuccess) {
         SparseArgs sp{b.tiles, b.grp, b.perm, b.xself, Tp, (int)(Tp / 128)};
         e = launch_attend_sparse_bf16(x->H, x->d, sp, x->sp_maps, T, x->sp_kmax2, x->a.zeros,

@@ -168,8 +168,8 @@ struct SparseBufs {
     __nv_bfloat16* Vs;
     float* kmax2;           // [H], zeroed by the caller
 };
-cudaError_t launch_annsa_pack(const SparseBufs& b, const void* Q, const void* K, const void* V, float scale_log2,
-                              cudaStream_t st);
+cudaError_t launch_annsa_pack(const SparseBufs& b, int nbits, const void* Q, const void* K, const void* V,
+                              float scale_log2, cudaStream_t st);
 
 // Host helpers (tc_runtime.cu).
 cudaError_t dev_alloc(void** p, size_t bytes);   // cudaMalloc with the TC_FAULT_ALLOC_AT injection
