@@ -399,13 +399,8 @@ cudaError_t prompt_t(const AnnView& a, const void* Kp, const void* Vp, const flo
 template <int D, int NBP>
 cudaError_t mark_t(const __nv_bfloat16* Q, int rows, int P, int F, const AnnView& a, const float* R,
                    const float* Rhost, const float* Rnorm_host, Stats* stats, cudaStream_t st) {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(annca_mark_kernel<D, NBP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             MarkSmem<D>::BYTES);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+    cudaError_t e = smem_attr_once(reinterpret_cast<const void*>(annca_mark_kernel<D, NBP>), MarkSmem<D>::BYTES);
+    if (e != cudaSuccess) return e;
     Planes<D, NBP> pl;
     for (int b = 0; b < NBP; ++b) {
         for (int i = 0; i < D; ++i) pl.v[b * D + i] = (b < a.nbits) ? Rhost[b * D + i] : 0.f;
@@ -660,16 +655,10 @@ __global__ void __launch_bounds__(kWarps * 32) annsa_pack_kernel(SparseBufs b, c
 
 cudaError_t launch_annsa_pack(const SparseBufs& b, int nbits, const void* Q, const void* K, const void* V,
                               float scale_log2, cudaStream_t st) {
-static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(annsa_order_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kMaxSparseT * 8);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(annsa_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (2 << kCountBits) * 4 + 32 * 32 * 4);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
+cudaError_t e = smem_attr_once(reinterpret_cast<const void*>(annsa_order_kernel), kMaxSparseT * 8);
+    if (e == cudaSuccess)
+        e = smem_attr_once(reinterpret_cast<const void*>(annsa_count_kernel), (2 << kCountBits) * 4 + 32 * 32 * 4);
+    if (e != cudaSuccess) return e;
     if (nbits <= kCountBits) {
         annsa_count_kernel<<<b.H, 1024, (2 << nbits) * 4 + 32 * 32 * 4, st>>>(b, nbits);
     } else {
@@ -677,7 +666,7 @@ static bool attr_set = false;
         while (n < b.T) n <<= 1;
         annsa_order_kernel<<<b.H, 1024, n * 8, st>>>(b);
     }
-    cudaError_t e = cudaGetLastError();
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int grid = grid_for_rows((int64_t)b.H * ((b.T + 127) / 128 * 128), kWarps * (32 / (b.d / 8)), 148 * 8);
     const auto* q = reinterpret_cast<const __nv_bfloat16*>(Q);

@@ -744,14 +744,7 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
 
 template <int D, int MODE>
 cudaError_t set_smem_attr() {
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(attend_bf16_duo_kernel<D, MODE>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, CfgU<D>::SMEM);
-        if (e != cudaSuccess) return e;
-        attr_set = true;
-    }
-    return cudaSuccess;
+    return smem_attr_once(reinterpret_cast<const void*>(attend_bf16_duo_kernel<D, MODE>), CfgU<D>::SMEM);
 }
 
 template <int D>

@@ -6,6 +6,9 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <set>
+#include <utility>
 #include <vector>
 
 namespace tc {
@@ -170,6 +173,22 @@ struct SparseBufs {
 };
 cudaError_t launch_annsa_pack(const SparseBufs& b, int nbits, const void* Q, const void* K, const void* V,
                               float scale_log2, cudaStream_t st);
+
+// Raises a kernel's dynamic shared-memory limit once per (device, kernel): function
+// attributes belong to each device's copy of the kernel, so a process that drives several
+// GPUs needs the call on each of them.
+inline cudaError_t smem_attr_once(const void* kern, int bytes) {
+    static std::mutex mu;
+    static std::set<std::pair<int, const void*>> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count({dev, kern})) return cudaSuccess;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.insert({dev, kern});
+    return e;
+}
 
 // Host helpers (tc_runtime.cu).
 cudaError_t dev_alloc(void** p, size_t bytes);   // cudaMalloc with the TC_FAULT_ALLOC_AT injection

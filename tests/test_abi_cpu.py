@@ -143,3 +143,7 @@ def test_annca_calls_reject_a_null_handle(tcmod):
     assert lib.tc_annca_kept(None, None, None, None, None, None, None, None) == tcmod.TC_EINVAL
     assert lib.tc_annca_sync(None) == tcmod.TC_EINVAL
     lib.tc_annca_destroy(None)
+
+
+def test_annsa_rejects_a_null_handle(tcmod):
+    assert tcmod.lib.tc_annsa_attend(None, None, None, None, 1, None, None) == tcmod.TC_EINVAL
