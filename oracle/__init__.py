@@ -24,3 +24,9 @@ from .annsa_oracle import (  # noqa: F401
     annsa_attention,
     same_bucket_groups,
 )
+from .lvsa_oracle import (  # noqa: F401
+    attended_frames,
+    global_frames,
+    local_window,
+    lvsa_attention,
+)
