@@ -363,13 +363,17 @@ def run_gpu(args):
     cbytes = args.steps * sum(commit_bytes(cfg, commit_counts))
     peaks, peak_kind = load_peaks()
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
-    traffic = None
+    traffic = traffic_earlier = None
     if os.path.exists(TRAFFIC_FILE):
         with open(TRAFFIC_FILE) as f:
             tr = json.load(f)
         # DRAM bytes per unit of work measured by ncu, scaled to an average launch here
-        traffic = tr.get("bytes_per_flop", 0) * (attn_flops_total / (args.steps * cfg.chunks * cfg.attends)) \
-            if tr.get("kernel") == ATTN_KERNEL else None
+        per_launch = tr.get("bytes_per_flop", 0) * (attn_flops_total / (args.steps * cfg.chunks * cfg.attends))
+        if tr.get("kernel") == ATTN_KERNEL:
+            if tr.get("current", True):
+                traffic = per_launch
+            else:   # counters of an earlier build of the kernel: context only
+                traffic_earlier = per_launch
 
     # dense baseline: the same attention kernel over the uncompressed history (no merges)
     dense_line = None
@@ -417,6 +421,7 @@ def run_gpu(args):
         "roofline": {"bound": "tensor", "kernel": ATTN_KERNEL, "achieved": attn_tflops,
                      "peak": peak, "unit": "TFLOP/s", "frac": attn_tflops / peak,
                      "peak_kind": f"{peak_kind} bf16 dense, sustained", "traffic": traffic,
+                     "traffic_earlier_build": traffic_earlier,
                      "flops_per_launch": attn_flops_total / (args.steps * cfg.chunks * cfg.attends),
                      "avg_launch_ms": 1000.0 * attn_sec / (args.steps * cfg.chunks * cfg.attends)},
         "merge": {"achieved_gbs": cbytes / app_sec / 1e9, "peak_gbs": float(peaks["hbm_gbs"]),

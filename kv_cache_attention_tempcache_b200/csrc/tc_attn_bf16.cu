@@ -5,6 +5,11 @@
 // summary, section 2.A: Lemma 5.1 makes averaged values with a logit shift by the
 // group size exact for identical keys. Computed in base 2: x = s * log2(e).
 //
+// Three modes share the kernel: self-attention over the TempCache (as above); AnnCA
+// cross-attention, where a CTA's keys are the prompt tokens kept for its frame (no
+// shift); and AnnSA same-bucket self-attention over a block put in bucket order, where a
+// CTA visits only the key tiles spanning its rows' buckets and masks every other bucket.
+//
 // One CTA = 128 query rows of one head, one CTA per SM (attend_bf16_duo_kernel below):
 // tcgen05.mma (kind::f16, cta_group::1) with operands staged by 3-D TMA in 128-byte
 // swizzled shared memory and fp32 accumulators in TMEM; two softmax teams on alternate
