@@ -288,6 +288,43 @@ tc_status tc_annca_sync(tc_annca_handle h);
 /* tc_annca_destroy - free every buffer of the handle. NULL-safe. Synchronises. */
 void tc_annca_destroy(tc_annca_handle h);
 
+/* ---- LVSA: frame-masked attention for long videos --------------------------- */
+
+/*
+ * LVSA (LVSA technical summary, section 2 "Mecanismo Central"): query frame t attends only
+ * to the frames A(t) = G_s u W(t). G_s = { g : g = step (mod T_per) } are the global frames
+ * of denoising step `step` (over T_per consecutive steps every frame is one exactly once);
+ * W(t) grows from {t} one frame at a time, on the side with fewer frames added so far
+ * (right first on a tie, the other side at the video's edge), until |G_s u W(t)| >= C or
+ * it covers all T frames. Query tokens of frame t attend (bidirectionally, plain softmax,
+ * bf16 tensor cores) to every token of the frames in A(t).
+ * Not yet run on a GPU in this build: see the design notes.
+ */
+typedef struct tc_lvsa_ctx* tc_lvsa_handle;
+
+/* tc_lvsa_create - H heads of dimension d (64 or 128), P tokens per frame (>= 1), anchor
+ * period T_per (>= 1), budget C frames (>= 1), softmax_scale 0 = 1/sqrt(d). */
+tc_status tc_lvsa_create(int32_t H, int32_t d, int32_t P, int32_t T_per, int32_t C,
+                         float softmax_scale, tc_lvsa_handle* out);
+
+/* tc_lvsa_attend - Q, K, V, out DEVICE [T P, H, d] bf16 (frame f = rows f P .. f P + P - 1),
+ * out not overlapping Q, K or V; step >= 0. Asynchronous on `stream` (a tile-list kernel
+ * and the attention kernel). Growing T past the largest earlier value reallocates (and
+ * synchronises first). TC_EINVAL unless T >= 1 and T P H < 2^31. */
+tc_status tc_lvsa_attend(tc_lvsa_handle h, const void* Q, const void* K, const void* V,
+                         int32_t T, int32_t step, void* out, tc_stream stream);
+
+/* tc_lvsa_frames - inspection of the last call (HOST buffers; synchronises): *T_out its T,
+ * nframes [T] = |A(t)|, frames [T*T] = A(t) ascending in frames[t*T .. t*T + nframes[t]). */
+tc_status tc_lvsa_frames(tc_lvsa_handle h, int32_t* T_out, int32_t* nframes, int32_t* frames);
+
+/* tc_lvsa_sync - synchronise the last stream; returns the sticky status (TC_ETIMEOUT if
+ * the attention kernel gave up on one of its barriers). */
+tc_status tc_lvsa_sync(tc_lvsa_handle h);
+
+/* tc_lvsa_destroy - free every buffer of the handle. NULL-safe. Synchronises. */
+void tc_lvsa_destroy(tc_lvsa_handle h);
+
 #ifdef __cplusplus
 }
 #endif

@@ -31,6 +31,7 @@ API = [
     "tc_get_hyperplanes", "tc_stats", "tc_merge_means_noalloc",
     "tc_annca_create", "tc_annca_set_prompt", "tc_annca_attend", "tc_annca_kept", "tc_annca_get_hyperplanes",
     "tc_annca_sync", "tc_annca_destroy", "tc_annsa_attend",
+    "tc_lvsa_create", "tc_lvsa_attend", "tc_lvsa_frames", "tc_lvsa_sync", "tc_lvsa_destroy",
 ]
 
 
@@ -73,6 +74,11 @@ def _load():
         "tc_annca_sync": (ctypes.c_int, [H]),
         "tc_annca_destroy": (None, [H]),
         "tc_annsa_attend": (ctypes.c_int, [H, vp, vp, vp, i64, vp, vp]),
+        "tc_lvsa_create": (ctypes.c_int, [i32, i32, i32, i32, i32, f32, ctypes.POINTER(H)]),
+        "tc_lvsa_attend": (ctypes.c_int, [H, vp, vp, vp, i32, i32, vp, vp]),
+        "tc_lvsa_frames": (ctypes.c_int, [H, ctypes.POINTER(i32), vp, vp]),
+        "tc_lvsa_sync": (ctypes.c_int, [H]),
+        "tc_lvsa_destroy": (None, [H]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -343,6 +349,59 @@ class AnnCA:
     def close(self):
         if getattr(self, "_h", None) is not None and self._h.value:
             lib.tc_annca_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class LVSA:
+    """LVSA frame-masked attention (LVSA summary, section 2): query frame t attends only to
+    the rotating global frames of the step and a local window around t extended to C
+    frames in all. Q, K, V are [T*P, H, d] torch.bfloat16 tensors."""
+
+    def __init__(self, H: int, d: int, P: int, T_per: int, C: int, softmax_scale: float = 0.0):
+        self.H, self.d, self.P = int(H), int(d), int(P)
+        self._h = ctypes.c_void_p()
+        _check(lib.tc_lvsa_create(self.H, self.d, self.P, int(T_per), int(C), float(softmax_scale),
+                                  ctypes.byref(self._h)), "tc_lvsa_create")
+
+    def attend(self, Q, K, V, step: int, out=None):
+        t = []
+        for x, name in ((Q, "Q"), (K, "K"), (V, "V")):
+            if x.dtype != torch.bfloat16 or x.dim() != 3 or x.shape[1] != self.H or x.shape[2] != self.d:
+                raise ValueError(f"{name} must be [T*P, {self.H}, {self.d}] bfloat16")
+            t.append((x if x.is_cuda else x.to("cuda", non_blocking=True)).contiguous())
+        Q, K, V = t
+        if Q.shape[0] % self.P:
+            raise ValueError("Q must hold whole frames")
+        if out is None:
+            out = torch.empty_like(Q)
+        self._keep = [Q, K, V]
+        _check(lib.tc_lvsa_attend(self._h, Q.data_ptr(), K.data_ptr(), V.data_ptr(), Q.shape[0] // self.P,
+                                  int(step), out.data_ptr(), TempCache._stream()), "tc_lvsa_attend")
+        return out
+
+    def frames(self):
+        """A(t) of the last call, as a list of arrays."""
+        T = ctypes.c_int32()
+        _check(lib.tc_lvsa_frames(self._h, ctypes.byref(T), None, None), "tc_lvsa_frames")
+        T = T.value
+        n = np.zeros(T, np.int32)
+        f = np.zeros(T * T, np.int32)
+        if T:
+            _check(lib.tc_lvsa_frames(self._h, None, _np_ptr(n), _np_ptr(f)), "tc_lvsa_frames")
+        return [f[t * T: t * T + n[t]].copy() for t in range(T)]
+
+    def sync(self):
+        _check(lib.tc_lvsa_sync(self._h), "tc_lvsa_sync")
+
+    def close(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            lib.tc_lvsa_destroy(self._h)
             self._h = ctypes.c_void_p()
 
     def __del__(self):

@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "_lib", "libtempcache.so")
-SOURCES = ["tc_runtime.cu", "tc_commit.cu", "tc_attn_bf16.cu", "tc_attn_f32.cu", "tc_noalloc.cu", "tc_annca.cu"]
+SOURCES = ["tc_runtime.cu", "tc_commit.cu", "tc_attn_bf16.cu", "tc_attn_f32.cu", "tc_noalloc.cu", "tc_annca.cu", "tc_lvsa.cu"]
 HEADERS = [os.path.join(CSRC, "tc_internal.h"), os.path.join(CSRC, "tc_device.cuh"),
            os.path.join(ROOT, "include", "tempcache.h")]
 

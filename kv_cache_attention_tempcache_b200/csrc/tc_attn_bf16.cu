@@ -260,7 +260,7 @@ struct CfgU {
 //               retired (up to three tiles ahead).
 //   warp 18     lane 0 TMA producer for the V ring (2 stages).
 //   warp 19     lane 0 issues O += P_i V_i in tile order.
-enum { kSelf = 0, kCross = 1, kSparse = 2 };   // kernel modes (see the prologue)
+enum { kSelf = 0, kCross = 1, kSparse = 2, kFrames = 3 };   // kernel modes (see the prologue)
 
 // A bucket code as a float's bits -> logit shift 0 when it equals the row's code, else
 // -inf (same-bucket mask of the sparse mode).
@@ -277,9 +277,11 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                        const float* __restrict__ bias2, const float* __restrict__ kmax2c,
                        const float* __restrict__ kmax2s, const float* __restrict__ bmaxh, int64_t capP,
                        const float* __restrict__ sbias, int64_t Ts, int64_t Tq, int H, int Pf, int Ff,
-                       const SparseArgs sp, __nv_bfloat16* __restrict__ out, float scale_log2, Stats* stats) {
+                       const SparseArgs sp, const FrameArgs fa, __nv_bfloat16* __restrict__ out, float scale_log2,
+                       Stats* stats) {
     constexpr bool CROSS = MODE == kCross;
     constexpr bool SPARSE = MODE == kSparse;
+    constexpr bool FRAMES = MODE == kFrames;
     using C = Cfg<D>;
     using L = CfgU<D>;
     constexpr int kWK = 16, kWQK = 17, kWV = 18, kWPV = 19;
@@ -306,9 +308,23 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
     // Sparse (same-bucket) self-attention: rows are in bucket order (packed, head-major);
     // CTA x covers packed rows [128 x, 128 x + 128) of head h, the keys are the packed
     // tiles [kt0, kt1) that hold its rows' buckets, masked per element to the same bucket.
+    // Frame mask (LVSA): the query rows are frames of Pf rows; CTA x covers rows of one
+    // frame f, and its keys are the token-major tiles listed for f (the frames f attends
+    // to, each run of consecutive frames tiled from its first row), rows past a run's end
+    // shifted by -inf.
     int q0, zc, kt0 = 0, nsp = 0;
     int64_t qend;
-    if constexpr (SPARSE) {
+    const int2* ftab = nullptr;
+    if constexpr (FRAMES) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");   // the tile lists of this call
+        const int tpf = (Pf + kBM - 1) / kBM;
+        const int f = blockIdx.x / tpf;
+        q0 = f * Pf + (blockIdx.x - f * tpf) * kBM;
+        qend = (int64_t)(f + 1) * Pf;
+        zc = h;
+        ftab = fa.tiles + (int64_t)f * fa.maxt;
+        nsp = fa.count[f];
+    } else if constexpr (SPARSE) {
         asm volatile("griddepcontrol.wait;" ::: "memory");   // the packing kernel's output
         q0 = blockIdx.x * kBM;
         qend = Tq;
@@ -330,8 +346,8 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         qend = Tq;
         zc = h;
     }
-    const int nc = SPARSE ? nsp : (Mdev[zc] + kBN - 1) / kBN;
-    const int ntiles = nc + ((CROSS || SPARSE) ? 0 : (int)((Ts + kBN - 1) / kBN));
+    const int nc = (SPARSE || FRAMES) ? nsp : (Mdev[zc] + kBN - 1) / kBN;
+    const int ntiles = nc + ((CROSS || SPARSE || FRAMES) ? 0 : (int)((Ts + kBN - 1) / kBN));
     if constexpr (CROSS) {
         if (ntiles == 0) {   // no key: the rows are the empty sum, zero
             constexpr int W = D / 8;   // 16-byte words per row
@@ -409,11 +425,17 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             const int st = i % nst;
             if (i >= nst && !mbar_wait(&empty[st], ((i / nst) - 1) & 1)) { *abort_flag = 1; break; }
             const bool cache = i < nc;
-            const int row0 = ((cache ? i : i - nc) + kt0) * kBN;
             mbar_expect_tx(&full[st], C::TILE);
-            for (int b = 0; b < C::NB; ++b)
-                tma_load_3d(ring + st * C::TILE + b * C::BOX, cache ? mc : ms, 64 * b, row0, cache ? zc : h,
-                            &full[st]);
+            if constexpr (FRAMES) {   // token-major keys and values
+                const int row0 = ftab[i].x;
+                for (int b = 0; b < C::NB; ++b)
+                    tma_load_3d(ring + st * C::TILE + b * C::BOX, mc, 64 * b, h, row0, &full[st]);
+            } else {
+                const int row0 = ((cache ? i : i - nc) + kt0) * kBN;
+                for (int b = 0; b < C::NB; ++b)
+                    tma_load_3d(ring + st * C::TILE + b * C::BOX, cache ? mc : ms, 64 * b, row0, cache ? zc : h,
+                                &full[st]);
+            }
             last = i;
         }
         if (kside) mbar_wait(&bars[U_QFULL], 0);
@@ -486,6 +508,7 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                                      : bias2 + (int64_t)zc * capP;
         const uint32_t gq = SPARSE ? sp.grp[(int64_t)h * sp.Tp + q0 + r] : 0u;
         auto bias_of = [&](int i) -> float {
+            if constexpr (FRAMES) return fa.masktab[ftab[i].y * kBN + r];
             return (i < nc) ? bias_h[(int64_t)i * kBN + r] : sbias[(int64_t)(i - nc) * kBN + r];
         };
         // Half 0 stages the log2 n row of each of its team's tiles and its quarter maxima
@@ -532,6 +555,7 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
             m_run = mfix;
             const uint64_t negm2 = pk2(-mfix, -mfix);
             auto bias_row = [&](int i) -> const float* {
+                if constexpr (FRAMES) return fa.masktab + ftab[i].y * kBN + 64 * g;
                 return ((i < nc) ? bias_h + (int64_t)i * kBN : sbias + (int64_t)(i - nc) * kBN) + 64 * g;
             };
             if (lane < 2 && t < ntiles) asm volatile("prefetch.global.L1 [%0];" ::"l"(bias_row(t) + 32 * lane));
@@ -770,7 +794,7 @@ cudaError_t launch_t(const CacheView& c, const StageView& s, const AttnMaps& m, 
     return cudaLaunchKernelEx(&cfg, attend_bf16_duo_kernel<D, kSelf>, m.q, m.kc, m.vc, m.ks, m.vs,
                               (const int32_t*)c.M, (const float*)c.bias2, (const float*)c.kmax2,
                               (const float*)c.kmax2s, (const float*)c.bmax, c.capP, (const float*)s.sbias, s.T, Tq,
-                              c.H, (int)Tq, 1, SparseArgs{}, out, scale_log2, stats);
+                              c.H, (int)Tq, 1, SparseArgs{}, FrameArgs{}, out, scale_log2, stats);
 }
 
 // Cross-attention over the kept prompt tokens: grid (F frames x tiles per frame, H),
@@ -795,7 +819,7 @@ cudaError_t launch_cross_t(const AnnView& a, const AttnMaps& m, int64_t Tq, int 
     return cudaLaunchKernelEx(&cfg, attend_bf16_duo_kernel<D, kCross>, m.q, m.kc, m.vc, m.kc, m.vc,
                               (const int32_t*)a.nsel, (const float*)a.sbias, (const float*)a.kmax2,
                               (const float*)a.zeros, (const float*)a.zeros, a.Lp, (const float*)nullptr, (int64_t)0,
-                              Tq, a.H, P, F, SparseArgs{}, out, scale_log2, stats);
+                              Tq, a.H, P, F, SparseArgs{}, FrameArgs{}, out, scale_log2, stats);
 }
 
 // Same-bucket self-attention over packed rows: grid (query tiles, H), a programmatic
@@ -818,7 +842,35 @@ cudaError_t launch_sparse_t(int H, const SparseArgs& sp, const AttnMaps& m, int6
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, attend_bf16_duo_kernel<D, kSparse>, m.q, m.kc, m.vc, m.kc, m.vc,
                               (const int32_t*)nullptr, (const float*)nullptr, kmax2, zeros, zeros, sp.Tp,
-                              (const float*)nullptr, (int64_t)0, T, H, (int)T, 1, sp, out, scale_log2, stats);
+                              (const float*)nullptr, (int64_t)0, T, H, (int)T, 1, sp, FrameArgs{}, out, scale_log2,
+                              stats);
+}
+
+// Frame-masked attention over token-major Q, K, V: grid (T frames x tiles per frame, H), a
+// programmatic dependent of the kernel that lists the tiles. `big` is one float of +inf:
+// with no bound of the key norms the kernel always takes the running softmax reference.
+template <int D>
+cudaError_t launch_frames_t(int H, const FrameArgs& fa, const AttnMaps& m, int T, int P, const float* big,
+                            const float* zeros, __nv_bfloat16* out, float scale_log2, Stats* stats,
+                            cudaStream_t st) {
+    cudaError_t e = set_smem_attr<D, kFrames>();
+    if (e != cudaSuccess) return e;
+    const int tpf = (P + kBM - 1) / kBM;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(T * tpf), (unsigned)H);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = CfgU<D>::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const int64_t N = (int64_t)T * P;
+    return cudaLaunchKernelEx(&cfg, attend_bf16_duo_kernel<D, kFrames>, m.q, m.kc, m.vc, m.kc, m.vc,
+                              (const int32_t*)nullptr, (const float*)nullptr, big, zeros, zeros, (int64_t)0,
+                              (const float*)nullptr, (int64_t)0, N, H, P, T, SparseArgs{}, fa, out, scale_log2,
+                              stats);
 }
 
 }  // namespace
@@ -834,6 +886,13 @@ cudaError_t launch_attend_cross_bf16(const AnnView& a, const AttnMaps& maps, int
                                      __nv_bfloat16* out, float scale_log2, Stats* stats, cudaStream_t st) {
     return a.d == 128 ? launch_cross_t<128>(a, maps, Tq, P, F, out, scale_log2, stats, st)
                       : launch_cross_t<64>(a, maps, Tq, P, F, out, scale_log2, stats, st);
+}
+
+cudaError_t launch_attend_frames_bf16(int H, int d, const FrameArgs& fa, const AttnMaps& maps, int T, int P,
+                                      const float* big, const float* zeros, __nv_bfloat16* out, float scale_log2,
+                                      Stats* stats, cudaStream_t st) {
+    return d == 128 ? launch_frames_t<128>(H, fa, maps, T, P, big, zeros, out, scale_log2, stats, st)
+                    : launch_frames_t<64>(H, fa, maps, T, P, big, zeros, out, scale_log2, stats, st);
 }
 
 cudaError_t launch_attend_sparse_bf16(int H, int d, const SparseArgs& sp, const AttnMaps& maps, int64_t T,

@@ -144,6 +144,15 @@ struct SparseArgs {
     int nqt;               // Tp / 128, the row stride of tiles
 };
 
+// LVSA frame-mask arrays read by the attention kernel's frame mode (tc_lvsa.cu): per query
+// frame, the key tiles that cover the frames it attends to.
+struct FrameArgs {
+    const int2* tiles;     // [T][maxt] (first token row, valid rows <= 128) of each key tile
+    const int32_t* count;  // [T] key tiles of each query frame
+    const float* masktab;  // [129][128]: row v holds 0 in its first v columns, -inf after
+    int maxt;
+};
+
 // Launchers (tc_annca.cu, tc_attn_bf16.cu).
 cudaError_t launch_annca_prompt(const AnnView& a, const void* Kp, const void* Vp, const float* R,
                                 const float* Rnorm, Stats* stats, cudaStream_t st);
@@ -153,6 +162,10 @@ cudaError_t launch_annca_select(const AnnView& a, const void* Q, int64_t Tq, int
                                 const float* Rhost, const float* Rnorm_host, Stats* stats, cudaStream_t st);
 cudaError_t launch_attend_cross_bf16(const AnnView& a, const AttnMaps& maps, int64_t Tq, int P, int F,
                                      __nv_bfloat16* out, float scale_log2, Stats* stats, cudaStream_t st);
+// maps.q / maps.kc / maps.vc: token-major Q, K, V [T P, H, d] (box 64 x 1 x 128).
+cudaError_t launch_attend_frames_bf16(int H, int d, const FrameArgs& fa, const AttnMaps& maps, int T, int P,
+                                      const float* big, const float* zeros, __nv_bfloat16* out, float scale_log2,
+                                      Stats* stats, cudaStream_t st);
 // maps.q: packed queries [H][Tp][d]; maps.kc / maps.vc: packed keys and values, same shape.
 cudaError_t launch_attend_sparse_bf16(int H, int d, const SparseArgs& sp, const AttnMaps& maps, int64_t T,
                                       const float* kmax2, const float* zeros, __nv_bfloat16* out,

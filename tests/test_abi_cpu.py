@@ -147,3 +147,25 @@ def test_annca_calls_reject_a_null_handle(tcmod):
 
 def test_annsa_rejects_a_null_handle(tcmod):
     assert tcmod.lib.tc_annsa_attend(None, None, None, None, 1, None, None) == tcmod.TC_EINVAL
+
+
+@pytest.mark.parametrize("args", [
+    (0, 128, 1560, 4, 21, 0.0),     # H < 1
+    (12, 96, 1560, 4, 21, 0.0),     # d not 64/128
+    (12, 128, 0, 4, 21, 0.0),       # P < 1
+    (12, 128, 1560, 0, 21, 0.0),    # T_per < 1
+    (12, 128, 1560, 4, 0, 0.0),     # C < 1
+    (12, 128, 1560, 4, 21, -1.0),   # negative scale
+])
+def test_lvsa_create_rejects_bad_arguments(tcmod, args):
+    h = ctypes.c_void_p()
+    assert tcmod.lib.tc_lvsa_create(*args, ctypes.byref(h)) == tcmod.TC_EINVAL
+    assert not h.value
+
+
+def test_lvsa_calls_reject_a_null_handle(tcmod):
+    lib = tcmod.lib
+    assert lib.tc_lvsa_attend(None, None, None, None, 1, 0, None, None) == tcmod.TC_EINVAL
+    assert lib.tc_lvsa_frames(None, None, None, None) == tcmod.TC_EINVAL
+    assert lib.tc_lvsa_sync(None) == tcmod.TC_EINVAL
+    lib.tc_lvsa_destroy(None)
