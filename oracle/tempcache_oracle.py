@@ -40,6 +40,15 @@ silent point is marked READING.
     value is the mean of its creating token and every later member, n their
     count. Committed entries precede new ones in index order, so exact ties
     still go to the lowest entry index.
+8c. Variant (option key_mode="mean"; the other half of the open point of 4): an
+    entry's key is the running mean of its members' keys, kept in fp32 the way a
+    device merge keeps means: k <- (n k + sum_{t in S} k_t) / (n + m), the sum taken
+    in fp32 in ascending t and every operation rounded to fp32 (READING). After the
+    commit the entry's code is recomputed from its new key (step 2) and it moves to
+    that bucket for later commits; matches inside one commit still see the keys as
+    they were before it (snapshot). Attention uses the mean key. Identical keys give
+    a mean equal to each of them exactly (bf16 keys, counts below 2^16), so Lemma
+    5.1's case is unchanged.
 10. Attention: out_t = sum_j w_tj v_j / sum_j w_tj with
     w_tj = exp(scale <q_t, k_j> + b_j - max), b_j = ln n_j for committed entries
     and 0 for staged tokens, scale = 1/sqrt(d), no mask (READING: the logit shift
@@ -152,6 +161,18 @@ def new_entry_members(u, match_row, e) -> np.ndarray:
     return np.concatenate([[u], np.nonzero(np.asarray(match_row) == e)[0]]).astype(np.int64)
 
 
+def mean_key_fp32(key, n, members) -> np.ndarray:
+    """Step 8c: (n key + sum of members' keys) / (n + m), the member sum taken in
+    ascending order in fp32 and every operation rounded to fp32; returned as fp64
+    holding the fp32 values."""
+    acc = np.zeros(np.asarray(key).shape, dtype=np.float32)
+    for row in np.asarray(members):
+        acc = (acc + np.asarray(row, dtype=np.float32)).astype(np.float32)
+    num = (np.float32(n) * np.asarray(key, dtype=np.float32)).astype(np.float32)
+    num = (num + acc).astype(np.float32)
+    return (num / np.float32(n + len(members))).astype(np.float32).astype(np.float64)
+
+
 def merge_decision(best, best_sim, tau) -> np.ndarray:
     """match = best where sim >= tau (tau as fp32 widened to fp64), else -1."""
     tau64 = np.float64(np.float32(tau))
@@ -212,8 +233,14 @@ class OracleTempCache:
     values widened to fp64).
     """
 
-    def __init__(self, H, d, nbits, tau, capacity, hyperplanes, scale=None, intra_chunk=False):
+    def __init__(self, H, d, nbits, tau, capacity, hyperplanes, scale=None, intra_chunk=False,
+                 key_mode="representative"):
         self.intra_chunk = bool(intra_chunk)
+        if key_mode not in ("representative", "mean"):
+            raise ValueError("key_mode is 'representative' or 'mean'")
+        if key_mode == "mean" and self.intra_chunk:
+            raise NotImplementedError("running-mean keys are defined for the snapshot commit")
+        self.key_mode = key_mode
         self.H, self.d, self.nbits = int(H), int(d), int(nbits)
         self.tau = float(tau)
         self.capacity = int(capacity)
@@ -256,6 +283,9 @@ class OracleTempCache:
                 total = n_old * st.values[j] + V[h, grp].sum(axis=0)
                 st.counts[j] = n_old + grp.size
                 st.values[j] = total / st.counts[j]
+                if self.key_mode == "mean":   # step 8c
+                    st.keys[j] = mean_key_fp32(st.keys[j], n_old, K[h, grp])
+                    st.codes[j] = simhash_codes(self.R, st.keys[j][None, :])[0]
             # step 8: append unmatched tokens in ascending t
             new = np.nonzero(unmatched[h])[0]
             dest[h, new] = st.size + np.arange(new.size)

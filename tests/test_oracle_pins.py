@@ -463,3 +463,112 @@ def test_planted_mistake_intra_without_creating_token_breaks_conservation(monkey
         total += f64(V)[:, 0].sum(0)
     _, vals, cnt, _ = o.export_head(0)
     assert np.abs((cnt[:, None] * vals).sum(0) - total).max() > 1e-6
+
+
+# ----------------------------------------------------------------------------- running-mean keys (step 8c)
+
+def _rollout(cfg, key_mode, chunks=None):
+    w = Workload(cfg)
+    R = f64(w.hyperplanes())
+    o = OracleTempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, R, key_mode=key_mode)
+    recs = []
+    for _ in range(chunks or cfg.chunks):
+        K, V = w.next_chunk()
+        recs.append(o.append_chunk(f64(K), f64(V)))
+    recs.append(o.flush())
+    return o, [r for r in recs if r is not None], R
+
+
+def test_mean_keys_of_identical_duplicates_change_nothing():
+    cfg = small_cfg(sigma=0.0, tau=1.0 - 1e-6, S=12, chunks=5)
+    a, ra, _ = _rollout(cfg, "representative")
+    b, rb, _ = _rollout(cfg, "mean")
+    for x, y in zip(ra, rb):
+        np.testing.assert_array_equal(x.match, y.match)
+        np.testing.assert_array_equal(x.dest, y.dest)
+    for h in range(cfg.H):
+        for u, v in zip(a.export_head(h), b.export_head(h)):
+            np.testing.assert_array_equal(u, v)
+    assert sum(int((r.match >= 0).sum()) for r in rb) > 0   # there were merges
+
+
+def _exact_code(R, key):
+    from fractions import Fraction
+    code = 0
+    for b in range(R.shape[0]):
+        s = sum(Fraction(float(R[b, i])) * Fraction(float(key[i])) for i in range(R.shape[1]))
+        code |= int(s >= 0) << b
+    return code
+
+
+def test_mean_keys_codes_follow_their_keys():
+    cfg = small_cfg(d=16, nbits=5, sigma=0.3, tau=0.8, S=6, chunks=4, P=24)
+    o, recs, R = _rollout(cfg, "mean")
+    moved = 0
+    for h in range(cfg.H):
+        keys, _, cnt, codes = o.export_head(h)
+        for k, c in zip(keys, codes):
+            assert int(c) == _exact_code(R, k)
+        np.testing.assert_array_equal(keys, keys.astype(np.float32).astype(np.float64))   # fp32 values
+        moved += int((cnt > 1).sum())
+    assert moved > 0
+
+
+def test_mean_keys_conserve_the_key_sum():
+    cfg = small_cfg(d=16, nbits=5, sigma=0.3, tau=0.8, S=6, chunks=4, P=24)
+    w = Workload(cfg)
+    total = np.zeros((cfg.H, cfg.d))
+    for _ in range(cfg.chunks):
+        K, _ = w.next_chunk()
+        total += f64(K).sum(axis=0)
+    o, _, _ = _rollout(cfg, "mean")
+    for h in range(cfg.H):
+        keys, _, cnt, _ = o.export_head(h)
+        got = (cnt[:, None] * keys).sum(axis=0)
+        assert np.abs(got - total[h]).max() <= 1e-4 * np.abs(total[h]).max() * cfg.T
+
+
+def test_mean_keys_worked_example():
+    """Hand geometry (one head, d = 2, one hyperplane along y, tau = 0.85): keys at 0, 20
+    and 40 degrees in three chunks. The 20-degree key merges into the first entry
+    (cos 20 = 0.94). With representative keys the 40-degree key then sees the 0-degree
+    key (cos 40 = 0.77 < 0.85) and is appended; with running-mean keys it sees their mean
+    at about 10 degrees (cos 30 = 0.87 >= 0.85) and merges too."""
+    def unit(deg):
+        return round_to_bf16(torch.tensor([[math.cos(math.radians(deg)), math.sin(math.radians(deg))]])).double().numpy()
+
+    R = np.array([[0.0, 1.0]])
+    ks = [unit(0), unit(20), unit(40)]
+    sizes = {}
+    for mode in ("representative", "mean"):
+        o = OracleTempCache(1, 2, 1, 0.85, 10, R, key_mode=mode)
+        for k in ks:
+            o.append_chunk(k[:, None, :], np.ones((1, 1, 2)))
+        o.flush()
+        sizes[mode] = int(o.cache_size()[0])
+        if mode == "mean":
+            keys, _, cnt, _ = o.export_head(0)
+            assert cnt.tolist() == [3]
+            np.testing.assert_allclose(keys[0], (ks[0][0] + ks[1][0] + ks[2][0]) / 3, rtol=0, atol=1e-6)
+    assert sizes == {"representative": 2, "mean": 1}
+
+
+def test_planted_stale_code_is_caught(monkeypatch):
+    real = orc.simhash_codes
+    calls = {"n": 0}
+
+    def stale_after_merge(R, X):
+        calls["n"] += 1
+        out = real(R, X)
+        return out ^ np.uint32(1) if np.asarray(X).shape[0] == 1 else out   # the mean key's code corrupted
+
+    monkeypatch.setattr(orc, "simhash_codes", stale_after_merge)
+    with pytest.raises(AssertionError):
+        test_mean_keys_codes_follow_their_keys()
+
+
+def test_planted_mean_without_old_count_is_caught(monkeypatch):
+    real = orc.mean_key_fp32
+    monkeypatch.setattr(orc, "mean_key_fp32", lambda key, n, members: real(key, 1, members))
+    with pytest.raises(AssertionError):
+        test_mean_keys_conserve_the_key_sum()
