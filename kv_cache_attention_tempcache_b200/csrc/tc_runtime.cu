@@ -5,6 +5,7 @@
 #include "tc_internal.h"
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -15,12 +16,12 @@ namespace tc {
 
 // ---- allocation with host-side fault injection (TC_FAULT_ALLOC_AT=n fails the
 // n-th allocation of the process, counting from 1), used by the failure tests.
-int g_alloc_calls = 0;
+std::atomic<int> g_alloc_calls{0};   // handles may be created from several host threads
 
 cudaError_t dev_alloc(void** p, size_t bytes) {
-    ++g_alloc_calls;
+    const int call = ++g_alloc_calls;
     const char* f = std::getenv("TC_FAULT_ALLOC_AT");
-    if (f && std::atoi(f) == g_alloc_calls) {
+    if (f && std::atoi(f) == call) {
         *p = nullptr;
         return cudaErrorMemoryAllocation;
     }
