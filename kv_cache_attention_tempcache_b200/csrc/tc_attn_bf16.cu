@@ -629,6 +629,11 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     for (int j = 0; j < 64; ++j)
                         if (__float_as_uint(ch[j]) != gq) sr[j] = __float_as_uint(-INFINITY);
                 }
+                if constexpr (FRAMES) {   // rows of frames outside A(t) do not count either
+                    const float* ch = sBias + (t * 3 + bb) * 128 + 64 * g;
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) sr[j] = __float_as_uint(__uint_as_float(sr[j]) + ch[j]);
+                }
 #pragma unroll
                 for (int j = 0; j < 64; j += 8) {
                     m4[0] = max3(m4[0], __uint_as_float(sr[j]), __uint_as_float(sr[j + 1]));
@@ -638,8 +643,8 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                 }
                 smax = fmaxf(max3(m4[0], m4[1], m4[2]), m4[3]);
             }
-            const float2 bm = SPARSE ? make_float2(0.f, 0.f)
-                                     : *reinterpret_cast<const float2*>(sBmax + (t * 3 + bb) * 4 + 2 * g);
+            const float2 bm = (SPARSE || FRAMES) ? make_float2(0.f, 0.f)
+                                                 : *reinterpret_cast<const float2*>(sBmax + (t * 3 + bb) * 4 + 2 * g);
             sUb[((t * 2 + u) * 2 + g) * 128 + r] = fmaf(smax, scale_log2, fmaxf(bm.x, bm.y));
             if (g == 0 && i + 2 < ntiles) stage_bias((k + 1) % 3, bnext);
             if (!bar_and(1 + t, 256, got)) { ok = false; break; }
@@ -847,8 +852,9 @@ cudaError_t launch_sparse_t(int H, const SparseArgs& sp, const AttnMaps& m, int6
 }
 
 // Frame-masked attention over token-major Q, K, V: grid (T frames x tiles per frame, H), a
-// programmatic dependent of the kernel that lists the tiles. `big` is one float of +inf:
-// with no bound of the key norms the kernel always takes the running softmax reference.
+// programmatic dependent of the kernel that lists the tiles. `big` holds H floats of +inf
+// (the per-head key-norm bound, read as big[h]) and `zeros` H zeros: with no bound of the
+// key norms the kernel always takes the running softmax reference.
 template <int D>
 cudaError_t launch_frames_t(int H, const FrameArgs& fa, const AttnMaps& m, int T, int P, const float* big,
                             const float* zeros, __nv_bfloat16* out, float scale_log2, Stats* stats,

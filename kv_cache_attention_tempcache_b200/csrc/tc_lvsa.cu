@@ -17,6 +17,7 @@
 #include "../../include/tempcache.h"
 #include "tc_internal.h"
 
+#include <algorithm>
 #include <cmath>
 #include <new>
 
@@ -85,7 +86,7 @@ struct tc_lvsa_ctx {
     float scale = 0.f;
     int device = 0;
     float* masktab = nullptr;   // [129][128]
-    float* consts = nullptr;    // [0] = +inf, [1 .. H] = 0
+    float* consts = nullptr;    // [0, H) = +inf (key-norm bound per head), [H, 2H) = 0
     Stats* stats = nullptr;
     int Tcap = 0, maxt = 0;     // frames the tables hold, tiles per frame
     int2* tiles = nullptr;
@@ -163,13 +164,13 @@ tc_status tc_lvsa_create(int32_t H, int32_t d, int32_t P, int32_t T_per, int32_t
     x->device = dev;
     x->scale = softmax_scale > 0.f ? softmax_scale : (float)(1.0 / std::sqrt((double)d));
     tc_status st;
-    if ((st = grab(x->masktab, 129 * 128 * 4)) || (st = grab(x->consts, (size_t)(H + 1) * 4)) ||
+    if ((st = grab(x->masktab, 129 * 128 * 4)) || (st = grab(x->consts, (size_t)2 * H * 4)) ||
         (st = grab(x->stats, sizeof(Stats)))) {
         delete x;
         return st;
     }
-    std::vector<float> c(H + 1, 0.f);
-    c[0] = INFINITY;
+    std::vector<float> c(2 * (size_t)H, 0.f);
+    std::fill(c.begin(), c.begin() + H, INFINITY);
     cudaError_t e;
     if ((e = cudaMemcpy(x->consts, c.data(), c.size() * 4, cudaMemcpyHostToDevice)) ||
         (e = cudaMemset(x->stats, 0, sizeof(Stats)))) {
@@ -232,7 +233,7 @@ tc_status tc_lvsa_attend(tc_lvsa_handle x, const void* Q, const void* K, const v
     cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) {
         FrameArgs fa{x->tiles, x->count, x->masktab, x->maxt};
-        e = launch_attend_frames_bf16(x->H, x->d, fa, m, T, x->P, x->consts, x->consts + 1,
+        e = launch_attend_frames_bf16(x->H, x->d, fa, m, T, x->P, x->consts, x->consts + x->H,
                                       static_cast<__nv_bfloat16*>(out),
                                       (float)((double)x->scale * 1.4426950408889634), x->stats, cs);
     }

@@ -2,9 +2,6 @@
 
 The frame sets A(t) are integer results: bit-exact. The output is bf16 tensor-core
 arithmetic: max-abs error <= 2e-2, mean-abs <= 2e-3 against fp64.
-
-The kernel path these tests drive has not yet had its first run on a GPU, so the module
-is skipped until that run has been made and checked.
 """
 import numpy as np
 import pytest
@@ -12,7 +9,7 @@ import torch
 
 from oracle import attended_frames, lvsa_attention
 
-pytestmark = [pytest.mark.gpu, pytest.mark.skip(reason="LVSA kernel not yet run on a GPU")]
+pytestmark = pytest.mark.gpu
 
 MAX_ABS, MEAN_ABS = 2e-2, 2e-3
 
