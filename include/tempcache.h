@@ -183,15 +183,21 @@ tc_status tc_stats(tc_handle h, uint64_t* kernel_launches, uint64_t* hash_rechec
  *   target  DEVICE [n_src] int32 destination row or -1 (skip); values outside
  *           [0, n_dst) are skipped too.
  *   mean    DEVICE [n_dst, d] fp32, updated in place; count DEVICE [n_dst] int32,
- *           updated in place. Rows no source targets are left as they are.
+ *           updated in place. Rows no source targets are left as they are. A row
+ *           with count 0 that some source targets becomes the plain mean of its
+ *           sources (its old contents, even NaN, are not read into the result).
  *   d       64 or 128.
+ *   src and target must not overlap mean or count, nor mean overlap count
+ *   (TC_EINVAL otherwise).
  * Limits: n_src <= 65536 and n_dst <= 262144; larger sizes return TC_EINVAL and
  * launch nothing. Scratch lives in a fixed device array of about 3.4 MB that every
  * GPU loading the library holds until the process exits; the call never calls
- * cudaMalloc, cudaFree or any allocating routine. The first call on a device looks
- * up that array's device address (make it before any stream capture). All calls
- * share the array: calls whose GPU work overlaps (other streams or host threads on
- * the same device) race and corrupt each other's results, so keep them ordered.
+ * cudaMalloc, cudaFree or any allocating routine. The first call in each CUDA
+ * context looks up that array's device address in that context and caches it per
+ * context (a device reset or another current context triggers a new lookup); make
+ * that first call before any stream capture. All calls share the array: calls whose
+ * GPU work overlaps (other streams or host threads on the same device) race and
+ * corrupt each other's results, so keep them ordered.
  * Asynchronous on `stream`; returns TC_ECUDA if a launch fails.
  */
 tc_status tc_merge_means_noalloc(const void* src, tc_dtype src_dtype, const int32_t* target,

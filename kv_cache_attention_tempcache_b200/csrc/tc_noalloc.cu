@@ -10,12 +10,14 @@
 // Scratch: one file-scope device array, kScratchWords 32-bit words (about 3.4 MB)
 // on every GPU that loads the library, held until the process exits. Host code
 // cannot pass the array's name to a kernel (on the host it is only a stand-in),
-// so the first call on each device looks up its device address with
-// cudaGetSymbolAddress while that device is current and caches it; make that first
-// call before any stream capture. Every call shares the array and it keeps the last
-// call's contents, so each call first clears the parts that must start at zero.
-// Two calls whose work overlaps on the GPU (different streams, or different host
-// threads on one device) race on the array and give wrong results.
+// so the first call in each CUDA context looks up the array's device address with
+// cudaGetSymbolAddress while that context is current and caches it together with the
+// context's unique id; a later call in another context (after cudaDeviceReset, or a
+// context the caller made current) looks the address up again. Make the first call
+// of a context before any stream capture. Every call shares the array and it keeps
+// the last call's contents, so each call first clears the parts that must start at
+// zero. Two calls whose work overlaps on the GPU (different streams, or different
+// host threads on one device) race on the array and give wrong results.
 #include "../../include/tempcache.h"
 #include "tc_internal.h"
 
@@ -52,19 +54,56 @@ Scratch carve(int32_t* base) {
     return s;
 }
 
-std::mutex g_mu;
-int32_t* g_addr[kMaxDevices] = {};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
 
-// Device address of the scratch array on the current device (looked up once).
+std::mutex g_mu;
+CtxGetCurrentFn g_ctx_current = nullptr;
+CtxGetIdFn g_ctx_id = nullptr;
+struct CachedAddr {
+    unsigned long long ctx_id;   // unique id of the context the address belongs to (0: none yet)
+    int32_t* addr;
+};
+CachedAddr g_addr[kMaxDevices] = {};
+
+// Device address of the scratch array in the current context of device `dev`, looked
+// up once per context: a context id that differs from the cached one (the device was
+// reset, or the caller made another context current) triggers a new lookup.
 cudaError_t scratch_address(int dev, int32_t** out) {
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_addr[dev]) {
-        void* p = nullptr;
-        cudaError_t e = cudaGetSymbolAddress(&p, g_merge_scratch);
-        if (e != cudaSuccess) return e;
-        g_addr[dev] = static_cast<int32_t*>(p);
+    if (!g_ctx_current || !g_ctx_id) {
+        void* f1 = nullptr;
+        void* f2 = nullptr;
+        cudaDriverEntryPointQueryResult q1, q2;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f1, cudaEnableDefault, &q1) != cudaSuccess ||
+            q1 != cudaDriverEntryPointSuccess || !f1 ||
+            cudaGetDriverEntryPoint("cuCtxGetId", &f2, cudaEnableDefault, &q2) != cudaSuccess ||
+            q2 != cudaDriverEntryPointSuccess || !f2)
+            return cudaErrorNotSupported;
+        g_ctx_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+        g_ctx_id = reinterpret_cast<CtxGetIdFn>(f2);
     }
-    *out = g_addr[dev];
+    // The context the runtime works in is the thread's current one (the caller's own,
+    // or the device's primary context); with none current yet, the runtime makes the
+    // primary context current on its first call, here cudaGetSymbolAddress.
+    CUcontext ctx = nullptr;
+    if (g_ctx_current(&ctx) != CUDA_SUCCESS) return cudaErrorDeviceUninitialized;
+    void* fresh = nullptr;
+    if (!ctx) {
+        cudaError_t e = cudaGetSymbolAddress(&fresh, g_merge_scratch);
+        if (e != cudaSuccess) return e;
+        if (g_ctx_current(&ctx) != CUDA_SUCCESS || !ctx) return cudaErrorDeviceUninitialized;
+    }
+    unsigned long long id = 0;
+    if (g_ctx_id(ctx, &id) != CUDA_SUCCESS || id == 0) return cudaErrorDeviceUninitialized;
+    if (g_addr[dev].ctx_id != id || !g_addr[dev].addr) {
+        if (!fresh) {
+            cudaError_t e = cudaGetSymbolAddress(&fresh, g_merge_scratch);
+            if (e != cudaSuccess) return e;
+        }
+        g_addr[dev] = CachedAddr{id, static_cast<int32_t*>(fresh)};
+    }
+    *out = g_addr[dev].addr;
     return cudaSuccess;
 }
 
@@ -137,12 +176,23 @@ __device__ __forceinline__ void na_load_row(const E* row, int lane, float (&x)[D
 }
 
 // One warp per touched destination: sum its sources in ascending source index in
-// fp32, then mean <- (n mean + sum) / (n + m), count <- n + m.
+// fp32, then mean <- (n mean + sum) / (n + m), count <- n + m (mean <- sum / m when
+// n = 0, so a row that was never written does not matter). The warp puts the sources
+// of its destination in ascending order: up to 32 in its lanes, up to kSortSmem in its
+// own shared-memory buffer (each id placed at its rank), and beyond that it visits
+// them by scanning target[] in source order, one 32-source window per ballot.
+constexpr int kMergeWarps = 8;
+constexpr int kSortSmem = 256;
+
 template <typename E, int D>
-__global__ void __launch_bounds__(256) na_merge(const E* __restrict__ src, float* __restrict__ mean,
-                                                int32_t* __restrict__ count, Scratch s) {
+__global__ void __launch_bounds__(kMergeWarps * 32) na_merge(const E* __restrict__ src,
+                                                            const int32_t* __restrict__ target, int n_src,
+                                                            float* __restrict__ mean, int32_t* __restrict__ count,
+                                                            Scratch s) {
     constexpr int EPL = D / 32;
-    const int lane = threadIdx.x & 31;
+    __shared__ int32_t sIds[kMergeWarps][kSortSmem];
+    __shared__ int32_t sSorted[kMergeWarps][kSortSmem];
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     const int ns = *s.ntouched;
     for (int w = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; w < ns; w += (gridDim.x * blockDim.x) >> 5) {
         const int j = s.touched[w];
@@ -150,32 +200,41 @@ __global__ void __launch_bounds__(256) na_merge(const E* __restrict__ src, float
         float acc[EPL];
 #pragma unroll
         for (int e = 0; e < EPL; ++e) acc[e] = 0.f;
+        auto add_row = [&](int i) {
+            float v[EPL];
+            na_load_row<E, D>(src + (size_t)i * D, lane, v);
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[e] = __fadd_rn(acc[e], v[e]);
+        };
         if (m <= 32) {
             const int id = (lane < m) ? s.seg[off + lane] : 0x7fffffff;
             int rank = 0;
             for (int k = 0; k < 32; ++k) rank += (__shfl_sync(0xffffffffu, id, k) < id);
             for (int q = 0; q < m; ++q) {
                 const int srcl = __ffs(__ballot_sync(0xffffffffu, rank == q)) - 1;
-                const int i = __shfl_sync(0xffffffffu, id, srcl);
-                float v[EPL];
-                na_load_row<E, D>(src + (size_t)i * D, lane, v);
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) acc[e] = __fadd_rn(acc[e], v[e]);
+                add_row(__shfl_sync(0xffffffffu, id, srcl));
             }
+        } else if (m <= kSortSmem) {
+            for (int p = lane; p < m; p += 32) sIds[wib][p] = s.seg[off + p];
+            __syncwarp();
+            for (int p = lane; p < m; p += 32) {
+                const int mine = sIds[wib][p];
+                int rank = 0;
+                for (int k = 0; k < m; ++k) rank += (sIds[wib][k] < mine);
+                sSorted[wib][rank] = mine;   // ids are distinct: ranks are a permutation
+            }
+            __syncwarp();
+            for (int q = 0; q < m; ++q) add_row(sSorted[wib][q]);
+            __syncwarp();   // the buffers are reused by this warp's next destination
         } else {
-            int last = -1;
-            for (int q = 0; q < m; ++q) {
-                int mn = 0x7fffffff;
-                for (int p = lane; p < m; p += 32) {
-                    const int id = s.seg[off + p];
-                    if (id > last && id < mn) mn = id;
+            for (int i0 = 0; i0 < n_src; i0 += 32) {
+                const bool hit = i0 + lane < n_src && target[i0 + lane] == j;
+                unsigned b = __ballot_sync(0xffffffffu, hit);
+                while (b) {
+                    const int k = __ffs(b) - 1;
+                    b &= b - 1;
+                    add_row(i0 + k);
                 }
-                for (int o = 16; o > 0; o >>= 1) mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-                float v[EPL];
-                na_load_row<E, D>(src + (size_t)mn * D, lane, v);
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) acc[e] = __fadd_rn(acc[e], v[e]);
-                last = mn;
             }
         }
         const int nold = count[j];
@@ -183,7 +242,7 @@ __global__ void __launch_bounds__(256) na_merge(const E* __restrict__ src, float
 #pragma unroll
         for (int e = 0; e < EPL; ++e) {
             float* p = mean + (size_t)j * D + lane * EPL + e;
-            *p = __fdiv_rn(__fadd_rn(__fmul_rn(fn, *p), acc[e]), ft);
+            *p = nold == 0 ? __fdiv_rn(acc[e], ft) : __fdiv_rn(__fadd_rn(__fmul_rn(fn, *p), acc[e]), ft);
         }
         if (lane == 0) count[j] = nold + m;
     }
@@ -196,8 +255,8 @@ cudaError_t run(const void* src, const int32_t* target, int n_src, float* mean, 
     na_count<<<gs, 256, 0, st>>>(target, n_src, n_dst, s);
     na_offsets<<<1, 1024, 0, st>>>(s);
     na_scatter<<<gs, 256, 0, st>>>(target, n_src, n_dst, s);
-    const int gm = (n_src + 7) / 8 > 1184 ? 1184 : (n_src + 7) / 8;
-    na_merge<E, D><<<gm, 256, 0, st>>>(reinterpret_cast<const E*>(src), mean, count, s);
+    const int gm = (n_src + kMergeWarps - 1) / kMergeWarps > 1184 ? 1184 : (n_src + kMergeWarps - 1) / kMergeWarps;
+    na_merge<E, D><<<gm, kMergeWarps * 32, 0, st>>>(reinterpret_cast<const E*>(src), target, n_src, mean, count, s);
     return cudaGetLastError();
 }
 
@@ -210,6 +269,18 @@ extern "C" tc_status tc_merge_means_noalloc(const void* src, tc_dtype src_dtype,
         (src_dtype != TC_BF16 && src_dtype != TC_F32) || n_src < 1 || n_dst < 1)
         return TC_EINVAL;
     if (n_src > kMaxSrc || n_dst > kMaxDst) return TC_EINVAL;  // beyond the fixed scratch
+    // The inputs must not overlap the rows the call writes.
+    const size_t esz = src_dtype == TC_BF16 ? 2 : 4;
+    auto overlap = [](const void* a, size_t na, const void* b, size_t nb) {
+        const char* x = static_cast<const char*>(a);
+        const char* y = static_cast<const char*>(b);
+        return x < y + nb && y < x + na;
+    };
+    const size_t src_b = (size_t)n_src * d * esz, tgt_b = (size_t)n_src * 4;
+    const size_t mean_b = (size_t)n_dst * d * 4, cnt_b = (size_t)n_dst * 4;
+    if (overlap(src, src_b, mean, mean_b) || overlap(src, src_b, count, cnt_b) || overlap(target, tgt_b, mean, mean_b) ||
+        overlap(target, tgt_b, count, cnt_b) || overlap(mean, mean_b, count, cnt_b))
+        return TC_EINVAL;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
         cudaGetLastError();

@@ -62,3 +62,79 @@ def test_noalloc_merge_rejects_sizes_beyond_its_scratch():
     p = buf.data_ptr()
     assert m.lib.tc_merge_means_noalloc(p, m.TC_F32, p, 65537, 128, p, p, 10, None) == m.TC_EINVAL
     assert m.lib.tc_merge_means_noalloc(p, m.TC_F32, p, 10, 128, p, p, 262145, None) == m.TC_EINVAL
+
+
+def _expected(src, target, mean, count):
+    """Sequential fp32 reference: sources summed in ascending index, then the mean update."""
+    mean = mean.copy()
+    count = count.copy()
+    for j in np.unique(target[(target >= 0) & (target < mean.shape[0])]):
+        ids = np.nonzero(target == j)[0]
+        acc = np.zeros(mean.shape[1], np.float32)
+        for i in ids:
+            acc = (acc + src[i].astype(np.float32)).astype(np.float32)
+        n = np.float32(count[j])
+        ft = np.float32(count[j] + ids.size)
+        if count[j] == 0:
+            mean[j] = (acc / ft).astype(np.float32)
+        else:
+            mean[j] = (((n * mean[j]).astype(np.float32) + acc).astype(np.float32) / ft).astype(np.float32)
+        count[j] += ids.size
+    return mean, count
+
+
+@pytest.mark.parametrize("dtype,d", [("f32", 64), ("bf16", 128), ("f32", 128)])
+def test_noalloc_merge_long_groups_in_source_order(dtype, d):
+    # one destination gets > 256 sources (scan path), one > 32 (shared-memory order),
+    # the rest small groups; a destination with count 0 holds NaN that must not leak
+    import kv_cache_attention_tempcache_b200 as m
+
+    rng = np.random.default_rng(7 + d)
+    n_src, n_dst = 3000, 400
+    target = rng.integers(-1, n_dst, n_src).astype(np.int32)
+    target[rng.choice(n_src, 700, replace=False)] = 5      # > 256 sources
+    target[rng.choice(np.nonzero(target != 5)[0], 100, replace=False)] = 17   # > 32 sources
+    src32 = rng.standard_normal((n_src, d)).astype(np.float32)
+    if dtype == "bf16":
+        src_t = torch.from_numpy(src32).to(torch.bfloat16)
+        src_np = src_t.float().numpy()
+        code = m.TC_BF16
+    else:
+        src_t = torch.from_numpy(src32)
+        src_np = src32
+        code = m.TC_F32
+    mean0 = rng.standard_normal((n_dst, d)).astype(np.float32)
+    count0 = rng.integers(0, 9, n_dst).astype(np.int32)
+    count0[17] = 0
+    mean0[17] = np.nan
+    exp_mean, exp_count = _expected(src_np, target, mean0, count0)
+    src_d = src_t.cuda()
+    tgt_d = torch.from_numpy(target).cuda()
+    for _ in range(2):   # two calls in a row on fresh copies
+        mean = torch.from_numpy(mean0.copy()).cuda()
+        count = torch.from_numpy(count0.copy()).cuda()
+        st = m.lib.tc_merge_means_noalloc(src_d.data_ptr(), code, tgt_d.data_ptr(), n_src, d, mean.data_ptr(),
+                                          count.data_ptr(), n_dst,
+                                          ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        assert st == m.TC_OK
+        torch.cuda.synchronize()
+        assert np.array_equal(count.cpu().numpy(), exp_count)
+        got = mean.cpu().numpy()
+        assert np.isfinite(got[17]).all()
+        assert np.abs(got - exp_mean).max() <= 1e-3
+        assert np.array_equal(got, exp_mean)   # same operations in the same order
+
+
+def test_noalloc_merge_rejects_overlapping_buffers():
+    import kv_cache_attention_tempcache_b200 as m
+
+    buf = torch.zeros(64 * 128, dtype=torch.float32, device="cuda")
+    tgt = torch.zeros(16, dtype=torch.int32, device="cuda")
+    cnt = torch.zeros(8, dtype=torch.int32, device="cuda")
+    p = buf.data_ptr()
+    # src rows [0, 16 * 64) overlap mean rows starting at the same address
+    assert m.lib.tc_merge_means_noalloc(p, m.TC_F32, tgt.data_ptr(), 16, 64, p, cnt.data_ptr(), 8,
+                                        None) == m.TC_EINVAL
+    # target overlaps count
+    assert m.lib.tc_merge_means_noalloc(p, m.TC_F32, tgt.data_ptr(), 16, 64, p + 16 * 64 * 4, tgt.data_ptr(), 8,
+                                        None) == m.TC_EINVAL
