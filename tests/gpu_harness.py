@@ -36,13 +36,17 @@ class ParityReport:
     sizes: list = field(default_factory=list)
 
 
-def compare_state(tc, o, rep: ParityReport, heads):
-    sizes_gpu = tc.cache_size()
+def compare_state(tc, o, rep: ParityReport, heads, oracle_heads):
+    """Cache contents of GPU heads `heads` against the oracle, whose head i is GPU head
+    oracle_heads[i]."""
+    sizes_gpu = tc.cache_size()[list(oracle_heads)]
     sizes_ref = o.cache_size()
     rep.size_mismatch += int((sizes_gpu != sizes_ref).sum())
-    for h in heads:
+    for i, h in enumerate(oracle_heads):
+        if h not in heads:
+            continue
         K, V32, n, code = tc.export_cache(h)
-        k_ref, v_ref, n_ref, c_ref = o.export_head(h)
+        k_ref, v_ref, n_ref, c_ref = o.export_head(i)
         if K.shape[0] != k_ref.shape[0]:
             rep.key_mismatch += 1
             continue
@@ -53,62 +57,75 @@ def compare_state(tc, o, rep: ParityReport, heads):
 
 
 def run_parity(cfg, chunks=None, attends=1, rows=None, state_heads=None, flush=True, device="cuda",
-               check_every_state=True, intra_chunk=False):
+               check_every_state=True, intra_chunk=False, oracle_heads=None, attn_chunks=None, q_scale=1.0,
+               key_mode="representative", on_chunk=None):
     """Run `chunks` chunks through both implementations and collect the differences.
 
-    rows: query rows checked per attend (None = all). state_heads: heads whose
-    cache contents are compared after every commit (None = all).
+    rows: query rows checked per attend (None = all). oracle_heads: the heads the oracle
+    follows (None = all; heads are independent, so the oracle may run a subset while the
+    GPU runs every head). state_heads: heads whose cache contents are compared (None =
+    every oracle head). attn_chunks: chunk indices whose attention is checked (None =
+    all; the GPU attends in every chunk). q_scale: queries multiplied by this factor
+    (then rounded to the storage type) to reach large logits. on_chunk(c, tc, o, w, K, V)
+    is called after each chunk's attention with that chunk's keys and values.
     """
     from kv_cache_attention_tempcache_b200 import TempCache
 
     chunks = cfg.chunks if chunks is None else chunks
+    oh = list(range(cfg.H)) if oracle_heads is None else list(oracle_heads)
     w = Workload(cfg, device=device)
     R = w.hyperplanes()
+    extra = {} if key_mode == "representative" else {"key_mode": key_mode}
     tc = TempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, dtype=cfg.dtype, hyperplanes=R.numpy(),
-                   intra_chunk=intra_chunk)
-    o = OracleTempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, R.double().numpy(),
-                        intra_chunk=intra_chunk)
-    heads = range(cfg.H) if state_heads is None else state_heads
+                   intra_chunk=intra_chunk, **extra)
+    o = OracleTempCache(len(oh), cfg.d, cfg.nbits, cfg.tau, cfg.capacity, R.double().numpy(),
+                        intra_chunk=intra_chunk, key_mode=key_mode)
+    heads = set(oh if state_heads is None else state_heads)
     rep = ParityReport()
     sum_abs, n_abs = 0.0, 0
+    sel = None if rows is None else np.asarray(rows)
+
+    def check_commit(rec):
+        codes, match, dest = tc.last_commit()
+        rep.commits += 1
+        rep.tokens += rec.match.size
+        rep.merges += int((rec.match >= 0).sum())
+        rep.code_mismatch += int((codes[oh] != rec.codes).sum())
+        rep.match_mismatch += int((match[oh] != rec.match).sum())
+        rep.dest_mismatch += int((dest[oh] != rec.dest).sum())
+
     for c in range(chunks):
         K, V = w.next_chunk()
-        rec = o.append_chunk(f64(K), f64(V))
+        rec = o.append_chunk(f64(K[:, oh]), f64(V[:, oh]))
         tc.append_chunk(K, V)
-        rep.code_mismatch += int((tc.staged_codes() != o.staged[2]).sum())
+        rep.code_mismatch += int((tc.staged_codes()[oh] != o.staged[2]).sum())
         if rec is not None:
-            codes, match, dest = tc.last_commit()
-            rep.commits += 1
-            rep.tokens += match.size
-            rep.merges += int((rec.match >= 0).sum())
-            rep.code_mismatch += int((codes != rec.codes).sum())
-            rep.match_mismatch += int((match != rec.match).sum())
-            rep.dest_mismatch += int((dest != rec.dest).sum())
+            check_commit(rec)
             if check_every_state or c == chunks - 1:
-                compare_state(tc, o, rep, heads)
+                compare_state(tc, o, rep, heads, oh)
             rep.sizes.append(o.cache_size().tolist())
         for a in range(attends):
             Q = w.queries(c, a)
+            if q_scale != 1.0:
+                Q = (Q.float() * q_scale).to(Q.dtype)
             out = tc.attend(Q)
-            sel = None if rows is None else np.asarray(rows)
-            ref = o.attend(f64(Q), rows=sel)
-            got = f64(out) if sel is None else f64(out[torch.as_tensor(sel, device=out.device)])
-            err = np.abs(got - ref)
+            if attn_chunks is not None and c not in attn_chunks:
+                continue
+            ref = o.attend(f64(Q[:, oh]), rows=sel)
+            got = out[:, oh] if sel is None else out[torch.as_tensor(sel, device=out.device)][:, oh]
+            err = np.abs(f64(got) - ref)
             rep.attn_max_err = max(rep.attn_max_err, float(err.max()))
             sum_abs += float(err.sum())
             n_abs += err.size
             rep.attn_checks += 1
+        if on_chunk is not None:
+            on_chunk(c, tc, o, w, K, V)
     if flush:
         rec = o.flush()
         tc.flush()
         if rec is not None:
-            codes, match, dest = tc.last_commit()
-            rep.commits += 1
-            rep.tokens += match.size
-            rep.code_mismatch += int((codes != rec.codes).sum())
-            rep.match_mismatch += int((match != rec.match).sum())
-            rep.dest_mismatch += int((dest != rec.dest).sum())
-            compare_state(tc, o, rep, heads)
+            check_commit(rec)
+            compare_state(tc, o, rep, heads, oh)
     rep.attn_mean_err = sum_abs / max(n_abs, 1)
     tc.sync()
     return rep, tc, o
