@@ -63,6 +63,16 @@ typedef struct {
                                   duplicates inside one chunk merge too (the other
                                   reading of the same passage). Costs one more kernel and
                                   4 * 2^nbits bytes per head.                             */
+    int32_t key_mode;          /* 0: an entry keeps the key that created it (section 2.A
+                                  says values are averaged; keys are read as kept). 1: an
+                                  entry's key is the running mean of its members' keys,
+                                  k <- (n k + sum k_t) / (n + m) in fp32 in ascending t
+                                  (the other reading of the same passage); the entry's
+                                  code is recomputed from the new key and it moves to that
+                                  bucket for later commits, attention uses the mean key.
+                                  Requires intra_chunk = 0. Costs 4 d bytes per entry
+                                  (bf16 storage), 4 * 2^nbits bytes per head and two more
+                                  kernels per commit.                                      */
 } tc_options;
 
 /*
@@ -87,12 +97,14 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
 
 /*
  * tc_append_chunk - feed the next chunk of T new tokens, K and V [T, H, d].
- * First commits the chunk staged by the previous call (section 2.A: each new key
- * is matched top-1 in its hash bucket among the entries committed before; a match
- * at cosine >= tau merges, v <- (n v + sum v_t)/(n + m), n <- n + m; unmatched
- * keys are appended in token order), then stages this chunk: copies it into the
- * library's head-major staging buffer and hashes its keys. Attention sees a staged
- * chunk raw, with logit shift 0.
+ * First commits the chunk staged by the previous call, then stages this chunk.
+ * Staging copies the chunk into the library's head-major staging buffer, hashes
+ * its keys and takes every merge decision (section 2.A: each new key is matched
+ * top-1 in its hash bucket among the entries committed before its commit, which
+ * are already final at staging; a match at cosine >= tau merges). The commit
+ * applies them: v <- (n v + sum v_t)/(n + m), n <- n + m for merges, unmatched
+ * keys appended in token order. Attention sees a staged chunk raw, with logit
+ * shift 0.
  * Asynchronous on `stream`, except when the committed cache might overflow its
  * capacity: then the call synchronises to learn the outcome and, if the commit
  * would overflow, returns TC_ECAPACITY with the cache unchanged, the previous
@@ -155,6 +167,10 @@ tc_status tc_debug_staged_codes(tc_handle h, int64_t* T_out, uint32_t* codes_HT)
  * Any pointer may be NULL. */
 tc_status tc_export_cache(tc_handle h, int32_t head, void* K, float* V32, int32_t* n,
                           uint32_t* code);
+
+/* Running-mean keys (key_mode 1): the fp32 key means of head `head`'s committed
+ * entries, HOST K32 [M*d]. TC_ESTATE for a handle with representative keys. */
+tc_status tc_export_key_means(tc_handle h, int32_t head, float* K32);
 
 /* The hash normals in use, HOST [nbits * d]. */
 tc_status tc_get_hyperplanes(tc_handle h, float* R);

@@ -28,7 +28,7 @@ TC_BF16, TC_F32 = 0, 1
 API = [
     "tc_create", "tc_create_ex", "tc_append_chunk", "tc_attend", "tc_flush", "tc_reset", "tc_cache_size", "tc_sync",
     "tc_destroy", "tc_status_string", "tc_debug_last_commit", "tc_debug_staged_codes", "tc_export_cache",
-    "tc_get_hyperplanes", "tc_stats", "tc_merge_means_noalloc",
+    "tc_get_hyperplanes", "tc_stats", "tc_merge_means_noalloc", "tc_export_key_means",
     "tc_annca_create", "tc_annca_set_prompt", "tc_annca_attend", "tc_annca_kept", "tc_annca_get_hyperplanes",
     "tc_annca_sync", "tc_annca_destroy", "tc_annsa_attend",
     "tc_lvsa_create", "tc_lvsa_attend", "tc_lvsa_frames", "tc_lvsa_sync", "tc_lvsa_destroy",
@@ -37,7 +37,8 @@ API = [
 
 class TCOptions(ctypes.Structure):
     _fields_ = [("dtype", ctypes.c_int), ("seed", ctypes.c_uint64), ("softmax_scale", ctypes.c_float),
-                ("hyperplanes", ctypes.POINTER(ctypes.c_float)), ("intra_chunk", ctypes.c_int32)]
+                ("hyperplanes", ctypes.POINTER(ctypes.c_float)), ("intra_chunk", ctypes.c_int32),
+                ("key_mode", ctypes.c_int32)]
 
 
 def _load():
@@ -62,6 +63,7 @@ def _load():
         "tc_debug_staged_codes": (ctypes.c_int, [H, ctypes.POINTER(i64), vp]),
         "tc_export_cache": (ctypes.c_int, [H, i32, vp, vp, vp, vp]),
         "tc_get_hyperplanes": (ctypes.c_int, [H, vp]),
+        "tc_export_key_means": (ctypes.c_int, [H, i32, vp]),
         "tc_stats": (ctypes.c_int, [H, ctypes.POINTER(ctypes.c_uint64), ctypes.POINTER(ctypes.c_uint64),
                                     ctypes.POINTER(ctypes.c_uint64)]),
         "tc_merge_means_noalloc": (ctypes.c_int, [vp, ctypes.c_int, vp, i32, i32, vp, vp, i32, vp]),
@@ -121,15 +123,20 @@ class TempCache:
     """
 
     def __init__(self, H: int, d: int, nbits: int, tau: float, capacity: int, dtype: str = "bf16",
-                 seed: int = 0, softmax_scale: float = 0.0, hyperplanes=None, intra_chunk: bool = False):
+                 seed: int = 0, softmax_scale: float = 0.0, hyperplanes=None, intra_chunk: bool = False,
+                 key_mode: str = "representative"):
+        if key_mode not in ("representative", "mean"):
+            raise ValueError("key_mode is 'representative' or 'mean'")
         self.H, self.d, self.nbits = int(H), int(d), int(nbits)
         self.dtype = dtype
+        self.key_mode = key_mode
         self.torch_dtype = torch.bfloat16 if dtype == "bf16" else torch.float32
         opt = TCOptions()
         opt.dtype = TC_BF16 if dtype == "bf16" else TC_F32
         opt.seed = int(seed)
         opt.softmax_scale = float(softmax_scale)
         opt.intra_chunk = 1 if intra_chunk else 0
+        opt.key_mode = 1 if key_mode == "mean" else 0
         self._R = None
         if hyperplanes is not None:
             R = np.ascontiguousarray(np.asarray(hyperplanes, dtype=np.float32).reshape(-1))
@@ -212,7 +219,8 @@ class TempCache:
         return codes
 
     def export_cache(self, head: int):
-        """(K [M,d] as fp32, V32 [M,d], n [M], code [M]) of one head's committed entries."""
+        """(K [M,d] as fp32, V32 [M,d], n [M], code [M]) of one head's committed entries.
+        With running-mean keys K holds the fp32 key means."""
         M = int(self.cache_size()[head])
         K = np.zeros((M, self.d), np.uint16 if self.dtype == "bf16" else np.float32)
         V = np.zeros((M, self.d), np.float32)
@@ -222,6 +230,9 @@ class TempCache:
                "tc_export_cache")
         if self.dtype == "bf16":
             K = (K.astype(np.uint32) << 16).view(np.float32)
+        if self.key_mode == "mean":
+            K = np.zeros((M, self.d), np.float32)
+            _check(lib.tc_export_key_means(self._h, head, _np_ptr(K)), "tc_export_key_means")
         return K, V, n, code
 
     def hyperplanes(self) -> np.ndarray:

@@ -1,19 +1,29 @@
-// TempCache commit path: stage + hash, bucketed top-1 search with the merge
-// decision, append in token order, and the deterministic list merge.
+// TempCache commit path: staging (copy + hash + bucketed top-1 search with the merge
+// decision), then, when the next chunk arrives, the commit (append in token order and
+// the deterministic list merge).
 //
 // FAST-AR technical summary, section 2.A "TempCache": each key of the current
 // chunk is hashed with locality-sensitive hashing, its top-1 neighbour among the
 // earlier cache entries is found, and near-duplicates above a similarity threshold
 // are merged with their values averaged; the rest extend the cache.
 //
+// When the decisions are taken. A chunk is committed one call after it was staged,
+// and nothing changes the cache in between, so the cache a staged token must be
+// matched against (the entries committed before its commit) is already final when
+// it is staged. The staging kernel therefore also hashes the keys and searches their
+// buckets while the keys are on chip; the commit kernel only applies the decisions:
+// it appends the unmatched tokens and merges the matched ones. Per chunk that is two
+// launches (plus the in-chunk dedupe of the intra_chunk option, and two re-bucketing
+// launches with running-mean keys).
+//
 // Exactness of the integer results. Every decision here (a hash bit, the best
 // candidate, merge or not) is defined on fp64 dot products summed in index order
-// 0..d-1 (products of bf16/fp32 values are exact in fp64). The kernels first
-// compute the same dots in fp32 and keep the fp32 decision only when it is
-// certified: when the fp32 value is farther from the decision boundary than a
-// rigorous bound on its rounding error. Otherwise they recompute the fp64 sums in
-// index order, the same sequence of IEEE operations as the definition, so codes,
-// matches and the append order are bit-identical to it.
+// 0..d-1 (products of bf16/fp32 values are exact in fp64). Hash bits are first
+// computed in fp32 and kept only outside a rigorous bound of their rounding error,
+// else recomputed in fp64 in index order. Similarities are computed in fp64 with the
+// value of the index-order sum: exactly in any order when the exponent-span rule
+// below holds, else as the index-order chain itself. Codes, matches and the append
+// order are therefore bit-identical to the definition.
 #include "tc_internal.h"
 #include "tc_device.cuh"
 
@@ -23,141 +33,9 @@ namespace tc {
 
 namespace {
 
-// ------------------------------------------------------------------ stage + hash
-//
-// One warp per input row r = t*H + h of the token-major chunk, four rows in flight.
-// The row is copied to the head-major staging buffer. Lane l keeps columns
-// [l*EPL, l*EPL + EPL) of every hyperplane in registers (as bf16 pairs: the normals
-// are bf16 values) and forms the partial dot products of its columns; a
-// reduce-scatter butterfly then leaves the full <R_b, k> (fp32) on lane b. Bit b
-// keeps the fp32 sign when
-//   |<R_b,k>| > 2 (d+2) u |R_b| |k|   (u = 2^-24; any summation order errs by at
-//                                      most (d+2) u sum|R_bi k_i| <= (d+2) u |R_b||k|,
-//                                      doubled for margin)
-// and otherwise lane b redoes the sum in fp64 in index order. Bit b = [<R_b,k> >= 0].
-
-template <typename E, int D, int NBP>
-__global__ void __launch_bounds__(kWarps * 32, NBP <= 8 ? 3 : (NBP <= 16 ? 2 : 1))
-stage_hash_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView c, StageView s,
-                  const float* __restrict__ R, const float* __restrict__ Rnorm, int32_t* ctr, Stats* stats) {
-    grid_dependency_wait();
-    constexpr int EPL = D / 32;
-    constexpr int ROWS = 2;
-    using IO = RowIO<E, EPL>;
-    __shared__ float sKey[kWarps][D];
-    const int nbits = c.nbits, H = c.H;
-    const int64_t T = s.T;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < s.TmaxP;
-         i += (int64_t)gridDim.x * blockDim.x)
-        s.sbias[i] = (i < T) ? 0.f : -INFINITY;
-    // The commit of this chunk starts from zeroed counters (every commit follows the
-    // staging of the chunk it commits; a refused commit is cleared by the host).
-    if (blockIdx.x == 0)
-        for (int i = threadIdx.x; i < kCtrInts(H); i += blockDim.x) ctr[i] = 0;
-    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-    uint32_t Rp[NBP][EPL / 2];   // hyperplane slices, bf16 pairs
-#pragma unroll
-    for (int b = 0; b < NBP; ++b)
-#pragma unroll
-        for (int e = 0; e < EPL / 2; ++e)
-            Rp[b][e] = (b < nbits) ? pack_bf16_exact(R[b * D + lane * EPL + 2 * e], R[b * D + lane * EPL + 2 * e + 1])
-                                   : 0u;
-    const bool mine = lane < nbits;   // lane b reports bit b
-    const float gam2 = 2.f * (float)(D + 2) * kU32;
-    const float rn = mine ? Rnorm[lane] : 0.f;
-    const unsigned mask = (nbits >= 32) ? 0xffffffffu : ((1u << nbits) - 1u);
-    const int64_t rows = T * H;
-    const int64_t stride = (int64_t)gridDim.x * kWarps;
-    int nq = 0;                    // rows queued for the bucket-head lookup
-    int64_t q_sidx = 0, q_bucket = 0;
-    float kmax = 0.f;              // largest |k|^2 this warp staged
-    for (int64_t r0 = (int64_t)blockIdx.x * kWarps + wib; r0 < rows; r0 += ROWS * stride) {
-        typename IO::V kv[ROWS], vv[ROWS];
-#pragma unroll
-        for (int q = 0; q < ROWS; ++q) {
-            const int64_t r = r0 + q * stride;
-            if (r < rows) {
-                kv[q] = IO::load(K + r * D, lane);
-                vv[q] = IO::load(V + r * D, lane);
-            }
-        }
-#pragma unroll
-        for (int q = 0; q < ROWS; ++q) {
-            const int64_t r = r0 + q * stride;
-            if (r >= rows) break;   // warp-uniform
-            const int64_t t = (uint32_t)r / (uint32_t)H;   // rows < 2^31 (host check): 32-bit division
-            const int h = (int)(r - t * H);
-            const int64_t sidx = (int64_t)h * s.TmaxP + t;
-            IO::store(reinterpret_cast<E*>(s.Ks) + sidx * D, lane, kv[q]);
-            IO::store(reinterpret_cast<E*>(s.Vs) + sidx * D, lane, vv[q]);
-            float x[EPL];
-            IO::to_float(kv[q], x);
-            float nk = 0.f;
-            float v[NBP];
-#pragma unroll
-            for (int e = 0; e < EPL; ++e) nk = fmaf(x[e], x[e], nk);
-#pragma unroll
-            for (int b = 0; b < NBP; ++b) {
-                float a = 0.f;
-#pragma unroll
-                for (int e = 0; e < EPL / 2; ++e) {
-                    a = fmaf(__uint_as_float(Rp[b][e] << 16), x[2 * e], a);
-                    a = fmaf(__uint_as_float(Rp[b][e] & 0xffff0000u), x[2 * e + 1], a);
-                }
-                v[b] = a;
-            }
-            nk = warp_sum(nk);
-            kmax = fmaxf(kmax, nk);
-            const float p = reduce_scatter<NBP>(v, lane);
-            const float err = gam2 * rn * sqrtf(nk) + 1e-30f;
-            const bool need = mine && !(fabsf(p) > err);   // inside the band (or not finite)
-            bool bit = p >= 0.f;
-            if (__any_sync(0xffffffffu, need)) {
-#pragma unroll
-                for (int e = 0; e < EPL; ++e) sKey[wib][lane * EPL + e] = x[e];
-                __syncwarp();
-                if (need) {   // exact: fp64, index order
-                    double acc = 0.0;
-                    const float* rb = R + lane * D;
-                    for (int i = 0; i < D; ++i) acc = fma((double)rb[i], (double)sKey[wib][i], acc);
-                    bit = (acc >= 0.0);
-                }
-                __syncwarp();
-            }
-            const unsigned code = __ballot_sync(0xffffffffu, mine && bit) & mask;
-            const unsigned nre = __popc(__ballot_sync(0xffffffffu, need));
-            if (lane == 0) {
-                s.scode[sidx] = code;
-                if (nre) atomicAdd(&stats->hash_rechecks, (unsigned long long)nre);
-            }
-            // The bucket-head lookups of up to 32 rows are batched, one row per lane, so
-            // their latencies overlap instead of stalling the warp once per row.
-            if (lane == nq) {
-                q_sidx = sidx;
-                q_bucket = ((int64_t)h << c.nbits) + code;
-            }
-            if (++nq == 32) {
-                s.sfirst[q_sidx] = c.bhead[q_bucket];
-                nq = 0;
-            }
-        }
-    }
-    if (lane < nq) s.sfirst[q_sidx] = c.bhead[q_bucket];
-    // one bound per block: |k|^2 of the staged keys, rounded up past the fp32 sums' error
-    __shared__ float sKmax[kWarps];
-    if (lane == 0) sKmax[wib] = kmax * (1.f + 1.f / 1024.f);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        float m = 0.f;
-        for (int w = 0; w < kWarps; ++w) m = fmaxf(m, sKmax[w]);
-        atomicMax(reinterpret_cast<int*>(c.kmax2s), __float_as_int(m));
-    }
-    grid_dependents_launch();
-}
-
 // ------------------------------------------------------------------ lane groups
 //
-// The search, append and merge kernels give each row to a group of 8 lanes: lane g
+// The dedupe, append and merge kernels give each row to a group of 8 lanes: lane g
 // of group q (lanes 8q .. 8q+7) holds elements [g*EPG, g*EPG + EPG) of the row, so
 // one warp works on four rows at once and every lane moves 16-byte words.
 template <typename E, int D>
@@ -210,12 +88,6 @@ struct GSlice {
     }
 };
 
-__device__ __forceinline__ float gsum(float v, unsigned gmask) {
-    v += __shfl_xor_sync(gmask, v, 4);
-    v += __shfl_xor_sync(gmask, v, 2);
-    v += __shfl_xor_sync(gmask, v, 1);
-    return v;
-}
 __device__ __forceinline__ double gsum64(double v, unsigned gmask) {
     v += __shfl_xor_sync(gmask, v, 4);
     v += __shfl_xor_sync(gmask, v, 2);
@@ -316,232 +188,329 @@ __device__ void publish_sizes(const CacheView& c, const StageView& s, int32_t* c
         }
     }
 }
+// ------------------------------------------------------------------ staging: copy, hash, search
+//
+// One warp per window of 32 consecutive tokens t0 .. t0+31 of one head h (the unit
+// of the append order). The warp
+//  1. copies the window's K rows into shared memory and, with its V rows, into the
+//     head-major staging buffer (16-byte words, eight in flight per lane);
+//  2. hashes: lane l takes token t0 + l and forms the nbits projections <R_b, k> in
+//     fp32, the normals being constant-bank operands of the FMAs (a kernel parameter);
+//     bit b keeps the fp32 sign when
+//       |<R_b,k>| > 2 (d+2) u |R_b| |k|   (u = 2^-24; any summation order errs by at
+//                                          most (d+2) u sum|R_bi k_i| <= (d+2) u |R_b||k|,
+//                                          doubled for margin)
+//     and otherwise the lane redoes the sum in fp64 in index order;
+//  3. searches: each lane walks its token's bucket list (the entries committed before
+//     this chunk's commit with the same code) and forms every cosine
+//     dot / sqrt(|k|^2 |e|^2) in fp64 with the value of the index-order sums; the best
+//     candidate (ties to the lowest entry index) merges when its cosine is >= tau;
+//  4. publishes: a matched token joins its target's merge list, the window's count of
+//     unmatched tokens is stored for the append order. The last block to finish turns
+//     the window counts into the new cache sizes and raises the abort flag when a head
+//     would exceed its capacity.
+// With the intra_chunk option step 4 keeps the best committed candidate and its
+// similarity instead, and groups the chunk's tokens by bucket for the dedupe kernel.
+//
+// Exact similarities of bf16 rows. A product of two bf16 values has at most 16
+// significant bits, so it is exact in fp32. When span(x) + span(y) <= kSpanLimit every
+// partial sum of the products is exact in fp64 (see gspan_bf16), so four fp64 partial
+// sums in any order give the bits of the index-order sum; otherwise the lane runs the
+// index-order chain. With running-mean keys an entry whose key is not a bf16 value
+// has span 255 and always takes the chain, over its fp32 key.
+template <int D, int NBP>
+struct StagePlanes {
+    float v[NBP * D];   // normals (bf16 values), rows past nbits zero
+    float rn[NBP];      // |R_b|, rounded up
+};
 
-// ------------------------------------------------------------------ search + decide
-//
-// One 8-lane group per staged token (h, t). Candidates are the committed entries of
-// the token's bucket: the list bhead/bnext holds exactly the entries committed
-// before this commit, and its head was read when the token was staged (nothing
-// changes the cache between staging and commit). The four groups of a warp walk
-// their lists in lockstep, so each step has four independent row loads in flight.
-// The grid is persistent (two blocks per SM).
-//
-// bf16 storage: every cosine is formed in fp64 exactly as the definition does
-// (dot / sqrt(|k|^2 |e|^2), each sum in index order): the sums are exact by the
-// span rule above (else the index-order chain), |e|^2 was stored the same way when
-// the entry was appended, and the division and square root are IEEE-rounded on
-// both sides. The best candidate (ties to the lowest entry index) merges when its
-// cosine is >= tau.
-//
-// fp32 storage: fp32 cosines first; with delta a rigorous bound on |sim32 - sim|
-// the fp32 result decides when best < tau - delta (no merge) or best > tau + delta
-// and best - second > 2 delta (merge into the unique best). Any other case
-// recomputes every candidate with the index-order chain.
-//
-// A matched token joins its target's merge list; unmatched tokens are counted per
-// 32-token window. The last block to finish turns the window counts into the new
-// cache sizes and raises the abort flag if some head would exceed its capacity.
 template <typename E, int D>
+struct StageSmem {
+    static constexpr int RB = D * (int)sizeof(E) + 16;   // row pitch: consecutive rows start 4 banks apart
+    static constexpr int WARP = 32 * RB;
+    static constexpr int BYTES = kWarps * WARP;
+};
+
+// Element i of a row in shared memory, as a float.
+template <typename E>
+__device__ __forceinline__ float srow_at(const uint8_t* row, int i) {
+    if constexpr (sizeof(E) == 2)
+        return __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(row)[i] << 16);
+    else
+        return reinterpret_cast<const float*>(row)[i];
+}
+
+// The floats packed in a 16-byte word of a row (8 bf16 values or 4 fp32 values).
+template <typename E>
+__device__ __forceinline__ void unpack16(const uint4& v, float (&x)[16 / sizeof(E)]) {
+    if constexpr (sizeof(E) == 2) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            x[2 * k] = __uint_as_float(w[k] << 16);
+            x[2 * k + 1] = __uint_as_float(w[k] & 0xffff0000u);
+        }
+    } else {
+        x[0] = __uint_as_float(v.x);
+        x[1] = __uint_as_float(v.y);
+        x[2] = __uint_as_float(v.z);
+        x[3] = __uint_as_float(v.w);
+    }
+}
+
+// Index-order fp64 sum of x_i y_i over a shared-memory row x and a global row y.
+template <typename E, typename F, int D>
+__device__ __forceinline__ double chain_dot(const uint8_t* x, const F* __restrict__ y) {
+    double acc = 0.0;
+#pragma unroll 8
+    for (int i = 0; i < D; ++i) {
+        float yi;
+        if constexpr (sizeof(F) == 2)
+            yi = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(y)[i] << 16);
+        else
+            yi = y[i];
+        acc = fma((double)srow_at<E>(x, i), (double)yi, acc);
+    }
+    return acc;
+}
+
+// Exact sum of x_i y_i of two bf16 rows (x in shared memory, y from global memory) when
+// the span rule holds: exact fp32 products, four fp64 partial sums.
+template <int D>
+__device__ __forceinline__ double span_dot(const uint8_t* x, const uint4* __restrict__ y) {
+    constexpr int W = D / 8;
+    uint4 yw[W];
+#pragma unroll
+    for (int c = 0; c < W; ++c) yw[c] = y[c];
+    double a0 = 0.0, a1 = 0.0, a2 = 0.0, a3 = 0.0;
+#pragma unroll
+    for (int c = 0; c < W; ++c) {
+        float xv[8], yv[8];
+        unpack16<__nv_bfloat16>(*reinterpret_cast<const uint4*>(x + 16 * c), xv);
+        unpack16<__nv_bfloat16>(yw[c], yv);
+        a0 += (double)(xv[0] * yv[0]) + (double)(xv[4] * yv[4]);
+        a1 += (double)(xv[1] * yv[1]) + (double)(xv[5] * yv[5]);
+        a2 += (double)(xv[2] * yv[2]) + (double)(xv[6] * yv[6]);
+        a3 += (double)(xv[3] * yv[3]) + (double)(xv[7] * yv[7]);
+    }
+    return (a0 + a1) + (a2 + a3);
+}
+
+template <typename E, int D, int NBP, bool INTRA, bool MEAN>
 __global__ void __launch_bounds__(kWarps * 32, 2)
-search_kernel(CacheView c, StageView s, float tau, double tau64, float delta, bool intra, int32_t* ctr,
-              Stats* stats) {
-    grid_dependency_wait();
-    using G = GSlice<E, D>;
-    constexpr int EPG = G::EPG;
-    const int lane = threadIdx.x & 31, gl = lane & 7, grp = lane >> 3;
-    const unsigned gmask = 0xFFu << (8 * grp);
-    const int H = c.H;
+stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView c, StageView s,
+                    const float* __restrict__ R, const __grid_constant__ StagePlanes<D, NBP> pl, double tau64,
+                    int32_t* ctr, Stats* stats) {
+    using S = StageSmem<E, D>;
+    constexpr int W = D * (int)sizeof(E) / 16;   // 16-byte words per row
+    constexpr int EPW = 16 / (int)sizeof(E);     // elements per word
+    extern __shared__ __align__(16) uint8_t ss_smem[];
+    __shared__ float sKmax[kWarps];
+    __shared__ unsigned sRe[kWarps][2];
+    grid_dependency_wait();   // the previous commit (and anything else before us in the stream)
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    uint8_t* rows = ss_smem + wib * S::WARP;
+    const int H = c.H, nbits = c.nbits;
     const int64_t T = s.T;
-    const int64_t rows = T * H;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < s.TmaxP;
+         i += (int64_t)gridDim.x * blockDim.x)
+        s.sbias[i] = (i < T) ? 0.f : -INFINITY;
+    const int nwin = (int)((T + 31) >> 5);
+    const float gam2 = 2.f * (float)(D + 2) * kU32;
     const E* Kc = reinterpret_cast<const E*>(c.Kc);
-    const E* Ks = reinterpret_cast<const E*>(s.Ks);
-    int32_t* ntouched = ctr;
-    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;   // global warp
-    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    // The next token's key row and list head are loaded while the current token's
-    // decision is published (its atomics wait for their old values).
-    G xn;
-    int first_n = -1;
-    auto fetch = [&](int64_t r4n) {
-        const int64_t rn = r4n + grp;
-        if (rn < rows) {
-            const int hn = (int)((uint32_t)rn / (uint32_t)T);
-            const int64_t sn = (int64_t)hn * s.TmaxP + (rn - (int64_t)hn * T);
-            xn.load(Ks + sn * D, gl);
-            first_n = s.sfirst[sn];
-        } else {
-            xn.zero();
-            first_n = -1;
-        }
-    };
-    fetch(gw * 4);
-    for (int64_t r4 = gw * 4; r4 < rows; r4 += nw * 4) {   // warp-uniform loop
-        const int64_t r = r4 + grp;
-        const bool valid = r < rows;
-        const int h = valid ? (int)((uint32_t)r / (uint32_t)T) : 0;
-        const int64_t t = valid ? r - (int64_t)h * T : 0;
-        const int64_t sidx = (int64_t)h * s.TmaxP + t;
-        const int64_t hrow = (int64_t)h * c.capP;
-        const G x = xn;
-        const int first = first_n;
-        const int Mh = valid ? c.M[h] : 0;
-        int m = -1, nslow = 0;
-        double best64 = -INFINITY;   // exact best committed similarity and its entry
-        int bj64 = -1;
-        if constexpr (sizeof(E) == 2) {
-            const int spx = gspan_bf16<D>(x, gmask);
-            double n1 = gsum64(lane_dot64(x, x), gmask);
-            if (2 * spx > kSpanLimit<D>) {
-                n1 = gchain_dot(x, x, gl, grp, gmask);
-                ++nslow;
-            }
-            double best = -INFINITY;
-            int bestj = -1, ncand = 0;
-            int j = first;
-            while (__any_sync(0xffffffffu, j >= 0)) {
-                const bool act = j >= 0;
-                G y;
-                int nxt = -1, spy = 0;
-                double n2 = 0.0;
-                if (act) {
-                    y.load(Kc + (hrow + j) * D, gl);
-                    nxt = c.bnext[hrow + j];
-                    n2 = c.knorm64[hrow + j];
-                    spy = c.kspan[hrow + j];   // stored at append
-                } else {
-                    y.zero();
-                }
-                double dot = gsum64(lane_dot64(x, y), gmask);
-                if (act) {
-                    if (spx + spy > kSpanLimit<D>) {
-                        dot = gchain_dot(x, y, gl, grp, gmask);
-                        ++nslow;
-                    }
-                    const double sim = (n1 > 0.0 && n2 > 0.0) ? dot / sqrt(n1 * n2) : 0.0;
-                    if (sim > best || (sim == best && j < bestj)) {
-                        best = sim;
-                        bestj = j;
-                    }
-                    if (++ncand > Mh) {   // a bucket list can never be longer than the cache
-                        if (gl == 0) atomicOr(&stats->error_bits, kErrBucketList);
-                        nxt = -1;
-                    }
-                }
-                j = nxt;
-            }
-            m = (bestj >= 0 && best >= tau64) ? bestj : -1;
-            best64 = best;
-            bj64 = bestj;
-        } else {
-            float nk = 0.f;
+    float kmax = 0.f;                 // largest fp32 |k|^2 this lane staged
+    unsigned hre = 0, mre = 0;        // hash bits and similarity sums that took the fp64 chain
+    for (int64_t item = (int64_t)blockIdx.x * kWarps + wib; item < (int64_t)H * nwin;
+         item += (int64_t)gridDim.x * kWarps) {   // warp-uniform
+        const int h = (int)(item / nwin);
+        const int w = (int)(item - (int64_t)h * nwin);
+        const int t0 = w * 32;
+        const int n = (T - t0 < 32) ? (int)(T - t0) : 32;
+        const int64_t sbase = (int64_t)h * s.TmaxP + t0;
+        // ---- 1. copy
+        {
+            uint4* ks = reinterpret_cast<uint4*>(reinterpret_cast<E*>(s.Ks) + sbase * D);
+            uint4* vs = reinterpret_cast<uint4*>(reinterpret_cast<E*>(s.Vs) + sbase * D);
+            const int nw = n * W;
+#pragma unroll 1
+            for (int q0 = 0; q0 < 32 * W; q0 += 4 * 32) {
+                uint4 kb[4], vb[4];
 #pragma unroll
-            for (int i = 0; i < EPG; ++i) nk = fmaf(x.at(i), x.at(i), nk);
-            nk = gsum(nk, gmask);
-            float best = -INFINITY, second = -INFINITY;
-            int bestj = -1, ncand = 0;
-            bool weird = false;
-            int j = first;
-            while (__any_sync(0xffffffffu, j >= 0)) {
-                const bool act = j >= 0;
-                G y;
-                int nxt = -1;
-                if (act) {
-                    y.load(Kc + (hrow + j) * D, gl);
-                    nxt = c.bnext[hrow + j];
-                } else {
-                    y.zero();
+                for (int u = 0; u < 4; ++u) {
+                    const int q = q0 + u * 32 + lane;
+                    if (q < nw) {
+                        const int row = q / W, col = q - row * W;
+                        const int64_t src = ((int64_t)(t0 + row) * H + h) * D;
+                        kb[u] = reinterpret_cast<const uint4*>(K + src)[col];
+                        vb[u] = reinterpret_cast<const uint4*>(V + src)[col];
+                    }
                 }
-                float dt = 0.f, ne = 0.f;
 #pragma unroll
-                for (int i = 0; i < EPG; ++i) {
-                    dt = fmaf(x.at(i), y.at(i), dt);
-                    ne = fmaf(y.at(i), y.at(i), ne);
-                }
-                dt = gsum(dt, gmask);
-                ne = gsum(ne, gmask);
-                if (act) {
-                    const float den = nk * ne;
-                    float sim = 0.f;
-                    if (nk > 1e-30f && ne > 1e-30f && den < 1e38f && fabsf(dt) < 1e38f)
-                        sim = dt / sqrtf(den);
-                    else
-                        weird = true;
-                    if (sim > best) {
-                        second = best;
-                        best = sim;
-                        bestj = j;
-                    } else if (sim > second) {
-                        second = sim;
-                    }
-                    if (++ncand > Mh) {
-                        if (gl == 0) atomicOr(&stats->error_bits, kErrBucketList);
-                        nxt = -1;
+                for (int u = 0; u < 4; ++u) {
+                    const int q = q0 + u * 32 + lane;
+                    if (q < nw) {
+                        const int row = q / W, col = q - row * W;
+                        *reinterpret_cast<uint4*>(rows + row * S::RB + col * 16) = kb[u];
+                        ks[q] = kb[u];
+                        vs[q] = vb[u];
                     }
                 }
-                j = nxt;
-            }
-            bool exact = false;
-            if (ncand > 0) {
-                if (intra) exact = true;   // the exact best similarity is needed
-                else if (!weird && best < tau - delta) m = -1;
-                else if (!weird && best > tau + delta && (ncand == 1 || best - second > 2.f * delta)) m = bestj;
-                else exact = true;
-            }
-            if (exact) {   // uniform inside the group
-                nslow = 1;
-                const double n1 = gchain_dot(x, x, gl, grp, gmask);
-                double bsim = -INFINITY;
-                int bj = -1, guard = 0;
-                for (int jj = first; jj >= 0; jj = c.bnext[hrow + jj]) {
-                    if (++guard > ncand) break;
-                    G y;
-                    y.load(Kc + (hrow + jj) * D, gl);
-                    const double dot = gchain_dot(x, y, gl, grp, gmask);
-                    const double n2 = c.knorm64[hrow + jj];
-                    const double sim = (n1 > 0.0 && n2 > 0.0) ? dot / sqrt(n1 * n2) : 0.0;
-                    if (sim > bsim || (sim == bsim && jj < bj)) {
-                        bsim = sim;
-                        bj = jj;
-                    }
-                }
-                m = (bj >= 0 && bsim >= tau64) ? bj : -1;
-                best64 = bsim;
-                bj64 = bj;
-            }
-        }
-        fetch(r4 + nw * 4);
-        if (intra) {
-            // Matching inside the chunk: keep the committed best for the dedupe kernel
-            // and group the chunk's tokens by bucket.
-            if (valid && gl == 0) {
-                s.match[sidx] = bj64;
-                s.bsim[sidx] = best64;
-                if (nslow) atomicAdd(&stats->match_rechecks, (unsigned long long)nslow);
-                const int old = atomicExch(&c.cbhead[((int64_t)h << c.nbits) + s.scode[sidx]], (int)t);
-                s.cbnext[sidx] = old;
-            }
-            __syncwarp();
-            continue;
-        }
-        if (valid && gl == 0) {
-            s.match[sidx] = m;
-            if (nslow) atomicAdd(&stats->match_rechecks, (unsigned long long)nslow);
-            if (m >= 0) {
-                const int old = atomicExch(&c.lhead[hrow + m], (int)t);
-                s.lnext[sidx] = old;
-                if (old < 0) s.touched[(int64_t)h * s.TmaxP + atomicAdd(&ntouched[h], 1)] = m;
-            } else {
-                atomicAdd(&s.wcnt[(int64_t)h * (s.TmaxP >> 5) + (t >> 5)], 1);
             }
         }
         __syncwarp();
+        // ---- 2. hash
+        const bool valid = lane < n;
+        const uint8_t* my = rows + lane * S::RB;
+        uint32_t code = 0;
+        int spx = 255;
+        if (valid) {
+            float acc[NBP];
+#pragma unroll
+            for (int b = 0; b < NBP; ++b) acc[b] = 0.f;
+            float n2 = 0.f;
+            int emax = 0, emin = 255;
+#pragma unroll
+            for (int cw = 0; cw < W; ++cw) {
+                const uint4 v4 = *reinterpret_cast<const uint4*>(my + cw * 16);
+                float x[EPW];
+                unpack16<E>(v4, x);
+                if constexpr (sizeof(E) == 2) {
+                    const uint32_t wd[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t lo = wd[k] & 0xffffu, hi = wd[k] >> 16;
+                        const int flo = max((int)((lo >> 7) & 0xffu), 1), fhi = max((int)((hi >> 7) & 0xffu), 1);
+                        if (lo & 0x7fffu) { emax = max(emax, flo); emin = min(emin, flo); }
+                        if (hi & 0x7fffu) { emax = max(emax, fhi); emin = min(emin, fhi); }
+                    }
+                }
+#pragma unroll
+                for (int k = 0; k < EPW; ++k) n2 = fmaf(x[k], x[k], n2);
+#pragma unroll
+                for (int b = 0; b < NBP; ++b) {
+                    float t = acc[b];
+#pragma unroll
+                    for (int k = 0; k < EPW; ++k) t = fmaf(pl.v[b * D + cw * EPW + k], x[k], t);
+                    acc[b] = t;
+                }
+            }
+            const float nx = sqrtf(n2);
+#pragma unroll
+            for (int b = 0; b < NBP; ++b) {
+                if (b >= nbits) break;
+                bool bit = acc[b] >= 0.f;
+                if (!(fabsf(acc[b]) > gam2 * pl.rn[b] * nx + 1e-30f)) {   // inside the band (or not finite)
+                    double s64 = 0.0;
+                    for (int i = 0; i < D; ++i) s64 = fma((double)R[b * D + i], (double)srow_at<E>(my, i), s64);
+                    bit = s64 >= 0.0;
+                    ++hre;
+                }
+                code |= (uint32_t)bit << b;
+            }
+            if constexpr (sizeof(E) == 2) spx = emax >= emin ? emax - emin + 7 : 0;
+            s.scode[sbase + lane] = code;
+            kmax = fmaxf(kmax, n2);
+        }
+        // ---- 3. search the bucket
+        const int64_t hrow = (int64_t)h * c.capP;
+        const int Mh = c.M[h];
+        int j = valid ? c.bhead[((int64_t)h << nbits) + code] : -1;
+        double best = -INFINITY, n1 = -1.0;
+        int bestj = -1, ncand = 0;
+        while (j >= 0) {   // per lane
+            const int nxt = c.bnext[hrow + j];
+            const double n2e = c.knorm64[hrow + j];
+            const int spy = c.kspan[hrow + j];
+            if (n1 < 0.0) {   // |x|^2 with the value of the index-order sum, once per token
+                if constexpr (sizeof(E) == 2) {
+                    if (2 * spx <= kSpanLimit<D>) {
+                        n1 = span_dot<D>(my, reinterpret_cast<const uint4*>(my));
+                    } else {
+                        n1 = chain_dot<E, __nv_bfloat16, D>(my, reinterpret_cast<const __nv_bfloat16*>(my));
+                        ++mre;
+                    }
+                } else {
+                    n1 = chain_dot<E, float, D>(my, reinterpret_cast<const float*>(my));
+                }
+            }
+            double dot;
+            if constexpr (sizeof(E) == 2) {
+                if (spx + spy <= kSpanLimit<D>) {
+                    dot = span_dot<D>(my, reinterpret_cast<const uint4*>(Kc + (hrow + j) * D));
+                } else {
+                    if constexpr (MEAN) dot = chain_dot<E, float, D>(my, c.K32 + (hrow + j) * D);
+                    else dot = chain_dot<E, __nv_bfloat16, D>(my, reinterpret_cast<const __nv_bfloat16*>(Kc) + (hrow + j) * D);
+                    ++mre;
+                }
+            } else {
+                dot = chain_dot<E, float, D>(my, reinterpret_cast<const float*>(Kc) + (hrow + j) * D);
+                ++mre;
+            }
+            const double sim = (n1 > 0.0 && n2e > 0.0) ? dot / sqrt(n1 * n2e) : 0.0;
+            if (sim > best || (sim == best && j < bestj)) {
+                best = sim;
+                bestj = j;
+            }
+            if (++ncand > Mh) {   // a bucket list can never be longer than the cache
+                atomicOr(&stats->error_bits, kErrBucketList);
+                break;
+            }
+            j = nxt;
+        }
+        // ---- 4. publish
+        const int64_t sidx = sbase + lane;
+        const int t = t0 + lane;
+        if constexpr (INTRA) {
+            if (valid) {
+                s.match[sidx] = bestj;
+                s.bsim[sidx] = best;
+                s.cbnext[sidx] = atomicExch(&c.cbhead[((int64_t)h << nbits) + code], t);
+            }
+            if (lane == 0) s.wcnt[(int64_t)h * (s.TmaxP >> 5) + w] = 0;   // counted by the dedupe kernel
+        } else {
+            const int m = (bestj >= 0 && best >= tau64) ? bestj : -1;
+            if (valid) {
+                s.match[sidx] = m;
+                if (m >= 0) {
+                    const int old = atomicExch(&c.lhead[hrow + m], t);
+                    s.lnext[sidx] = old;
+                    if (old < 0) s.touched[(int64_t)h * s.TmaxP + atomicAdd(&ctr[h], 1)] = m;
+                }
+            }
+            const unsigned un = __ballot_sync(0xffffffffu, valid && m < 0);
+            if (lane == 0) s.wcnt[(int64_t)h * (s.TmaxP >> 5) + w] = __popc(un);
+        }
+        __syncwarp();   // the rows buffer is refilled by the warp's next window
+    }
+    // one bound per block: |k|^2 of the staged keys, rounded up past the fp32 sums' error
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        kmax = fmaxf(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+        hre += __shfl_xor_sync(0xffffffffu, hre, o);
+        mre += __shfl_xor_sync(0xffffffffu, mre, o);
+    }
+    if (lane == 0) {
+        sKmax[wib] = kmax * (1.f + 1.f / 1024.f);
+        sRe[wib][0] = hre;
+        sRe[wib][1] = mre;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float m = 0.f;
+        unsigned a = 0, b = 0;
+        for (int q = 0; q < kWarps; ++q) {
+            m = fmaxf(m, sKmax[q]);
+            a += sRe[q][0];
+            b += sRe[q][1];
+        }
+        atomicMax(reinterpret_cast<int*>(c.kmax2s), __float_as_int(m));
+        if (a) atomicAdd(&stats->hash_rechecks, (unsigned long long)a);
+        if (b) atomicAdd(&stats->match_rechecks, (unsigned long long)b);
     }
     grid_dependents_launch();
-    if (!intra) publish_sizes(c, s, ctr);
+    if (!INTRA) publish_sizes(c, s, ctr);
 }
 
-// Exact fp64 cosine of two rows held by a lane group (the similarity of the
-// definition; bf16 rows use the exact-sum rule, other rows the index-order chain).
 template <typename E, int D>
 __device__ __forceinline__ double gexact_dot(const GSlice<E, D>& a, int spa, const GSlice<E, D>& b, int spb, int gl,
                                              int grp, unsigned gmask) {
@@ -711,156 +680,193 @@ __device__ __forceinline__ double gnorm64(const GSlice<E, D>& x, int span, int g
     return gchain_dot(x, x, gl, grp, gmask);
 }
 
-// ------------------------------------------------------------------ append
+// ------------------------------------------------------------------ commit: append + merge
 //
-// One warp per 32-token window of one head. Unmatched tokens of the window take
-// consecutive entries in token order: dest = M_h + (unmatched tokens of earlier
-// windows) + (unmatched lanes below). Each becomes an entry (key, value mean, n = 1,
-// log2 n = 0, code, |k|^2 with the value of the fp64 index-order sum) and is pushed
-// on its bucket's list; lane groups copy two rows each per pass.
-template <typename E, int D>
-__global__ void __launch_bounds__(kWarps * 32, 3) append_kernel(CacheView c, StageView s, const int32_t* ctr) {
-    grid_dependency_wait();
-    grid_dependents_launch();   // the merge only needs this kernel's completion
-    using G = GSlice<E, D>;
-    constexpr int EPG = G::EPG;
-    __shared__ int sSrc[kWarps][32];
-    const int H = c.H;
-    if (ctr[2 * H]) return;  // commit aborted: nothing changes
-    const int lane = threadIdx.x & 31, gl = lane & 7, grp = lane >> 3, wib = threadIdx.x >> 5;
-    const unsigned gmask = 0xFFu << (8 * grp);
-    const int64_t T = s.T;
-    const int nwin = (int)((T + 31) >> 5);
-    const E* Ks = reinterpret_cast<const E*>(s.Ks);
-    const E* Vs = reinterpret_cast<const E*>(s.Vs);
-    const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t wg = gw; wg < (int64_t)H * nwin; wg += nw) {
-        const int h = (int)(wg / nwin);
-        const int w = (int)(wg - (int64_t)h * nwin);
-        const int32_t* wc = s.wcnt + (int64_t)h * (s.TmaxP >> 5);
-        int prefix = 0;
-#pragma unroll 4
-        for (int q = lane; q < w; q += 32) prefix += wc[q];   // independent loads, unrolled
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) prefix += __shfl_xor_sync(0xffffffffu, prefix, o);
-        const int64_t t = (int64_t)w * 32 + lane;
-        const bool valid = t < T;
-        const int64_t sidx = (int64_t)h * s.TmaxP + t;
-        const int m = valid ? s.match[sidx] : 0;
-        const bool un = valid && m == -1;   // -2 - u: joins the entry token u creates
-        const unsigned bal = __ballot_sync(0xffffffffu, un);
-        const int rank = __popc(bal & ((1u << lane) - 1u));
-        const int base = c.M[h] + prefix;
-        if (valid) {
-            if (m >= -1) s.dest[sidx] = un ? base + rank : m;
-            s.lcode[sidx] = s.scode[sidx];
-        }
-        if (un) sSrc[wib][rank] = lane;
-        __syncwarp();
-        const int nun = __popc(bal);
-        const int64_t hrow = (int64_t)h * c.capP;
-        const int64_t wrow = (int64_t)h * s.TmaxP + (int64_t)w * 32;
-        float kmax = 0.f;   // largest |k|^2 of the entries this warp creates
-        for (int k0 = 0; k0 < nun; k0 += 8) {   // warp-uniform
-            G kr[2], vr[2];
-            int64_t st[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int k = k0 + 4 * u + grp;
-                st[u] = k < nun ? wrow + sSrc[wib][k] : -1;
-                if (st[u] >= 0) {
-                    kr[u].load(Ks + st[u] * D, gl);
-                    vr[u].load(Vs + st[u] * D, gl);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                if (st[u] < 0) continue;   // group-uniform
-                const int k = k0 + 4 * u + grp;
-                const int64_t e = hrow + base + k;
-                kr[u].store(reinterpret_cast<E*>(c.Kc) + e * D, gl);
-                float4* v32 = reinterpret_cast<float4*>(c.V32 + e * D + gl * EPG);
-                int members = 0;   // later tokens of this chunk that joined this new entry
-                const int64_t sbase = (int64_t)h * s.TmaxP;
-                int tm = s.ichead[st[u]];
-                if (tm < 0) {
-                    vr[u].store(reinterpret_cast<E*>(c.Vc) + e * D, gl);
-#pragma unroll
-                    for (int q = 0; q < EPG / 4; ++q)
-                        v32[q] = make_float4(vr[u].at(4 * q), vr[u].at(4 * q + 1), vr[u].at(4 * q + 2),
-                                             vr[u].at(4 * q + 3));
-                } else {   // group-uniform: mean of the creating token and its members, in t order
-                    float acc[EPG];
-#pragma unroll
-                    for (int i = 0; i < EPG; ++i) acc[i] = 0.f;
-                    for (; tm >= 0; tm = s.icnext[sbase + tm]) {
-                        G vm;
-                        vm.load(Vs + (sbase + tm) * D, gl);
-#pragma unroll
-                        for (int i = 0; i < EPG; ++i) acc[i] = __fadd_rn(acc[i], vm.at(i));
-                        if (gl == 0) {
-                            s.match[sbase + tm] = base + k;
-                            s.dest[sbase + tm] = base + k;
-                        }
-                        if (++members > (int)T) break;
-                    }
-                    const float ft = (float)(1 + members);
-                    float nv[EPG];
-#pragma unroll
-                    for (int i = 0; i < EPG; ++i) nv[i] = __fdiv_rn(__fadd_rn(vr[u].at(i), acc[i]), ft);
-#pragma unroll
-                    for (int q = 0; q < EPG / 4; ++q)
-                        v32[q] = make_float4(nv[4 * q], nv[4 * q + 1], nv[4 * q + 2], nv[4 * q + 3]);
-                    G out;
-                    out.from_floats(nv);
-                    out.store(reinterpret_cast<E*>(c.Vc) + e * D, gl);
-                    if (gl == 0) s.ichead[st[u]] = -1;
-                }
-                int span = 255;
-                if constexpr (sizeof(E) == 2) span = min(gspan_bf16<D>(kr[u], gmask), 255);
-                const double nk = gnorm64(kr[u], span, gl, grp, gmask);
-                kmax = fmaxf(kmax, __double2float_ru(nk));
-                if (gl == 0) {
-                    const uint32_t code = s.scode[st[u]];
-                    c.knorm64[e] = nk;
-                    c.kspan[e] = (uint8_t)span;
-                    c.cnt[e] = 1 + members;
-                    c.bias2[e] = log2f((float)(1 + members));
-                    if (members) atomicMax(reinterpret_cast<int*>(&c.bmax[h]), __float_as_int(log2f((float)(1 + members))));
-                    c.code[e] = code;
-                    c.bnext[e] = atomicExch(&c.bhead[((int64_t)h << c.nbits) + code], base + k);
-                }
-            }
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) kmax = fmaxf(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-        if (lane == 0 && nun > 0) atomicMax(reinterpret_cast<int*>(&c.kmax2[h]), __float_as_int(kmax));
-        __syncwarp();
-    }
-}
-
-// ------------------------------------------------------------------ merge
+// One kernel applies the decisions the staging of the chunk took. Its warps take work
+// items in order: first the 32-token windows of every head (append), then groups of
+// four slots of the per-head lists of touched entries (merge). The two kinds write
+// disjoint entries (new ones at M_h and beyond, merged ones below M_h). The last block
+// to finish publishes the new sizes and clears the per-commit counters.
 //
-// One lane group per entry touched by merges. The matched tokens' values are
-// summed in fp32 in ascending token order (whatever order the atomics built the
-// list in), then v <- (n v + sum) / (n + m), n <- n + m (Lemma 5.1: the merged
-// entry carries the mean of its group and the group size). Lists of up to 8 tokens
-// are ordered inside the group; longer ones go to the whole warp, which orders up
-// to kListSmem tokens in shared memory and otherwise gathers them by scanning the
-// head's match targets in token order. The kernel also leaves the per-commit state
-// ready for the next commit (lists emptied, window counts zeroed, sizes published).
+// Append: unmatched tokens of a window take consecutive entries in token order:
+// dest = M_h + (unmatched tokens of earlier windows) + (unmatched lanes below). Each
+// becomes an entry (key, value mean, n = 1, log2 n = 0, code, |k|^2 with the value of
+// the fp64 index-order sum) and is pushed on its bucket's list; lane groups copy two
+// rows each per pass. With the intra_chunk option an entry created in the commit also
+// averages the later tokens of the chunk that merged into it.
+//
+// Merge: one lane group per touched entry. The matched tokens' values are summed in
+// fp32 in ascending token order (whatever order the atomics built the list in), then
+// v <- (n v + sum) / (n + m), n <- n + m (Lemma 5.1: the merged entry carries the mean
+// of its group and the group size). Lists of up to 8 tokens are ordered inside the
+// group; longer ones go to the whole warp, which orders up to kListSmem tokens in
+// shared memory and otherwise gathers them by scanning the head's match targets in
+// token order. With running-mean keys every merge goes to the whole warp, which also
+// averages the keys the same way in fp32, re-hashes the new key and records the entry
+// when its code changed (the re-bucketing kernels then move it).
 constexpr int kListSmem = 256;
 
+template <typename E, int D, bool MEAN>
+struct CommitArgs {
+    CacheView c;
+    StageView s;
+    const float* R;       // device normals (fp64 re-checks of the new keys' codes)
+    const float* Rnorm;   // |R_b|, rounded up
+    int32_t* ctr;
+    Stats* stats;
+};
+
 template <typename E, int D>
-__device__ void merge_long_list(const CacheView& c, const StageView& s, int h, int j, int32_t* sIds,
-                                int32_t* sSorted, int lane) {
+__device__ __forceinline__ void append_window(const CacheView& c, const StageView& s, int h, int w, int* sSrc,
+                                              int lane) {
+    using G = GSlice<E, D>;
+    constexpr int EPG = G::EPG;
+    const int gl = lane & 7, grp = lane >> 3;
+    const unsigned gmask = 0xFFu << (8 * grp);
+    const int64_t T = s.T;
+    const E* Ks = reinterpret_cast<const E*>(s.Ks);
+    const E* Vs = reinterpret_cast<const E*>(s.Vs);
+    const int32_t* wc = s.wcnt + (int64_t)h * (s.TmaxP >> 5);
+    int prefix = 0;
+#pragma unroll 4
+    for (int q = lane; q < w; q += 32) prefix += wc[q];   // independent loads, unrolled
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) prefix += __shfl_xor_sync(0xffffffffu, prefix, o);
+    const int64_t t = (int64_t)w * 32 + lane;
+    const bool valid = t < T;
+    const int64_t sidx = (int64_t)h * s.TmaxP + t;
+    const int m = valid ? s.match[sidx] : 0;
+    const bool un = valid && m == -1;   // -2 - u: joins the entry token u creates
+    const unsigned bal = __ballot_sync(0xffffffffu, un);
+    const int rank = __popc(bal & ((1u << lane) - 1u));
+    const int base = c.M[h] + prefix;
+    if (valid) {
+        if (m >= -1) {
+            s.dest[sidx] = un ? base + rank : m;
+            s.lmatch[sidx] = m;
+        }
+        s.lcode[sidx] = s.scode[sidx];
+    }
+    if (un) sSrc[rank] = lane;
+    __syncwarp();
+    const int nun = __popc(bal);
+    const int64_t hrow = (int64_t)h * c.capP;
+    const int64_t wrow = (int64_t)h * s.TmaxP + (int64_t)w * 32;
+    float kmax = 0.f;   // largest |k|^2 of the entries this warp creates
+    for (int k0 = 0; k0 < nun; k0 += 8) {   // warp-uniform
+        G kr[2], vr[2];
+        int64_t st[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int k = k0 + 4 * u + grp;
+            st[u] = k < nun ? wrow + sSrc[k] : -1;
+            if (st[u] >= 0) {
+                kr[u].load(Ks + st[u] * D, gl);
+                vr[u].load(Vs + st[u] * D, gl);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            if (st[u] < 0) continue;   // group-uniform
+            const int k = k0 + 4 * u + grp;
+            const int64_t e = hrow + base + k;
+            kr[u].store(reinterpret_cast<E*>(c.Kc) + e * D, gl);
+            if (c.K32 && (void*)c.K32 != c.Kc) {   // running-mean keys, bf16 storage: the fp32 key
+                float4* k32 = reinterpret_cast<float4*>(c.K32 + e * D + gl * EPG);
+#pragma unroll
+                for (int q = 0; q < EPG / 4; ++q)
+                    k32[q] = make_float4(kr[u].at(4 * q), kr[u].at(4 * q + 1), kr[u].at(4 * q + 2), kr[u].at(4 * q + 3));
+            }
+            float4* v32 = reinterpret_cast<float4*>(c.V32 + e * D + gl * EPG);
+            int members = 0;   // later tokens of this chunk that joined this new entry
+            const int64_t sbase = (int64_t)h * s.TmaxP;
+            int tm = s.ichead[st[u]];
+            if (tm < 0) {
+                vr[u].store(reinterpret_cast<E*>(c.Vc) + e * D, gl);
+#pragma unroll
+                for (int q = 0; q < EPG / 4; ++q)
+                    v32[q] = make_float4(vr[u].at(4 * q), vr[u].at(4 * q + 1), vr[u].at(4 * q + 2),
+                                         vr[u].at(4 * q + 3));
+            } else {   // group-uniform: mean of the creating token and its members, in t order
+                float acc[EPG];
+#pragma unroll
+                for (int i = 0; i < EPG; ++i) acc[i] = 0.f;
+                for (; tm >= 0; tm = s.icnext[sbase + tm]) {
+                    G vm;
+                    vm.load(Vs + (sbase + tm) * D, gl);
+#pragma unroll
+                    for (int i = 0; i < EPG; ++i) acc[i] = __fadd_rn(acc[i], vm.at(i));
+                    if (gl == 0) {
+                        s.lmatch[sbase + tm] = base + k;
+                        s.dest[sbase + tm] = base + k;
+                    }
+                    if (++members > (int)T) break;
+                }
+                const float ft = (float)(1 + members);
+                float nv[EPG];
+#pragma unroll
+                for (int i = 0; i < EPG; ++i) nv[i] = __fdiv_rn(__fadd_rn(vr[u].at(i), acc[i]), ft);
+#pragma unroll
+                for (int q = 0; q < EPG / 4; ++q)
+                    v32[q] = make_float4(nv[4 * q], nv[4 * q + 1], nv[4 * q + 2], nv[4 * q + 3]);
+                G out;
+                out.from_floats(nv);
+                out.store(reinterpret_cast<E*>(c.Vc) + e * D, gl);
+                if (gl == 0) s.ichead[st[u]] = -1;
+            }
+            int span = 255;
+            if constexpr (sizeof(E) == 2) span = min(gspan_bf16<D>(kr[u], gmask), 255);
+            const double nk = gnorm64(kr[u], span, gl, grp, gmask);
+            kmax = fmaxf(kmax, __double2float_ru(nk));
+            if (gl == 0) {
+                const uint32_t code = s.scode[st[u]];
+                c.knorm64[e] = nk;
+                c.kspan[e] = (uint8_t)span;
+                c.cnt[e] = 1 + members;
+                c.bias2[e] = log2f((float)(1 + members));
+                if (members) atomicMax(reinterpret_cast<int*>(&c.bmax[h]), __float_as_int(log2f((float)(1 + members))));
+                c.code[e] = code;
+                c.bnext[e] = atomicExch(&c.bhead[((int64_t)h << c.nbits) + code], base + k);
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) kmax = fmaxf(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    if (lane == 0 && nun > 0) atomicMax(reinterpret_cast<int*>(&c.kmax2[h]), __float_as_int(kmax));
+    __syncwarp();
+}
+
+// Index-order fp64 sum of x_i^2 (or of <R_b, x>) over a row spread across the warp,
+// lane l holding elements [l EPL, l EPL + EPL): each lane continues the previous
+// lane's sum. Every lane gets the result.
+template <int EPL>
+__device__ __forceinline__ double warp_chain(const float (&a)[EPL], const float (&b)[EPL], int lane) {
+    double acc = 0.0;
+#pragma unroll 1
+    for (int k = 0; k < 32; ++k) {
+        if (lane == k) {
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) acc = fma((double)a[i], (double)b[i], acc);
+        }
+        acc = __shfl_sync(0xffffffffu, acc, k);
+    }
+    return acc;
+}
+
+// One touched entry j of head h, merged by the whole warp (lane l: elements
+// [l EPL, l EPL + EPL)). MEAN: the key is averaged too, then re-hashed.
+template <typename E, int D, bool MEAN>
+__device__ void merge_entry_warp(const CommitArgs<E, D, MEAN>& a, int h, int j, int32_t* sIds, int32_t* sSorted,
+                                 int lane) {
+    const CacheView& c = a.c;
+    const StageView& s = a.s;
     constexpr int EPL = D / 32;
     using IO = RowIO<E, EPL>;
     const int64_t T = s.T;
     const int64_t sbase = (int64_t)h * s.TmaxP;
     const int64_t e = (int64_t)h * c.capP + j;
     const E* Vs = reinterpret_cast<const E*>(s.Vs);
+    const E* Ks = reinterpret_cast<const E*>(s.Ks);
     int L = 0, id = 0x7fffffff;
     for (int tt = c.lhead[e]; tt >= 0; tt = s.lnext[sbase + tt]) {
         if (L < 32 && lane == L) id = tt;
@@ -869,14 +875,20 @@ __device__ void merge_long_list(const CacheView& c, const StageView& s, int h, i
         if (L > (int)T) break;   // a list is never longer than the chunk
     }
     __syncwarp();
-    float acc[EPL];
+    float acc[EPL], kacc[EPL];
 #pragma unroll
-    for (int q = 0; q < EPL; ++q) acc[q] = 0.f;
+    for (int q = 0; q < EPL; ++q) acc[q] = kacc[q] = 0.f;
     auto add_row = [&](int tt) {
         float v[EPL];
         IO::to_float(IO::load(Vs + (sbase + tt) * D, lane), v);
 #pragma unroll
         for (int q = 0; q < EPL; ++q) acc[q] = __fadd_rn(acc[q], v[q]);
+        if constexpr (MEAN) {
+            float k[EPL];
+            IO::to_float(IO::load(Ks + (sbase + tt) * D, lane), k);
+#pragma unroll
+            for (int q = 0; q < EPL; ++q) kacc[q] = __fadd_rn(kacc[q], k[q]);
+        }
     };
     if (L <= 32) {
         int rank = 0;
@@ -886,8 +898,8 @@ __device__ void merge_long_list(const CacheView& c, const StageView& s, int h, i
             add_row(__shfl_sync(0xffffffffu, id, src));
         }
     } else if (L <= kListSmem) {
-        for (int a = lane; a < L; a += 32) {
-            const int mine = sIds[a];
+        for (int p = lane; p < L; p += 32) {
+            const int mine = sIds[p];
             int rank = 0;
             for (int b = 0; b < L; ++b) rank += (sIds[b] < mine);
             sSorted[rank] = mine;
@@ -916,6 +928,84 @@ __device__ void merge_long_list(const CacheView& c, const StageView& s, int h, i
         c.V32[e * D + lane * EPL + q] = nv[q];
     }
     IO::store(reinterpret_cast<E*>(c.Vc) + e * D, lane, IO::from_float(nv));
+    if constexpr (MEAN) {
+        // k <- (n k + sum k_t) / (n + m) in fp32, the same operations as the values
+        float nk[EPL];
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) {
+            const float old = c.K32[e * D + lane * EPL + q];
+            nk[q] = __fdiv_rn(__fadd_rn(__fmul_rn(fn, old), kacc[q]), ft);
+            c.K32[e * D + lane * EPL + q] = nk[q];
+        }
+        const typename IO::V kst = IO::from_float(nk);
+        IO::store(reinterpret_cast<E*>(c.Kc) + e * D, lane, kst);
+        // the storage copy's |k|^2 bounds the attention logits
+        float ks[EPL];
+        IO::to_float(kst, ks);
+        float ks2 = 0.f;
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) ks2 = fmaf(ks[q], ks[q], ks2);
+        ks2 = warp_sum(ks2);
+        // span of the new key when every element is a bf16 value (else 255: the search
+        // then takes the chain over the fp32 key)
+        bool exact16 = true;
+        int emax = 0, emin = 255;
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) {
+            const uint32_t u = __float_as_uint(nk[q]);
+            exact16 = exact16 && (u & 0xffffu) == 0u;
+            const uint32_t hb = u >> 16;
+            if (hb & 0x7fffu) {
+                const int f = max((int)((hb >> 7) & 0xffu), 1);
+                emax = max(emax, f);
+                emin = min(emin, f);
+            }
+        }
+        exact16 = __all_sync(0xffffffffu, exact16) && sizeof(E) == 2;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, o));
+            emin = min(emin, __shfl_xor_sync(0xffffffffu, emin, o));
+        }
+        const int span = exact16 ? min(emax >= emin ? emax - emin + 7 : 0, 255) : 255;
+        const double n64 = warp_chain<EPL>(nk, nk, lane);
+        // the code of the new key: fp32 projections, certified, else fp64 in index order
+        float n2 = 0.f;
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) n2 = fmaf(nk[q], nk[q], n2);
+        const float nx = sqrtf(warp_sum(n2));
+        const float gam2 = 2.f * (float)(D + 2) * kU32;
+        uint32_t code = 0;
+        unsigned nre = 0;
+        for (int b = 0; b < c.nbits; ++b) {
+            float rb[EPL];
+#pragma unroll
+            for (int q = 0; q < EPL; ++q) rb[q] = a.R[b * D + lane * EPL + q];
+            float p = 0.f;
+#pragma unroll
+            for (int q = 0; q < EPL; ++q) p = fmaf(rb[q], nk[q], p);
+            p = warp_sum(p);
+            bool bit = p >= 0.f;
+            if (!(fabsf(p) > gam2 * a.Rnorm[b] * nx + 1e-30f)) {   // warp-uniform
+                bit = warp_chain<EPL>(rb, nk, lane) >= 0.0;
+                ++nre;
+            }
+            code |= (uint32_t)bit << b;
+        }
+        if (lane == 0) {
+            c.knorm64[e] = n64;
+            c.kspan[e] = (uint8_t)span;
+            atomicMax(reinterpret_cast<int*>(&c.kmax2[h]), __float_as_int(ks2 * (1.f + 1.f / 1024.f)));
+            if (nre) atomicAdd(&a.stats->hash_rechecks, (unsigned long long)nre);
+            const uint32_t oc = c.code[e];
+            if (code != oc) {   // the entry leaves its bucket after this commit
+                c.code[e] = code;
+                const int slot = atomicAdd(&a.ctr[2 * c.H + 4 + h], 1);
+                s.moved[sbase + slot] = j;
+                s.movedold[sbase + slot] = oc;
+            }
+        }
+    }
     __syncwarp();
     if (lane == 0) {
         c.cnt[e] = ntot;
@@ -926,182 +1016,323 @@ __device__ void merge_long_list(const CacheView& c, const StageView& s, int h, i
     __syncwarp();
 }
 
-template <typename E, int D>
-__global__ void __launch_bounds__(kWarps * 32, 3) merge_kernel(CacheView c, StageView s, int32_t* ctr) {
-    grid_dependency_wait();
+// Four touched-list slots q4 .. q4+3 (slot q = h T + i is the i-th touched entry of
+// head h, when i < ctr[h]), one lane group each; lists longer than 8 tokens (every
+// list with running-mean keys) go to the whole warp afterwards.
+template <typename E, int D, bool MEAN>
+__device__ __forceinline__ void merge_quad(const CommitArgs<E, D, MEAN>& a, int64_t q4, int32_t* sIds,
+                                           int32_t* sSorted, int lane) {
+    const CacheView& c = a.c;
+    const StageView& s = a.s;
     using G = GSlice<E, D>;
     constexpr int EPG = G::EPG;
-    __shared__ int32_t sIds[kWarps][kListSmem];
-    __shared__ int32_t sSorted[kWarps][kListSmem];
-    const int H = c.H;
-    const bool aborted = ctr[2 * H] != 0;
-    const int lane = threadIdx.x & 31, gl = lane & 7, grp = lane >> 3, wib = threadIdx.x >> 5;
+    const int gl = lane & 7, grp = lane >> 3;
     const unsigned gmask = 0xFFu << (8 * grp);
     const int64_t T = s.T;
+    const int H = c.H;
     const E* Vs = reinterpret_cast<const E*>(s.Vs);
-    if (aborted)   // a refused commit leaves no member chains behind (matching inside the chunk)
-        for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < (int64_t)H * T;
-             q += (int64_t)gridDim.x * blockDim.x)
-            s.ichead[(q / T) * s.TmaxP + (q % T)] = -1;
-    if (!aborted && blockIdx.x == 0)
-        for (int hh = threadIdx.x; hh < H; hh += blockDim.x) c.M[hh] = ctr[H + hh];
-    const int nwin = (int)((T + 31) >> 5);
-    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < (int64_t)H * nwin;
-         q += (int64_t)gridDim.x * blockDim.x)
-        s.wcnt[(q / nwin) * (s.TmaxP >> 5) + (q % nwin)] = 0;
+    const int64_t q = q4 + grp;
+    int h = 0, j = -1;
+    bool act = false, big = false;
+    if (q < (int64_t)H * T) {
+        h = (int)((uint32_t)q / (uint32_t)T);
+        const int slot = (int)(q - (int64_t)h * T);
+        act = slot < a.ctr[h];
+        if (act) j = s.touched[(int64_t)h * s.TmaxP + slot];
+    }
+    if (act && MEAN) {
+        big = true;
+    } else if (act) {   // group-uniform
+        const int64_t sbase = (int64_t)h * s.TmaxP;
+        const int64_t e = (int64_t)h * c.capP + j;
+        const float4* v32p = reinterpret_cast<const float4*>(c.V32 + e * D + gl * EPG);
+        float4 old[EPG / 4];
+#pragma unroll
+        for (int k = 0; k < EPG / 4; ++k) old[k] = v32p[k];
+        const int nold = c.cnt[e];
+        int L = 0, id = 0x7fffffff;
+        for (int tt = c.lhead[e]; tt >= 0; tt = s.lnext[sbase + tt]) {
+            if (gl == L) id = tt;
+            if (++L > 8) break;
+        }
+        if (L > 8) {
+            big = true;
+        } else {
+            int rank = 0;
+            for (int k = 0; k < L; ++k) rank += (__shfl_sync(gmask, id, 8 * grp + k) < id);
+            int srt = 0;   // lane gl gets the gl-th smallest token
+            for (int k = 0; k < L; ++k) {
+                const int idk = __shfl_sync(gmask, id, 8 * grp + k);
+                const int rk = __shfl_sync(gmask, rank, 8 * grp + k);
+                if (rk == gl) srt = idk;
+            }
+            float acc[EPG];
+#pragma unroll
+            for (int i = 0; i < EPG; ++i) acc[i] = 0.f;
+            G cur;
+            cur.load(Vs + (sbase + __shfl_sync(gmask, srt, 8 * grp)) * D, gl);
+            for (int k = 0; k < L; ++k) {
+                G nxt;
+                const int tn = __shfl_sync(gmask, srt, 8 * grp + ((k + 1) & 7));
+                if (k + 1 < L) nxt.load(Vs + (sbase + tn) * D, gl);
+#pragma unroll
+                for (int i = 0; i < EPG; ++i) acc[i] = __fadd_rn(acc[i], cur.at(i));
+                cur = nxt;
+            }
+            const int ntot = nold + L;
+            const float fn = (float)nold, ft = (float)ntot;
+            float nv[EPG];
+#pragma unroll
+            for (int k = 0; k < EPG / 4; ++k) {
+                nv[4 * k] = __fdiv_rn(__fadd_rn(__fmul_rn(fn, old[k].x), acc[4 * k]), ft);
+                nv[4 * k + 1] = __fdiv_rn(__fadd_rn(__fmul_rn(fn, old[k].y), acc[4 * k + 1]), ft);
+                nv[4 * k + 2] = __fdiv_rn(__fadd_rn(__fmul_rn(fn, old[k].z), acc[4 * k + 2]), ft);
+                nv[4 * k + 3] = __fdiv_rn(__fadd_rn(__fmul_rn(fn, old[k].w), acc[4 * k + 3]), ft);
+            }
+            float4* v32w = reinterpret_cast<float4*>(c.V32 + e * D + gl * EPG);
+#pragma unroll
+            for (int k = 0; k < EPG / 4; ++k)
+                v32w[k] = make_float4(nv[4 * k], nv[4 * k + 1], nv[4 * k + 2], nv[4 * k + 3]);
+            G out;
+            out.from_floats(nv);
+            out.store(reinterpret_cast<E*>(c.Vc) + e * D, gl);
+            if (gl == 0) {
+                c.cnt[e] = ntot;
+                c.bias2[e] = log2f(ft);
+                c.lhead[e] = -1;
+                atomicMax(reinterpret_cast<int*>(&c.bmax[h]), __float_as_int(log2f(ft)));   // log2 n >= 0
+            }
+        }
+    }
+    __syncwarp();
+    unsigned bigm = __ballot_sync(0xffffffffu, big && gl == 0);
+    while (bigm) {
+        const int src = __ffs(bigm) - 1;
+        bigm &= bigm - 1;
+        const int bh = __shfl_sync(0xffffffffu, h, src);
+        const int bj = __shfl_sync(0xffffffffu, j, src);
+        merge_entry_warp<E, D, MEAN>(a, bh, bj, sIds, sSorted, lane);
+    }
+}
+
+// The last block of a grid to finish (every thread calls this once, after its last
+// update). With `sizes`, it publishes the new cache sizes. With `clear_lo` it clears
+// the counters [0, 2H+4) (touched lists, sizes, abort flag and tickets); with
+// `clear_moved`, the moved-entry counters [2H+4, 3H+4); its own ticket always.
+__device__ void commit_done(const CacheView& c, int32_t* ctr, int ticket, bool sizes, bool clear_lo,
+                            bool clear_moved) {
+    const int H = c.H;
+    __shared__ bool last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicAdd(&ctr[ticket], 1) == (int)gridDim.x - 1;
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    if (sizes)
+        for (int h = threadIdx.x; h < H; h += blockDim.x) c.M[h] = __ldcg(&ctr[H + h]);
+    __syncthreads();
+    if (clear_lo)
+        for (int i = threadIdx.x; i < 2 * H + 4; i += blockDim.x) ctr[i] = 0;
+    if (clear_moved)
+        for (int i = 2 * H + 4 + threadIdx.x; i < 3 * H + 4; i += blockDim.x) ctr[i] = 0;
+    if (threadIdx.x == 0) ctr[ticket] = 0;
+}
+
+template <typename E, int D, bool MEAN>
+__global__ void __launch_bounds__(kWarps * 32, 2) commit_kernel(const CommitArgs<E, D, MEAN> a) {
+    grid_dependency_wait();
+    __shared__ int sSrc[kWarps][32];
+    __shared__ int32_t sIds[kWarps][kListSmem];
+    __shared__ int32_t sSorted[kWarps][kListSmem];
+    const CacheView& c = a.c;
+    const StageView& s = a.s;
+    const int H = c.H;
+    if (__ldcg(&a.ctr[2 * H])) return;   // refused: nothing changes, the decisions stay for a retry
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const int64_t T = s.T;
+    const int64_t nA = (int64_t)H * ((T + 31) >> 5);
+    const int64_t nM = ((int64_t)H * T + 3) / 4;
     const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t q4 = gw * 4; q4 < (int64_t)H * T; q4 += nw * 4) {   // warp-uniform
-        const int64_t q = q4 + grp;
-        int h = 0, j = -1;
-        bool act = false, big = false;
-        if (q < (int64_t)H * T) {
-            h = (int)((uint32_t)q / (uint32_t)T);
-            const int slot = (int)(q - (int64_t)h * T);
-            act = slot < ctr[h];
-            if (act) j = s.touched[(int64_t)h * s.TmaxP + slot];
+    for (int64_t it = gw; it < nA + nM; it += nw) {   // warp-uniform
+        if (it < nA) {
+            const int64_t nwin = (T + 31) >> 5;
+            append_window<E, D>(c, s, (int)(it / nwin), (int)(it % nwin), sSrc[wib], lane);
+        } else {
+            merge_quad<E, D, MEAN>(a, (it - nA) * 4, sIds[wib], sSorted[wib], lane);
         }
-        if (act) {   // group-uniform
-            const int64_t sbase = (int64_t)h * s.TmaxP;
-            const int64_t e = (int64_t)h * c.capP + j;
-            if (!aborted) {
-                const float4* v32p = reinterpret_cast<const float4*>(c.V32 + e * D + gl * EPG);
-                float4 old[EPG / 4];
-#pragma unroll
-                for (int k = 0; k < EPG / 4; ++k) old[k] = v32p[k];
-                const int nold = c.cnt[e];
-                int L = 0, id = 0x7fffffff;
-                for (int tt = c.lhead[e]; tt >= 0; tt = s.lnext[sbase + tt]) {
-                    if (gl == L) id = tt;
-                    if (++L > 8) break;
-                }
-                if (L > 8) {
-                    big = true;
-                } else {
-                    int rank = 0;
-                    for (int k = 0; k < L; ++k) rank += (__shfl_sync(gmask, id, 8 * grp + k) < id);
-                    int srt = 0;   // lane gl gets the gl-th smallest token
-                    for (int k = 0; k < L; ++k) {
-                        const int idk = __shfl_sync(gmask, id, 8 * grp + k);
-                        const int rk = __shfl_sync(gmask, rank, 8 * grp + k);
-                        if (rk == gl) srt = idk;
-                    }
-                    float acc[EPG];
-#pragma unroll
-                    for (int i = 0; i < EPG; ++i) acc[i] = 0.f;
-                    G cur;
-                    cur.load(Vs + (sbase + __shfl_sync(gmask, srt, 8 * grp)) * D, gl);
-                    for (int k = 0; k < L; ++k) {
-                        G nxt;
-                        const int tn = __shfl_sync(gmask, srt, 8 * grp + ((k + 1) & 7));
-                        if (k + 1 < L) nxt.load(Vs + (sbase + tn) * D, gl);
-#pragma unroll
-                        for (int i = 0; i < EPG; ++i) acc[i] = __fadd_rn(acc[i], cur.at(i));
-                        cur = nxt;
-                    }
-                    const int ntot = nold + L;
-                    const float fn = (float)nold, ft = (float)ntot;
-                    float nv[EPG];
-#pragma unroll
-                    for (int k = 0; k < EPG / 4; ++k) {
-                        nv[4 * k] = __fdiv_rn(__fadd_rn(__fmul_rn(fn, old[k].x), acc[4 * k]), ft);
-                        nv[4 * k + 1] = __fdiv_rn(__fadd_rn(__fmul_rn(fn, old[k].y), acc[4 * k + 1]), ft);
-                        nv[4 * k + 2] = __fdiv_rn(__fadd_rn(__fmul_rn(fn, old[k].z), acc[4 * k + 2]), ft);
-                        nv[4 * k + 3] = __fdiv_rn(__fadd_rn(__fmul_rn(fn, old[k].w), acc[4 * k + 3]), ft);
-                    }
-                    float4* v32w = reinterpret_cast<float4*>(c.V32 + e * D + gl * EPG);
-#pragma unroll
-                    for (int k = 0; k < EPG / 4; ++k)
-                        v32w[k] = make_float4(nv[4 * k], nv[4 * k + 1], nv[4 * k + 2], nv[4 * k + 3]);
-                    G out;
-                    out.from_floats(nv);
-                    out.store(reinterpret_cast<E*>(c.Vc) + e * D, gl);
-                    if (gl == 0) {
-                        c.cnt[e] = ntot;
-                        c.bias2[e] = log2f(ft);
-                        atomicMax(reinterpret_cast<int*>(&c.bmax[h]), __float_as_int(log2f(ft)));   // log2 n >= 0
-                    }
-                }
+    }
+    grid_dependents_launch();
+    commit_done(c, a.ctr, 2 * H + 2, true, true, !MEAN);
+}
+
+// ------------------------------------------------------------------ re-bucketing (running-mean keys)
+//
+// An entry whose merged key changed code leaves its old bucket and joins the new one.
+// Unlink: for every moved entry, the first thread to claim the old bucket rebuilds that
+// bucket's list without the entries whose code is no longer the bucket's (so one thread
+// owns each list). Push: every moved entry is pushed on its new bucket's list and the
+// claims are released; the last block clears the moved-entry counters.
+__global__ void rebucket_unlink_kernel(CacheView c, StageView s, const int32_t* ctr, int32_t* claim, Stats* stats) {
+    grid_dependency_wait();
+    const int H = c.H;
+    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < (int64_t)H * s.TmaxP;
+         q += (int64_t)gridDim.x * blockDim.x) {
+        const int h = (int)(q / s.TmaxP);
+        const int idx = (int)(q - (int64_t)h * s.TmaxP);
+        if (idx >= __ldcg(&ctr[2 * H + 4 + h])) continue;
+        const uint32_t oc = s.movedold[q];
+        const int64_t b = ((int64_t)h << c.nbits) + oc;
+        if (atomicExch(&claim[b], 1) != 0) continue;
+        const int64_t hrow = (int64_t)h * c.capP;
+        const int Mh = c.M[h];
+        int head = -1, tail = -1, guard = 0;
+        for (int e = c.bhead[b]; e >= 0;) {
+            const int nx = c.bnext[hrow + e];
+            if (c.code[hrow + e] == oc) {
+                if (tail < 0) head = e;
+                else c.bnext[hrow + tail] = e;
+                tail = e;
             }
-            __syncwarp(gmask);
-            if (!big && gl == 0) c.lhead[e] = -1;
+            if (++guard > Mh) {
+                atomicOr(&stats->error_bits, kErrBucketList);
+                break;
+            }
+            e = nx;
         }
-        // lists longer than 8 tokens: the whole warp, one list at a time
-        unsigned bigm = __ballot_sync(0xffffffffu, big && gl == 0);
-        while (bigm) {
-            const int src = __ffs(bigm) - 1;
-            bigm &= bigm - 1;
-            const int bh = __shfl_sync(0xffffffffu, h, src);
-            const int bj = __shfl_sync(0xffffffffu, j, src);
-            merge_long_list<E, D>(c, s, bh, bj, sIds[wib], sSorted[wib], lane);
-        }
+        if (tail >= 0) c.bnext[hrow + tail] = -1;
+        c.bhead[b] = head;
     }
     grid_dependents_launch();
 }
 
-template <typename E, int D, int NBP>
-cudaError_t stage_hash_n(const CacheView& c, const StageView& s, const void* K, const void* V, const float* R,
-                         const float* Rnorm, int32_t* ctr, Stats* stats, cudaStream_t st) {
-    const int64_t rows = s.T * c.H;
-    const int grid = grid_for_rows(rows > s.TmaxP ? rows : s.TmaxP, 4 * kWarps, 148 * 8);
-    return launch_pdl(stage_hash_kernel<E, D, NBP>, grid, kWarps * 32, st, reinterpret_cast<const E*>(K),
-                      reinterpret_cast<const E*>(V), c, s, R, Rnorm, ctr, stats);
-}
-
-template <typename E, int D>
-cudaError_t stage_hash_t(const CacheView& c, const StageView& s, const void* K, const void* V,
-                         const float* R, const float* Rnorm, int32_t* ctr, Stats* stats, cudaStream_t st) {
-    if (c.nbits <= 8) return stage_hash_n<E, D, 8>(c, s, K, V, R, Rnorm, ctr, stats, st);
-    if (c.nbits <= 16) return stage_hash_n<E, D, 16>(c, s, K, V, R, Rnorm, ctr, stats, st);
-    return stage_hash_n<E, D, 32>(c, s, K, V, R, Rnorm, ctr, stats, st);
-}
-
-// The counters start at zero: the staging kernel of the chunk cleared them.
-template <typename E, int D>
-cudaError_t commit_t(const CacheView& c, const StageView& s, float tau, bool intra, int32_t* ctr, Stats* stats,
-                     int* launches, cudaStream_t st) {
+__global__ void rebucket_push_kernel(CacheView c, StageView s, int32_t* ctr, int32_t* claim) {
+    grid_dependency_wait();
     const int H = c.H;
-    const int64_t rows = s.T * H;
-    // delta bounds |sim32 - sim| (see the search kernel): 2 x (2 (d+2) u + 3 u).
-    const float delta = 2.f * (2.f * (float)(D + 2) * kU32 + 3.f * kU32);
-    const int sgrid = grid_for_rows(rows, 4 * kWarps, 148 * 2);
-    cudaError_t e = launch_pdl(search_kernel<E, D>, sgrid, kWarps * 32, st, c, s, tau, (double)tau, delta, intra,
-                               ctr, stats);
-    if (e == cudaSuccess && intra) {
-        e = launch_pdl(dedupe_kernel<E, D>, sgrid, kWarps * 32, st, c, s, (double)tau, ctr, stats);
+    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < (int64_t)H * s.TmaxP;
+         q += (int64_t)gridDim.x * blockDim.x) {
+        const int h = (int)(q / s.TmaxP);
+        const int idx = (int)(q - (int64_t)h * s.TmaxP);
+        if (idx >= __ldcg(&ctr[2 * H + 4 + h])) continue;
+        const int j = s.moved[q];
+        const int64_t e = (int64_t)h * c.capP + j;
+        c.bnext[e] = atomicExch(&c.bhead[((int64_t)h << c.nbits) + c.code[e]], j);
+        claim[((int64_t)h << c.nbits) + s.movedold[q]] = 0;
+    }
+    grid_dependents_launch();
+    commit_done(c, ctr, 2 * H + 3, false, false, true);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl_smem(void (*kern)(KArgs...), int grid, int block, int smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)block);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+template <typename E, int D, int NBP, bool INTRA, bool MEAN>
+cudaError_t stage_n(const CacheView& c, const StageView& s, const void* K, const void* V, const float* R,
+                    const float* Rhost, const float* Rnorm_host, float tau, int32_t* ctr, Stats* stats,
+                    int* launches, cudaStream_t st) {
+    auto kern = stage_search_kernel<E, D, NBP, INTRA, MEAN>;
+    constexpr int smem = StageSmem<E, D>::BYTES;
+    cudaError_t e = smem_attr_once(reinterpret_cast<const void*>(kern), smem);
+    if (e != cudaSuccess) return e;
+    StagePlanes<D, NBP> pl;
+    for (int b = 0; b < NBP; ++b) {
+        for (int i = 0; i < D; ++i) pl.v[b * D + i] = b < c.nbits ? Rhost[b * D + i] : 0.f;
+        pl.rn[b] = b < c.nbits ? Rnorm_host[b] : 0.f;
+    }
+    const int64_t items = (int64_t)c.H * ((s.T + 31) / 32);
+    const int grid = grid_for_rows(items > s.TmaxP / kWarps ? items : s.TmaxP / kWarps, kWarps, 148 * 2);
+    e = launch_pdl_smem(kern, grid, kWarps * 32, smem, st, reinterpret_cast<const E*>(K),
+                        reinterpret_cast<const E*>(V), c, s, R, pl, (double)tau, ctr, stats);
+    *launches += 1;
+    if (e == cudaSuccess && INTRA) {
+        const int dgrid = grid_for_rows(s.T * c.H, 4 * kWarps, 148 * 2);
+        e = launch_pdl(dedupe_kernel<E, D>, dgrid, kWarps * 32, st, c, s, (double)tau, ctr, stats);
         *launches += 1;
     }
-    const int64_t wins = (int64_t)H * ((s.T + 31) / 32);
-    if (e == cudaSuccess)
-        e = launch_pdl(append_kernel<E, D>, grid_for_rows(wins, kWarps, 148 * 16), kWarps * 32, st, c, s,
-                       (const int32_t*)ctr);
-    if (e == cudaSuccess)
-        e = launch_pdl(merge_kernel<E, D>, grid_for_rows(rows, kWarps, 148 * 8), kWarps * 32, st, c, s, ctr);
-    *launches += 3;
+    return e;
+}
+
+template <typename E, int D, bool INTRA, bool MEAN>
+cudaError_t stage_t(const CacheView& c, const StageView& s, const void* K, const void* V, const float* R,
+                    const float* Rhost, const float* Rnorm_host, float tau, int32_t* ctr, Stats* stats,
+                    int* launches, cudaStream_t st) {
+    if (c.nbits <= 8)
+        return stage_n<E, D, 8, INTRA, MEAN>(c, s, K, V, R, Rhost, Rnorm_host, tau, ctr, stats, launches, st);
+    if (c.nbits <= 16)
+        return stage_n<E, D, 16, INTRA, MEAN>(c, s, K, V, R, Rhost, Rnorm_host, tau, ctr, stats, launches, st);
+    return stage_n<E, D, 32, INTRA, MEAN>(c, s, K, V, R, Rhost, Rnorm_host, tau, ctr, stats, launches, st);
+}
+
+template <typename E, int D>
+cudaError_t stage_mode(const CacheView& c, const StageView& s, bool intra, bool mean, const void* K, const void* V,
+                       const float* R, const float* Rhost, const float* Rnorm_host, float tau, int32_t* ctr,
+                       Stats* stats, int* launches, cudaStream_t st) {
+    if (intra) return stage_t<E, D, true, false>(c, s, K, V, R, Rhost, Rnorm_host, tau, ctr, stats, launches, st);
+    if (mean) return stage_t<E, D, false, true>(c, s, K, V, R, Rhost, Rnorm_host, tau, ctr, stats, launches, st);
+    return stage_t<E, D, false, false>(c, s, K, V, R, Rhost, Rnorm_host, tau, ctr, stats, launches, st);
+}
+
+template <typename E, int D, bool MEAN>
+cudaError_t commit_t(const CacheView& c, const StageView& s, const float* R, const float* Rnorm, int32_t* ctr,
+                     int32_t* claim, Stats* stats, int* launches, cudaStream_t st) {
+    const int64_t items = (int64_t)c.H * ((s.T + 31) / 32) + ((int64_t)c.H * s.T + 3) / 4;
+    const int grid = grid_for_rows(items, kWarps, 148 * 2);
+    CommitArgs<E, D, MEAN> a{c, s, R, Rnorm, ctr, stats};
+    cudaError_t e = launch_pdl(commit_kernel<E, D, MEAN>, grid, kWarps * 32, st, a);
+    *launches += 1;
+    if (MEAN && e == cudaSuccess) {
+        const int rgrid = grid_for_rows((int64_t)c.H * s.TmaxP, 256, 148 * 2);
+        e = launch_pdl(rebucket_unlink_kernel, rgrid, 256, st, c, s, (const int32_t*)ctr, claim, stats);
+        if (e == cudaSuccess) e = launch_pdl(rebucket_push_kernel, rgrid, 256, st, c, s, ctr, claim);
+        *launches += 2;
+    }
     return e;
 }
 
 }  // namespace
 
-cudaError_t launch_stage_hash(const CacheView& c, const StageView& s, int dtype, const void* K,
-                              const void* V, const float* R, const float* Rnorm, int32_t* ctr, Stats* stats,
-                              cudaStream_t st) {
-    if (dtype == 0) {
-        return c.d == 128 ? stage_hash_t<__nv_bfloat16, 128>(c, s, K, V, R, Rnorm, ctr, stats, st)
-                          : stage_hash_t<__nv_bfloat16, 64>(c, s, K, V, R, Rnorm, ctr, stats, st);
-    }
-    return c.d == 128 ? stage_hash_t<float, 128>(c, s, K, V, R, Rnorm, ctr, stats, st)
-                      : stage_hash_t<float, 64>(c, s, K, V, R, Rnorm, ctr, stats, st);
+cudaError_t launch_stage(const CacheView& c, const StageView& s, int dtype, bool intra, bool mean, const void* K,
+                         const void* V, const float* R, const float* Rhost, const float* Rnorm_host, float tau,
+                         int32_t* ctr, Stats* stats, int* launches, cudaStream_t st) {
+    if (dtype == 0)
+        return c.d == 128 ? stage_mode<__nv_bfloat16, 128>(c, s, intra, mean, K, V, R, Rhost, Rnorm_host, tau, ctr,
+                                                           stats, launches, st)
+                          : stage_mode<__nv_bfloat16, 64>(c, s, intra, mean, K, V, R, Rhost, Rnorm_host, tau, ctr,
+                                                          stats, launches, st);
+    return c.d == 128 ? stage_mode<float, 128>(c, s, intra, mean, K, V, R, Rhost, Rnorm_host, tau, ctr, stats,
+                                               launches, st)
+                      : stage_mode<float, 64>(c, s, intra, mean, K, V, R, Rhost, Rnorm_host, tau, ctr, stats,
+                                              launches, st);
 }
 
-cudaError_t launch_commit(const CacheView& c, const StageView& s, int dtype, float tau, bool intra, int32_t* ctr,
-                          Stats* stats, int* launches, cudaStream_t st) {
+cudaError_t launch_commit(const CacheView& c, const StageView& s, int dtype, bool mean, const float* R,
+                          const float* Rnorm, int32_t* ctr, int32_t* claim, Stats* stats, int* launches,
+                          cudaStream_t st) {
     if (dtype == 0) {
-        return c.d == 128 ? commit_t<__nv_bfloat16, 128>(c, s, tau, intra, ctr, stats, launches, st)
-                          : commit_t<__nv_bfloat16, 64>(c, s, tau, intra, ctr, stats, launches, st);
+        if (c.d == 128)
+            return mean ? commit_t<__nv_bfloat16, 128, true>(c, s, R, Rnorm, ctr, claim, stats, launches, st)
+                        : commit_t<__nv_bfloat16, 128, false>(c, s, R, Rnorm, ctr, claim, stats, launches, st);
+        return mean ? commit_t<__nv_bfloat16, 64, true>(c, s, R, Rnorm, ctr, claim, stats, launches, st)
+                    : commit_t<__nv_bfloat16, 64, false>(c, s, R, Rnorm, ctr, claim, stats, launches, st);
     }
-    return c.d == 128 ? commit_t<float, 128>(c, s, tau, intra, ctr, stats, launches, st)
-                      : commit_t<float, 64>(c, s, tau, intra, ctr, stats, launches, st);
+    if (c.d == 128)
+        return mean ? commit_t<float, 128, true>(c, s, R, Rnorm, ctr, claim, stats, launches, st)
+                    : commit_t<float, 128, false>(c, s, R, Rnorm, ctr, claim, stats, launches, st);
+    return mean ? commit_t<float, 64, true>(c, s, R, Rnorm, ctr, claim, stats, launches, st)
+                : commit_t<float, 64, false>(c, s, R, Rnorm, ctr, claim, stats, launches, st);
 }
 
 }  // namespace tc

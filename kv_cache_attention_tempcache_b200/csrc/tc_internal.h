@@ -19,7 +19,9 @@ struct CacheView {
     int H, d, nbits;
     int64_t capP;          // padded capacity per head
     int64_t capacity;      // usable entries per head
-    void* Kc;              // [H][capP][d] storage type, representative keys
+    void* Kc;              // [H][capP][d] storage type, entry keys (the attention operand)
+    float* K32;            // [H][capP][d] fp32 key means with running-mean keys (bf16 storage; the
+                           // same array as Kc with fp32 storage); null with representative keys
     void* Vc;              // [H][capP][d] storage type, value means (attention operand)
     float* V32;            // [H][capP][d] fp32 value means (master copy)
     int32_t* cnt;          // [H][capP] group sizes n
@@ -47,10 +49,10 @@ struct StageView {
     void* Ks;              // [H][TmaxP][d]
     void* Vs;              // [H][TmaxP][d]
     uint32_t* scode;       // [H][TmaxP] hash codes of the staged tokens
-    int32_t* sfirst;       // [H][TmaxP] newest committed entry of the token's bucket (-1 = empty), read at
-                           // staging; the cache cannot change between staging and commit
     float* sbias;          // [TmaxP] 0 for t < T, -inf beyond
-    int32_t* match;        // [H][TmaxP] merge target or -1 (last commit)
+    int32_t* match;        // [H][TmaxP] merge target or -1 of each staged token, decided at staging
+                           // (the cache cannot change between staging and commit)
+    int32_t* lmatch;       // [H][TmaxP] merge targets of the last committed chunk
     int32_t* dest;         // [H][TmaxP] entry each token ended in (last commit)
     uint32_t* lcode;       // [H][TmaxP] codes of the last committed chunk
     int32_t* lnext;        // [H][TmaxP] next (older) token of the same merge list
@@ -63,15 +65,21 @@ struct StageView {
     int32_t* ichead;       // [H][TmaxP] first token merging into the entry this token created (-1: none)
     int32_t* ictail;       // [H][TmaxP] last such token
     int32_t* icnext;       // [H][TmaxP] next token merging into the same new entry
+    // running-mean keys: entries whose merged key changed code in the last commit
+    int32_t* moved;        // [H][TmaxP] entry
+    uint32_t* movedold;    // [H][TmaxP] its code before the commit
 };
 
-// Per-commit counters (int32; zeroed by the staging kernel of the chunk a commit
-// commits, and by the host after a refused commit):
-//   ctr[0, H)   entries touched by merges, per head
-//   ctr[H, 2H)  cache size after the commit, per head
-//   ctr[2H]     abort flag: some head would exceed its capacity
-//   ctr[2H+1]   blocks of the search kernel that have finished
-__host__ __device__ constexpr int kCtrInts(int H) { return 2 * H + 2; }
+// Per-commit counters (int32). The staging kernels of a chunk fill them and the last
+// kernel of that chunk's commit clears them (the host clears them on a reset):
+//   ctr[0, H)        entries touched by merges, per head
+//   ctr[H, 2H)       cache size after the commit, per head
+//   ctr[2H]          abort flag: some head would exceed its capacity
+//   ctr[2H+1]        ticket of the staging kernel that publishes the sizes
+//   ctr[2H+2]        ticket of the commit kernel
+//   ctr[2H+3]        ticket of the last re-bucketing kernel (running-mean keys)
+//   ctr[2H+4, 3H+4)  entries whose key changed code, per head (running-mean keys)
+__host__ __device__ constexpr int kCtrInts(int H) { return 3 * H + 4; }
 
 // Sticky device-side statistics and error bits.
 enum : unsigned { kErrBucketList = 1u, kErrTimeout = 2u };
@@ -82,12 +90,16 @@ struct Stats {
     unsigned int pad;
 };
 
-// Launchers (tc_commit.cu).
-cudaError_t launch_stage_hash(const CacheView& c, const StageView& s, int dtype,
-                              const void* K, const void* V, const float* R, const float* Rnorm,
-                              int32_t* ctr, Stats* stats, cudaStream_t st);
-cudaError_t launch_commit(const CacheView& c, const StageView& s, int dtype, float tau, bool intra_chunk,
-                          int32_t* ctr, Stats* stats, int* launches, cudaStream_t st);
+// Launchers (tc_commit.cu). launch_stage copies, hashes and searches the chunk s.T
+// (plus the in-chunk dedupe when intra); launch_commit applies the staged chunk's
+// decisions (plus the re-bucketing with running-mean keys). R: device normals;
+// Rhost, Rnorm_host: host copies of the normals and of |R_b| (rounded up).
+cudaError_t launch_stage(const CacheView& c, const StageView& s, int dtype, bool intra, bool mean, const void* K,
+                         const void* V, const float* R, const float* Rhost, const float* Rnorm_host, float tau,
+                         int32_t* ctr, Stats* stats, int* launches, cudaStream_t st);
+cudaError_t launch_commit(const CacheView& c, const StageView& s, int dtype, bool mean, const float* R,
+                          const float* Rnorm, int32_t* ctr, int32_t* claim, Stats* stats, int* launches,
+                          cudaStream_t st);
 
 // Launchers (tc_attn_f32.cu, tc_attn_bf16.cu).
 cudaError_t launch_attend_f32(const CacheView& c, const StageView& s, const float* Q,

@@ -120,6 +120,8 @@ struct tc_ctx {
     float tau = 0.f, scale = 0.f;
     tc_dtype dtype = TC_BF16;
     bool intra = false;            // commits also match inside the chunk
+    bool mean = false;             // entry keys are running means of their members' keys
+    int32_t* claim = nullptr;      // [H << nbits] bucket claims of the re-bucketing (running-mean keys)
     int64_t capacity = 0, capP = 0;
     int device = 0;
     CacheView c{};
@@ -129,6 +131,7 @@ struct tc_ctx {
     float* R = nullptr;
     float* Rnorm = nullptr;
     std::vector<float> Rhost;
+    std::vector<float> Rnorm_host; // |R_b| rounded up
     std::vector<int64_t> m_upper;  // per-head upper bound of the committed size
     int64_t T_staged = 0, last_commit_T = 0;
     bool appended = false;
@@ -155,8 +158,9 @@ struct tc_ctx {
         return TC_OK;
     }
     void free_staging() {
-        void* ptrs[] = {s.Ks,    s.Vs,     s.scode,  s.sfirst, s.sbias,  s.match,  s.dest,   s.lcode,
-                        s.lnext, s.wcnt,   s.touched, s.bsim,  s.cbnext, s.crnext, s.ichead, s.ictail, s.icnext};
+        void* ptrs[] = {s.Ks,     s.Vs,     s.scode,  s.sbias,  s.match,  s.lmatch, s.dest,  s.lcode,
+                        s.lnext,  s.wcnt,   s.touched, s.bsim,  s.cbnext, s.crnext, s.ichead, s.ictail,
+                        s.icnext, s.moved,  s.movedold};
         for (void* p : ptrs) {
             if (!p) continue;
             owned.erase(std::remove(owned.begin(), owned.end(), p), owned.end());
@@ -207,13 +211,15 @@ tc_status ensure_staging(tc_ctx* x, int64_t T) {
     tc_ctx& c = *x;
     tc_status st = TC_OK;
     if ((st = c.alloc(&c.s.Ks, rowsH * x->d * x->esize)) || (st = c.alloc(&c.s.Vs, rowsH * x->d * x->esize)) ||
-        (st = c.alloc((void**)&c.s.scode, rowsH * 4)) || (st = c.alloc((void**)&c.s.sfirst, rowsH * 4)) || (st = c.alloc((void**)&c.s.sbias, P * 4)) ||
-        (st = c.alloc((void**)&c.s.match, rowsH * 4)) || (st = c.alloc((void**)&c.s.dest, rowsH * 4)) ||
+        (st = c.alloc((void**)&c.s.scode, rowsH * 4)) || (st = c.alloc((void**)&c.s.sbias, P * 4)) ||
+        (st = c.alloc((void**)&c.s.match, rowsH * 4)) || (st = c.alloc((void**)&c.s.lmatch, rowsH * 4)) ||
+        (st = c.alloc((void**)&c.s.dest, rowsH * 4)) ||
         (st = c.alloc((void**)&c.s.lcode, rowsH * 4)) || (st = c.alloc((void**)&c.s.lnext, rowsH * 4)) ||
         (st = c.alloc((void**)&c.s.wcnt, rowsH / 32 * 4)) || (st = c.alloc((void**)&c.s.touched, rowsH * 4)) ||
         (st = c.alloc((void**)&c.s.bsim, rowsH * 8)) || (st = c.alloc((void**)&c.s.cbnext, rowsH * 4)) ||
         (st = c.alloc((void**)&c.s.crnext, rowsH * 4)) || (st = c.alloc((void**)&c.s.ichead, rowsH * 4)) ||
-        (st = c.alloc((void**)&c.s.ictail, rowsH * 4)) || (st = c.alloc((void**)&c.s.icnext, rowsH * 4))) {
+        (st = c.alloc((void**)&c.s.ictail, rowsH * 4)) || (st = c.alloc((void**)&c.s.icnext, rowsH * 4)) ||
+        (x->mean && ((st = c.alloc((void**)&c.s.moved, rowsH * 4)) || (st = c.alloc((void**)&c.s.movedold, rowsH * 4))))) {
         x->free_staging();
         return st;
     }
@@ -241,34 +247,30 @@ tc_status encode_stage_maps(tc_ctx* x) {
     return TC_OK;
 }
 
-// Commit the staged chunk. May synchronise (see tc_append_chunk).
+// Commit the staged chunk: apply the decisions its staging took. When the worst case
+// could overflow the capacity, first synchronise and read the staging's verdict; a
+// refused commit launches nothing and leaves the chunk staged with its decisions.
 tc_status commit_staged(tc_ctx* x, cudaStream_t st) {
     if (x->T_staged == 0) return TC_OK;
-    StageView s = x->s;
-    s.T = x->T_staged;
-    int launches = 0;
-    cudaError_t e = launch_commit(x->c, s, (int)x->dtype, x->tau, x->intra, x->ctr, x->stats, &launches, st);
-    x->launches += launches;
-    if (e != cudaSuccess) return cuda_status(e);
     int64_t worst = 0;
     for (int64_t m : x->m_upper) worst = std::max(worst, m);
     if (worst + x->T_staged > x->capacity) {
-        // The commit might overflow: learn the outcome now.
         if (cudaStreamSynchronize(st) != cudaSuccess) return cuda_status(cudaGetLastError());
         std::vector<int32_t> ctr(kCtrInts(x->H));
-        std::vector<int32_t> M(x->H);
-        if (cudaMemcpy(ctr.data(), x->ctr, ctr.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess ||
-            cudaMemcpy(M.data(), x->c.M, M.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+        if (cudaMemcpy(ctr.data(), x->ctr, ctr.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
             return cuda_status(cudaGetLastError());
-        for (int h = 0; h < x->H; ++h) x->m_upper[h] = M[h];
-        if (ctr[2 * x->H]) {
-            // Nothing changed and the chunk stays staged; clear the counters for a retry.
-            if (cudaMemset(x->ctr, 0, ctr.size() * 4) != cudaSuccess) return cuda_status(cudaGetLastError());
-            return TC_ECAPACITY;
-        }
+        if (ctr[2 * x->H]) return TC_ECAPACITY;
+        for (int h = 0; h < x->H; ++h) x->m_upper[h] = ctr[x->H + h];
     } else {
         for (auto& m : x->m_upper) m += x->T_staged;
     }
+    StageView s = x->s;
+    s.T = x->T_staged;
+    int launches = 0;
+    cudaError_t e = launch_commit(x->c, s, (int)x->dtype, x->mean, x->R, x->Rnorm, x->ctr, x->claim, x->stats,
+                                  &launches, st);
+    x->launches += launches;
+    if (e != cudaSuccess) return cuda_status(e);
     x->last_commit_T = x->T_staged;
     x->T_staged = 0;
     return TC_OK;
@@ -308,11 +310,12 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
                        tc_handle* out) {
     if (!out) return TC_EINVAL;
     *out = nullptr;
-    tc_options o{TC_BF16, 0, 0.f, nullptr, 0};
+    tc_options o{TC_BF16, 0, 0.f, nullptr, 0, 0};
     if (opt) o = *opt;
     if (H < 1 || H > 4096 || (d != 64 && d != 128) || nbits < 1 || nbits > 24 || !(tau >= -1.f && tau <= 2.f) ||
         capacity < 1 || capacity > (int64_t)1 << 30 || (o.dtype != TC_BF16 && o.dtype != TC_F32) ||
-        !(o.softmax_scale >= 0.f) || !std::isfinite(o.softmax_scale) || (o.intra_chunk != 0 && o.intra_chunk != 1))
+        !(o.softmax_scale >= 0.f) || !std::isfinite(o.softmax_scale) || (o.intra_chunk != 0 && o.intra_chunk != 1) ||
+        (o.key_mode != 0 && o.key_mode != 1) || (o.key_mode == 1 && o.intra_chunk == 1))
         return TC_EINVAL;
     if (o.hyperplanes) {
         for (int i = 0; i < nbits * d; ++i)
@@ -339,6 +342,7 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
     x->tau = tau;
     x->dtype = o.dtype;
     x->intra = o.intra_chunk != 0;
+    x->mean = o.key_mode == 1;
     x->esize = (o.dtype == TC_BF16) ? 2 : 4;
     x->capacity = capacity;
     x->capP = round_up(capacity, 128);
@@ -352,7 +356,9 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
 
     // Memory budget: refuse early instead of failing halfway.
     const size_t rows = (size_t)H * x->capP;
-    const size_t need = rows * d * (2 * x->esize + 4) + rows * (4 * 7 + 1) + ((size_t)H << nbits) * 4;
+    const bool k32 = x->mean && o.dtype == TC_BF16;   // fp32 key means beside the bf16 keys
+    const size_t need = rows * d * (2 * x->esize + 4 + (k32 ? 4 : 0)) + rows * (4 * 7 + 1) +
+                        ((size_t)H << nbits) * 4 * (x->mean ? 2 : 1);
     size_t fr = 0, tot = 0;
     if (cudaMemGetInfo(&fr, &tot) != cudaSuccess) {
         cudaGetLastError();
@@ -378,6 +384,8 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
         (st = x->alloc((void**)&c.M, (size_t)H * 4)) || (st = x->alloc((void**)&c.kmax2, (size_t)H * 4)) ||
         (st = x->alloc((void**)&c.kmax2s, 4)) || (st = x->alloc((void**)&c.bmax, (size_t)H * 4)) ||
         (x->intra && (st = x->alloc((void**)&c.cbhead, ((size_t)H << nbits) * 4))) ||
+        (k32 && (st = x->alloc((void**)&c.K32, rows * d * 4))) ||
+        (x->mean && (st = x->alloc((void**)&x->claim, ((size_t)H << nbits) * 4))) ||
         (st = x->alloc((void**)&x->ctr, (size_t)kCtrInts(H) * 4)) ||
         (st = x->alloc((void**)&x->stats, sizeof(Stats))) ||
         (st = x->alloc((void**)&x->R, (size_t)nbits * d * 4)) || (st = x->alloc((void**)&x->Rnorm, nbits * 4))) {
@@ -386,6 +394,7 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
     }
     // Rows past the committed entries stay zero (finite attention operands) with
     // log2 n = -inf (masked); empty buckets hold -1.
+    if (x->mean && !k32) c.K32 = static_cast<float*>(c.Kc);   // fp32 storage: the keys are the means
     std::vector<float> rnorm(nbits);
     for (int b = 0; b < nbits; ++b) {
         double s2 = 0.0;
@@ -401,12 +410,15 @@ tc_status tc_create_ex(int32_t H, int32_t d, int32_t nbits, float tau, int64_t c
         (e = cudaMemset(c.M, 0, (size_t)H * 4)) || (e = cudaMemset(c.kmax2, 0, (size_t)H * 4)) ||
         (e = cudaMemset(c.kmax2s, 0, 4)) || (e = cudaMemset(c.bmax, 0, (size_t)H * 4)) ||
         (x->intra && (e = cudaMemset(c.cbhead, 0xff, ((size_t)H << nbits) * 4))) || (e = cudaMemset(x->ctr, 0, (size_t)kCtrInts(H) * 4)) ||
+        (k32 && (e = cudaMemset(c.K32, 0, rows * d * 4))) ||
+        (x->mean && (e = cudaMemset(x->claim, 0, ((size_t)H << nbits) * 4))) ||
         (e = cudaMemset(x->stats, 0, sizeof(Stats))) ||
         (e = cudaMemcpy(x->R, x->Rhost.data(), (size_t)nbits * d * 4, cudaMemcpyHostToDevice)) ||
         (e = cudaMemcpy(x->Rnorm, rnorm.data(), nbits * 4, cudaMemcpyHostToDevice))) {
         delete x;
         return cuda_status(e);
     }
+    x->Rnorm_host = rnorm;
     fill_f32<<<1024, 256>>>(c.bias2, (int64_t)rows, 1, 0, -INFINITY);
     if ((e = cudaDeviceSynchronize()) != cudaSuccess) {
         delete x;
@@ -440,9 +452,11 @@ tc_status tc_append_chunk(tc_handle x, const void* K, const void* V, int64_t T, 
     x->s.T = T;
     if ((st = encode_stage_maps(x))) return st;
     cudaError_t e = cudaMemsetAsync(x->c.kmax2s, 0, 4, cs);   // the staged keys' bound starts over
+    int launches = 0;
     if (e == cudaSuccess)
-        e = launch_stage_hash(x->c, x->s, (int)x->dtype, K, V, x->R, x->Rnorm, x->ctr, x->stats, cs);
-    x->launches += 1;
+        e = launch_stage(x->c, x->s, (int)x->dtype, x->intra, x->mean, K, V, x->R, x->Rhost.data(),
+                         x->Rnorm_host.data(), x->tau, x->ctr, x->stats, &launches, cs);
+    x->launches += launches;
     if (e != cudaSuccess) return cuda_status(e);
     x->T_staged = T;
     x->appended = true;
@@ -512,6 +526,14 @@ tc_status tc_reset(tc_handle x, tc_stream stream) {
     upto = std::min(round_up(upto, 128), x->capP);
     cudaError_t e = cudaMemsetAsync(x->c.bhead, 0xff, ((size_t)x->H << x->nbits) * 4, cs);
     if (e == cudaSuccess) e = cudaMemsetAsync(x->c.M, 0, (size_t)x->H * 4, cs);
+    if (e == cudaSuccess) e = cudaMemsetAsync(x->ctr, 0, (size_t)kCtrInts(x->H) * 4, cs);
+    if (e == cudaSuccess && x->T_staged > 0) {
+        // a staged chunk's decisions are dropped: its merge lists on committed entries,
+        // in-chunk member chains and bucket groups
+        e = cudaMemsetAsync(x->c.lhead, 0xff, (size_t)x->H * x->capP * 4, cs);
+        if (e == cudaSuccess) e = cudaMemsetAsync(x->s.ichead, 0xff, (size_t)x->H * x->s.TmaxP * 4, cs);
+        if (e == cudaSuccess && x->intra) e = cudaMemsetAsync(x->c.cbhead, 0xff, ((size_t)x->H << x->nbits) * 4, cs);
+    }
     if (e == cudaSuccess) e = cudaMemsetAsync(x->c.kmax2, 0, (size_t)x->H * 4, cs);
     if (e == cudaSuccess) e = cudaMemsetAsync(x->c.bmax, 0, (size_t)x->H * 4, cs);
     if (e == cudaSuccess && upto > 0) {
@@ -571,7 +593,7 @@ tc_status tc_debug_last_commit(tc_handle x, int64_t* T_out, uint32_t* codes_HT, 
         cudaError_t e = cudaSuccess;
         if (codes_HT && (e = cudaMemcpy(codes_HT + h * T, x->s.lcode + off, T * 4, cudaMemcpyDeviceToHost)))
             return cuda_status(e);
-        if (match_HT && (e = cudaMemcpy(match_HT + h * T, x->s.match + off, T * 4, cudaMemcpyDeviceToHost)))
+        if (match_HT && (e = cudaMemcpy(match_HT + h * T, x->s.lmatch + off, T * 4, cudaMemcpyDeviceToHost)))
             return cuda_status(e);
         if (dest_HT && (e = cudaMemcpy(dest_HT + h * T, x->s.dest + off, T * 4, cudaMemcpyDeviceToHost)))
             return cuda_status(e);
@@ -610,6 +632,20 @@ tc_status tc_export_cache(tc_handle x, int32_t head, void* K, float* V32, int32_
     if (n && (e = cudaMemcpy(n, x->c.cnt + row, (size_t)M * 4, cudaMemcpyDeviceToHost))) return cuda_status(e);
     if (code && (e = cudaMemcpy(code, x->c.code + row, (size_t)M * 4, cudaMemcpyDeviceToHost)))
         return cuda_status(e);
+    return TC_OK;
+}
+
+tc_status tc_export_key_means(tc_handle x, int32_t head, float* K32) {
+    tc_status st = tc_sync(x);
+    if (st) return st;
+    if (head < 0 || head >= x->H || !K32) return TC_EINVAL;
+    if (!x->mean) return TC_ESTATE;
+    int32_t M = 0;
+    if (cudaMemcpy(&M, x->c.M + head, 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return cuda_status(cudaGetLastError());
+    const size_t row = (size_t)head * x->capP;
+    if (cudaMemcpy(K32, x->c.K32 + row * x->d, (size_t)M * x->d * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return cuda_status(cudaGetLastError());
     return TC_OK;
 }
 

@@ -34,6 +34,7 @@ class ParityReport:
     attn_checks: int = 0
     merges: int = 0
     sizes: list = field(default_factory=list)
+    records: list = field(default_factory=list)   # the oracle's commit records (keep_records=True)
 
 
 def compare_state(tc, o, rep: ParityReport, heads, oracle_heads):
@@ -58,7 +59,7 @@ def compare_state(tc, o, rep: ParityReport, heads, oracle_heads):
 
 def run_parity(cfg, chunks=None, attends=1, rows=None, state_heads=None, flush=True, device="cuda",
                check_every_state=True, intra_chunk=False, oracle_heads=None, attn_chunks=None, q_scale=1.0,
-               key_mode="representative", on_chunk=None):
+               key_mode="representative", on_chunk=None, keep_records=False):
     """Run `chunks` chunks through both implementations and collect the differences.
 
     rows: query rows checked per attend (None = all). oracle_heads: the heads the oracle
@@ -86,6 +87,8 @@ def run_parity(cfg, chunks=None, attends=1, rows=None, state_heads=None, flush=T
     sel = None if rows is None else np.asarray(rows)
 
     def check_commit(rec):
+        if keep_records:
+            rep.records.append(rec)
         codes, match, dest = tc.last_commit()
         rep.commits += 1
         rep.tokens += rec.match.size
