@@ -3,14 +3,16 @@
 
 A step is one full rollout of the workload from an empty cache: 40 chunks of 3
 frames (4680 tokens, 12 heads, d = 128, bf16), each chunk one tc_append_chunk
-(commit of the previous chunk: hash, bucket search, merge, append; staging of this
-one) followed by 4 tc_attend calls. value = frames processed by all ranks / the
+(commit of the previous chunk: append and merge; staging of this one: copy, hash,
+bucket search and merge decisions) followed by 4 tc_attend calls. value = frames processed by all ranks / the
 slowest rank's device time. Inputs are generated before timing and stay resident
 in HBM (3.5 GB of distinct K, V, Q per rollout, far larger than the 126 MB L2).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
   python bench.py --workload annca-wan1.3b     (AnnCA cross-attention, its own line)
   python bench.py --workload annsa-wan1.3b     (AnnSA same-bucket self-attention, its own line)
+  python bench.py --workload lvsa-wan1.3b      (LVSA frame-masked attention, its own line)
+  python bench.py --key-mode mean              (running-mean keys, its own line)
 
 N > 1 runs under torchrun: each rank runs an independent rollout (its own seed);
 there is no collective in the data path, only the max-over-ranks of the timing.
@@ -169,18 +171,30 @@ def rollout(tc, chunks, outs, events=None):
 
 
 def sizes_per_chunk(tc, chunks, outs, cfg):
-    """Committed entries per head seen by the attends of each chunk, and commit counts."""
+    """Committed entries per head seen by the attends of each chunk, and per append call
+    the counts its algorithmic bytes depend on: tokens appended, tokens merged and
+    entries touched by the commit it runs (of the previous chunk), and the candidates
+    the staging search of this chunk visits (the committed entries in each staged
+    token's bucket, counted here from the exported codes)."""
     tc.reset()
     sizes, commit = [], []
     for K, V, Qs in chunks:
         tc.append_chunk(K, V)
         sizes.append(tc.cache_size().copy())
         _, match, _ = tc.last_commit()
+        staged = tc.staged_codes()
+        cand = 0
+        for h in range(cfg.H):
+            codes = tc.export_cache(h)[3]
+            if codes.size:
+                u, n = np.unique(codes, return_counts=True)
+                pos = np.clip(np.searchsorted(u, staged[h]), 0, u.size - 1)
+                cand += int(np.where(u[pos] == staged[h], n[pos], 0).sum())
         if match.size:
             touched = sum(len(np.unique(match[h][match[h] >= 0])) for h in range(cfg.H))
-            commit.append(((match < 0).sum(), (match >= 0).sum(), touched, match.shape[1]))
+            commit.append((int((match < 0).sum()), int((match >= 0).sum()), touched, match.shape[1], cand))
         else:
-            commit.append((0, 0, 0, 0))
+            commit.append((0, 0, 0, 0, cand))
         for a, Q in enumerate(Qs):
             tc.attend(Q, out=outs[a])
     return sizes, commit
@@ -193,59 +207,64 @@ def attn_flops(cfg, sizes):
 
 
 def commit_bytes(cfg, commit_counts, b=2):
-    """Algorithmic bytes of one tc_append_chunk: staging copy + hash, reading every
-    staged key once for the search, appending unmatched rows (K, V, fp32 V) and
-    updating merged entries (read the matched V rows, read+write fp32 V, write V)."""
+    """Algorithmic bytes of each tc_append_chunk call, which commits the previous chunk
+    and stages this one:
+      staging   read K and V, write the head-major copies: 4 T H d b; per token its code,
+                decision and bucket head: 12 T H;
+      search    per candidate visited, its key row, |k|^2, next link and span: d b + 13;
+                per merged token its merge-list link: 8;
+      append    per new entry: read the staged K and V rows, write K, V and the fp32 V
+                mean: 4 d b + 4 d; its scalars (n, log2 n, code, |k|^2, span, list
+                links): 29;
+      merge     per merged token its staged V row and list link: d b + 4; per touched
+                entry the fp32 mean read and written, the storage copy written and its
+                scalars: 8 d + d b + 12;
+      exports   per committed token its code, target and entry index: 12 (the commit's
+                reads of the staged codes and decisions: 8)."""
     T, H, d = cfg.T, cfg.H, cfg.d
     total = []
-    for u, m, e, Tc in commit_counts:
-        stage = 4 * T * H * d * b + 4 * T * H
-        search = Tc * H * d * b + 8 * Tc * H if Tc else 0
-        append = u * (2 * d * b + 2 * d * b + 4 * d + 16)
-        merge = m * (d * b + 4) + e * (2 * 4 * d + d * b + 8)
-        total.append(stage + search + append + merge)
+    for u, m, e, Tc, cand in commit_counts:
+        stage = 4 * T * H * d * b + 12 * T * H
+        search = cand * (d * b + 13) + 8 * m
+        append = u * (4 * d * b + 4 * d + 29)
+        merge = m * (d * b + 4) + e * (8 * d + d * b + 12)
+        exports = 20 * Tc * H
+        total.append(stage + search + append + merge + exports)
     return total
 
 
 # ----------------------------------------------------------------------------- CPU oracle leg
 
-def oracle_sample(cfg, chunks_cpu, R, n_chunks, rows_per_attend, time_budget_s, warmup_chunks=0):
-    """Time the CPU oracle over consecutive chunks of the rollout.
+def oracle_rollout(cfg, R, chunks, heads, rows_per_call, seed=0):
+    """Time the CPU oracle over one whole rollout, on a subset of the heads.
 
-    Every chunk runs the oracle's full merge path; attention runs on
-    `rows_per_attend` query rows per call and its time is scaled to all rows.
-    Returns (frames/s, chunks timed, description).
+    Heads are independent, so the oracle follows `heads` through every chunk: each
+    chunk's full merge path (hash, bucket search, merge, append) is timed, and one of the
+    chunk's attention calls on `rows_per_call` sampled query rows, its time scaled to all
+    rows and all calls. The sum is scaled to all H heads. Inputs are converted to fp64
+    outside the timed sections. Returns (frames/s, description).
     """
     from oracle import OracleTempCache
 
-    o = OracleTempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, R.astype(np.float64))
-    rng = np.random.default_rng(0)
-    total, timed = 0.0, 0
-    for c, (K, V, Qs) in enumerate(chunks_cpu):
-        if c >= warmup_chunks + n_chunks:
-            break
+    f = lambda x: x[:, heads].to(torch.float64).cpu().numpy()  # noqa: E731
+    o = OracleTempCache(len(heads), cfg.d, cfg.nbits, cfg.tau, cfg.capacity, R.astype(np.float64))
+    rng = np.random.default_rng(seed)
+    t_merge = t_attn = 0.0
+    for K, V, Qs in chunks:
+        k, v = f(K), f(V)
         t0 = time.perf_counter()
-        o.append_chunk(K, V)
-        t_merge = time.perf_counter() - t0
-        t_attn = 0.0
-        for Q in Qs:
-            rows = np.sort(rng.choice(cfg.T, size=min(rows_per_attend, cfg.T), replace=False))
-            t1 = time.perf_counter()
-            o.attend(Q, rows=rows)
-            t_attn += (time.perf_counter() - t1) * (cfg.T / len(rows))
-        if c >= warmup_chunks:
-            total += t_merge + t_attn
-            timed += 1
-        if total > time_budget_s and timed >= 1:
-            break
-    desc = (f"chunks {warmup_chunks}..{warmup_chunks + timed - 1} of the {WORKLOAD} rollout: full oracle "
-            f"merge path; attention on {rows_per_attend} of {cfg.T} query rows per call, time scaled to all rows")
-    return cfg.F * timed / total, timed, desc
-
-
-def cpu_inputs(chunks):
-    f = lambda x: x.to(torch.float64).cpu().numpy()  # noqa: E731
-    return [(f(K), f(V), [f(Q) for Q in Qs]) for K, V, Qs in chunks]
+        o.append_chunk(k, v)
+        t_merge += time.perf_counter() - t0
+        rows = np.sort(rng.choice(cfg.T, size=min(rows_per_call, cfg.T), replace=False))
+        q = Qs[0][torch.as_tensor(rows, device=Qs[0].device)][:, heads].to(torch.float64).cpu().numpy()
+        t1 = time.perf_counter()
+        o.attend(q)
+        t_attn += (time.perf_counter() - t1) * (cfg.T / len(rows)) * cfg.attends
+    total = (t_merge + t_attn) * cfg.H / len(heads)
+    desc = (f"one whole {cfg.name} rollout ({len(chunks)} chunks) on heads {list(heads)} of {cfg.H}, scaled to all "
+            f"heads: full oracle merge path every chunk; attention timed on {rows_per_call} of {cfg.T} query rows "
+            f"of one call per chunk, scaled to all rows and {cfg.attends} calls")
+    return cfg.F * len(chunks) / total, desc
 
 
 def describe(cfg) -> str:
@@ -258,15 +277,22 @@ def run_reference(args):
     if rank != 0:
         return
     cfg = CONFIGS[WORKLOAD]
-    R, chunks = generate_inputs(cfg.replace(chunks=args.warmup + args.steps), "cpu", cfg.seed)
-    value, timed, desc = oracle_sample(cfg, cpu_inputs(chunks), R, args.steps, 64, float("inf"),
-                                       warmup_chunks=args.warmup)
+    R, chunks = generate_inputs(cfg, "cpu", cfg.seed)
+    for _ in range(args.warmup):
+        oracle_rollout(cfg, R, chunks, [0], 32)
+    t = 0.0
+    for k in range(args.steps):   # each step: the whole rollout on one head, scaled to all 12
+        value_k, desc = oracle_rollout(cfg, R, chunks, [k % cfg.H], 32, seed=k)
+        t += cfg.F * cfg.chunks / value_k
+    value = cfg.F * cfg.chunks * args.steps / t
     cores = len(os.sched_getaffinity(0))
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * cfg.F / value,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": describe(cfg), "step": "one chunk (commit + 4 attends) of the rollout"},
+        "config": {"workload": describe(cfg),
+                   "step": f"one {cfg.chunks}-chunk rollout ({cfg.F * cfg.chunks} frames) from an empty cache, "
+                           "timed on one head (head k mod 12 at step k) and scaled to all heads"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -315,12 +341,14 @@ def run_gpu(args):
     init_dist(world, "nccl")
     dev = torch.device("cuda", local)
     cfg = CONFIGS[args.workload]
-    headline = args.workload == WORKLOAD and not args.profile and not args.intra_chunk
+    headline = (args.workload == WORKLOAD and not args.profile and not args.intra_chunk
+                and args.key_mode == "representative")
     if args.chunks:
         cfg = cfg.replace(chunks=args.chunks, capacity=min(cfg.capacity, args.chunks * cfg.T))
     R, chunks = generate_inputs(cfg, dev, rank_seed(cfg.seed, rank))
     input_gb = cfg.chunks * cfg.T * cfg.H * cfg.d * 2 * (2 + cfg.attends) / 1e9
-    tc = TempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, hyperplanes=R, intra_chunk=args.intra_chunk)
+    tc = TempCache(cfg.H, cfg.d, cfg.nbits, cfg.tau, cfg.capacity, hyperplanes=R, intra_chunk=args.intra_chunk,
+                   key_mode=args.key_mode)
     outs = [torch.empty(cfg.T, cfg.H, cfg.d, dtype=torch.bfloat16, device=dev) for _ in range(cfg.attends)]
 
     sizes, commit_counts = sizes_per_chunk(tc, chunks, outs, cfg)
@@ -405,9 +433,7 @@ def run_gpu(args):
     cores = len(os.sched_getaffinity(0))
     cpu = None
     if world == 1 and not args.no_cpu_baseline and headline:
-        cpu_chunks = cpu_inputs(chunks[:6])
-        v, n, desc = oracle_sample(cfg, cpu_chunks, R, n_chunks=5, rows_per_attend=256, time_budget_s=20.0,
-                                   warmup_chunks=1)
+        v, desc = oracle_rollout(cfg, R, chunks, [0, cfg.H // 2], 32)
         cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -417,14 +443,18 @@ def run_gpu(args):
                    "step": f"one {cfg.chunks}-chunk rollout ({cfg.F * cfg.chunks} frames) from an empty cache",
                    "l2": f"inputs larger than L2 ({input_gb:.1f} GB of distinct K, V, Q per rollout)",
                    "parallelism": f"independent rollout per rank x{world}",
-                   "commit": "matches inside the chunk too" if args.intra_chunk else "snapshot of earlier commits"},
+                   "commit": "matches inside the chunk too" if args.intra_chunk else "snapshot of earlier commits",
+                   "keys": "running means of the members' keys" if args.key_mode == "mean"
+                           else "the key that created the entry"},
         "roofline": {"bound": "tensor", "kernel": ATTN_KERNEL, "achieved": attn_tflops,
                      "peak": peak, "unit": "TFLOP/s", "frac": attn_tflops / peak,
                      "peak_kind": f"{peak_kind} bf16 dense, sustained", "traffic": traffic,
                      "traffic_earlier_build": traffic_earlier,
                      "flops_per_launch": attn_flops_total / (args.steps * cfg.chunks * cfg.attends),
                      "avg_launch_ms": 1000.0 * attn_sec / (args.steps * cfg.chunks * cfg.attends)},
-        "merge": {"achieved_gbs": cbytes / app_sec / 1e9, "peak_gbs": float(peaks["hbm_gbs"]),
+        "merge": {"kernels": "stage_search_kernel (copy, hash, bucket search) + commit_kernel (append, merge)"
+                             + (" + rebucket kernels" if args.key_mode == "mean" else ""),
+                  "achieved_gbs": cbytes / app_sec / 1e9, "peak_gbs": float(peaks["hbm_gbs"]),
                   "frac": cbytes / app_sec / 1e9 / float(peaks["hbm_gbs"]),
                   "bytes_per_chunk": cbytes / (args.steps * cfg.chunks),
                   "avg_append_ms": 1000.0 * app_sec / (args.steps * cfg.chunks)},
@@ -724,6 +754,124 @@ def run_annsa(args):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- LVSA leg
+
+LVSA_METRIC = "LVSA frame-masked attention frames/s at Wan-1.3B shape, 6x horizon (126 frames, C = 21)"
+
+
+def run_lvsa(args):
+    """One step = one tc_lvsa_attend call (one denoising step s = k) over a 126-frame
+    latent video of the Wan-2.1-1.3B layer shape (6x its 21-frame training horizon):
+    every query frame attends to C = 21 frames (rotating anchors every T_per = 21
+    frames plus its expanded window)."""
+    from kv_cache_attention_tempcache_b200 import LVSA
+    from oracle import attended_frames
+
+    rank, world, local = dist_info()
+    torch.cuda.set_device(local)
+    init_dist(world, "nccl")
+    dev = torch.device("cuda", local)
+    T, P, H, d, T_per, C = 126, 1560, 12, 128, 21, 21
+    g = torch.Generator(device=dev).manual_seed(rank_seed(2024, rank))
+    Q, K, V = (torch.randn(T * P, H, d, generator=g, device=dev).to(torch.bfloat16) for _ in range(3))
+    out = torch.empty_like(Q)
+    lv = LVSA(H, d, P, T_per, C)
+    dense = LVSA(H, d, P, 1, T)   # every frame attends to every frame: the same kernel, dense
+
+    def flops_of(Cb, Tp, s):
+        return 4.0 * P * P * d * H * sum(len(a) for a in attended_frames(T, Tp, Cb, s))
+
+    for k in range(args.warmup):
+        lv.attend(Q, K, V, k, out=out)
+    torch.cuda.synchronize()
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    marks = [(ev(), ev()) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0, t1 = ev(), ev()
+    t0.record()
+    for k in range(args.steps):
+        marks[k][0].record()
+        lv.attend(Q, K, V, k, out=out)
+        marks[k][1].record()
+    t1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    sec = t0.elapsed_time(t1) / 1000.0
+    sec_max = max_over_ranks(sec, world, dev)
+    value = aggregate_rate(T * args.steps, world, sec_max)
+    call_sec = sum(a.elapsed_time(b) for a, b in marks) / 1000.0 / args.steps
+    flops = float(np.mean([flops_of(C, T_per, k) for k in range(args.steps)]))
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    # dense baseline: the same kernel with every frame attended
+    dense.attend(Q, K, V, 0, out=out)
+    torch.cuda.synchronize()
+    d0, d1 = ev(), ev()
+    d0.record()
+    dense.attend(Q, K, V, 0, out=out)
+    d1.record()
+    torch.cuda.synchronize()
+    dense_sec = d0.elapsed_time(d1) / 1000.0
+    dense_flops = flops_of(T, 1, 0)
+    # end to end: Q, K, V from pinned host memory, the output read back
+    hq, hk, hv = (x.cpu().pin_memory() for x in (Q, K, V))
+    ho = torch.empty_like(hq).pin_memory()
+    ho.copy_(lv.attend(hq, hk, hv, 0), non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = ev(), ev()
+    e0.record()
+    ho.copy_(lv.attend(hq, hk, hv, 1), non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_sec = max_over_ranks(e0.elapsed_time(e1) / 1000.0, world, dev)
+    nb = T * P * H * d * 2
+    if rank != 0:
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        from oracle import biased_attention
+        A = attended_frames(T, T_per, C, 0)
+        t, h = T // 2, 0
+        keys = np.concatenate([np.arange(f * P, (f + 1) * P) for f in A[t]])
+        f64 = lambda x: x.to(torch.float64).cpu().numpy()  # noqa: E731
+        q, kk, vv = f64(Q[t * P:(t + 1) * P, h]), f64(K[keys, h]), f64(V[keys, h])
+        tc0 = time.perf_counter()
+        biased_attention(q, kk, vv, np.zeros(keys.size), 1.0 / math.sqrt(d))
+        tcpu = (time.perf_counter() - tc0) * T * H
+        cpu = {"value": T / tcpu, "unit": UNIT, "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+               "sample": f"query frame {t} of head {h} in full (its {len(A[t])} frames of keys), scaled to "
+                         f"{T} frames x {H} heads"}
+    line = {
+        "metric": LVSA_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * sec_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"lvsa-wan1.3b: T={T} frames x P={P} tokens, H={H} d={d}, T_per={T_per}, C={C}, "
+                               "Q K V ~ N(0,1) bf16",
+                   "step": "one tc_lvsa_attend call (denoising step s = k)",
+                   "l2": f"inputs larger than L2 ({3 * nb / 1e9:.2f} GB of Q, K, V)",
+                   "parallelism": f"independent layer per rank x{world}"},
+        "roofline": {"bound": "tensor", "kernel": "attend_bf16_duo_kernel (frame mode)", "achieved": flops / call_sec / 1e12,
+                     "peak": peak, "unit": "TFLOP/s", "frac": flops / call_sec / 1e12 / peak,
+                     "peak_kind": f"{peak_kind} bf16 dense, sustained", "traffic": None,
+                     "flops_per_call": flops, "avg_call_ms": 1000.0 * call_sec},
+        "dense_baseline": {"value": T / dense_sec, "unit": UNIT, "attn_tflops": dense_flops / dense_sec / 1e12,
+                           "note": "same kernel with C = T (every frame attends to every frame)"},
+        "cpu_baseline": cpu,
+        "e2e": {"value": aggregate_rate(T, world, e2e_sec), "unit": UNIT, "h2d_bytes_per_step": 3 * nb,
+                "d2h_bytes_per_step": nb},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+    }
+    lv.close()
+    dense.close()
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -737,12 +885,15 @@ def main():
                     help="rollout length in chunks (default: the workload's); profiling runs use fewer")
     ap.add_argument("--workload", default=WORKLOAD,
                     choices=[k for k, v in CONFIGS.items() if v.dtype == "bf16"] + ["annca-wan1.3b",
-                                                                                      "annsa-wan1.3b"],
+                                                                                      "annsa-wan1.3b",
+                                                                                      "lvsa-wan1.3b"],
                     help="synthetic workload; only the default one adds the dense, end-to-end and CPU legs "
                          "(annca-wan1.3b: AnnCA cross-attention, with its own legs)")
     ap.add_argument("--series", action="store_true", help="add per-chunk commit and attention times")
     ap.add_argument("--intra-chunk", action="store_true",
                     help="commits also match tokens against entries created earlier in the same commit")
+    ap.add_argument("--key-mode", default="representative", choices=["representative", "mean"],
+                    help="mean: an entry's key is the running mean of its members' keys")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
@@ -750,6 +901,8 @@ def main():
         run_annca(args)
     elif args.workload == "annsa-wan1.3b":
         run_annsa(args)
+    elif args.workload == "lvsa-wan1.3b":
+        run_lvsa(args)
     else:
         run_gpu(args)
     if torch.distributed.is_initialized():

@@ -195,7 +195,7 @@ __device__ void publish_sizes(const CacheView& c, const StageView& s, int32_t* c
 //  1. copies the window's K rows into shared memory and, with its V rows, into the
 //     head-major staging buffer (16-byte words, eight in flight per lane);
 //  2. hashes: lane l takes token t0 + l and forms the nbits projections <R_b, k> in
-//     fp32, the normals being constant-bank operands of the FMAs (a kernel parameter);
+//     fp32, the normals broadcast from a copy in shared memory;
 //     bit b keeps the fp32 sign when
 //       |<R_b,k>| > 2 (d+2) u |R_b| |k|   (u = 2^-24; any summation order errs by at
 //                                          most (d+2) u sum|R_bi k_i| <= (d+2) u |R_b||k|,
@@ -260,7 +260,7 @@ __device__ __forceinline__ void unpack16(const uint4& v, float (&x)[16 / sizeof(
 
 // Index-order fp64 sum of x_i y_i over a shared-memory row x and a global row y.
 template <typename E, typename F, int D>
-__device__ __forceinline__ double chain_dot(const uint8_t* x, const F* __restrict__ y) {
+__device__ __noinline__ double chain_dot(const uint8_t* x, const F* __restrict__ y) {
     double acc = 0.0;
 #pragma unroll 8
     for (int i = 0; i < D; ++i) {
@@ -277,7 +277,7 @@ __device__ __forceinline__ double chain_dot(const uint8_t* x, const F* __restric
 // Exact sum of x_i y_i of two bf16 rows (x in shared memory, y from global memory) when
 // the span rule holds: exact fp32 products, four fp64 partial sums.
 template <int D>
-__device__ __forceinline__ double span_dot(const uint8_t* x, const uint4* __restrict__ y) {
+__device__ __noinline__ double span_dot(const uint8_t* x, const uint4* __restrict__ y) {
     constexpr int W = D / 8;
     uint4 yw[W];
 #pragma unroll
@@ -296,17 +296,60 @@ __device__ __forceinline__ double span_dot(const uint8_t* x, const uint4* __rest
     return (a0 + a1) + (a2 + a3);
 }
 
+// fp32 sum of x_i y_i of a bf16 row in shared memory and a bf16 row from global memory
+// (exact products, rounded sums in four chains: within (d+2) u |x||y| of the exact sum).
+template <int D>
+__device__ __forceinline__ float dot32_bf16(const uint8_t* x, const uint4* __restrict__ y) {
+    constexpr int W = D / 8;
+    uint4 yw[W];
+#pragma unroll
+    for (int c = 0; c < W; ++c) yw[c] = y[c];
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+    for (int c = 0; c < W; ++c) {
+        float xv[8], yv[8];
+        unpack16<__nv_bfloat16>(*reinterpret_cast<const uint4*>(x + 16 * c), xv);
+        unpack16<__nv_bfloat16>(yw[c], yv);
+        a0 = fmaf(xv[0], yv[0], fmaf(xv[4], yv[4], a0));
+        a1 = fmaf(xv[1], yv[1], fmaf(xv[5], yv[5], a1));
+        a2 = fmaf(xv[2], yv[2], fmaf(xv[6], yv[6], a2));
+        a3 = fmaf(xv[3], yv[3], fmaf(xv[7], yv[7], a3));
+    }
+    return (a0 + a1) + (a2 + a3);
+}
+
+// The same with an fp32 row y (running-mean keys that are not bf16 values).
+template <typename E, int D>
+__device__ __forceinline__ float dot32_f32(const uint8_t* x, const float* __restrict__ y) {
+    float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll 4
+    for (int i = 0; i < D; i += 4) {
+        const float4 yv = *reinterpret_cast<const float4*>(y + i);
+        a0 = fmaf(srow_at<E>(x, i), yv.x, a0);
+        a1 = fmaf(srow_at<E>(x, i + 1), yv.y, a1);
+        a2 = fmaf(srow_at<E>(x, i + 2), yv.z, a2);
+        a3 = fmaf(srow_at<E>(x, i + 3), yv.w, a3);
+    }
+    return (a0 + a1) + (a2 + a3);
+}
+
 template <typename E, int D, int NBP, bool INTRA, bool MEAN>
 __global__ void __launch_bounds__(kWarps * 32, 2)
 stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView c, StageView s,
-                    const float* __restrict__ R, const __grid_constant__ StagePlanes<D, NBP> pl, double tau64,
+                    const float* __restrict__ R, const __grid_constant__ StagePlanes<D, NBP> pl, float tau,
                     int32_t* ctr, Stats* stats) {
     using S = StageSmem<E, D>;
+    const double tau64 = (double)tau;
+    // delta bounds |sim32 - sim| of the fp32 cosines: 2 x (2 (d+2) u + 3 u)
+    const float delta = 2.f * (2.f * (float)(D + 2) * kU32 + 3.f * kU32);
     constexpr int W = D * (int)sizeof(E) / 16;   // 16-byte words per row
     constexpr int EPW = 16 / (int)sizeof(E);     // elements per word
     extern __shared__ __align__(16) uint8_t ss_smem[];
     __shared__ float sKmax[kWarps];
     __shared__ unsigned sRe[kWarps][2];
+    __shared__ __align__(16) float sR[NBP * D];   // the normals (rows past nbits zero)
+    for (int i = threadIdx.x; i < NBP * D; i += blockDim.x) sR[i] = pl.v[i];
+    __syncthreads();
     grid_dependency_wait();   // the previous commit (and anything else before us in the stream)
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     uint8_t* rows = ss_smem + wib * S::WARP;
@@ -363,13 +406,13 @@ stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView 
         const uint8_t* my = rows + lane * S::RB;
         uint32_t code = 0;
         int spx = 255;
+        float n2 = 0.f;
         if (valid) {
             float acc[NBP];
 #pragma unroll
             for (int b = 0; b < NBP; ++b) acc[b] = 0.f;
-            float n2 = 0.f;
-            int emax = 0, emin = 255;
-#pragma unroll
+            uint32_t emax2 = 0u, emin2 = 0x7f807f80u;   // exponent fields of both bf16 halves
+#pragma unroll 1
             for (int cw = 0; cw < W; ++cw) {
                 const uint4 v4 = *reinterpret_cast<const uint4*>(my + cw * 16);
                 float x[EPW];
@@ -378,19 +421,25 @@ stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView 
                     const uint32_t wd[4] = {v4.x, v4.y, v4.z, v4.w};
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const uint32_t lo = wd[k] & 0xffffu, hi = wd[k] >> 16;
-                        const int flo = max((int)((lo >> 7) & 0xffu), 1), fhi = max((int)((hi >> 7) & 0xffu), 1);
-                        if (lo & 0x7fffu) { emax = max(emax, flo); emin = min(emin, flo); }
-                        if (hi & 0x7fffu) { emax = max(emax, fhi); emin = min(emin, fhi); }
+                        const uint32_t f = wd[k] & 0x7f807f80u;
+                        emax2 = __vmaxu2(emax2, f);
+                        emin2 = __vminu2(emin2, f);
                     }
                 }
 #pragma unroll
                 for (int k = 0; k < EPW; ++k) n2 = fmaf(x[k], x[k], n2);
 #pragma unroll
                 for (int b = 0; b < NBP; ++b) {
+                    const float* rb = sR + b * D + cw * EPW;   // same address on every lane: broadcast
                     float t = acc[b];
 #pragma unroll
-                    for (int k = 0; k < EPW; ++k) t = fmaf(pl.v[b * D + cw * EPW + k], x[k], t);
+                    for (int k = 0; k < EPW; k += 4) {
+                        const float4 r4 = *reinterpret_cast<const float4*>(rb + k);
+                        t = fmaf(r4.x, x[k], t);
+                        t = fmaf(r4.y, x[k + 1], t);
+                        t = fmaf(r4.z, x[k + 2], t);
+                        t = fmaf(r4.w, x[k + 3], t);
+                    }
                     acc[b] = t;
                 }
             }
@@ -407,21 +456,24 @@ stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView 
                 }
                 code |= (uint32_t)bit << b;
             }
-            if constexpr (sizeof(E) == 2) spx = emax >= emin ? emax - emin + 7 : 0;
+            if constexpr (sizeof(E) == 2) {
+                // span from the exponent fields; a zero element counts as field 0, which only
+                // widens the span (the exact-sum rule then sends the row to the chain)
+                const int emax = (int)max(emax2 >> 23, (emax2 >> 7) & 0xffu);
+                const int emin = max((int)min(emin2 >> 23, (emin2 >> 7) & 0xffu), 0);
+                spx = emax >= 1 ? emax - emin + 7 + (emin == 0 ? 1 : 0) : 0;
+            }
             s.scode[sbase + lane] = code;
             kmax = fmaxf(kmax, n2);
         }
         // ---- 3. search the bucket
         const int64_t hrow = (int64_t)h * c.capP;
         const int Mh = c.M[h];
-        int j = valid ? c.bhead[((int64_t)h << nbits) + code] : -1;
-        double best = -INFINITY, n1 = -1.0;
-        int bestj = -1, ncand = 0;
-        while (j >= 0) {   // per lane
-            const int nxt = c.bnext[hrow + j];
-            const double n2e = c.knorm64[hrow + j];
-            const int spy = c.kspan[hrow + j];
-            if (n1 < 0.0) {   // |x|^2 with the value of the index-order sum, once per token
+        const int head = valid ? c.bhead[((int64_t)h << nbits) + code] : -1;
+        double n1 = -1.0;   // exact |x|^2, formed when first needed
+        // exact fp64 cosine of the lane's token with entry j (the value of the definition)
+        auto exact_sim = [&](int j) -> double {
+            if (n1 < 0.0) {
                 if constexpr (sizeof(E) == 2) {
                     if (2 * spx <= kSpanLimit<D>) {
                         n1 = span_dot<D>(my, reinterpret_cast<const uint4*>(my));
@@ -433,8 +485,10 @@ stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView 
                     n1 = chain_dot<E, float, D>(my, reinterpret_cast<const float*>(my));
                 }
             }
+            const double n2e = c.knorm64[hrow + j];
             double dot;
             if constexpr (sizeof(E) == 2) {
+                const int spy = c.kspan[hrow + j];
                 if (spx + spy <= kSpanLimit<D>) {
                     dot = span_dot<D>(my, reinterpret_cast<const uint4*>(Kc + (hrow + j) * D));
                 } else {
@@ -446,16 +500,101 @@ stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView 
                 dot = chain_dot<E, float, D>(my, reinterpret_cast<const float*>(Kc) + (hrow + j) * D);
                 ++mre;
             }
-            const double sim = (n1 > 0.0 && n2e > 0.0) ? dot / sqrt(n1 * n2e) : 0.0;
-            if (sim > best || (sim == best && j < bestj)) {
-                best = sim;
-                bestj = j;
+            return (n1 > 0.0 && n2e > 0.0) ? dot / sqrt(n1 * n2e) : 0.0;
+        };
+        double best = -INFINITY;   // exact best similarity (intra_chunk and exact paths)
+        int bestj = -1, m = -1;
+        if constexpr (INTRA || sizeof(E) != 2) {
+            // every candidate exactly: the in-chunk dedupe needs the exact best similarity,
+            // and fp32 rows have no certified shortcut here
+            int ncand = 0;
+            for (int j = head; j >= 0;) {   // per lane
+                const int nxt = c.bnext[hrow + j];
+                const double sim = exact_sim(j);
+                if (sim > best || (sim == best && j < bestj)) {
+                    best = sim;
+                    bestj = j;
+                }
+                if (++ncand > Mh) {   // a bucket list can never be longer than the cache
+                    atomicOr(&stats->error_bits, kErrBucketList);
+                    break;
+                }
+                j = nxt;
             }
-            if (++ncand > Mh) {   // a bucket list can never be longer than the cache
-                atomicOr(&stats->error_bits, kErrBucketList);
-                break;
+            m = (bestj >= 0 && best >= tau64) ? bestj : -1;
+        } else {
+            // fp32 cosines first. With delta a rigorous bound on |sim32 - sim|, the fp32
+            // result decides when its best is below tau - delta (no merge), or above
+            // tau + delta and ahead of every other candidate by more than 2 delta (merge into
+            // it). Otherwise the candidates within 2 delta of the fp32 best (the only ones
+            // that can be the exact best) are recomputed exactly.
+            float b32 = -INFINITY, s32 = -INFINITY;
+            int bj = -1, ncand = 0;
+            bool weird = !(n2 > 1e-30f && n2 < 1e30f);
+            for (int j = head; j >= 0;) {   // per lane
+                const int nxt = c.bnext[hrow + j];
+                const float ne = (float)c.knorm64[hrow + j];
+                float dt;
+                if constexpr (MEAN) {
+                    if (c.kspan[hrow + j] == 255) dt = dot32_f32<E, D>(my, c.K32 + (hrow + j) * D);
+                    else dt = dot32_bf16<D>(my, reinterpret_cast<const uint4*>(Kc + (hrow + j) * D));
+                } else {
+                    dt = dot32_bf16<D>(my, reinterpret_cast<const uint4*>(Kc + (hrow + j) * D));
+                }
+                if (nxt >= 0) {   // the next candidate's row (two 128-byte lines for d = 128)
+                    const E* nr = Kc + (hrow + nxt) * D;
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(nr));
+                    if (D * sizeof(E) > 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(nr + 128 / sizeof(E)));
+                }
+                weird = weird || !(ne > 1e-30f && ne < 1e30f && fabsf(dt) < 1e30f);
+                const float sim = dt / sqrtf(n2 * ne);
+                if (sim > b32 || (sim == b32 && j < bj)) {
+                    s32 = b32;
+                    b32 = sim;
+                    bj = j;
+                } else if (sim > s32) {
+                    s32 = sim;
+                }
+                if (++ncand > Mh) {
+                    atomicOr(&stats->error_bits, kErrBucketList);
+                    break;
+                }
+                j = nxt;
             }
-            j = nxt;
+            if (ncand == 0) {
+                m = -1;
+            } else if (!weird && b32 < tau - delta) {
+                m = -1;
+            } else if (!weird && b32 > tau + delta && (ncand == 1 || b32 - s32 > 2.f * delta)) {
+                m = bj;
+            } else {   // exact recheck of the candidates that can still be the best
+                int guard = 0;
+                for (int j = head; j >= 0;) {
+                    const int nxt = c.bnext[hrow + j];
+                    bool near = weird;
+                    if (!weird) {
+                        const float ne = (float)c.knorm64[hrow + j];
+                        float dt;
+                        if constexpr (MEAN) {
+                            if (c.kspan[hrow + j] == 255) dt = dot32_f32<E, D>(my, c.K32 + (hrow + j) * D);
+                            else dt = dot32_bf16<D>(my, reinterpret_cast<const uint4*>(Kc + (hrow + j) * D));
+                        } else {
+                            dt = dot32_bf16<D>(my, reinterpret_cast<const uint4*>(Kc + (hrow + j) * D));
+                        }
+                        near = dt / sqrtf(n2 * ne) >= b32 - 2.f * delta;
+                    }
+                    if (near) {
+                        const double sim = exact_sim(j);
+                        if (sim > best || (sim == best && j < bestj)) {
+                            best = sim;
+                            bestj = j;
+                        }
+                    }
+                    if (++guard > ncand) break;
+                    j = nxt;
+                }
+                m = (bestj >= 0 && best >= tau64) ? bestj : -1;
+            }
         }
         // ---- 4. publish
         const int64_t sidx = sbase + lane;
@@ -468,7 +607,6 @@ stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView 
             }
             if (lane == 0) s.wcnt[(int64_t)h * (s.TmaxP >> 5) + w] = 0;   // counted by the dedupe kernel
         } else {
-            const int m = (bestj >= 0 && best >= tau64) ? bestj : -1;
             if (valid) {
                 s.match[sidx] = m;
                 if (m >= 0) {
@@ -836,28 +974,11 @@ __device__ __forceinline__ void append_window(const CacheView& c, const StageVie
     __syncwarp();
 }
 
-// Index-order fp64 sum of x_i^2 (or of <R_b, x>) over a row spread across the warp,
-// lane l holding elements [l EPL, l EPL + EPL): each lane continues the previous
-// lane's sum. Every lane gets the result.
-template <int EPL>
-__device__ __forceinline__ double warp_chain(const float (&a)[EPL], const float (&b)[EPL], int lane) {
-    double acc = 0.0;
-#pragma unroll 1
-    for (int k = 0; k < 32; ++k) {
-        if (lane == k) {
-#pragma unroll
-            for (int i = 0; i < EPL; ++i) acc = fma((double)a[i], (double)b[i], acc);
-        }
-        acc = __shfl_sync(0xffffffffu, acc, k);
-    }
-    return acc;
-}
-
 // One touched entry j of head h, merged by the whole warp (lane l: elements
 // [l EPL, l EPL + EPL)). MEAN: the key is averaged too, then re-hashed.
 template <typename E, int D, bool MEAN>
 __device__ void merge_entry_warp(const CommitArgs<E, D, MEAN>& a, int h, int j, int32_t* sIds, int32_t* sSorted,
-                                 int lane) {
+                                 float* sRow, int lane) {
     const CacheView& c = a.c;
     const StageView& s = a.s;
     constexpr int EPL = D / 32;
@@ -968,30 +1089,39 @@ __device__ void merge_entry_warp(const CommitArgs<E, D, MEAN>& a, int h, int j, 
             emin = min(emin, __shfl_xor_sync(0xffffffffu, emin, o));
         }
         const int span = exact16 ? min(emax >= emin ? emax - emin + 7 : 0, 255) : 255;
-        const double n64 = warp_chain<EPL>(nk, nk, lane);
-        // the code of the new key: fp32 projections, certified, else fp64 in index order
+        // One lane per hash bit forms <R_b, k> in fp32 over the key staged in shared memory,
+        // keeps its sign outside the rounding bound and otherwise redoes it in fp64 in index
+        // order; lane 31 meanwhile forms |k|^2 as the index-order fp64 chain (nbits <= 24).
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) sRow[lane * EPL + q] = nk[q];
         float n2 = 0.f;
 #pragma unroll
         for (int q = 0; q < EPL; ++q) n2 = fmaf(nk[q], nk[q], n2);
         const float nx = sqrtf(warp_sum(n2));
+        __syncwarp();
         const float gam2 = 2.f * (float)(D + 2) * kU32;
-        uint32_t code = 0;
-        unsigned nre = 0;
-        for (int b = 0; b < c.nbits; ++b) {
-            float rb[EPL];
-#pragma unroll
-            for (int q = 0; q < EPL; ++q) rb[q] = a.R[b * D + lane * EPL + q];
+        bool bit = false, re = false;
+        double n64 = 0.0;
+        if (lane < c.nbits) {
+            const float* rb = a.R + lane * D;
             float p = 0.f;
-#pragma unroll
-            for (int q = 0; q < EPL; ++q) p = fmaf(rb[q], nk[q], p);
-            p = warp_sum(p);
-            bool bit = p >= 0.f;
-            if (!(fabsf(p) > gam2 * a.Rnorm[b] * nx + 1e-30f)) {   // warp-uniform
-                bit = warp_chain<EPL>(rb, nk, lane) >= 0.0;
-                ++nre;
+#pragma unroll 8
+            for (int i = 0; i < D; ++i) p = fmaf(rb[i], sRow[i], p);
+            bit = p >= 0.f;
+            if (!(fabsf(p) > gam2 * a.Rnorm[lane] * nx + 1e-30f)) {
+                double acc = 0.0;
+                for (int i = 0; i < D; ++i) acc = fma((double)rb[i], (double)sRow[i], acc);
+                bit = acc >= 0.0;
+                re = true;
             }
-            code |= (uint32_t)bit << b;
+        } else if (lane == 31) {
+#pragma unroll 8
+            for (int i = 0; i < D; ++i) n64 = fma((double)sRow[i], (double)sRow[i], n64);
         }
+        n64 = __shfl_sync(0xffffffffu, n64, 31);
+        const uint32_t code = __ballot_sync(0xffffffffu, bit) & (c.nbits >= 32 ? 0xffffffffu : ((1u << c.nbits) - 1u));
+        const unsigned nre = __popc(__ballot_sync(0xffffffffu, re));
+        __syncwarp();   // sRow is reused by the warp's next entry
         if (lane == 0) {
             c.knorm64[e] = n64;
             c.kspan[e] = (uint8_t)span;
@@ -1021,7 +1151,7 @@ __device__ void merge_entry_warp(const CommitArgs<E, D, MEAN>& a, int h, int j, 
 // list with running-mean keys) go to the whole warp afterwards.
 template <typename E, int D, bool MEAN>
 __device__ __forceinline__ void merge_quad(const CommitArgs<E, D, MEAN>& a, int64_t q4, int32_t* sIds,
-                                           int32_t* sSorted, int lane) {
+                                           int32_t* sSorted, float* sRow, int lane) {
     const CacheView& c = a.c;
     const StageView& s = a.s;
     using G = GSlice<E, D>;
@@ -1111,7 +1241,7 @@ __device__ __forceinline__ void merge_quad(const CommitArgs<E, D, MEAN>& a, int6
         bigm &= bigm - 1;
         const int bh = __shfl_sync(0xffffffffu, h, src);
         const int bj = __shfl_sync(0xffffffffu, j, src);
-        merge_entry_warp<E, D, MEAN>(a, bh, bj, sIds, sSorted, lane);
+        merge_entry_warp<E, D, MEAN>(a, bh, bj, sIds, sSorted, sRow, lane);
     }
 }
 
@@ -1145,6 +1275,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) commit_kernel(const CommitArgs
     __shared__ int sSrc[kWarps][32];
     __shared__ int32_t sIds[kWarps][kListSmem];
     __shared__ int32_t sSorted[kWarps][kListSmem];
+    __shared__ float sRow[kWarps][MEAN ? D : 1];   // running-mean keys: the new key, for the re-hash
     const CacheView& c = a.c;
     const StageView& s = a.s;
     const int H = c.H;
@@ -1160,7 +1291,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) commit_kernel(const CommitArgs
             const int64_t nwin = (T + 31) >> 5;
             append_window<E, D>(c, s, (int)(it / nwin), (int)(it % nwin), sSrc[wib], lane);
         } else {
-            merge_quad<E, D, MEAN>(a, (it - nA) * 4, sIds[wib], sSorted[wib], lane);
+            merge_quad<E, D, MEAN>(a, (it - nA) * 4, sIds[wib], sSorted[wib], sRow[wib], lane);
         }
     }
     grid_dependents_launch();
@@ -1255,7 +1386,7 @@ cudaError_t stage_n(const CacheView& c, const StageView& s, const void* K, const
     const int64_t items = (int64_t)c.H * ((s.T + 31) / 32);
     const int grid = grid_for_rows(items > s.TmaxP / kWarps ? items : s.TmaxP / kWarps, kWarps, 148 * 2);
     e = launch_pdl_smem(kern, grid, kWarps * 32, smem, st, reinterpret_cast<const E*>(K),
-                        reinterpret_cast<const E*>(V), c, s, R, pl, (double)tau, ctr, stats);
+                        reinterpret_cast<const E*>(V), c, s, R, pl, tau, ctr, stats);
     *launches += 1;
     if (e == cudaSuccess && INTRA) {
         const int dgrid = grid_for_rows(s.T * c.H, 4 * kWarps, 148 * 2);
