@@ -209,8 +209,7 @@ struct MarkSmem {
 };
 
 // The normals as fp32 [NBP][D] (zero rows past nbits) and their rounded-up norms, passed
-// by value: a kernel parameter sits in the constant bank, so with every index known at
-// compile time each FMA reads its normal as a constant operand, with no load.
+// by value; the mark kernel copies the normals into shared memory once per block.
 template <int D, int NBP>
 struct Planes {
     float v[NBP * D];
@@ -231,6 +230,9 @@ annca_mark_kernel(const __nv_bfloat16* __restrict__ Q, int rows, int P, int F, A
     constexpr int W = D / 8;   // 16-byte words per row
     extern __shared__ __align__(16) uint8_t mk_smem[];
     uint8_t* sRows = mk_smem;
+    __shared__ __align__(16) float sR[NBP * D];   // the normals, broadcast to every lane
+    for (int i = threadIdx.x; i < NBP * D; i += blockDim.x) sR[i] = pl.v[i];
+    __syncthreads();
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     const int nbits = a.nbits;
     grid_dependency_wait();
@@ -252,7 +254,7 @@ annca_mark_kernel(const __nv_bfloat16* __restrict__ Q, int rows, int P, int F, A
 #pragma unroll
             for (int b = 0; b < NBP; ++b) acc[b] = 0.f;
             float n2 = 0.f;
-#pragma unroll
+#pragma unroll 1
             for (int c = 0; c < W; ++c) {
                 const uint4 v = *reinterpret_cast<const uint4*>(rowp + c * 16);
                 const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
@@ -266,9 +268,17 @@ annca_mark_kernel(const __nv_bfloat16* __restrict__ Q, int rows, int P, int F, A
                 for (int k = 0; k < 8; ++k) n2 = fmaf(x[k], x[k], n2);
 #pragma unroll
                 for (int b = 0; b < NBP; ++b) {
+                    const float4 r0 = *reinterpret_cast<const float4*>(sR + b * D + c * 8);
+                    const float4 r1 = *reinterpret_cast<const float4*>(sR + b * D + c * 8 + 4);
                     float t = acc[b];
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) t = fmaf(pl.v[b * D + c * 8 + k], x[k], t);
+                    t = fmaf(r0.x, x[0], t);
+                    t = fmaf(r0.y, x[1], t);
+                    t = fmaf(r0.z, x[2], t);
+                    t = fmaf(r0.w, x[3], t);
+                    t = fmaf(r1.x, x[4], t);
+                    t = fmaf(r1.y, x[5], t);
+                    t = fmaf(r1.z, x[6], t);
+                    t = fmaf(r1.w, x[7], t);
                     acc[b] = t;
                 }
             }
@@ -610,10 +620,19 @@ __global__ void __launch_bounds__(kWarps * 32) annsa_pack_kernel(SparseBufs b, c
     uint4* Qs4 = reinterpret_cast<uint4*>(b.Qs);
     uint4* Ks4 = reinterpret_cast<uint4*>(b.Ks);
     uint4* Vs4 = reinterpret_cast<uint4*>(b.Vs);
-    const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t rr0 = (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5) * RPW; rr0 < rows; rr0 += nw * RPW) {
+    // each block packs one contiguous range of rows (one or two heads), and gathers the
+    // heads' |k|^2 bounds in shared memory: one atomic per head and block, not per row
+    constexpr int kSlots = 4;
+    __shared__ float sK[kSlots];
+    if (threadIdx.x < kSlots) sK[threadIdx.x] = 0.f;
+    __syncthreads();
+    const int64_t per = ((rows + gridDim.x - 1) / gridDim.x + RPW - 1) / RPW * RPW;
+    const int64_t rb0 = (int64_t)blockIdx.x * per, rb1 = min(rows, rb0 + per);
+    const int hlo = (int)(min(rb0, rows - 1) / Tr);
+    const int wib = threadIdx.x >> 5;
+    for (int64_t rr0 = rb0 + (int64_t)wib * RPW; rr0 < rb1; rr0 += (int64_t)kWarps * RPW) {
         const int64_t rr = rr0 + sub;
-        const bool live = rr < rows;
+        const bool live = rr < rb1;
         const int h = live ? (int)(rr / Tr) : 0;
         const int64_t r = (int64_t)h * b.Tp + (rr - (int64_t)h * Tr);
         const int32_t t = live ? b.perm[r] : -1;
@@ -645,9 +664,14 @@ __global__ void __launch_bounds__(kWarps * 32) annsa_pack_kernel(SparseBufs b, c
         }
         if (live && w == 0) {
             b.xself[r] = qk * scale_log2;
-            atomicMax(reinterpret_cast<int*>(b.kmax2 + h), __float_as_int(kk * (1.f + 1.f / 1024.f)));
+            const float kb = kk * (1.f + 1.f / 1024.f);   // floats >= 0 order like their bits
+            if (h - hlo < kSlots) atomicMax(reinterpret_cast<int*>(sK + (h - hlo)), __float_as_int(kb));
+            else atomicMax(reinterpret_cast<int*>(b.kmax2 + h), __float_as_int(kb));
         }
     }
+    __syncthreads();
+    if (threadIdx.x < kSlots && hlo + (int)threadIdx.x < b.H && sK[threadIdx.x] > 0.f)
+        atomicMax(reinterpret_cast<int*>(b.kmax2 + hlo + threadIdx.x), __float_as_int(sK[threadIdx.x]));
     grid_dependents_launch();
 }
 

@@ -224,11 +224,14 @@ struct StagePlanes {
     float rn[NBP];      // |R_b|, rounded up
 };
 
+constexpr int kStageWarps = 4;   // warps per block of the staging kernel
+constexpr int kCandKeep = 8;     // candidates whose fp32 cosine a lane keeps for the exact recheck
+
 template <typename E, int D>
 struct StageSmem {
     static constexpr int RB = D * (int)sizeof(E) + 16;   // row pitch: consecutive rows start 4 banks apart
     static constexpr int WARP = 32 * RB;
-    static constexpr int BYTES = kWarps * WARP;
+    static constexpr int BYTES = kStageWarps * WARP;
 };
 
 // Element i of a row in shared memory, as a float.
@@ -271,6 +274,15 @@ __device__ __noinline__ double chain_dot(const uint8_t* x, const F* __restrict__
             yi = y[i];
         acc = fma((double)srow_at<E>(x, i), (double)yi, acc);
     }
+    return acc;
+}
+
+// Index-order fp64 sum of y_i^2 over an fp32 row in global memory.
+template <int D>
+__device__ __noinline__ double chain_dot_ff(const float* __restrict__ y) {
+    double acc = 0.0;
+#pragma unroll 8
+    for (int i = 0; i < D; ++i) acc = fma((double)y[i], (double)y[i], acc);
     return acc;
 }
 
@@ -334,7 +346,7 @@ __device__ __forceinline__ float dot32_f32(const uint8_t* x, const float* __rest
 }
 
 template <typename E, int D, int NBP, bool INTRA, bool MEAN>
-__global__ void __launch_bounds__(kWarps * 32, 2)
+__global__ void __launch_bounds__(kStageWarps * 32, 4)
 stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView c, StageView s,
                     const float* __restrict__ R, const __grid_constant__ StagePlanes<D, NBP> pl, float tau,
                     int32_t* ctr, Stats* stats) {
@@ -345,9 +357,11 @@ stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView 
     constexpr int W = D * (int)sizeof(E) / 16;   // 16-byte words per row
     constexpr int EPW = 16 / (int)sizeof(E);     // elements per word
     extern __shared__ __align__(16) uint8_t ss_smem[];
-    __shared__ float sKmax[kWarps];
-    __shared__ unsigned sRe[kWarps][2];
+    __shared__ float sKmax[kStageWarps];
+    __shared__ unsigned sRe[kStageWarps][2];
     __shared__ __align__(16) float sR[NBP * D];   // the normals (rows past nbits zero)
+    __shared__ int sCj[kStageWarps][kCandKeep][32];     // per lane: its first candidates ...
+    __shared__ float sCs[kStageWarps][kCandKeep][32];   // ... and their fp32 cosines
     for (int i = threadIdx.x; i < NBP * D; i += blockDim.x) sR[i] = pl.v[i];
     __syncthreads();
     grid_dependency_wait();   // the previous commit (and anything else before us in the stream)
@@ -363,8 +377,8 @@ stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView 
     const E* Kc = reinterpret_cast<const E*>(c.Kc);
     float kmax = 0.f;                 // largest fp32 |k|^2 this lane staged
     unsigned hre = 0, mre = 0;        // hash bits and similarity sums that took the fp64 chain
-    for (int64_t item = (int64_t)blockIdx.x * kWarps + wib; item < (int64_t)H * nwin;
-         item += (int64_t)gridDim.x * kWarps) {   // warp-uniform
+    for (int64_t item = (int64_t)blockIdx.x * kStageWarps + wib; item < (int64_t)H * nwin;
+         item += (int64_t)gridDim.x * kStageWarps) {   // warp-uniform
         const int h = (int)(item / nwin);
         const int w = (int)(item - (int64_t)h * nwin);
         const int t0 = w * 32;
@@ -485,10 +499,13 @@ stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView 
                     n1 = chain_dot<E, float, D>(my, reinterpret_cast<const float*>(my));
                 }
             }
-            const double n2e = c.knorm64[hrow + j];
+            double n2e = c.knorm64[hrow + j];
             double dot;
             if constexpr (sizeof(E) == 2) {
                 const int spy = c.kspan[hrow + j];
+                if constexpr (MEAN) {   // a merged key outside the exact-sum rule stores only an fp32 |k|^2
+                    if (spy == 255) n2e = chain_dot_ff<D>(c.K32 + (hrow + j) * D);
+                }
                 if (spx + spy <= kSpanLimit<D>) {
                     dot = span_dot<D>(my, reinterpret_cast<const uint4*>(Kc + (hrow + j) * D));
                 } else {
@@ -548,6 +565,10 @@ stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView 
                 }
                 weird = weird || !(ne > 1e-30f && ne < 1e30f && fabsf(dt) < 1e30f);
                 const float sim = dt / sqrtf(n2 * ne);
+                if (ncand < kCandKeep) {
+                    sCj[wib][ncand][lane] = j;
+                    sCs[wib][ncand][lane] = sim;
+                }
                 if (sim > b32 || (sim == b32 && j < bj)) {
                     s32 = b32;
                     b32 = sim;
@@ -567,6 +588,18 @@ stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView 
                 m = -1;
             } else if (!weird && b32 > tau + delta && (ncand == 1 || b32 - s32 > 2.f * delta)) {
                 m = bj;
+            } else if (!weird && ncand <= kCandKeep) {   // exact recheck of the kept candidates near the best
+                for (int q = 0; q < ncand; ++q) {
+                    if (sCs[wib][q][lane] >= b32 - 2.f * delta) {
+                        const int j = sCj[wib][q][lane];
+                        const double sim = exact_sim(j);
+                        if (sim > best || (sim == best && j < bestj)) {
+                            best = sim;
+                            bestj = j;
+                        }
+                    }
+                }
+                m = (bestj >= 0 && best >= tau64) ? bestj : -1;
             } else {   // exact recheck of the candidates that can still be the best
                 int guard = 0;
                 for (int j = head; j >= 0;) {
@@ -607,13 +640,22 @@ stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView 
             }
             if (lane == 0) s.wcnt[(int64_t)h * (s.TmaxP >> 5) + w] = 0;   // counted by the dedupe kernel
         } else {
+            bool first = false;   // this token starts its target's merge list: a new touched entry
             if (valid) {
                 s.match[sidx] = m;
                 if (m >= 0) {
                     const int old = atomicExch(&c.lhead[hrow + m], t);
                     s.lnext[sidx] = old;
-                    if (old < 0) s.touched[(int64_t)h * s.TmaxP + atomicAdd(&ctr[h], 1)] = m;
+                    first = old < 0;
                 }
+            }
+            // one atomic per window for the new touched entries (a counter shared by the head)
+            const unsigned fb = __ballot_sync(0xffffffffu, first);
+            if (fb) {
+                int base = 0;
+                if (lane == __ffs(fb) - 1) base = atomicAdd(&ctr[h], __popc(fb));
+                base = __shfl_sync(0xffffffffu, base, __ffs(fb) - 1);
+                if (first) s.touched[(int64_t)h * s.TmaxP + base + __popc(fb & ((1u << lane) - 1u))] = m;
             }
             const unsigned un = __ballot_sync(0xffffffffu, valid && m < 0);
             if (lane == 0) s.wcnt[(int64_t)h * (s.TmaxP >> 5) + w] = __popc(un);
@@ -636,7 +678,7 @@ stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView 
     if (threadIdx.x == 0) {
         float m = 0.f;
         unsigned a = 0, b = 0;
-        for (int q = 0; q < kWarps; ++q) {
+        for (int q = 0; q < kStageWarps; ++q) {
             m = fmaxf(m, sKmax[q]);
             a += sRe[q][0];
             b += sRe[q][1];
@@ -844,6 +886,14 @@ __device__ __forceinline__ double gnorm64(const GSlice<E, D>& x, int span, int g
 // when its code changed (the re-bucketing kernels then move it).
 constexpr int kListSmem = 256;
 
+constexpr int kHeadSlots = 64;   // heads whose bounds a commit block gathers in shared memory
+
+// max into a per-block slot of head h when it has one, else straight into the global bound
+__device__ __forceinline__ void bound_max(float* slots, float* global_h, int h, float v) {
+    if (h < kHeadSlots) atomicMax(reinterpret_cast<int*>(slots + h), __float_as_int(v));   // floats >= 0
+    else atomicMax(reinterpret_cast<int*>(global_h), __float_as_int(v));
+}
+
 template <typename E, int D, bool MEAN>
 struct CommitArgs {
     CacheView c;
@@ -978,7 +1028,7 @@ __device__ __forceinline__ void append_window(const CacheView& c, const StageVie
 // [l EPL, l EPL + EPL)). MEAN: the key is averaged too, then re-hashed.
 template <typename E, int D, bool MEAN>
 __device__ void merge_entry_warp(const CommitArgs<E, D, MEAN>& a, int h, int j, int32_t* sIds, int32_t* sSorted,
-                                 float* sRow, int lane) {
+                                 float* sRow, float* sBm, float* sKm, int lane) {
     const CacheView& c = a.c;
     const StageView& s = a.s;
     constexpr int EPL = D / 32;
@@ -1088,44 +1138,70 @@ __device__ void merge_entry_warp(const CommitArgs<E, D, MEAN>& a, int h, int j, 
             emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, o));
             emin = min(emin, __shfl_xor_sync(0xffffffffu, emin, o));
         }
-        const int span = exact16 ? min(emax >= emin ? emax - emin + 7 : 0, 255) : 255;
-        // One lane per hash bit forms <R_b, k> in fp32 over the key staged in shared memory,
-        // keeps its sign outside the rounding bound and otherwise redoes it in fp64 in index
-        // order; lane 31 meanwhile forms |k|^2 as the index-order fp64 chain (nbits <= 24).
-#pragma unroll
-        for (int q = 0; q < EPL; ++q) sRow[lane * EPL + q] = nk[q];
+        int span = exact16 ? min(emax >= emin ? emax - emin + 7 : 0, 255) : 255;
+        // |k|^2: exact (any order) when the key is a bf16 row within the exponent-span rule;
+        // otherwise the fp32 sum is stored and the span set to 255, which makes the search
+        // form the exact value (the index-order chain over the fp32 key) whenever it needs it.
         float n2 = 0.f;
-#pragma unroll
-        for (int q = 0; q < EPL; ++q) n2 = fmaf(nk[q], nk[q], n2);
-        const float nx = sqrtf(warp_sum(n2));
-        __syncwarp();
-        const float gam2 = 2.f * (float)(D + 2) * kU32;
-        bool bit = false, re = false;
         double n64 = 0.0;
-        if (lane < c.nbits) {
-            const float* rb = a.R + lane * D;
-            float p = 0.f;
-#pragma unroll 8
-            for (int i = 0; i < D; ++i) p = fmaf(rb[i], sRow[i], p);
-            bit = p >= 0.f;
-            if (!(fabsf(p) > gam2 * a.Rnorm[lane] * nx + 1e-30f)) {
-                double acc = 0.0;
-                for (int i = 0; i < D; ++i) acc = fma((double)rb[i], (double)sRow[i], acc);
-                bit = acc >= 0.0;
-                re = true;
-            }
-        } else if (lane == 31) {
-#pragma unroll 8
-            for (int i = 0; i < D; ++i) n64 = fma((double)sRow[i], (double)sRow[i], n64);
+#pragma unroll
+        for (int q = 0; q < EPL; ++q) {
+            n2 = fmaf(nk[q], nk[q], n2);
+            n64 += (double)(nk[q] * nk[q]);   // exact products when nk holds bf16 values
         }
-        n64 = __shfl_sync(0xffffffffu, n64, 31);
-        const uint32_t code = __ballot_sync(0xffffffffu, bit) & (c.nbits >= 32 ? 0xffffffffu : ((1u << c.nbits) - 1u));
-        const unsigned nre = __popc(__ballot_sync(0xffffffffu, re));
-        __syncwarp();   // sRow is reused by the warp's next entry
+        n2 = warp_sum(n2);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) n64 += __shfl_xor_sync(0xffffffffu, n64, o);
+        if (!(exact16 && 2 * span <= kSpanLimit<D>)) {
+            span = 255;
+            if constexpr (sizeof(E) == 2) {
+                n64 = (double)n2;
+            } else {   // fp32 storage (the search takes the exact path for every candidate): the chain here
+#pragma unroll
+                for (int q = 0; q < EPL; ++q) sRow[lane * EPL + q] = nk[q];
+                __syncwarp();
+                double acc = 0.0;
+                if (lane == 0)
+                    for (int i = 0; i < D; ++i) acc = fma((double)sRow[i], (double)sRow[i], acc);
+                n64 = __shfl_sync(0xffffffffu, acc, 0);
+                __syncwarp();
+            }
+        }
+        // the code of the new key: partial projections of the lane's elements, a
+        // reduce-scatter leaves <R_b, k> (fp32) on lane b, kept outside the rounding bound
+        // and otherwise redone in fp64 in index order over the key staged in shared memory
+        float v[32];
+#pragma unroll
+        for (int b = 0; b < 32; ++b) {
+            float t = 0.f;
+            if (b < c.nbits) {
+#pragma unroll
+                for (int q = 0; q < EPL; ++q) t = fmaf(a.R[b * D + lane * EPL + q], nk[q], t);
+            }
+            v[b] = t;
+        }
+        const float p = reduce_scatter<32>(v, lane);
+        const float nx = sqrtf(n2);
+        const float gam2 = 2.f * (float)(D + 2) * kU32;
+        bool bit = p >= 0.f;
+        const bool need = lane < c.nbits && !(fabsf(p) > gam2 * a.Rnorm[lane] * nx + 1e-30f);
+        if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+            for (int q = 0; q < EPL; ++q) sRow[lane * EPL + q] = nk[q];
+            __syncwarp();
+            if (need) {
+                double acc = 0.0;
+                for (int i = 0; i < D; ++i) acc = fma((double)a.R[lane * D + i], (double)sRow[i], acc);
+                bit = acc >= 0.0;
+            }
+            __syncwarp();   // sRow is reused by the warp's next entry
+        }
+        const uint32_t code = __ballot_sync(0xffffffffu, lane < c.nbits && bit);
+        const unsigned nre = __popc(__ballot_sync(0xffffffffu, need));
         if (lane == 0) {
             c.knorm64[e] = n64;
             c.kspan[e] = (uint8_t)span;
-            atomicMax(reinterpret_cast<int*>(&c.kmax2[h]), __float_as_int(ks2 * (1.f + 1.f / 1024.f)));
+            bound_max(sKm, &c.kmax2[h], h, ks2 * (1.f + 1.f / 1024.f));
             if (nre) atomicAdd(&a.stats->hash_rechecks, (unsigned long long)nre);
             const uint32_t oc = c.code[e];
             if (code != oc) {   // the entry leaves its bucket after this commit
@@ -1141,7 +1217,7 @@ __device__ void merge_entry_warp(const CommitArgs<E, D, MEAN>& a, int h, int j, 
         c.cnt[e] = ntot;
         c.bias2[e] = log2f(ft);
         c.lhead[e] = -1;
-        atomicMax(reinterpret_cast<int*>(&c.bmax[h]), __float_as_int(log2f(ft)));   // log2 n >= 0
+        bound_max(sBm, &c.bmax[h], h, log2f(ft));   // log2 n >= 0
     }
     __syncwarp();
 }
@@ -1151,7 +1227,7 @@ __device__ void merge_entry_warp(const CommitArgs<E, D, MEAN>& a, int h, int j, 
 // list with running-mean keys) go to the whole warp afterwards.
 template <typename E, int D, bool MEAN>
 __device__ __forceinline__ void merge_quad(const CommitArgs<E, D, MEAN>& a, int64_t q4, int32_t* sIds,
-                                           int32_t* sSorted, float* sRow, int lane) {
+                                           int32_t* sSorted, float* sRow, float* sBm, float* sKm, int lane) {
     const CacheView& c = a.c;
     const StageView& s = a.s;
     using G = GSlice<E, D>;
@@ -1230,7 +1306,7 @@ __device__ __forceinline__ void merge_quad(const CommitArgs<E, D, MEAN>& a, int6
                 c.cnt[e] = ntot;
                 c.bias2[e] = log2f(ft);
                 c.lhead[e] = -1;
-                atomicMax(reinterpret_cast<int*>(&c.bmax[h]), __float_as_int(log2f(ft)));   // log2 n >= 0
+                bound_max(sBm, &c.bmax[h], h, log2f(ft));   // log2 n >= 0
             }
         }
     }
@@ -1241,7 +1317,7 @@ __device__ __forceinline__ void merge_quad(const CommitArgs<E, D, MEAN>& a, int6
         bigm &= bigm - 1;
         const int bh = __shfl_sync(0xffffffffu, h, src);
         const int bj = __shfl_sync(0xffffffffu, j, src);
-        merge_entry_warp<E, D, MEAN>(a, bh, bj, sIds, sSorted, sRow, lane);
+        merge_entry_warp<E, D, MEAN>(a, bh, bj, sIds, sSorted, sRow, sBm, sKm, lane);
     }
 }
 
@@ -1276,10 +1352,13 @@ __global__ void __launch_bounds__(kWarps * 32, 2) commit_kernel(const CommitArgs
     __shared__ int32_t sIds[kWarps][kListSmem];
     __shared__ int32_t sSorted[kWarps][kListSmem];
     __shared__ float sRow[kWarps][MEAN ? D : 1];   // running-mean keys: the new key, for the re-hash
+    __shared__ float sBm[kHeadSlots], sKm[kHeadSlots];   // this block's bounds of log2 n and |k|^2 per head
     const CacheView& c = a.c;
     const StageView& s = a.s;
     const int H = c.H;
     if (__ldcg(&a.ctr[2 * H])) return;   // refused: nothing changes, the decisions stay for a retry
+    for (int i = threadIdx.x; i < kHeadSlots; i += blockDim.x) sBm[i] = sKm[i] = 0.f;
+    __syncthreads();
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     const int64_t T = s.T;
     const int64_t nA = (int64_t)H * ((T + 31) >> 5);
@@ -1291,8 +1370,13 @@ __global__ void __launch_bounds__(kWarps * 32, 2) commit_kernel(const CommitArgs
             const int64_t nwin = (T + 31) >> 5;
             append_window<E, D>(c, s, (int)(it / nwin), (int)(it % nwin), sSrc[wib], lane);
         } else {
-            merge_quad<E, D, MEAN>(a, (it - nA) * 4, sIds[wib], sSorted[wib], sRow[wib], lane);
+            merge_quad<E, D, MEAN>(a, (it - nA) * 4, sIds[wib], sSorted[wib], sRow[wib], sBm, sKm, lane);
         }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < H && i < kHeadSlots; i += blockDim.x) {
+        if (sBm[i] > 0.f) atomicMax(reinterpret_cast<int*>(&c.bmax[i]), __float_as_int(sBm[i]));
+        if (sKm[i] > 0.f) atomicMax(reinterpret_cast<int*>(&c.kmax2[i]), __float_as_int(sKm[i]));
     }
     grid_dependents_launch();
     commit_done(c, a.ctr, 2 * H + 2, true, true, !MEAN);
@@ -1384,8 +1468,8 @@ cudaError_t stage_n(const CacheView& c, const StageView& s, const void* K, const
         pl.rn[b] = b < c.nbits ? Rnorm_host[b] : 0.f;
     }
     const int64_t items = (int64_t)c.H * ((s.T + 31) / 32);
-    const int grid = grid_for_rows(items > s.TmaxP / kWarps ? items : s.TmaxP / kWarps, kWarps, 148 * 2);
-    e = launch_pdl_smem(kern, grid, kWarps * 32, smem, st, reinterpret_cast<const E*>(K),
+    const int grid = grid_for_rows(items, kStageWarps, 148 * 4);
+    e = launch_pdl_smem(kern, grid, kStageWarps * 32, smem, st, reinterpret_cast<const E*>(K),
                         reinterpret_cast<const E*>(V), c, s, R, pl, tau, ctr, stats);
     *launches += 1;
     if (e == cudaSuccess && INTRA) {
