@@ -852,9 +852,9 @@ cudaError_t launch_sparse_t(int H, const SparseArgs& sp, const AttnMaps& m, int6
 }
 
 // Frame-masked attention over token-major Q, K, V: grid (T frames x tiles per frame, H), a
-// programmatic dependent of the kernel that lists the tiles. `big` holds H floats of +inf
-// (the per-head key-norm bound, read as big[h]) and `zeros` H zeros: with no bound of the
-// key norms the kernel always takes the running softmax reference.
+// programmatic dependent of the kernels that list the tiles and bound the keys. `big` holds
+// the per-head bound of |k|^2 (read as big[h]) and `zeros` H zeros (no group sizes, no
+// staged keys): rows whose logit bound stays small take the fixed softmax reference.
 template <int D>
 cudaError_t launch_frames_t(int H, const FrameArgs& fa, const AttnMaps& m, int T, int P, const float* big,
                             const float* zeros, __nv_bfloat16* out, float scale_log2, Stats* stats,

@@ -421,7 +421,24 @@ stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView 
         uint32_t code = 0;
         int spx = 255;
         float n2 = 0.f;
-        if (valid) {
+        if (valid && sizeof(E) == 4) {   // fp32 storage (small workloads): plain loops
+            for (int i = 0; i < D; ++i) n2 = fmaf(srow_at<E>(my, i), srow_at<E>(my, i), n2);
+            const float nx = sqrtf(n2);
+            for (int b = 0; b < nbits; ++b) {
+                float a = 0.f;
+                for (int i = 0; i < D; ++i) a = fmaf(sR[b * D + i], srow_at<E>(my, i), a);
+                bool bit = a >= 0.f;
+                if (!(fabsf(a) > gam2 * pl.rn[b] * nx + 1e-30f)) {
+                    double s64 = 0.0;
+                    for (int i = 0; i < D; ++i) s64 = fma((double)R[b * D + i], (double)srow_at<E>(my, i), s64);
+                    bit = s64 >= 0.0;
+                    ++hre;
+                }
+                code |= (uint32_t)bit << b;
+            }
+            s.scode[sbase + lane] = code;
+            kmax = fmaxf(kmax, n2);
+        } else if (valid) {
             float acc[NBP];
 #pragma unroll
             for (int b = 0; b < NBP; ++b) acc[b] = 0.f;
@@ -1484,6 +1501,8 @@ template <typename E, int D, bool INTRA, bool MEAN>
 cudaError_t stage_t(const CacheView& c, const StageView& s, const void* K, const void* V, const float* R,
                     const float* Rhost, const float* Rnorm_host, float tau, int32_t* ctr, Stats* stats,
                     int* launches, cudaStream_t st) {
+    if constexpr (sizeof(E) == 4)   // fp32 storage hashes with plain loops: one width of normals
+        return stage_n<E, D, 32, INTRA, MEAN>(c, s, K, V, R, Rhost, Rnorm_host, tau, ctr, stats, launches, st);
     if (c.nbits <= 8)
         return stage_n<E, D, 8, INTRA, MEAN>(c, s, K, V, R, Rhost, Rnorm_host, tau, ctr, stats, launches, st);
     if (c.nbits <= 16)

@@ -12,8 +12,10 @@
 //
 // Kernels: lvsa_tiles_kernel (one thread per query frame) builds A(t) and the list of
 // token-major key tiles covering it (each run of consecutive frames tiled from its first
-// row); the attention kernel of tc_attn_bf16.cu in its frame mode then runs each query
-// frame's rows against its tiles, rows past a run's end shifted by -inf.
+// row); lvsa_kbound_kernel bounds |k|^2 per head over the call's keys; the attention
+// kernel of tc_attn_bf16.cu in its frame mode then runs each query frame's rows against its
+// tiles, rows past a run's end shifted by -inf, with the fixed softmax reference whenever
+// the rows' logit bounds allow it.
 #include "../../include/tempcache.h"
 #include "tc_internal.h"
 
@@ -68,6 +70,47 @@ __global__ void lvsa_tiles_kernel(int T, int P, int T_per, int C, int s, int max
     nframes[t] = n;
 }
 
+// Upper bound of |k|^2 per head over the keys K [N, H, d] (bf16), rounded up past the fp32
+// sums' error: the attention kernel's fixed softmax reference needs it. Each block takes one
+// contiguous range of rows r = n H + h (W = d / 8 lanes per row) and gathers its heads'
+// maxima in shared memory, one atomic per head and block.
+template <int D>
+__global__ void __launch_bounds__(256) lvsa_kbound_kernel(const __nv_bfloat16* __restrict__ K, int64_t rows, int H,
+                                                          float* kmax2) {
+    constexpr int W = D / 8, RPW = 32 / W, kSlots = 64;
+    __shared__ float sK[kSlots];
+    for (int i = threadIdx.x; i < kSlots; i += blockDim.x) sK[i] = 0.f;
+    __syncthreads();
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5, sub = lane / W, w = lane % W;
+    const int64_t per = ((rows + gridDim.x - 1) / gridDim.x + RPW - 1) / RPW * RPW;
+    const int64_t r0 = (int64_t)blockIdx.x * per, r1 = min(rows, r0 + per);
+    const uint4* K4 = reinterpret_cast<const uint4*>(K);
+    for (int64_t rr = r0 + (int64_t)wib * RPW; rr < r1; rr += (int64_t)(blockDim.x >> 5) * RPW) {   // warp-uniform
+        const int64_t r = rr + sub;
+        float kk = 0.f;
+        if (r < r1) {
+            const uint4 v = K4[r * W + w];
+            const uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float lo = __uint_as_float(wd[e] << 16), hi = __uint_as_float(wd[e] & 0xffff0000u);
+                kk = fmaf(lo, lo, fmaf(hi, hi, kk));
+            }
+        }
+#pragma unroll
+        for (int o = 1; o < W; o <<= 1) kk += __shfl_xor_sync(0xffffffffu, kk, o);
+        if (r < r1 && w == 0) {
+            const int h = (int)(r % H);
+            const float kb = kk * (1.f + 1.f / 1024.f);   // floats >= 0 order like their bits
+            if (h < kSlots) atomicMax(reinterpret_cast<int*>(sK + h), __float_as_int(kb));
+            else atomicMax(reinterpret_cast<int*>(kmax2 + h), __float_as_int(kb));
+        }
+    }
+    __syncthreads();
+    for (int h = threadIdx.x; h < H && h < kSlots; h += blockDim.x)
+        if (sK[h] > 0.f) atomicMax(reinterpret_cast<int*>(kmax2 + h), __float_as_int(sK[h]));
+}
+
 }  // namespace
 
 }  // namespace tc
@@ -86,7 +129,8 @@ struct tc_lvsa_ctx {
     float scale = 0.f;
     int device = 0;
     float* masktab = nullptr;   // [129][128]
-    float* consts = nullptr;    // [0, H) = +inf (key-norm bound per head), [H, 2H) = 0
+    float* consts = nullptr;    // [0, H) = 0
+    float* kmax2 = nullptr;     // [H] bound of |k|^2 per head of the last call's keys
     Stats* stats = nullptr;
     int Tcap = 0, maxt = 0;     // frames the tables hold, tiles per frame
     int2* tiles = nullptr;
@@ -106,7 +150,7 @@ struct tc_lvsa_ctx {
     }
     ~tc_lvsa_ctx() {
         free_tables();
-        void* ps[] = {masktab, consts, stats};
+        void* ps[] = {masktab, consts, kmax2, stats};
         for (void* p : ps) if (p) cudaFree(p);
         magic = 0;
     }
@@ -164,13 +208,13 @@ tc_status tc_lvsa_create(int32_t H, int32_t d, int32_t P, int32_t T_per, int32_t
     x->device = dev;
     x->scale = softmax_scale > 0.f ? softmax_scale : (float)(1.0 / std::sqrt((double)d));
     tc_status st;
-    if ((st = grab(x->masktab, 129 * 128 * 4)) || (st = grab(x->consts, (size_t)2 * H * 4)) ||
+    if ((st = grab(x->masktab, 129 * 128 * 4)) || (st = grab(x->consts, (size_t)H * 4)) ||
+        (st = grab(x->kmax2, (size_t)H * 4)) ||
         (st = grab(x->stats, sizeof(Stats)))) {
         delete x;
         return st;
     }
-    std::vector<float> c(2 * (size_t)H, 0.f);
-    std::fill(c.begin(), c.begin() + H, INFINITY);
+    std::vector<float> c((size_t)H, 0.f);
     cudaError_t e;
     if ((e = cudaMemcpy(x->consts, c.data(), c.size() * 4, cudaMemcpyHostToDevice)) ||
         (e = cudaMemset(x->stats, 0, sizeof(Stats)))) {
@@ -231,9 +275,20 @@ tc_status tc_lvsa_attend(tc_lvsa_handle x, const void* Q, const void* K, const v
     lvsa_tiles_kernel<<<(T + 127) / 128, 128, 0, cs>>>(T, x->P, x->T_per, x->C, step, x->maxt, x->tiles, x->count,
                                                        x->nframes, x->frames);
     cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaMemsetAsync(x->kmax2, 0, (size_t)x->H * 4, cs);
+    if (e == cudaSuccess) {
+        const int64_t rows = N * x->H;
+        const int rpb = 8 * (32 / (x->d / 8));   // rows a 256-thread block takes per step
+        int grid = (int)std::min<int64_t>((rows + rpb - 1) / rpb, 148 * 8);
+        if (x->d == 128)
+            lvsa_kbound_kernel<128><<<grid, 256, 0, cs>>>(static_cast<const __nv_bfloat16*>(K), rows, x->H, x->kmax2);
+        else
+            lvsa_kbound_kernel<64><<<grid, 256, 0, cs>>>(static_cast<const __nv_bfloat16*>(K), rows, x->H, x->kmax2);
+        e = cudaGetLastError();
+    }
     if (e == cudaSuccess) {
         FrameArgs fa{x->tiles, x->count, x->masktab, x->maxt};
-        e = launch_attend_frames_bf16(x->H, x->d, fa, m, T, x->P, x->consts, x->consts + x->H,
+        e = launch_attend_frames_bf16(x->H, x->d, fa, m, T, x->P, x->kmax2, x->consts,
                                       static_cast<__nv_bfloat16*>(out),
                                       (float)((double)x->scale * 1.4426950408889634), x->stats, cs);
     }
