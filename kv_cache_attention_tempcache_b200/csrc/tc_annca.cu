@@ -600,6 +600,109 @@ __global__ void __launch_bounds__(1024) annsa_count_kernel(SparseBufs b, int nbi
     }
 }
 
+// The same order for codes of at most kSegBits bits without serialising the warps: each
+// of the 32 warps takes one contiguous segment of the tokens and counts its segment's codes
+// in its own row of a [32][2^nbits] table; a column scan turns the table into each warp's
+// first position per code (bucket start + the counts of the earlier segments), and every
+// warp then places its tokens in order, ranking equal codes inside each 32-token step with
+// a match mask. Positions fit 16 bits (T <= kMaxSparseT).
+constexpr int kSegBits = 10;
+
+__global__ void __launch_bounds__(1024) annsa_segcount_kernel(SparseBufs b, int nbits) {
+    extern __shared__ uint16_t sg_smem[];
+    const int ncodes = 1 << nbits;
+    uint16_t* hist = sg_smem;                                                   // [32][ncodes]
+    int32_t* cstart = reinterpret_cast<int32_t*>(sg_smem + 32 * ncodes);         // [ncodes]
+    int32_t* ccount = cstart + ncodes;                                          // [ncodes]
+    __shared__ int wsum[32];
+    const int h = blockIdx.x, T = (int)b.T;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const unsigned lt = (1u << lane) - 1u;
+    for (int i = threadIdx.x; i < 32 * ncodes; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    const int seg = (T + 31) / 32, t0 = min(T, warp * seg), t1 = min(T, t0 + seg);
+    for (int base = t0; base < t1; base += 32) {   // warp-uniform
+        const int t = base + lane;
+        const bool valid = t < t1;
+        const uint32_t c = valid ? b.codes[(int64_t)t * b.H + h] : 0xffffffffu;
+        const unsigned same = __match_any_sync(0xffffffffu, c);
+        if (valid && lane == __ffs(same) - 1) hist[warp * ncodes + c] += (uint16_t)__popc(same);
+        __syncwarp();
+    }
+    __syncthreads();
+    // bucket sizes, their exclusive scan (bucket starts), then per code the first position of
+    // every warp's segment
+    const int per = (ncodes + blockDim.x - 1) / blockDim.x;
+    const int c0 = min(ncodes, (int)threadIdx.x * per), c1 = min(ncodes, c0 + per);
+    int run = 0;
+    for (int c = c0; c < c1; ++c) {
+        int tot = 0;
+        for (int w = 0; w < 32; ++w) tot += hist[w * ncodes + c];
+        ccount[c] = tot;
+        run += tot;
+    }
+    int inc = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+    }
+    if (lane == 31) wsum[warp] = inc;
+    __syncthreads();
+    if (warp == 0) {
+        int y = wsum[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int z = __shfl_up_sync(0xffffffffu, y, o);
+            if (lane >= o) y += z;
+        }
+        wsum[lane] = y;
+    }
+    __syncthreads();
+    int pos = (warp > 0 ? wsum[warp - 1] : 0) + inc - run;
+    for (int c = c0; c < c1; ++c) {
+        cstart[c] = pos;
+        int cur = pos;
+        for (int w = 0; w < 32; ++w) {
+            const int n = hist[w * ncodes + c];
+            hist[w * ncodes + c] = (uint16_t)cur;   // warp w's next position for code c
+            cur += n;
+        }
+        pos += ccount[c];
+    }
+    __syncthreads();
+    for (int base = t0; base < t1; base += 32) {   // warp-uniform
+        const int t = base + lane;
+        const bool valid = t < t1;
+        const uint32_t c = valid ? b.codes[(int64_t)t * b.H + h] : 0xffffffffu;
+        const unsigned same = __match_any_sync(0xffffffffu, c);
+        const int lead = __ffs(same) - 1;
+        int first = 0;
+        if (valid && lane == lead) {
+            first = hist[warp * ncodes + c];
+            hist[warp * ncodes + c] = (uint16_t)(first + __popc(same));
+        }
+        first = __shfl_sync(0xffffffffu, first, lead);
+        if (valid) {
+            const int64_t o = (int64_t)h * b.Tp + first + __popc(same & lt);
+            b.perm[o] = t;
+            b.grp[o] = c;
+        }
+        __syncwarp();
+    }
+    for (int64_t i = T + threadIdx.x; i < b.Tp; i += blockDim.x) {
+        b.perm[(int64_t)h * b.Tp + i] = -1;
+        b.grp[(int64_t)h * b.Tp + i] = 0xffffffffu;
+    }
+    __syncthreads();   // (this block's own global writes, read back below)
+    const int nqt = (int)(b.Tp / 128);
+    for (int k = threadIdx.x; k < (T + 127) / 128; k += blockDim.x) {
+        const int f = 128 * k, l = min(f + 127, T - 1);
+        const uint32_t cf = b.grp[(int64_t)h * b.Tp + f], cl = b.grp[(int64_t)h * b.Tp + l];
+        b.tiles[(int64_t)h * nqt + k] = make_int2(cstart[cf] / 128, (cstart[cl] + ccount[cl] + 127) / 128);
+    }
+}
+
 // One warp per packed row r = h Tp + i: copy the token's q, k, v rows (zeros past T),
 // its own logit scale log2(e) <q, k> (the first softmax reference when the kernel cannot
 // use a fixed one) and the head's bound of |k|^2.
@@ -683,7 +786,12 @@ cudaError_t e = smem_attr_once(reinterpret_cast<const void*>(annsa_order_kernel)
     if (e == cudaSuccess)
         e = smem_attr_once(reinterpret_cast<const void*>(annsa_count_kernel), (2 << kCountBits) * 4 + 32 * 32 * 4);
     if (e != cudaSuccess) return e;
-    if (nbits <= kCountBits) {
+    if (nbits <= kSegBits) {
+        const int smem = 32 * (2 << nbits) + 8 * (1 << nbits);   // [32][2^nbits] u16 + two [2^nbits] i32
+        e = smem_attr_once(reinterpret_cast<const void*>(annsa_segcount_kernel), 32 * (2 << kSegBits) + 8 * (1 << kSegBits));
+        if (e != cudaSuccess) return e;
+        annsa_segcount_kernel<<<b.H, 1024, smem, st>>>(b, nbits);
+    } else if (nbits <= kCountBits) {
         annsa_count_kernel<<<b.H, 1024, (2 << nbits) * 4 + 32 * 32 * 4, st>>>(b, nbits);
     } else {
         int n = 1;

@@ -62,6 +62,11 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// One arrival worth `count` (a warp arriving for its lanes after a __syncwarp).
+__device__ __forceinline__ void mbar_arrive_n(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
     uint32_t done;
     asm volatile(
@@ -244,10 +249,13 @@ struct CfgU {
 // One CTA = 128 query rows of one head.
 //   TMEM: score buffers S_b = [128 b, 128 b + 128) (tile i uses b = i mod 3) and one
 //         output accumulator O = [384, 384 + D).
-//   warps 0-15  softmax, two teams of eight warps: team t takes tiles t, t + 2, ...;
-//               thread (t, g, r) owns columns [64 g, 64 g + 64) of query row r (TMEM
-//               lane r), so every SM sub-partition runs two warps of each team and the
-//               teams' phases interleave. Per tile the halves agree on an upper bound of
+//   warps 0-15  softmax. With the fixed reference (every row's logit bound <= 60, the
+//               common case) all sixteen warps take every tile: thread (t, g, r) owns key
+//               columns [32 (2 t + g), 32 (2 t + g) + 32) of query row r (TMEM lane r).
+//               Otherwise two teams of eight warps: team t takes tiles t, t + 2, ...;
+//               thread (t, g, r) owns columns [64 g, 64 g + 64) of query row r, so every
+//               SM sub-partition runs two warps of each team and the teams' phases
+//               interleave. Per tile the halves agree on an upper bound of
 //               the row max (max raw score * scale + max log2 n) at a team barrier.
 //               The reference m is shared by both teams and changes lazily: tile i keeps
 //               the reference of tile i - 1 (published by the other team through shared
@@ -463,11 +471,12 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         mbar_wait(&bars[U_DRAIN], 0);
     } else if (warp == kWPV && lane == 0) {
         // ---------------------------------------------------------------- PV issuer
-        // O += P_i V_i; keys [16 kk, 16 kk + 16) of P sit at column 128 b + 64 (kk / 4) +
-        // 8 (kk % 4): each half's probabilities over its own first S columns.
-        // With the fixed reference the keys of half 0 go in as soon as that half's P is
-        // written; with the online reference a tile may rescale all of O first, so both
-        // halves must be done.
+        // O += P_i V_i. With the online reference keys [16 kk, 16 kk + 16) of P sit at
+        // column 128 b + 64 (kk / 4) + 8 (kk % 4), each half's probabilities over its own
+        // first S columns, and both halves must be done (a tile may rescale all of O
+        // first). With the fixed reference they sit at 128 b + 32 (kk / 2) + 8 (kk % 2),
+        // each quarter's over its own first columns, and the keys of quarters 0-1 go in as
+        // soon as those are written.
         const uint32_t aV = smem_u32(sV);
         bool ok = true, fixed = false;
         for (int i = 0; i < ntiles && !*abort_flag; ++i) {
@@ -484,8 +493,9 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
                     if (!mbar_wait(&bars[U_PFULL + 2 * b + 1], (i / 3) & 1)) { ok = false; break; }
                     tc_fence_after();
                 }
-                mma_ts(tO, tmem + b * 128 + 64 * (kk >> 2) + 8 * (kk & 3), sdesc(aVs + kk * 2048, C::BOX, 1024),
-                       C::IDESC_PV, (i > 0 || kk > 0));
+                const uint32_t pcol = fixed ? 32 * (kk >> 1) + 8 * (kk & 1) : 64 * (kk >> 2) + 8 * (kk & 3);
+                mma_ts(tO, tmem + b * 128 + pcol, sdesc(aVs + kk * 2048, C::BOX, 1024), C::IDESC_PV,
+                       (i > 0 || kk > 0));
             }
             if (!ok) break;
             tc_commit(&bars[U_VEMPTY + st]);
@@ -552,56 +562,59 @@ attend_bf16_duo_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_con
         const bool fixed = bar_and(3, 512, ok && mfix <= 60.f);   // uniform over the CTA
         if (threadIdx.x == 0) *sFixed = fixed ? 1 : 0;             // before thread 0's first P
         if (fixed) {
+            // No max pass and no agreement between threads: all sixteen warps take every
+            // tile, thread (t, g, r) the key columns [32 (2 t + g), 32 (2 t + g) + 32) of row
+            // r, so a tile's exponentials spread over the whole SM. P goes over the first 16
+            // columns of each quarter; the PV issuer starts the keys of quarters 0-1 (team 0)
+            // once those are written.
             m_run = mfix;
             const uint64_t negm2 = pk2(-mfix, -mfix);
+            const int qc = 32 * (2 * t + g);
             auto bias_row = [&](int i) -> const float* {
-                if constexpr (FRAMES) return fa.masktab + ftab[i].y * kBN + 64 * g;
-                return ((i < nc) ? bias_h + (int64_t)i * kBN : sbias + (int64_t)(i - nc) * kBN) + 64 * g;
+                if constexpr (FRAMES) return fa.masktab + ftab[i].y * kBN + qc;
+                return ((i < nc) ? bias_h + (int64_t)i * kBN : sbias + (int64_t)(i - nc) * kBN) + qc;
             };
-            if (lane < 2 && t < ntiles) asm volatile("prefetch.global.L1 [%0];" ::"l"(bias_row(t) + 32 * lane));
-            for (int i = t; i < ntiles; i += 2) {
+            if (lane == 0 && ntiles > 0) asm volatile("prefetch.global.L1 [%0];" ::"l"(bias_row(0)));
+            uint64_t sumA = pk2(0.f, 0.f), sumB = pk2(0.f, 0.f);
+            for (int i = 0; i < ntiles; ++i) {
                 const int b = i % 3;
                 const bool got = __all_sync(0xffffffffu, !*abort_flag && mbar_wait(&bars[U_SFULL + b], (i / 3) & 1));
                 if (!got) { ok = false; *abort_flag = 1; break; }
                 tc_fence_after();
-                if (lane < 2 && i + 2 < ntiles)
-                    asm volatile("prefetch.global.L1 [%0];" ::"l"(bias_row(i + 2) + 32 * lane));
-                const uint32_t tS = tmem + b * 128 + 64 * g + lane_base;
+                if (lane == 0 && i + 1 < ntiles) asm volatile("prefetch.global.L1 [%0];" ::"l"(bias_row(i + 1)));
+                const uint32_t tS = tmem + b * 128 + qc + lane_base;
                 const float4* brow = reinterpret_cast<const float4*>(bias_row(i));   // (codes when sparse)
-                uint64_t sumA = pk2(0.f, 0.f), sumB = pk2(0.f, 0.f);
-#pragma unroll 1
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    uint32_t sr[32];
-                    TC_LD32(tS + 32 * h2, sr);
-                    tc_wait_ld();
-                    uint32_t pk[16];
+                uint32_t sr[32];
+                TC_LD32(tS, sr);
+                tc_wait_ld();
+                uint32_t pk[16];
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4) {
-                        float4 b4 = __ldg(brow + 8 * h2 + j / 4);
-                        if constexpr (SPARSE) b4 = mask4(b4, gq);
-                        const uint64_t x01 = fma2(pk2(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), c2,
-                                                  add2(pk2(b4.x, b4.y), negm2));
-                        const uint64_t x23 = fma2(pk2(__uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3])), c2,
-                                                  add2(pk2(b4.z, b4.w), negm2));
-                        float a0, a1, a2, a3;
-                        up2(x01, a0, a1);
-                        up2(x23, a2, a3);
-                        const float p0 = ex2(a0), p1 = ex2(a1), p2 = ex2(a2), p3 = ex2(a3);
-                        sumA = add2(sumA, pk2(p0, p1));
-                        sumB = add2(sumB, pk2(p2, p3));
-                        pk[j / 2] = cvt_bf16x2(p0, p1);
-                        pk[j / 2 + 1] = cvt_bf16x2(p2, p3);
-                    }
-                    TC_ST16(tS + 16 * h2, pk);
+                for (int j = 0; j < 32; j += 4) {
+                    float4 b4 = __ldg(brow + j / 4);
+                    if constexpr (SPARSE) b4 = mask4(b4, gq);
+                    const uint64_t x01 = fma2(pk2(__uint_as_float(sr[j]), __uint_as_float(sr[j + 1])), c2,
+                                              add2(pk2(b4.x, b4.y), negm2));
+                    const uint64_t x23 = fma2(pk2(__uint_as_float(sr[j + 2]), __uint_as_float(sr[j + 3])), c2,
+                                              add2(pk2(b4.z, b4.w), negm2));
+                    float a0, a1, a2, a3;
+                    up2(x01, a0, a1);
+                    up2(x23, a2, a3);
+                    const float p0 = ex2(a0), p1 = ex2(a1), p2 = ex2(a2), p3 = ex2(a3);
+                    sumA = add2(sumA, pk2(p0, p1));
+                    sumB = add2(sumB, pk2(p2, p3));
+                    pk[j / 2] = cvt_bf16x2(p0, p1);
+                    pk[j / 2 + 1] = cvt_bf16x2(p2, p3);
                 }
-                float s0, s1, s2, s3;
-                up2(sumA, s0, s1);
-                up2(sumB, s2, s3);
-                l_run += (s0 + s1) + (s2 + s3);
+                TC_ST16(tS, pk);
                 tc_wait_st();
                 tc_fence_before();
-                mbar_arrive(&bars[U_PFULL + 2 * b + g]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive_n(&bars[U_PFULL + 2 * b + t], 16);   // 8 warps x 16 = 128
             }
+            float s0, s1, s2, s3;
+            up2(sumA, s0, s1);
+            up2(sumB, s2, s3);
+            l_run = (s0 + s1) + (s2 + s3);
         } else {
         float bnext = 0.f;
         if (g == 0) {

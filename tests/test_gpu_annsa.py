@@ -62,6 +62,15 @@ def test_mostly_singleton_buckets():
     assert sum((s == 1).sum() for s in sizes[0]) > 0
 
 
+@pytest.mark.parametrize("nbits", [10, 12, 14])
+def test_every_ordering_path(nbits):
+    # codes of <= 10 bits are ordered by per-warp segment counts, <= 13 by one shared count,
+    # wider ones by a sort; a ragged token count (2 x 700) in each
+    cfg = CROSS_CONFIGS["annca-tiny"].replace(H=2, d=128, P=700, F=2, nbits=nbits, sigma=0.5,
+                                              seed=3020 + nbits)
+    run(cfg)
+
+
 def test_large_logits_take_the_running_reference():
     # |q| max|k| scale log2(e) ~ 130 > 60: the kernel cannot use the fixed softmax
     # reference and starts each row's running reference at its own logit
