@@ -463,6 +463,16 @@ cudaError_t select_t(const AnnView& a, const void* Qv, int64_t Tq, int P, int F,
 
 constexpr int kMaxSparseT = 16384;   // tokens per block (the ordering sorts in shared memory)
 
+// Start of every ordering kernel (one block per head h, launched as a programmatic
+// dependent of the previous kernel in the stream, which may be the previous call's
+// attention reading the arrays rewritten here): wait for it, clear the head's key bound
+// for the packing kernel, and let the packing kernel be scheduled.
+__device__ __forceinline__ void order_prologue(const SparseBufs& b, int h) {
+    grid_dependency_wait();
+    if (threadIdx.x == 0) b.kmax2[h] = 0.f;
+    grid_dependents_launch();
+}
+
 // One block per head: bitonic sort of (code, token); per packed row its token and code;
 // per query tile the key tiles from the start of its first row's bucket to the end of its
 // last row's bucket.
@@ -470,6 +480,7 @@ __global__ void __launch_bounds__(1024) annsa_order_kernel(SparseBufs b) {
     extern __shared__ unsigned long long okey[];
     const int h = blockIdx.x;
     const int T = (int)b.T;
+    order_prologue(b, h);
     int n = 1;
     while (n < T) n <<= 1;
     for (int i = threadIdx.x; i < n; i += blockDim.x)
@@ -532,6 +543,7 @@ __global__ void __launch_bounds__(1024) annsa_count_kernel(SparseBufs b, int nbi
     __shared__ int wsum[32];
     const int h = blockIdx.x, T = (int)b.T;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    order_prologue(b, h);
     for (int c = threadIdx.x; c < ncodes; c += blockDim.x) cnt[c] = 0;
     __syncthreads();
     for (int t = threadIdx.x; t < T; t += blockDim.x) atomicAdd(&cnt[b.codes[(int64_t)t * b.H + h]], 1);
@@ -600,45 +612,95 @@ __global__ void __launch_bounds__(1024) annsa_count_kernel(SparseBufs b, int nbi
     }
 }
 
-// The same order for codes of at most kSegBits bits without serialising the warps: each
-// of the 32 warps takes one contiguous segment of the tokens and counts its segment's codes
-// in its own row of a [32][2^nbits] table; a column scan turns the table into each warp's
-// first position per code (bucket start + the counts of the earlier segments), and every
-// warp then places its tokens in order, ranking equal codes inside each 32-token step with
-// a match mask. Positions fit 16 bits (T <= kMaxSparseT).
+// The same order for codes of at most kSegBits bits, spread over kOrdBlocks blocks per head
+// in two kernels. Block (h, j) owns the contiguous token range [j S, j S + S), S =
+// ceil(T / kOrdBlocks). The first kernel counts each code over every block's range; the
+// second sums, per code, all blocks' counts (the bucket size) and the earlier blocks' ones
+// (this block's offset inside the bucket), scans the bucket sizes into bucket starts, counts
+// its range again per warp (each warp a contiguous sub-range, one 16-byte row of eight
+// counts per code) and places its tokens in order, ranking equal codes inside each 32-token
+// step with a match mask. Positions fit 16 bits (T <= kMaxSparseT).
 constexpr int kSegBits = 10;
+constexpr int kOrdBlocks = 8;
+constexpr int kOrdSteps = kMaxSparseT / kOrdBlocks / 8 / 32;   // 32-token steps of one warp's sub-range, at most
 
-__global__ void __launch_bounds__(1024) annsa_segcount_kernel(SparseBufs b, int nbits) {
-    extern __shared__ uint16_t sg_smem[];
-    const int ncodes = 1 << nbits;
-    uint16_t* hist = sg_smem;                                                   // [32][ncodes]
-    int32_t* cstart = reinterpret_cast<int32_t*>(sg_smem + 32 * ncodes);         // [ncodes]
-    int32_t* ccount = cstart + ncodes;                                          // [ncodes]
-    __shared__ int wsum[32];
-    const int h = blockIdx.x, T = (int)b.T;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const unsigned lt = (1u << lane) - 1u;
-    for (int i = threadIdx.x; i < 32 * ncodes; i += blockDim.x) hist[i] = 0;
+__device__ __forceinline__ void ord_range(int T, int j, int& a, int& e) {
+    const int S = (T + kOrdBlocks - 1) / kOrdBlocks;
+    a = min(T, j * S);
+    e = min(T, a + S);
+}
+
+__device__ __forceinline__ int ord_code_at(const int32_t* cstart, int ncodes, int f) {
+    int lo = 0, hi = ncodes;   // the last code whose bucket starts at or before packed row f
+    while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (cstart[mid] <= f) lo = mid + 1;
+        else hi = mid;
+    }
+    return lo - 1;
+}
+
+__global__ void __launch_bounds__(256) annsa_bcount_kernel(SparseBufs b, int nbits) {
+    extern __shared__ int32_t bc_smem[];   // [ncodes]
+    const int ncodes = 1 << nbits, h = blockIdx.x / kOrdBlocks, j = blockIdx.x % kOrdBlocks;
+    order_prologue(b, h);
+    for (int c = threadIdx.x; c < ncodes; c += blockDim.x) bc_smem[c] = 0;
     __syncthreads();
-    const int seg = (T + 31) / 32, t0 = min(T, warp * seg), t1 = min(T, t0 + seg);
-    for (int base = t0; base < t1; base += 32) {   // warp-uniform
-        const int t = base + lane;
-        const bool valid = t < t1;
-        const uint32_t c = valid ? b.codes[(int64_t)t * b.H + h] : 0xffffffffu;
+    int a, e;
+    ord_range((int)b.T, j, a, e);
+    for (int t = a + threadIdx.x; t < e; t += blockDim.x) atomicAdd(&bc_smem[b.codes[(int64_t)t * b.H + h]], 1);
+    __syncthreads();
+    int32_t* dst = b.bcnt + ((int64_t)h * kOrdBlocks + j) * ncodes;
+    for (int c = threadIdx.x; c < ncodes; c += blockDim.x) dst[c] = bc_smem[c];
+}
+
+__global__ void __launch_bounds__(256) annsa_bplace_kernel(SparseBufs b, int nbits) {
+    extern __shared__ __align__(16) int32_t bp_smem[];
+    const int ncodes = 1 << nbits, h = blockIdx.x / kOrdBlocks, j = blockIdx.x % kOrdBlocks;
+    int32_t* cstart = bp_smem;                                       // [ncodes] bucket start
+    int32_t* ctot = cstart + ncodes;                                 // [ncodes] bucket size
+    uint16_t* wh = reinterpret_cast<uint16_t*>(ctot + ncodes);       // [ncodes][8] per-warp counts
+    __shared__ int wsum[8];
+    const int T = (int)b.T, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const unsigned lt = (1u << lane) - 1u;
+    grid_dependency_wait();   // the counts of every block
+    grid_dependents_launch();
+    int a, e;
+    ord_range(T, j, a, e);
+    const int sub = (e - a + 7) / 8, w0 = min(e, a + warp * sub), w1 = min(e, w0 + sub);
+    uint32_t cc[kOrdSteps];
+#pragma unroll
+    for (int k = 0; k < kOrdSteps; ++k) {
+        const int t = w0 + 32 * k + lane;
+        cc[k] = (t < w1) ? b.codes[(int64_t)t * b.H + h] : 0xffffffffu;
+    }
+    for (int i = threadIdx.x; i < ncodes; i += blockDim.x) reinterpret_cast<uint4*>(wh)[i] = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < kOrdSteps; ++k) {
+        if (w0 + 32 * k >= w1) break;   // warp-uniform
+        const uint32_t c = cc[k];
+        const bool valid = w0 + 32 * k + lane < w1;
         const unsigned same = __match_any_sync(0xffffffffu, c);
-        if (valid && lane == __ffs(same) - 1) hist[warp * ncodes + c] += (uint16_t)__popc(same);
+        if (valid && lane == __ffs(same) - 1) wh[c * 8 + warp] += (uint16_t)__popc(same);
         __syncwarp();
     }
-    __syncthreads();
-    // bucket sizes, their exclusive scan (bucket starts), then per code the first position of
-    // every warp's segment
+    // per code: bucket size and this block's offset in it from the blocks' counts; the bucket
+    // starts by a block scan (consecutive codes per thread)
     const int per = (ncodes + blockDim.x - 1) / blockDim.x;
     const int c0 = min(ncodes, (int)threadIdx.x * per), c1 = min(ncodes, c0 + per);
+    const int32_t* cnt = b.bcnt + (int64_t)h * kOrdBlocks * ncodes;
     int run = 0;
     for (int c = c0; c < c1; ++c) {
-        int tot = 0;
-        for (int w = 0; w < 32; ++w) tot += hist[w * ncodes + c];
-        ccount[c] = tot;
+        int tot = 0, off = 0;
+#pragma unroll
+        for (int jj = 0; jj < kOrdBlocks; ++jj) {
+            const int n = cnt[jj * ncodes + c];
+            tot += n;
+            off += (jj < j) ? n : 0;
+        }
+        ctot[c] = tot;
+        cstart[c] = off;   // (for now: this block's offset inside the bucket)
         run += tot;
     }
     int inc = run;
@@ -648,39 +710,38 @@ __global__ void __launch_bounds__(1024) annsa_segcount_kernel(SparseBufs b, int 
         if (lane >= o) inc += y;
     }
     if (lane == 31) wsum[warp] = inc;
-    __syncthreads();
-    if (warp == 0) {
-        int y = wsum[lane];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int z = __shfl_up_sync(0xffffffffu, y, o);
-            if (lane >= o) y += z;
-        }
-        wsum[lane] = y;
-    }
-    __syncthreads();
-    int pos = (warp > 0 ? wsum[warp - 1] : 0) + inc - run;
+    __syncthreads();   // (also: every warp's counts)
+    int pos = inc - run;
+    for (int w = 0; w < warp; ++w) pos += wsum[w];
     for (int c = c0; c < c1; ++c) {
+        const int off = cstart[c];
         cstart[c] = pos;
-        int cur = pos;
-        for (int w = 0; w < 32; ++w) {
-            const int n = hist[w * ncodes + c];
-            hist[w * ncodes + c] = (uint16_t)cur;   // warp w's next position for code c
-            cur += n;
+        uint4* row = reinterpret_cast<uint4*>(wh + c * 8);
+        uint4 v = *row;
+        uint32_t wd[4] = {v.x, v.y, v.z, v.w};
+        uint32_t cur = (uint32_t)(pos + off);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {   // warps 2 q and 2 q + 1: their first positions for code c
+            const uint32_t f0 = cur, f1 = f0 + (wd[q] & 0xffffu);
+            cur = f1 + (wd[q] >> 16);
+            wd[q] = f0 | (f1 << 16);
         }
-        pos += ccount[c];
+        *row = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        pos += ctot[c];
     }
     __syncthreads();
-    for (int base = t0; base < t1; base += 32) {   // warp-uniform
-        const int t = base + lane;
-        const bool valid = t < t1;
-        const uint32_t c = valid ? b.codes[(int64_t)t * b.H + h] : 0xffffffffu;
+#pragma unroll
+    for (int k = 0; k < kOrdSteps; ++k) {
+        if (w0 + 32 * k >= w1) break;   // warp-uniform
+        const int t = w0 + 32 * k + lane;
+        const bool valid = t < w1;
+        const uint32_t c = cc[k];
         const unsigned same = __match_any_sync(0xffffffffu, c);
         const int lead = __ffs(same) - 1;
         int first = 0;
         if (valid && lane == lead) {
-            first = hist[warp * ncodes + c];
-            hist[warp * ncodes + c] = (uint16_t)(first + __popc(same));
+            first = wh[c * 8 + warp];
+            wh[c * 8 + warp] = (uint16_t)(first + __popc(same));
         }
         first = __shfl_sync(0xffffffffu, first, lead);
         if (valid) {
@@ -690,16 +751,17 @@ __global__ void __launch_bounds__(1024) annsa_segcount_kernel(SparseBufs b, int 
         }
         __syncwarp();
     }
-    for (int64_t i = T + threadIdx.x; i < b.Tp; i += blockDim.x) {
+    for (int64_t i = T + (int64_t)j * blockDim.x + threadIdx.x; i < b.Tp; i += (int64_t)kOrdBlocks * blockDim.x) {
         b.perm[(int64_t)h * b.Tp + i] = -1;
         b.grp[(int64_t)h * b.Tp + i] = 0xffffffffu;
     }
-    __syncthreads();   // (this block's own global writes, read back below)
+    // per query tile the key tiles from its first row's bucket start to its last row's
+    // bucket end (the rows' codes found from the bucket starts); block j takes tiles j, j + 8, ...
     const int nqt = (int)(b.Tp / 128);
-    for (int k = threadIdx.x; k < (T + 127) / 128; k += blockDim.x) {
+    for (int k = j + kOrdBlocks * (int)threadIdx.x; k < (T + 127) / 128; k += kOrdBlocks * blockDim.x) {
         const int f = 128 * k, l = min(f + 127, T - 1);
-        const uint32_t cf = b.grp[(int64_t)h * b.Tp + f], cl = b.grp[(int64_t)h * b.Tp + l];
-        b.tiles[(int64_t)h * nqt + k] = make_int2(cstart[cf] / 128, (cstart[cl] + ccount[cl] + 127) / 128);
+        const int cf = ord_code_at(cstart, ncodes, f), cl = ord_code_at(cstart, ncodes, l);
+        b.tiles[(int64_t)h * nqt + k] = make_int2(cstart[cf] / 128, (cstart[cl] + ctot[cl] + 127) / 128);
     }
 }
 
@@ -787,18 +849,17 @@ cudaError_t e = smem_attr_once(reinterpret_cast<const void*>(annsa_order_kernel)
         e = smem_attr_once(reinterpret_cast<const void*>(annsa_count_kernel), (2 << kCountBits) * 4 + 32 * 32 * 4);
     if (e != cudaSuccess) return e;
     if (nbits <= kSegBits) {
-        const int smem = 32 * (2 << nbits) + 8 * (1 << nbits);   // [32][2^nbits] u16 + two [2^nbits] i32
-        e = smem_attr_once(reinterpret_cast<const void*>(annsa_segcount_kernel), 32 * (2 << kSegBits) + 8 * (1 << kSegBits));
-        if (e != cudaSuccess) return e;
-        annsa_segcount_kernel<<<b.H, 1024, smem, st>>>(b, nbits);
+        const int ncodes = 1 << nbits;   // shared memory: counts; starts, sizes and [ncodes][8] uint16
+        e = launch_pdl_smem(annsa_bcount_kernel, b.H * kOrdBlocks, 256, ncodes * 4, st, b, nbits);
+        if (e == cudaSuccess)
+            e = launch_pdl_smem(annsa_bplace_kernel, b.H * kOrdBlocks, 256, ncodes * 24, st, b, nbits);
     } else if (nbits <= kCountBits) {
-        annsa_count_kernel<<<b.H, 1024, (2 << nbits) * 4 + 32 * 32 * 4, st>>>(b, nbits);
+        e = launch_pdl_smem(annsa_count_kernel, b.H, 1024, (2 << nbits) * 4 + 32 * 32 * 4, st, b, nbits);
     } else {
         int n = 1;
         while (n < b.T) n <<= 1;
-        annsa_order_kernel<<<b.H, 1024, n * 8, st>>>(b);
+        e = launch_pdl_smem(annsa_order_kernel, b.H, 1024, n * 8, st, b);
     }
-    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const int grid = grid_for_rows((int64_t)b.H * ((b.T + 127) / 128 * 128), kWarps * (32 / (b.d / 8)), 148 * 8);
     const auto* q = reinterpret_cast<const __nv_bfloat16*>(Q);
@@ -895,7 +956,7 @@ struct tc_annca_ctx {
         a.Zmax = 0;
     }
     void free_sparse() {
-        void* ps[] = {sb.perm, sb.grp, sb.tiles, sb.xself, sb.Qs, sb.Ks, sb.Vs};
+        void* ps[] = {sb.perm, sb.grp, sb.tiles, sb.xself, sb.Qs, sb.Ks, sb.Vs, sb.bcnt};
         for (void* p : ps) if (p) cudaFree(p);
         sb = SparseBufs{};
         sp_Tp = 0;
@@ -1177,6 +1238,7 @@ tc_status tc_annsa_attend(tc_annca_handle x, const void* Q, const void* K, const
             (st = x->grab(b.tiles, rows / 128 * sizeof(int2))) || (st = x->grab(b.xself, rows * 4)) ||
             (st = x->grab(b.Qs, rows * x->d * 2)) || (st = x->grab(b.Ks, rows * x->d * 2)) ||
             (st = x->grab(b.Vs, rows * x->d * 2)) ||
+            (x->nbits <= kSegBits && (st = x->grab(b.bcnt, (size_t)x->H * kOrdBlocks * ((size_t)1 << x->nbits) * 4))) ||
             (!x->sp_kmax2 && (st = x->grab(x->sp_kmax2, (size_t)x->H * 4)))) {
             x->free_sparse();
             return st;
@@ -1201,8 +1263,7 @@ tc_status tc_annsa_attend(tc_annca_handle x, const void* Q, const void* K, const
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     x->last_stream = cs;
     const float scale_log2 = (float)((double)x->scale * 1.4426950408889634);
-    cudaError_t e = cudaMemsetAsync(x->sp_kmax2, 0, (size_t)x->H * 4, cs);
-    if (e == cudaSuccess) e = launch_annsa_pack(b, x->nbits, Q, K, V, scale_log2, cs);
+    cudaError_t e = launch_annsa_pack(b, x->nbits, Q, K, V, scale_log2, cs);   // (clears the key bounds first)
     if (e == cudaSuccess) {
         SparseArgs sp{b.tiles, b.grp, b.perm, b.xself, Tp, (int)(Tp / 128)};
         e = launch_attend_sparse_bf16(x->H, x->d, sp, x->sp_maps, T, x->sp_kmax2, x->a.zeros,

@@ -1456,21 +1456,6 @@ __global__ void rebucket_push_kernel(CacheView c, StageView s, int32_t* ctr, int
     commit_done(c, ctr, 2 * H + 3, false, false, true);
 }
 
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl_smem(void (*kern)(KArgs...), int grid, int block, int smem, cudaStream_t st, Args... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3((unsigned)block);
-    cfg.dynamicSmemBytes = (size_t)smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
-}
-
 template <typename E, int D, int NBP, bool INTRA, bool MEAN>
 cudaError_t stage_n(const CacheView& c, const StageView& s, const void* K, const void* V, const float* R,
                     const float* Rhost, const float* Rnorm_host, float tau, int32_t* ctr, Stats* stats,

@@ -92,11 +92,11 @@ __device__ __forceinline__ void grid_dependents_launch() {
 }
 
 template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int block, cudaStream_t st, Args... args) {
+cudaError_t launch_pdl_smem(void (*kern)(KArgs...), int grid, int block, int smem, cudaStream_t st, Args... args) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3((unsigned)block);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -104,6 +104,11 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int block, cudaStream_t
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), int grid, int block, cudaStream_t st, Args... args) {
+    return launch_pdl_smem(kern, grid, block, 0, st, args...);
 }
 
 inline int grid_for_rows(int64_t rows, int per_block, int max_blocks) {

@@ -194,7 +194,8 @@ struct SparseBufs {
     __nv_bfloat16* Qs;      // [H][Tp][d]
     __nv_bfloat16* Ks;
     __nv_bfloat16* Vs;
-    float* kmax2;           // [H], zeroed by the caller
+    float* kmax2;           // [H], cleared by the ordering kernel
+    int32_t* bcnt;          // [H][blocks][2^nbits] per-block code counts of the ordering (short codes)
 };
 cudaError_t launch_annsa_pack(const SparseBufs& b, int nbits, const void* Q, const void* K, const void* V,
                               float scale_log2, cudaStream_t st);
