@@ -10,7 +10,7 @@
 //                         bound |k|^2 per head.
 //   annca_sort_kernel     once per prompt: sort each head's (code, token) pairs; every
 //                         prompt token learns where its code's run starts.
-//   annca_mark_kernel     per call: one lane per query row hashes it, then looks its code
+//   annca_mark_kernel     per call: two lanes per query row hash it, then look its code
 //                         up (a table of the head's codes for nbits <= 16, else a binary
 //                         search of its sorted codes) and, if the prompt has that code,
 //                         stamps the bucket with the call's number for the query's frame
@@ -200,12 +200,12 @@ __device__ __forceinline__ void flag_bucket(const AnnView& a, int h, int64_t z, 
     }
 }
 
-// Shared memory of the mark kernel: per warp 32 staged rows (row stride padded by 16
+// Shared memory of the mark kernel: per warp 16 staged rows (row stride padded by 16
 // bytes so that lanes reading their own rows hit distinct banks).
 template <int D>
 struct MarkSmem {
     static constexpr int RB = D * 2 + 16;
-    static constexpr int BYTES = kWarps * 32 * RB;
+    static constexpr int BYTES = kWarps * 16 * RB;
 };
 
 // The normals as fp32 [NBP][D] (zero rows past nbits) and their rounded-up norms, passed
@@ -216,43 +216,49 @@ struct Planes {
     float rn[NBP];
 };
 
-// One lane per query row, 32 consecutive rows r = t H + h per warp: the warp copies
-// its rows (one contiguous block of the token-major input) into shared memory with
-// coalesced loads, then every lane forms the NBP projections of its own row in fp32
-// (normals broadcast from shared memory), keeps the sign of each bit outside its
-// rounding bound and recomputes the rest in fp64 in index order. The code is stored
-// token-major, and the lane stamps its code's prompt bucket for its frame.
+// Two lanes per query row, 16 consecutive rows r = t H + h per warp: the warp copies its
+// rows (one contiguous block of the token-major input) into shared memory with coalesced
+// loads, then lane 2 i + u forms projections u NBP/2 ... u NBP/2 + NBP/2 - 1 of row i in
+// fp32 (normals broadcast from shared memory; the second half of the normals sits 16 bytes
+// further so that the two lanes' loads fall in different banks), keeps the sign of each bit
+// outside its rounding bound and recomputes the rest in fp64 in index order. The code is
+// stored token-major, and the row's even lane stamps its code's prompt bucket for its frame.
 template <int D, int NBP>
 __global__ void __launch_bounds__(kWarps * 32)
 annca_mark_kernel(const __nv_bfloat16* __restrict__ Q, int rows, int P, int F, AnnView a,
                   const float* __restrict__ R, const __grid_constant__ Planes<D, NBP> pl, Stats* stats) {
     using S = MarkSmem<D>;
-    constexpr int W = D / 8;   // 16-byte words per row
+    constexpr int W = D / 8;        // 16-byte words per row
+    constexpr int HB = NBP / 2;     // projections per lane
+    static_assert(NBP % 2 == 0, "two lanes per row");
     extern __shared__ __align__(16) uint8_t mk_smem[];
     uint8_t* sRows = mk_smem;
-    __shared__ __align__(16) float sR[NBP * D];   // the normals, broadcast to every lane
-    for (int i = threadIdx.x; i < NBP * D; i += blockDim.x) sR[i] = pl.v[i];
+    __shared__ __align__(16) float sR[NBP * D + 4];   // the normals; bits >= HB start 4 floats later
+    for (int i = threadIdx.x; i < NBP * D; i += blockDim.x) sR[i + (i >= HB * D ? 4 : 0)] = pl.v[i];
     __syncthreads();
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const int half = lane & 1, ri = lane >> 1;
+    const float* myR = sR + half * (HB * D + 4);
     const int nbits = a.nbits;
     grid_dependency_wait();
-    uint8_t* mine = sRows + wib * 32 * S::RB;
+    uint8_t* mine = sRows + wib * 16 * S::RB;
     const float gam2 = 2.f * (float)(D + 2) * kU32;
     unsigned rechecks = 0;
-    for (int base = (blockIdx.x * kWarps + wib) * 32; base < rows; base += gridDim.x * kWarps * 32) {
-        const int n = min(32, rows - base);
+    for (int base = (blockIdx.x * kWarps + wib) * 16; base < rows; base += gridDim.x * kWarps * 16) {
+        const int n = min(16, rows - base);
         const uint4* src = reinterpret_cast<const uint4*>(Q + (int64_t)base * D);
-#pragma unroll 4
+#pragma unroll 8
         for (int w = lane; w < n * W; w += 32) {
             const int row = w / W, col = w - row * W;
             *reinterpret_cast<uint4*>(mine + row * S::RB + col * 16) = src[w];
         }
         __syncwarp();
-        if (lane < n) {
-            const uint8_t* rowp = mine + lane * S::RB;
-            float acc[NBP];
+        uint32_t code = 0;
+        if (ri < n) {
+            const uint8_t* rowp = mine + ri * S::RB;
+            float acc[HB];
 #pragma unroll
-            for (int b = 0; b < NBP; ++b) acc[b] = 0.f;
+            for (int b = 0; b < HB; ++b) acc[b] = 0.f;
             float n2 = 0.f;
 #pragma unroll 1
             for (int c = 0; c < W; ++c) {
@@ -267,9 +273,9 @@ annca_mark_kernel(const __nv_bfloat16* __restrict__ Q, int rows, int P, int F, A
 #pragma unroll
                 for (int k = 0; k < 8; ++k) n2 = fmaf(x[k], x[k], n2);
 #pragma unroll
-                for (int b = 0; b < NBP; ++b) {
-                    const float4 r0 = *reinterpret_cast<const float4*>(sR + b * D + c * 8);
-                    const float4 r1 = *reinterpret_cast<const float4*>(sR + b * D + c * 8 + 4);
+                for (int b = 0; b < HB; ++b) {
+                    const float4 r0 = *reinterpret_cast<const float4*>(myR + b * D + c * 8);
+                    const float4 r1 = *reinterpret_cast<const float4*>(myR + b * D + c * 8 + 4);
                     float t = acc[b];
                     t = fmaf(r0.x, x[0], t);
                     t = fmaf(r0.y, x[1], t);
@@ -285,23 +291,29 @@ annca_mark_kernel(const __nv_bfloat16* __restrict__ Q, int rows, int P, int F, A
             // |<R_b,x>| > 2 (d+2) u |R_b||x| certifies the fp32 sign (any summation order
             // errs by at most (d+2) u |R_b||x|; doubled for margin); else fp64, index order
             const float nx = sqrtf(n2);
-            uint32_t code = 0;
 #pragma unroll
-            for (int b = 0; b < NBP; ++b) {
+            for (int k = 0; k < HB; ++k) {
+                const int b = half * HB + k;
                 if (b >= nbits) break;
-                bool bit = acc[b] >= 0.f;
-                if (!(fabsf(acc[b]) > gam2 * pl.rn[b] * nx + 1e-30f)) {
+                bool bit = acc[k] >= 0.f;
+                if (!(fabsf(acc[k]) > gam2 * pl.rn[b] * nx + 1e-30f)) {
+                    // (the shared copy holds the bf16 normals exactly; products are exact in fp64)
+                    const float* Rb = myR + k * D;
                     double s64 = 0.0;
+#pragma unroll 8
                     for (int i = 0; i < D; ++i) {
                         const uint16_t u = *reinterpret_cast<const uint16_t*>(rowp + 2 * i);
-                        s64 = fma((double)R[b * D + i], (double)__uint_as_float((uint32_t)u << 16), s64);
+                        s64 = fma((double)Rb[i], (double)__uint_as_float((uint32_t)u << 16), s64);
                     }
                     bit = s64 >= 0.0;
                     ++rechecks;
                 }
                 code |= (uint32_t)bit << b;
             }
-            const int r = base + lane;
+        }
+        code |= __shfl_xor_sync(0xffffffffu, code, 1);   // the two halves' bits
+        if (ri < n && half == 0) {
+            const int r = base + ri;
             a.qcode[r] = code;
             const int t = (int)((uint32_t)r / (uint32_t)a.H);
             const int h = r - t * a.H;
@@ -416,7 +428,7 @@ cudaError_t mark_t(const __nv_bfloat16* Q, int rows, int P, int F, const AnnView
         for (int i = 0; i < D; ++i) pl.v[b * D + i] = (b < a.nbits) ? Rhost[b * D + i] : 0.f;
         pl.rn[b] = (b < a.nbits) ? Rnorm_host[b] : 0.f;
     }
-    const int grid = (rows + kWarps * 32 - 1) / (kWarps * 32);
+    const int grid = (rows + kWarps * 16 - 1) / (kWarps * 16);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kWarps * 32);
@@ -437,6 +449,7 @@ cudaError_t select_t(const AnnView& a, const void* Qv, int64_t Tq, int P, int F,
     const int rows = (int)(Tq * a.H);   // < 2^31 (host check)
     cudaError_t e;
     if (a.nbits <= 8) e = mark_t<D, 8>(Q, rows, P, F, a, R, Rhost, Rnorm_host, stats, st);
+    else if (a.nbits <= 12) e = mark_t<D, 12>(Q, rows, P, F, a, R, Rhost, Rnorm_host, stats, st);
     else if (a.nbits <= 16) e = mark_t<D, 16>(Q, rows, P, F, a, R, Rhost, Rnorm_host, stats, st);
     else e = mark_t<D, 24>(Q, rows, P, F, a, R, Rhost, Rnorm_host, stats, st);
     if (e != cudaSuccess) return e;

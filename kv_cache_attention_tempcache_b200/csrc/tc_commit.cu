@@ -430,7 +430,7 @@ stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView 
                 bool bit = a >= 0.f;
                 if (!(fabsf(a) > gam2 * pl.rn[b] * nx + 1e-30f)) {
                     double s64 = 0.0;
-                    for (int i = 0; i < D; ++i) s64 = fma((double)R[b * D + i], (double)srow_at<E>(my, i), s64);
+                    for (int i = 0; i < D; ++i) s64 = fma((double)sR[b * D + i], (double)srow_at<E>(my, i), s64);
                     bit = s64 >= 0.0;
                     ++hre;
                 }
@@ -480,8 +480,10 @@ stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView 
                 if (b >= nbits) break;
                 bool bit = acc[b] >= 0.f;
                 if (!(fabsf(acc[b]) > gam2 * pl.rn[b] * nx + 1e-30f)) {   // inside the band (or not finite)
+                    // (the shared copy holds the bf16 normals exactly; products are exact in fp64)
                     double s64 = 0.0;
-                    for (int i = 0; i < D; ++i) s64 = fma((double)R[b * D + i], (double)srow_at<E>(my, i), s64);
+#pragma unroll 8
+                    for (int i = 0; i < D; ++i) s64 = fma((double)sR[b * D + i], (double)srow_at<E>(my, i), s64);
                     bit = s64 >= 0.0;
                     ++hre;
                 }
