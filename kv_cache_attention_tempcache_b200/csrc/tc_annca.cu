@@ -226,7 +226,7 @@ struct Planes {
 template <int D, int NBP>
 __global__ void __launch_bounds__(kWarps * 32)
 annca_mark_kernel(const __nv_bfloat16* __restrict__ Q, int rows, int P, int F, AnnView a,
-                  const float* __restrict__ R, const __grid_constant__ Planes<D, NBP> pl, Stats* stats) {
+                  const __grid_constant__ Planes<D, NBP> pl, Stats* stats) {
     using S = MarkSmem<D>;
     constexpr int W = D / 8;        // 16-byte words per row
     constexpr int HB = NBP / 2;     // projections per lane
@@ -439,7 +439,7 @@ cudaError_t mark_t(const __nv_bfloat16* Q, int rows, int P, int F, const AnnView
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, annca_mark_kernel<D, NBP>, Q, rows, P, F, a, R, pl, stats);
+    return cudaLaunchKernelEx(&cfg, annca_mark_kernel<D, NBP>, Q, rows, P, F, a, pl, stats);
 }
 
 template <int D>

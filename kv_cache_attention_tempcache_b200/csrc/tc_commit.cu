@@ -348,7 +348,7 @@ __device__ __forceinline__ float dot32_f32(const uint8_t* x, const float* __rest
 template <typename E, int D, int NBP, bool INTRA, bool MEAN>
 __global__ void __launch_bounds__(kStageWarps * 32, 4)
 stage_search_kernel(const E* __restrict__ K, const E* __restrict__ V, CacheView c, StageView s,
-                    const float* __restrict__ R, const __grid_constant__ StagePlanes<D, NBP> pl, float tau,
+                    const __grid_constant__ StagePlanes<D, NBP> pl, float tau,
                     int32_t* ctr, Stats* stats) {
     using S = StageSmem<E, D>;
     const double tau64 = (double)tau;
@@ -1474,7 +1474,7 @@ cudaError_t stage_n(const CacheView& c, const StageView& s, const void* K, const
     const int64_t items = (int64_t)c.H * ((s.T + 31) / 32);
     const int grid = grid_for_rows(items, kStageWarps, 148 * 4);
     e = launch_pdl_smem(kern, grid, kStageWarps * 32, smem, st, reinterpret_cast<const E*>(K),
-                        reinterpret_cast<const E*>(V), c, s, R, pl, tau, ctr, stats);
+                        reinterpret_cast<const E*>(V), c, s, pl, tau, ctr, stats);
     *launches += 1;
     if (e == cudaSuccess && INTRA) {
         const int dgrid = grid_for_rows(s.T * c.H, 4 * kWarps, 148 * 2);
