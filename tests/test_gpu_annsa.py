@@ -71,6 +71,14 @@ def test_every_ordering_path(nbits):
     run(cfg)
 
 
+@pytest.mark.parametrize("P", [5, 129])
+def test_blocks_with_few_tokens(P):
+    # T = 5 leaves most of the eight ordering blocks of a head empty; T = 129 puts one token
+    # past the first 128-row tile
+    cfg = CROSS_CONFIGS["annca-tiny"].replace(H=2, P=P, F=1, nbits=6, seed=3030 + P)
+    run(cfg)
+
+
 def test_large_logits_take_the_running_reference():
     # |q| max|k| scale log2(e) ~ 130 > 40: the kernel cannot use the fixed softmax
     # reference and starts each row's running reference at its own logit
