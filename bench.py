@@ -737,8 +737,8 @@ def run_annsa(args):
                    "l2": f"inputs larger than L2 ({calls * 3 * cfg.T * cfg.H * cfg.d * 2 / 1e9:.2f} GB of "
                          "distinct Q, K, V per step)",
                    "parallelism": f"independent layer per rank x{world}"},
-        "roofline": {"bound": "tensor", "kernel": "annsa_order_kernel + annsa_pack_kernel + attend_bf16_duo_kernel "
-                                                  "(sparse), one call",
+        "roofline": {"bound": "tensor", "kernel": "annsa_bcount_kernel + annsa_bplace_kernel + annsa_pack_kernel + "
+                                                  "attend_bf16_duo_kernel (sparse), one call",
                      "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
                      "peak_kind": f"{peak_kind} bf16 dense, burst", "traffic": None,
                      "flops_per_call": float(np.mean(flops)), "avg_call_us": 1e6 * call_sec},
