@@ -13,7 +13,7 @@
 //   annca_mark_kernel     per call: two lanes per query row hash it, then look its code
 //                         up (a table of the head's codes for nbits <= 16, else a binary
 //                         search of its sorted codes) and, if the prompt has that code,
-//                         stamps the bucket with the call's number for the query's frame
+//                         stamp the bucket with the call's number for the query's frame
 //                         (written only while the stamp differs, so the many queries of
 //                         one bucket rarely store).
 //   annca_pack_kernel     per call: a few blocks per (head, frame) list the prompt tokens
