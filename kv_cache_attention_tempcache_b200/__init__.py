@@ -114,12 +114,95 @@ def _np_ptr(a: np.ndarray):
     return a.ctypes.data_as(ctypes.c_void_p)
 
 
+class _HostCopies:
+    """Side streams for host tensors, one pair per device. A host input is copied on the
+    H2D stream and the current stream waits for that copy; a host output is filled on the
+    D2H stream once the current stream has produced it. The kernels of one call then
+    overlap the transfers of the next (and of the previous call's result). The device
+    copies are tied to the streams that use them (record_stream), so the caching allocator
+    reuses their memory only after that work."""
+
+    _per_device = {}
+
+    def __init__(self, dev: int):
+        self.h2d = torch.cuda.Stream(dev)
+        self.d2h = torch.cuda.Stream(dev)
+
+    @classmethod
+    def get(cls) -> "_HostCopies":
+        dev = torch.cuda.current_device()
+        if dev not in cls._per_device:
+            cls._per_device[dev] = cls(dev)
+        return cls._per_device[dev]
+
+    def to_device(self, x: torch.Tensor) -> torch.Tensor:
+        cur = torch.cuda.current_stream()
+        with torch.cuda.stream(self.h2d):
+            xd = x.to("cuda", non_blocking=True)
+        cur.wait_stream(self.h2d)
+        xd.record_stream(cur)
+        return xd
+
+    def to_host(self, xd: torch.Tensor, out: torch.Tensor):
+        self.d2h.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(self.d2h):
+            out.copy_(xd, non_blocking=True)
+        xd.record_stream(self.d2h)
+
+    def join(self):
+        cur = torch.cuda.current_stream()
+        cur.wait_stream(self.h2d)
+        cur.wait_stream(self.d2h)
+
+    def synchronize(self):
+        self.h2d.synchronize()
+        self.d2h.synchronize()
+
+
+def host_copy_streams():
+    """(H2D stream, D2H stream) that host inputs and outputs of this package use on the
+    current device. A caller timing an end-to-end region makes the H2D stream wait for its
+    start event so that no copy begins before it."""
+    io = _HostCopies.get()
+    return io.h2d, io.d2h
+
+
+def join_host_copies():
+    """Make the current stream wait for every host copy issued so far on this device."""
+    _HostCopies.get().join()
+
+
+def _to_device(x: torch.Tensor) -> torch.Tensor:
+    return x if x.is_cuda else _HostCopies.get().to_device(x)
+
+
+def _out_for(Q: torch.Tensor, out: torch.Tensor | None):
+    """(device output to compute into, host tensor to fill afterwards or None)."""
+    if out is None:
+        return torch.empty_like(Q), None
+    if out.shape != Q.shape or out.dtype != Q.dtype:
+        raise ValueError("out must match Q in shape and dtype")
+    if out.is_cuda:
+        return out, None
+    return torch.empty_like(Q), out
+
+
+def _finish(out: torch.Tensor, host: torch.Tensor | None) -> torch.Tensor:
+    if host is None:
+        return out
+    _HostCopies.get().to_host(out, host)
+    return host
+
+
 class TempCache:
     """One attention layer's TempCache on the current CUDA device.
 
     K, V, Q are [T, H, d] torch tensors in the storage dtype (torch.bfloat16 or
-    torch.float32). CUDA tensors are used in place; CPU tensors are copied to the
-    device on the current stream first (the end-to-end path).
+    torch.float32). CUDA tensors are used in place. CPU tensors (the end-to-end path;
+    pinned memory for asynchronous copies) are copied to the device on a side stream that
+    the current stream waits for; a CPU `out` of attend() is filled from a second side
+    stream after the kernels, and holds the result once sync() or join_host_copies() and
+    the current stream have completed.
     """
 
     def __init__(self, H: int, d: int, nbits: int, tau: float, capacity: int, dtype: str = "bf16",
@@ -153,9 +236,7 @@ class TempCache:
             raise TypeError(f"{name} must be {self.torch_dtype}, got {x.dtype}")
         if x.dim() != 3 or x.shape[1] != self.H or x.shape[2] != self.d:
             raise ValueError(f"{name} must be [T, {self.H}, {self.d}], got {tuple(x.shape)}")
-        if not x.is_cuda:
-            x = x.to("cuda", non_blocking=True)
-        return x.contiguous()
+        return _to_device(x.contiguous())
 
     @staticmethod
     def _stream():
@@ -177,10 +258,9 @@ class TempCache:
 
     def attend(self, Q: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
         Q = self._dev(Q, "Q")
-        if out is None:
-            out = torch.empty_like(Q)
+        out, host = _out_for(Q, out)
         _check(lib.tc_attend(self._h, Q.data_ptr(), Q.shape[0], out.data_ptr(), self._stream()), "tc_attend")
-        return out
+        return _finish(out, host)
 
     def flush(self):
         _check(lib.tc_flush(self._h, self._stream()), "tc_flush")
@@ -191,6 +271,11 @@ class TempCache:
 
     def sync(self):
         _check(lib.tc_sync(self._h), "tc_sync")
+        if torch.cuda.is_available() and torch.cuda.is_initialized():
+            _HostCopies.get().synchronize()
+
+    def join_host_copies(self):
+        join_host_copies()
 
     def cache_size(self) -> np.ndarray:
         out = np.zeros(self.H, dtype=np.int64)
@@ -292,9 +377,7 @@ class AnnCA:
             raise TypeError(f"{name} must be torch.bfloat16, got {x.dtype}")
         if x.dim() != 3 or x.shape[1] != self.H or x.shape[2] != self.d:
             raise ValueError(f"{name} must be [n, {self.H}, {self.d}], got {tuple(x.shape)}")
-        if not x.is_cuda:
-            x = x.to("cuda", non_blocking=True)
-        return x.contiguous()
+        return _to_device(x.contiguous())
 
     def set_prompt(self, Kp: torch.Tensor, Vp: torch.Tensor):
         Kp = self._dev(Kp, "Kp")
@@ -307,11 +390,10 @@ class AnnCA:
 
     def attend(self, Q: torch.Tensor, P: int, out: torch.Tensor | None = None) -> torch.Tensor:
         Q = self._dev(Q, "Q")
-        if out is None:
-            out = torch.empty_like(Q)
+        out, host = _out_for(Q, out)
         _check(lib.tc_annca_attend(self._h, Q.data_ptr(), Q.shape[0], int(P), out.data_ptr(), TempCache._stream()),
                "tc_annca_attend")
-        return out
+        return _finish(out, host)
 
     def kept(self):
         """Inspection of the last attend: (keep [H, F, L] bool, query codes [H, T], prompt codes [H, L])."""
@@ -342,12 +424,11 @@ class AnnCA:
         V = self._dev(V, "V")
         if not (Q.shape == K.shape == V.shape):
             raise ValueError("Q, K and V shapes differ")
-        if out is None:
-            out = torch.empty_like(Q)
+        out, host = _out_for(Q, out)
         self._keep_sa = [Q, K, V]
         _check(lib.tc_annsa_attend(self._h, Q.data_ptr(), K.data_ptr(), V.data_ptr(), Q.shape[0], out.data_ptr(),
                                    TempCache._stream()), "tc_annsa_attend")
-        return out
+        return _finish(out, host)
 
     def hyperplanes(self) -> np.ndarray:
         R = np.zeros((self.nbits, self.d), np.float32)
@@ -356,6 +437,8 @@ class AnnCA:
 
     def sync(self):
         _check(lib.tc_annca_sync(self._h), "tc_annca_sync")
+        if torch.cuda.is_available() and torch.cuda.is_initialized():
+            _HostCopies.get().synchronize()
 
     def close(self):
         if getattr(self, "_h", None) is not None and self._h.value:
@@ -385,16 +468,15 @@ class LVSA:
         for x, name in ((Q, "Q"), (K, "K"), (V, "V")):
             if x.dtype != torch.bfloat16 or x.dim() != 3 or x.shape[1] != self.H or x.shape[2] != self.d:
                 raise ValueError(f"{name} must be [T*P, {self.H}, {self.d}] bfloat16")
-            t.append((x if x.is_cuda else x.to("cuda", non_blocking=True)).contiguous())
+            t.append(_to_device(x.contiguous()))
         Q, K, V = t
         if Q.shape[0] % self.P:
             raise ValueError("Q must hold whole frames")
-        if out is None:
-            out = torch.empty_like(Q)
+        out, host = _out_for(Q, out)
         self._keep = [Q, K, V]
         _check(lib.tc_lvsa_attend(self._h, Q.data_ptr(), K.data_ptr(), V.data_ptr(), Q.shape[0] // self.P,
                                   int(step), out.data_ptr(), TempCache._stream()), "tc_lvsa_attend")
-        return out
+        return _finish(out, host)
 
     def frames(self):
         """A(t) of the last call, as a list of arrays."""
@@ -409,6 +491,8 @@ class LVSA:
 
     def sync(self):
         _check(lib.tc_lvsa_sync(self._h), "tc_lvsa_sync")
+        if torch.cuda.is_available() and torch.cuda.is_initialized():
+            _HostCopies.get().synchronize()
 
     def close(self):
         if getattr(self, "_h", None) is not None and self._h.value:
