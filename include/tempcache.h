@@ -43,7 +43,7 @@ typedef enum {
     TC_ECUDA = 4,      /* a CUDA runtime or driver call failed                     */
     TC_ESTATE = 5,     /* call not valid in the current state                      */
     TC_ETIMEOUT = 6,   /* a kernel gave up waiting on one of its own barriers      */
-    TC_ENOTIMPL = 7,   /* combination not supported by this build                  */
+    TC_ENOTIMPL = 7,   /* combination of options the library does not support      */
     TC_EDEVICE = 8     /* no usable sm_100 device                                  */
 } tc_status;
 
@@ -320,7 +320,6 @@ void tc_annca_destroy(tc_annca_handle h);
  * (right first on a tie, the other side at the video's edge), until |G_s u W(t)| >= C or
  * it covers all T frames. Query tokens of frame t attend (bidirectionally, plain softmax,
  * bf16 tensor cores) to every token of the frames in A(t).
- * Not yet run on a GPU in this build: see the design notes.
  */
 typedef struct tc_lvsa_ctx* tc_lvsa_handle;
 
