@@ -79,6 +79,13 @@ def test_blocks_with_few_tokens(P):
     run(cfg)
 
 
+def test_largest_block():
+    # T = 16 383, one short of the largest block: every warp of the ordering takes all of
+    # its 32-token steps
+    cfg = CROSS_CONFIGS["annca-tiny"].replace(H=1, d=128, P=5461, F=3, nbits=10, sigma=0.5, seed=3040)
+    run(cfg)
+
+
 def test_large_logits_take_the_running_reference():
     # |q| max|k| scale log2(e) ~ 130 > 40: the kernel cannot use the fixed softmax
     # reference and starts each row's running reference at its own logit
